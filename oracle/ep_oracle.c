@@ -1,0 +1,225 @@
+/*
+ * ep_oracle.c -- CPU oracle for MoE expert-parallel dispatch and combine.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the plain, slow, single-threaded
+ * statement of what the dispatch and combine calls compute. It exists so that
+ * tests, the smoke check and the CPU baseline of the bench can check the CUDA
+ * path against it. Nothing in the product links or calls it, and it shares no
+ * header, helper, table or constant with the CUDA path.
+ *
+ * Sources (mori pages):
+ *   - "MORI JIT v2" design page, §3.2 (EpCfg: worldSize, hiddenDim,
+ *     maxTokPerRank, numExpertPerRank, numExpertPerToken, maxRecv with
+ *     0 meaning worldSize*maxTokPerRank and serving as the stride of the flat
+ *     receive index, dtype, useWeights), §3.5 (validity rules), §3.7 (dispatch
+ *     moves bytes only; combine reduces), §8 (destPe = expert / numExpertPerRank).
+ *   - mori PR #599 "Perf/ep disp 1250 ship", the per-optimisation list:
+ *     dedup of (token, destPe), the per-destination histogram, the
+ *     three-field per-token meta record, the receive count that is stored
+ *     rather than accumulated.
+ *
+ * Readings where the pages leave a step open (each one is also listed in the
+ * design notes of the repository):
+ *   - Slots of one destination are ordered by (source rank, source token)
+ *     ascending. The pages reserve slots with an atomic fetch_add, whose order
+ *     is not defined.
+ *   - A token's set of destinations P(r,t) is the set of destPe over its valid
+ *     topk entries; an entry < 0 is masked; an entry >= E is a contract
+ *     violation: it is reported in the status word and treated as masked.
+ *   - Per-destination weight w(r,t,pe) = fold over topk position j ascending
+ *     of s = s + w_j (float32, s0 = +0.0f) over the entries that map to pe;
+ *     1.0f when useWeights is 0.
+ *   - Meta record per (pe, slot), array of structs with 3 + k int32 fields:
+ *     source rank, source token, weight sum (float32 bits), then for every topk
+ *     position j the local expert id (expert - pe*numExpertPerRank) when entry
+ *     j maps to pe, else -1.
+ *   - Combine: out[r][t] = bf16_rne( fold over pe in P(r,t) ascending of
+ *     acc = fmaf(w(r,t,pe), y[pe][slot], acc) ), acc0 = +0.0f; a token with an
+ *     empty P gets a zero row.
+ *   - Receive rows and meta past recv_count[pe] are not written.
+ *
+ * Floating point: the pages fix float32 accumulation with bfloat16 output, so
+ * the oracle computes in float32 with one fused multiply-add per term (C99
+ * fmaf, correctly rounded) and converts with round-to-nearest-even. Build with
+ * -ffp-contract=off so that the compiler fuses nothing else.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int32_t worldSize;
+    int32_t hiddenDim;
+    int32_t maxTokPerRank;
+    int32_t numExpertPerRank;
+    int32_t numExpertPerToken;
+    int32_t maxRecv;
+    int32_t dtype;
+    int32_t useWeights;
+} OracleCfg;
+
+enum {
+    ORACLE_OK = 0,
+    ORACLE_ERR_ARG = -1,
+    ORACLE_ERR_NOMEM = -2,
+    ORACLE_STATUS_EXPERT_RANGE = 1, /* positive: an id >= E was seen (masked) */
+};
+
+/* bfloat16 <-> float32, from the formats: bf16 is the top half of a float32. */
+static float bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round a float32 to bfloat16, nearest with ties to even. A NaN keeps its sign
+ * and is forced quiet. */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u)
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t lower = u & 0xffffu;
+    uint32_t upper = u >> 16;
+    /* above half: round up; exactly half: round up only when upper is odd */
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))
+        upper += 1u;
+    return (uint16_t)upper;
+}
+
+static int cfg_ok(const OracleCfg *c)
+{
+    if (!c) return 0;
+    if (c->worldSize <= 0 || c->hiddenDim <= 0 || c->maxTokPerRank <= 0) return 0;
+    if (c->numExpertPerRank <= 0 || c->numExpertPerToken <= 0) return 0;
+    if (c->dtype != 0) return 0; /* bf16 only */
+    return 1;
+}
+
+static int64_t recv_cap(const OracleCfg *c)
+{
+    return c->maxRecv == 0 ? (int64_t)c->worldSize * c->maxTokPerRank : c->maxRecv;
+}
+
+int oracle_recv_capacity(const OracleCfg *c)
+{
+    return cfg_ok(c) ? (int)recv_cap(c) : ORACLE_ERR_ARG;
+}
+
+/*
+ * Dispatch. Shapes (all row-major, C order):
+ *   x          uint16 [W][T][h]          bf16 bits
+ *   topk_idx   int32  [W][T][k]
+ *   topk_w     float  [W][T][k]          may be NULL when useWeights == 0
+ *   recv_x     uint16 [W][R][h]          R = maxRecv (or W*T)
+ *   recv_meta  int32  [W][R][3+k]
+ *   recv_count int32  [W]
+ *   slotmap    int32  [W][T][W]          slot of (r,t) at pe, or -1
+ *   wsum       float  [W][T][W]          w(r,t,pe), 0 where absent
+ * Returns 0, ORACLE_STATUS_EXPERT_RANGE when an id >= E was masked, or a
+ * negative error.
+ */
+int oracle_dispatch(const OracleCfg *c, const uint16_t *x, const int32_t *topk_idx,
+                    const float *topk_w, uint16_t *recv_x, int32_t *recv_meta,
+                    int32_t *recv_count, int32_t *slotmap, float *wsum)
+{
+    if (!cfg_ok(c) || !x || !topk_idx || !recv_x || !recv_meta || !recv_count ||
+        !slotmap || !wsum)
+        return ORACLE_ERR_ARG;
+    if (c->useWeights && !topk_w) return ORACLE_ERR_ARG;
+
+    const int64_t W = c->worldSize, T = c->maxTokPerRank, h = c->hiddenDim;
+    const int64_t nEpr = c->numExpertPerRank, k = c->numExpertPerToken;
+    const int64_t E = W * nEpr, R = recv_cap(c), M = 3 + k;
+    int status = ORACLE_OK;
+
+    int64_t *next = (int64_t *)calloc((size_t)W, sizeof *next);
+    if (!next) return ORACLE_ERR_NOMEM;
+
+    /* Tokens in (source rank, source token) ascending order; every destination
+     * hands out its slots in that order. */
+    for (int64_t r = 0; r < W; ++r) {
+        for (int64_t t = 0; t < T; ++t) {
+            const int64_t g = r * T + t;
+            const int32_t *ids = topk_idx + g * k;
+            for (int64_t pe = 0; pe < W; ++pe) {
+                int hit = 0;
+                float s = 0.0f;
+                for (int64_t j = 0; j < k; ++j) {
+                    int32_t e = ids[j];
+                    if (e < 0) continue;
+                    if (e >= E) { status = ORACLE_STATUS_EXPERT_RANGE; continue; }
+                    if (e / nEpr != pe) continue;
+                    hit = 1;
+                    if (c->useWeights) s = s + topk_w[g * k + j];
+                }
+                if (!c->useWeights) s = 1.0f;
+                if (!hit) {
+                    slotmap[g * W + pe] = -1;
+                    wsum[g * W + pe] = 0.0f;
+                    continue;
+                }
+                if (next[pe] >= R) { free(next); return ORACLE_ERR_ARG; }
+                const int64_t slot = next[pe]++;
+                memcpy(recv_x + (pe * R + slot) * h, x + g * h, (size_t)h * sizeof(uint16_t));
+                int32_t *meta = recv_meta + (pe * R + slot) * M;
+                meta[0] = (int32_t)r;
+                meta[1] = (int32_t)t;
+                memcpy(&meta[2], &s, sizeof s);
+                for (int64_t j = 0; j < k; ++j) {
+                    int32_t e = ids[j];
+                    meta[3 + j] = (e >= 0 && e < E && e / nEpr == pe) ? (int32_t)(e - pe * nEpr) : -1;
+                }
+                slotmap[g * W + pe] = (int32_t)slot;
+                wsum[g * W + pe] = s;
+            }
+        }
+    }
+    for (int64_t pe = 0; pe < W; ++pe) recv_count[pe] = (int32_t)next[pe];
+    free(next);
+    return status;
+}
+
+/*
+ * Combine. y has recv_x's layout; slotmap and wsum are what oracle_dispatch
+ * wrote; out is uint16 [W][T][h] bf16 bits.
+ */
+int oracle_combine(const OracleCfg *c, const uint16_t *y, const int32_t *slotmap,
+                   const float *wsum, uint16_t *out)
+{
+    if (!cfg_ok(c) || !y || !slotmap || !wsum || !out) return ORACLE_ERR_ARG;
+    const int64_t W = c->worldSize, T = c->maxTokPerRank, h = c->hiddenDim;
+    const int64_t R = recv_cap(c);
+    float *acc = (float *)malloc((size_t)h * sizeof *acc);
+    if (!acc) return ORACLE_ERR_NOMEM;
+
+    for (int64_t g = 0; g < W * T; ++g) {
+        for (int64_t i = 0; i < h; ++i) acc[i] = 0.0f;
+        for (int64_t pe = 0; pe < W; ++pe) {
+            const int32_t slot = slotmap[g * W + pe];
+            if (slot < 0) continue;
+            const float w = wsum[g * W + pe];
+            const uint16_t *row = y + (pe * R + slot) * h;
+            for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, bf16_to_f32(row[i]), acc[i]);
+        }
+        for (int64_t i = 0; i < h; ++i) out[g * h + i] = f32_to_bf16_rne(acc[i]);
+    }
+    free(acc);
+    return ORACLE_OK;
+}
+
+/* The two format conversions, exported so that tests can pin them against an
+ * independent implementation. */
+void oracle_f32_to_bf16(const float *in, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = f32_to_bf16_rne(in[i]);
+}
+
+void oracle_bf16_to_f32(const uint16_t *in, float *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = bf16_to_f32(in[i]);
+}

@@ -1,0 +1,511 @@
+"""Pins for the CPU oracle: checks that tie it to something other than itself.
+
+Each ``pin_*`` function takes an oracle library handle (``lib=None`` is the
+real oracle; the mutant tests pass copies with planted mistakes) and raises
+AssertionError when the oracle disagrees with:
+
+* a second, independent formulation of dispatch on tiny inputs (Python sets,
+  ``sorted`` order, dict slots) -- ``pin_bruteforce_*``;
+* exact rational arithmetic for the float32 fused-multiply-add fold of
+  combine and the float32 weight sums -- ``pin_combine_exact_fma``;
+* float64 bounds -- ``pin_combine_fp64_bound``;
+* closed forms: the identity-expert round trip without weights is exactly
+  bf16(|P| * x) (the "analytic golden" of the MORI JIT v2 design page, §10);
+  with softmax weights it is x * sum_j w_j within the tolerance; W=1 reduces
+  dispatch to the identity permutation of routed tokens;
+* invariants: conservation of routed rows, one meta record per
+  (rank, token, destPe), slot order, the bound of mori PR #599 on unique
+  copies (max_tokens * min(world_size, topk)), capacity;
+* the two figures the pages print about this routing: the 311 MB staging copy
+  (MORI JIT v2 design page §8) and the ~1374 null writes (mori PR #599);
+* torch's independent float32 -> bfloat16 conversion.
+"""
+from __future__ import annotations
+
+import math
+import os
+import sys
+from fractions import Fraction
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import oracle  # noqa: E402
+from synth.inputs import Workload, make_inputs, workload  # noqa: E402
+
+U32 = 2.0 ** -24  # unit roundoff of float32
+
+
+# ---------------------------------------------------------------- helpers
+def f32_from_bits(b):
+    return np.asarray(b, dtype=np.uint32).view(np.float32)
+
+
+def bf16_bits_to_f64(b):
+    """Exact value of bf16 bit patterns (bf16 = top half of a float32)."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def torch_bf16_bits(f32):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(f32, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def random_small_case(rng, W=None):
+    """A tiny random problem with masked entries, duplicate expert ids,
+    occasional out-of-range-free ids and arbitrary-sign weights."""
+    W = W or int(rng.integers(1, 6))
+    T = int(rng.integers(1, 7))
+    nEpr = int(rng.integers(1, 5))
+    k = int(rng.integers(1, 6))
+    h = 8 * int(rng.integers(1, 4))
+    E = W * nEpr
+    idx = rng.integers(-2, E, size=(W, T, k)).astype(np.int32)  # with replacement: duplicates
+    w = rng.standard_normal((W, T, k)).astype(np.float32)
+    use_w = int(rng.integers(0, 2))
+    maxRecv = [0, W * T, W * T + 3][int(rng.integers(0, 3))]
+    xb = rng.integers(0, 1 << 16, size=(W, T, h)).astype(np.uint16)
+    # keep x finite and far from overflow: exponents >= 2^113 lose their top exponent bit
+    xb = np.where((xb & 0x7F80) >= 0x7880, xb & 0xBFFF, xb).astype(np.uint16)
+    cfg = dict(worldSize=W, hiddenDim=h, maxTokPerRank=T, numExpertPerRank=nEpr,
+               numExpertPerToken=k, maxRecv=maxRecv, dtype=0, useWeights=use_w)
+    return cfg, xb, idx, (w if use_w else None)
+
+
+def brute_routes(cfg, idx):
+    """Second formulation of dispatch's routing, from set semantics:
+    the (destPe, srcRank, srcToken) triples of all valid entries, deduplicated
+    by a set, ordered by ``sorted``; slots numbered per destination."""
+    W, T, k = cfg["worldSize"], cfg["maxTokPerRank"], cfg["numExpertPerToken"]
+    nEpr = cfg["numExpertPerRank"]
+    E = W * nEpr
+    triples = set()
+    for r in range(W):
+        for t in range(T):
+            for j in range(k):
+                e = int(idx[r, t, j])
+                if 0 <= e < E:
+                    triples.add((e // nEpr, r, t))
+    slot, count = {}, [0] * W
+    for pe, r, t in sorted(triples):
+        slot[(pe, r, t)] = count[pe]
+        count[pe] += 1
+    return slot, count
+
+
+# ---------------------------------------------------------------- pins
+def pin_bruteforce_dispatch(lib=None, n_cases=40, seed=11):
+    rng = np.random.default_rng(seed)
+    for _ in range(n_cases):
+        cfg, xb, idx, w = random_small_case(rng)
+        W, T, k, nEpr, h = (cfg[n] for n in ("worldSize", "maxTokPerRank", "numExpertPerToken",
+                                             "numExpertPerRank", "hiddenDim"))
+        R = oracle.recv_capacity(cfg)
+        canary_x = np.full((W, R, h), 0xABCD, dtype=np.uint16)
+        canary_m = np.full((W, R, 3 + k), 0x5EADBEEF, dtype=np.int32)
+        res = oracle.dispatch(cfg, xb, idx, w, recv_x=canary_x, recv_meta=canary_m, lib=lib)
+        slot, count = brute_routes(cfg, idx)
+        assert list(res["recv_count"]) == count, (res["recv_count"], count)
+        for r in range(W):
+            for t in range(T):
+                for pe in range(W):
+                    s = slot.get((pe, r, t), -1)
+                    assert res["slotmap"][r, t, pe] == s
+                    if s < 0:
+                        assert res["wsum"][r, t, pe] == 0.0
+                        continue
+                    assert np.array_equal(res["recv_x"][pe, s], xb[r, t])
+                    meta = res["recv_meta"][pe, s]
+                    assert meta[0] == r and meta[1] == t
+                    # local expert ids: the position-j id, reduced modulo nEpr, where it lives on pe
+                    for j in range(k):
+                        e = int(idx[r, t, j])
+                        want = (e % nEpr) if (0 <= e < W * nEpr and e // nEpr == pe) else -1
+                        assert meta[3 + j] == want
+                    # weight sum: fp32 fold vs exact sum (bound), exact when one term
+                    terms = [float(w[r, t, j]) for j in range(k)
+                             if w is not None and 0 <= idx[r, t, j] < W * nEpr and idx[r, t, j] // nEpr == pe]
+                    got = float(res["wsum"][r, t, pe])
+                    assert np.float32(got).view(np.int32) == meta[2]
+                    if w is None:
+                        assert got == 1.0
+                    else:
+                        exact = math.fsum(terms)
+                        bound = max(len(terms) - 1, 0) * U32 * (sum(abs(v) for v in terms) + abs(exact))
+                        assert abs(got - exact) <= bound + 1e-45, (got, exact, bound)
+                        if len(terms) == 1:
+                            assert got == terms[0]
+        # untouched past recv_count
+        for pe in range(W):
+            n = count[pe]
+            assert np.all(res["recv_x"][pe, n:] == 0xABCD)
+            assert np.all(res["recv_meta"][pe, n:] == 0x5EADBEEF)
+
+
+def pin_bruteforce_weight_sum_order(lib=None):
+    """The weight sum is the float32 fold in topk order, s0=+0: with three
+    weights whose float32 sum depends on the order, the oracle must return the
+    left-to-right value (computed here with exact rationals and RNE)."""
+    w = np.array([[[1.0, 2.0 ** -24, 2.0 ** -24]]], dtype=np.float32)
+    idx = np.array([[[0, 1, 2]]], dtype=np.int32)
+    cfg = dict(worldSize=1, hiddenDim=8, maxTokPerRank=1, numExpertPerRank=4,
+               numExpertPerToken=3, maxRecv=0, dtype=0, useWeights=1)
+    res = oracle.dispatch(cfg, np.zeros((1, 1, 8), np.uint16), idx, w, lib=lib)
+    # left to right: (1 + 2^-24) rounds to 1 (tie to even), + 2^-24 rounds to 1 again.
+    s = Fraction(0)
+    for v in w[0, 0]:
+        s = round_fraction_to_f32(s + Fraction(float(v)))
+    assert float(res["wsum"][0, 0, 0]) == float(s) == 1.0
+
+
+def round_fraction_to_f32(q: Fraction) -> Fraction:
+    """Round an exact rational to the nearest float32 (ties to even), by
+    integer arithmetic on the significand. Handles subnormals; no overflow
+    handling (the inputs used here stay far from it)."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    # now 2^e <= a < 2^(e+1); float32 keeps 24 significant bits, exponent >= -126
+    lsb_exp = max(e, -126) - 23
+    scaled = a / (Fraction(2) ** lsb_exp)
+    n, rem = divmod(scaled.numerator, scaled.denominator)
+    twice = 2 * rem
+    if twice > scaled.denominator or (twice == scaled.denominator and n % 2 == 1):
+        n += 1
+    return sign * Fraction(n) * Fraction(2) ** lsb_exp
+
+
+def round_fraction_to_bf16(q: Fraction) -> Fraction:
+    """Nearest bfloat16 (8 significant bits, same exponent range as float32)."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    lsb_exp = max(e, -126) - 7
+    scaled = a / (Fraction(2) ** lsb_exp)
+    n, rem = divmod(scaled.numerator, scaled.denominator)
+    twice = 2 * rem
+    if twice > scaled.denominator or (twice == scaled.denominator and n % 2 == 1):
+        n += 1
+    return sign * Fraction(n) * Fraction(2) ** lsb_exp
+
+
+def pin_combine_exact_fma(lib=None, seed=5):
+    """Combine equals, bit for bit, the fold acc = RNE32(w*y + acc) over pe
+    ascending, evaluated with exact rationals, then RNE to bfloat16."""
+    wl = workload("tiny")
+    d = make_inputs(wl)
+    cfg = wl.cfg()
+    res = oracle.dispatch(cfg, d["x"], d["topk_idx"], d["topk_w"], lib=lib)
+    rng = np.random.default_rng(seed)
+    # an arbitrary expert output (not the identity) so that terms differ
+    y = res["recv_x"].copy()
+    n = int(res["recv_count"].max())
+    y[:, :n] = rng.integers(0, 1 << 16, size=y[:, :n].shape).astype(np.uint16)
+    y = np.where((y & 0x7F80) == 0x7F80, y & 0x807F, y).astype(np.uint16)
+    out = oracle.combine(cfg, y, res["slotmap"], res["wsum"], lib=lib)
+    W, T, h = wl.W, wl.max_tok, wl.h
+    yv = bf16_bits_to_f64(y)
+    outv = bf16_bits_to_f64(out)
+    for r in range(W):
+        for t in range(T):
+            for i in range(h):
+                acc = Fraction(0)
+                for pe in range(W):
+                    s = int(res["slotmap"][r, t, pe])
+                    if s < 0:
+                        continue
+                    acc = round_fraction_to_f32(Fraction(float(res["wsum"][r, t, pe])) * Fraction(float(yv[pe, s, i])) + acc)
+                want = round_fraction_to_bf16(acc)
+                assert Fraction(float(outv[r, t, i])) == want, (r, t, i, float(want), outv[r, t, i])
+
+
+def fma_sensitive_case():
+    """One token on two destinations whose combine result, in bf16, depends on
+    the product w*y being fused into the add (one rounding) rather than rounded
+    first: w1=a on a row of 1.0, then w2 on a row of 1.25, with a + w2*1.25
+    just above the float32 midpoint next to the bf16 tie 1 + 2^-8.
+    Returns (cfg, topk_idx, topk_w, y) with y in the receive layout."""
+    a = np.array([0x393D0800], np.uint32).view(np.float32)[0]
+    w2 = np.array([0x3F4D9027], np.uint32).view(np.float32)[0]
+    h = 8
+    cfg = dict(worldSize=2, hiddenDim=h, maxTokPerRank=1, numExpertPerRank=1,
+               numExpertPerToken=2, maxRecv=0, dtype=0, useWeights=1)
+    idx = np.array([[[0, 1]], [[-1, -1]]], dtype=np.int32)
+    w = np.array([[[a, w2]], [[0, 0]]], dtype=np.float32)
+    y = np.zeros((2, 2, h), dtype=np.uint16)
+    y[0, 0, :] = 0x3F80  # 1.0
+    y[1, 0, :] = 0x3FA0  # 1.25
+    return cfg, idx, w, y
+
+
+def pin_combine_single_rounding_case(lib=None):
+    """The crafted case above: the exact fold with one rounding per term gives
+    1 + 2^-7 (bf16 0x3F81); rounding the product first would give 1.0."""
+    cfg, idx, w, y = fma_sensitive_case()
+    res = oracle.dispatch(cfg, np.zeros((2, 1, 8), np.uint16), idx, w, lib=lib)
+    out = oracle.combine(cfg, y, res["slotmap"], res["wsum"], lib=lib)
+    acc = Fraction(0)
+    for pe, yv in ((0, 1.0), (1, 1.25)):
+        acc = round_fraction_to_f32(Fraction(float(w[0, 0, pe])) * Fraction(yv) + acc)
+    want = round_fraction_to_bf16(acc)
+    assert want == 1 + Fraction(1, 128)
+    assert np.all(out[0, 0] == 0x3F81), out[0, 0]
+    assert np.all(out[1, 0] == 0)
+
+
+def pin_combine_fp64_bound(lib=None, seed=7):
+    """Combine against the float64 sum of w*y: fp32 fold error plus one bf16 rounding."""
+    rng = np.random.default_rng(seed)
+    for _ in range(10):
+        cfg, xb, idx, w = random_small_case(rng)
+        res = oracle.dispatch(cfg, xb, idx, w, lib=lib)
+        y = res["recv_x"]
+        out = oracle.combine(cfg, y, res["slotmap"], res["wsum"], lib=lib)
+        W, T = cfg["worldSize"], cfg["maxTokPerRank"]
+        yv = bf16_bits_to_f64(y)
+        outv = bf16_bits_to_f64(out)
+        for r in range(W):
+            for t in range(T):
+                ref = np.zeros(cfg["hiddenDim"])
+                mag = np.zeros(cfg["hiddenDim"])
+                m = 0
+                for pe in range(W):
+                    s = int(res["slotmap"][r, t, pe])
+                    if s < 0:
+                        continue
+                    m += 1
+                    term = float(res["wsum"][r, t, pe]) * yv[pe, s]
+                    ref += term
+                    mag += np.abs(term)
+                tol = 2.0 ** -8 * np.abs(ref) + 2 * m * U32 * mag + 2.0 ** -132
+                assert np.all(np.abs(outv[r, t] - ref) <= tol), (r, t)
+                if m == 0:
+                    assert np.all(out[r, t] == 0)
+
+
+def pin_roundtrip_unweighted_exact(lib=None):
+    """Identity experts, no weights: out = bf16(|P| * x) exactly, since |P|*x
+    is exact in float32 for |P| <= 32. |P| is counted from the ids here."""
+    for name in ("latency8", "tiny"):
+        wl = workload(name).replace(use_weights=False)
+        d = make_inputs(wl)
+        cfg = wl.cfg()
+        res = oracle.dispatch(cfg, d["x"], d["topk_idx"], None, lib=lib)
+        out = oracle.combine(cfg, res["recv_x"], res["slotmap"], res["wsum"], lib=lib)
+        idx = d["topk_idx"]
+        m = np.zeros(idx.shape[:2], dtype=np.float32)
+        for r in range(wl.W):
+            for t in range(wl.max_tok):
+                m[r, t] = len({int(e) // wl.n_epr for e in idx[r, t] if 0 <= e < wl.E})
+        xf = bf16_bits_to_f64(d["x"]).astype(np.float32)
+        want = torch_bf16_bits(xf * m[..., None])
+        live = m > 0
+        assert np.array_equal(out[live], want[live])
+        assert np.all(out[~live] == 0)  # absent tokens: +0 rows
+
+
+def pin_roundtrip_weighted(lib=None):
+    """Identity experts with softmax weights: out ~= x * sum_j w_j (the
+    weights of a fully routed token sum to 1), within 2^-7|ref| + 1e-3."""
+    wl = workload("tiny")
+    for seed in range(4):
+        d = make_inputs(wl.replace(seed=seed))
+        cfg = wl.cfg()
+        res = oracle.dispatch(cfg, d["x"], d["topk_idx"], d["topk_w"], lib=lib)
+        out = oracle.combine(cfg, res["recv_x"], res["slotmap"], res["wsum"], lib=lib)
+        ref = bf16_bits_to_f64(d["x"]) * d["topk_w"].astype(np.float64).sum(-1, keepdims=True)
+        assert np.all(np.abs(bf16_bits_to_f64(out) - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-3)
+
+
+def pin_single_rank(lib=None):
+    """W=1: dispatch is the identity permutation of the routed tokens; combine
+    is bf16(fp32(wsum * x)) per routed token (one term: fma(w, x, 0) is one
+    float32 rounding of the product), zero for unrouted ones."""
+    rng = np.random.default_rng(3)
+    T, h, k, nEpr = 9, 16, 3, 4
+    idx = rng.integers(-1, nEpr, size=(1, T, k)).astype(np.int32)
+    idx[0, 2] = -1
+    w = rng.random((1, T, k)).astype(np.float32)
+    xb = torch_bf16_bits(rng.standard_normal((1, T, h)).astype(np.float32))
+    cfg = dict(worldSize=1, hiddenDim=h, maxTokPerRank=T, numExpertPerRank=nEpr,
+               numExpertPerToken=k, maxRecv=0, dtype=0, useWeights=1)
+    res = oracle.dispatch(cfg, xb, idx, w, lib=lib)
+    routed = [t for t in range(T) if (idx[0, t] >= 0).any()]
+    assert res["recv_count"][0] == len(routed)
+    for s, t in enumerate(routed):
+        assert np.array_equal(res["recv_x"][0, s], xb[0, t])
+    out = oracle.combine(cfg, res["recv_x"], res["slotmap"], res["wsum"], lib=lib)
+    xf = bf16_bits_to_f64(xb).astype(np.float32)
+    for t in range(T):
+        if t in routed:
+            prod = np.float32(res["wsum"][0, t, 0]) * xf[0, t]  # one float32 rounding
+            assert np.array_equal(out[0, t], torch_bf16_bits(prod))
+        else:
+            assert np.all(out[0, t] == 0)
+
+
+def pin_invariants(lib=None):
+    """Conservation, uniqueness, order, unique-copy bound, capacity -- on the
+    routing of the measured workloads (hidden shrunk to 8: routing does not
+    depend on it)."""
+    for name in ("pr599", "skewed", "latency8"):
+        wl = workload(name).replace(h=8)
+        d = make_inputs(wl)
+        cfg = wl.cfg()
+        res = oracle.dispatch(cfg, d["x"], d["topk_idx"], d["topk_w"], lib=lib)
+        idx = d["topk_idx"]
+        valid = idx >= 0
+        pe_of = np.where(valid, idx // wl.n_epr, -1)
+        hits = np.zeros((wl.W, wl.max_tok, wl.W), dtype=bool)
+        for j in range(wl.k):
+            for pe in range(wl.W):
+                hits[:, :, pe] |= pe_of[:, :, j] == pe
+        # conservation of routed rows and per-destination counts
+        assert res["recv_count"].sum() == hits.sum()
+        assert np.array_equal(res["recv_count"], hits.sum(axis=(0, 1)))
+        assert np.all(res["recv_count"] <= oracle.recv_capacity(cfg))
+        # unique-copy bound of mori PR #599: per source rank <= ct * min(W, k)
+        assert np.all(hits.sum(axis=(1, 2)) <= wl.ct * min(wl.W, wl.k))
+        for pe in range(wl.W):
+            n = res["recv_count"][pe]
+            meta = res["recv_meta"][pe, :n]
+            key = meta[:, 0].astype(np.int64) * wl.max_tok + meta[:, 1]
+            assert np.all(np.diff(key) > 0)  # (srcRank, token) strictly ascending: unique + ordered
+            r_, t_ = np.nonzero(hits[:, :, pe])
+            assert np.array_equal(np.sort(key), r_.astype(np.int64) * wl.max_tok + t_)
+            # local expert ids rebuild the routed expert ids
+            loc = meta[:, 3:]
+            src = idx[meta[:, 0], meta[:, 1]]
+            assert np.all((loc == -1) | ((loc >= 0) & (loc < wl.n_epr)))
+            assert np.array_equal(np.where(loc >= 0, pe * wl.n_epr + loc, -1),
+                                  np.where((src >= 0) & (src // wl.n_epr == pe), src, -1))
+            # the slot map points back at these records
+            assert np.array_equal(res["slotmap"][meta[:, 0], meta[:, 1], pe], np.arange(n))
+
+
+def pin_page_staging_copy(lib=None):
+    """MORI JIT v2 design page §8: a 311 MB staging copy at EP8, hidden 7168,
+    topk 8, 4096 tokens/rank = the rows one rank receives x 14336 bytes."""
+    from conftest import read_golden
+    g = read_golden("staging_copy_ep8_h7168_topk8.txt")
+    wl = workload("main").replace(h=8)
+    assert (wl.W, wl.max_tok, wl.k, wl.n_epr) == (g["world_size"], g["tokens_per_rank"], g["topk"],
+                                                  g["experts_per_rank"])
+    d = make_inputs(wl, with_x=False)
+    cfg = wl.cfg()
+    x = np.zeros((wl.W, wl.max_tok, wl.h), np.uint16)
+    res = oracle.dispatch(cfg, x, d["topk_idx"], d["topk_w"], lib=lib)
+    per_rank_rows = res["recv_count"].sum() / wl.W
+    mb = per_rank_rows * g["hidden"] * g["bytes_per_element"] / 1e6
+    # sampling spread of the mean over 32768 tokens is ~0.3 MB; rounding 0.5 MB
+    assert abs(mb - g["staging_copy_mb"]) <= g["rounding_mb"] + 1.5, mb
+
+
+def pin_page_null_writes(lib=None):
+    """mori PR #599: ~1374 null writes per rank at EP4, ct=512, topk=6 -- one
+    per topk entry that the (token, destPe) dedup drops."""
+    from conftest import read_golden
+    g = read_golden("null_writes_ep4_ct512_topk6.txt")
+    wl = Workload("nullw", W=g["world_size"], max_tok=g["tokens_per_rank"], ct=g["tokens_per_rank"],
+                  h=8, n_epr=g["experts_per_rank"], k=g["topk"], routing="uniform",
+                  use_weights=True, max_recv=0, seed=0)
+    dups = []
+    for seed in range(8):
+        w2 = wl.replace(seed=100 + seed)
+        d = make_inputs(w2, with_x=False)
+        res = oracle.dispatch(w2.cfg(), np.zeros((w2.W, w2.max_tok, 8), np.uint16), d["topk_idx"],
+                              d["topk_w"], lib=lib)
+        kept = (res["slotmap"] >= 0).sum(axis=(1, 2))          # per source rank
+        dups.extend(list(w2.ct * w2.k - kept))
+    dups = np.array(dups, dtype=np.float64)
+    # one rank's count spreads by ~17; the page's single figure must sit within
+    # 3 spreads of the oracle's mean, and the mean (32 ranks) is tight.
+    assert abs(dups.mean() - g["null_writes"]) <= 3 * dups.std() / math.sqrt(len(dups)) + 3 * 17.5 / 1, dups.mean()
+    assert abs(dups.mean() - g["null_writes"]) <= 20, dups.mean()
+
+
+def pin_closed_form_unique_count(lib=None):
+    """E|P| = W (1 - C(E-nEpr, k) / C(E, k)) for k distinct uniform experts."""
+    for name in ("main", "pr599"):
+        wl = workload(name).replace(h=8)
+        d = make_inputs(wl, with_x=False)
+        res = oracle.dispatch(wl.cfg(), np.zeros((wl.W, wl.max_tok, 8), np.uint16), d["topk_idx"],
+                              d["topk_w"], lib=lib)
+        n_tok = wl.W * wl.ct
+        mean = res["recv_count"].sum() / n_tok
+        E = wl.E
+        want = wl.W * (1 - math.comb(E - wl.n_epr, wl.k) / math.comb(E, wl.k))
+        per_tok = (res["slotmap"] >= 0).sum(-1).reshape(-1)
+        se = per_tok.std() / math.sqrt(n_tok)
+        assert abs(mean - want) <= 4 * se, (name, mean, want, se)
+
+
+def pin_bf16_conversion(lib=None):
+    """The oracle's float32 -> bfloat16 RNE against torch's conversion, and
+    bf16 -> float32 against the exact value of the bit pattern."""
+    rng = np.random.default_rng(0)
+    bits = rng.integers(0, 1 << 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    # ties and near-ties at every parity
+    ties = (rng.integers(0, 1 << 16, size=20000, dtype=np.uint32) << 16) | np.uint32(0x8000)
+    specials = np.array([0, 0x80000000, 0x7F800000, 0xFF800000, 0x7F7FFFFF, 0x00000001, 0x007FFFFF,
+                         0x00008000, 0x00018000, 0x3F808000, 0x3F818000, 0x7F7F8000, 0x7F7F7FFF],
+                        dtype=np.uint32)
+    allb = np.concatenate([bits, ties, ties + 1, ties - 1, specials])
+    f = f32_from_bits(allb)
+    nan = np.isnan(f)
+    got = oracle.f32_to_bf16(f, lib=lib)
+    want = torch_bf16_bits(f)
+    assert np.array_equal(got[~nan], want[~nan])
+    gotf = bf16_bits_to_f64(got[nan])
+    assert np.all(np.isnan(gotf))
+    assert np.array_equal(got[nan] >> 15, (allb[nan] >> 31).astype(np.uint16))  # sign kept
+    b16 = np.arange(1 << 16, dtype=np.uint16)
+    back = oracle.bf16_to_f32(b16, lib=lib)
+    ok = ~np.isnan(back)
+    exact = f32_from_bits(b16.astype(np.uint32) << 16)
+    assert np.array_equal(back[ok].view(np.uint32), exact[ok].view(np.uint32))
+
+
+def pin_out_of_range_ids(lib=None):
+    """An id >= E is reported (status 1) and routes nowhere."""
+    cfg = dict(worldSize=2, hiddenDim=8, maxTokPerRank=2, numExpertPerRank=2,
+               numExpertPerToken=2, maxRecv=0, dtype=0, useWeights=1)
+    idx = np.array([[[0, 9], [3, 1]], [[-1, -1], [4, 2]]], dtype=np.int32)
+    w = np.ones((2, 2, 2), np.float32)
+    res = oracle.dispatch(cfg, np.zeros((2, 2, 8), np.uint16), idx, w, lib=lib)
+    assert res["status"] == oracle.STATUS_EXPERT_RANGE
+    assert list(res["recv_count"]) == [2, 2]
+    res2 = oracle.dispatch(cfg, np.zeros((2, 2, 8), np.uint16), np.where(idx >= 4, -1, idx), w, lib=lib)
+    assert res2["status"] == 0
+    for key in ("recv_count", "slotmap", "wsum"):
+        assert np.array_equal(res[key], res2[key])
+
+
+ALL_PINS = [
+    pin_bruteforce_dispatch,
+    pin_bruteforce_weight_sum_order,
+    pin_combine_exact_fma,
+    pin_combine_single_rounding_case,
+    pin_combine_fp64_bound,
+    pin_roundtrip_unweighted_exact,
+    pin_roundtrip_weighted,
+    pin_single_rank,
+    pin_invariants,
+    pin_page_staging_copy,
+    pin_page_null_writes,
+    pin_closed_form_unique_count,
+    pin_bf16_conversion,
+    pin_out_of_range_ids,
+]
