@@ -1,0 +1,420 @@
+"""Benchmark: one step = ep_dispatch -> identity expert (y = recv_x) ->
+ep_combine over W=8 virtual EP ranks on one B200, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload main|pr599|skewed|latency1|latency8|mid] [--no-cpu-baseline]
+
+Prints one JSON line (rank 0). Timing: W untimed warm-up steps, then K steps,
+each bracketed by CUDA events on the launching stream (dispatch and combine
+separately); a 256 MB buffer is rewritten between steps outside the events
+(L2 flush; the main workload's inputs are larger than L2 as well). Barrier +
+synchronize on both sides; the reported time is the max over ranks. N > 1
+runs N independent replicas, one per GPU (each GPU holds all W virtual ranks).
+
+--impl reference times the CPU oracle (the plain C statement of the method)
+on this host's cores, on a bounded sample of the same workload (see
+``ref_sample``), scaled to the full step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth.inputs import make_inputs, workload  # noqa: E402
+
+METRIC = "dispatch+combine µs and HBM GB/s (% of B200 peak) at W=8 ct=4096 h=7168 topk8"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ["combine_ep_dispatch_05_b200/csrc/ep_kernels.cu",
+                  "combine_ep_dispatch_05_b200/csrc/ep_abi.cu",
+                  "combine_ep_dispatch_05_b200/csrc/ep_internal.h"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="main")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def get_workload(name):
+    if name == "mid":  # the main shape at 1024 tokens/rank: the small ncu case
+        return workload("main").replace(name="mid", max_tok=1024, ct=1024, max_recv=8192)
+    return workload(name)
+
+
+def describe(wl) -> dict:
+    return {"workload": f"{wl.name}: W={wl.W} ct={wl.ct} h={wl.h} topk={wl.k} "
+                        f"E={wl.E} ({wl.n_epr}/rank) {wl.routing} routing, bf16 rows",
+            "world_size": wl.W, "tokens_per_rank": wl.ct, "max_tok_per_rank": wl.max_tok,
+            "hidden": wl.h, "topk": wl.k, "experts": wl.E, "max_recv": wl.max_recv,
+            "use_weights": wl.use_weights,
+            "l2": "256 MB buffer rewritten between steps outside the events; inputs larger than L2"}
+
+
+def dispatch_bytes(wl, U, n_routed):
+    row, G, k, W = wl.h * 2, wl.W * wl.max_tok, wl.k, wl.W
+    return (n_routed * row                    # read each routed x row once
+            + U * row                         # write every received row
+            + G * k * 4 * (1 + int(wl.use_weights))  # topk ids (+ weights)
+            + U * (3 + k) * 4                 # meta records
+            + 4 * W)                          # recv_count
+
+
+def combine_bytes(wl, U):
+    row, G = wl.h * 2, wl.W * wl.max_tok
+    return (U * row       # read every received row of y
+            + G * row     # write every out row
+            + U * 8)      # (slot, weight) of each received row
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, wl_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[kernel]
+        if e.get("source_sha") != source_hash():
+            return None
+        return e["per_launch_bytes"].get(wl_name)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.t0 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # samples under load: the top 3/4 of power draw
+        cut = sorted(power)[len(power) // 4] if len(power) >= 4 else min(power)
+        loaded = [s for s, p in zip(sm, power) if p >= cut] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power), "reasons": sorted(reasons)}
+
+
+def dist_setup(n):
+    if n <= 1 and "RANK" not in os.environ:
+        return 0, 1, 0, None
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    return rank, world, local, dist
+
+
+def max_over_ranks(val: float, dist, device) -> float:
+    if dist is None:
+        return val
+    import torch
+    t = torch.tensor([val], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ reference arm
+def ref_sample(wl, frac_den=8):
+    """The bounded sample the CPU oracle runs per reference step: the same
+    workload with 1/frac_den of the tokens per rank (same routing law, same
+    hidden size and capacity per token), so every per-token cost is the same;
+    the step time is scaled back by the token ratio."""
+    ct = max(1, wl.ct // frac_den)
+    mt = max(1, wl.max_tok // frac_den)
+    sample = wl.replace(ct=ct, max_tok=mt, max_recv=wl.W * mt)
+    scale = (wl.W * wl.max_tok) / (sample.W * sample.max_tok)
+    return sample, scale, (f"{wl.name} shape with {mt} of {wl.max_tok} tokens per rank "
+                           f"(maxRecv {wl.W * mt}), time x {scale:g}")
+
+
+def time_oracle(wl, inputs, steps, scale=1.0):
+    import oracle
+    cfg = wl.cfg()
+    R = oracle.recv_capacity(cfg)
+    recv_x = np.zeros((wl.W, R, wl.h), dtype=np.uint16)
+    recv_meta = np.zeros((wl.W, R, 3 + wl.k), dtype=np.int32)
+    idx = inputs["topk_idx"]
+    ts = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        r = oracle.dispatch(cfg, inputs["x"], idx, inputs["topk_w"], recv_x=recv_x, recv_meta=recv_meta)
+        oracle.combine(cfg, r["recv_x"], r["slotmap"], r["wsum"])
+        ts.append((time.perf_counter() - t0) * scale)
+    return ts
+
+
+def run_reference(args, wl):
+    rank, world, local, dist = dist_setup(args.gpus)
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    swl, scale, sample = ref_sample(wl)
+    inputs = make_inputs(swl)
+    time_oracle(swl, inputs, args.warmup, scale)
+    ts = time_oracle(swl, inputs, args.steps, scale)
+    us = statistics.mean(ts) * 1e6
+    cores = 1
+    line = {"metric": METRIC, "value": us, "unit": "us", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": describe(wl), "impl": "reference",
+            "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, wl):
+    import torch
+    rank, world, local, dist = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist is not None:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    from combine_ep_dispatch_05_b200 import build as epbuild
+    if rank == 0 or dist is None:
+        epbuild.build()
+    if dist is not None:
+        dist.barrier()
+    import combine_ep_dispatch_05_b200 as ep
+
+    cfg = wl.cfg()
+    inputs = make_inputs(wl)
+    plan = ep.ep_plan_create(cfg)
+    info = ep.ep_plan_info(plan)
+    W, T, h, k, R = wl.W, wl.max_tok, wl.h, wl.k, info.maxRecv
+    x = torch.from_numpy(inputs["x"].view(np.int16)).to(dev)
+    idx = torch.from_numpy(inputs["topk_idx"]).to(dev)
+    w = torch.from_numpy(inputs["topk_w"]).to(dev) if inputs["topk_w"] is not None else None
+    recv_x = torch.empty((W, R, h), dtype=torch.int16, device=dev)
+    recv_meta = torch.empty((W, R, 3 + k), dtype=torch.int32, device=dev)
+    recv_count = torch.empty((W,), dtype=torch.int32, device=dev)
+    out = torch.empty((W, T, h), dtype=torch.int16, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    s = torch.cuda.current_stream(dev)
+
+    def step():
+        ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, s)
+        ep.ep_combine(plan, recv_x, out, s)  # identity expert: y = recv_x
+
+    for i in range(max(args.warmup, 0)):
+        flush.fill_(i)
+        step()
+    torch.cuda.synchronize(dev)
+    err = ep.ep_plan_check_error(plan)
+    if err:
+        raise RuntimeError(f"device error word {err} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i + 1)
+        evs[i][0].record(s)
+        ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, s)
+        evs[i][1].record(s)
+        ep.ep_combine(plan, recv_x, out, s)
+        evs[i][2].record(s)
+    torch.cuda.synchronize(dev)
+    t_wall = time.perf_counter() - t_wall
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    t_disp = [evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps)]
+    t_comb = [evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps)]
+    disp_ms = statistics.mean(t_disp)
+    comb_ms = statistics.mean(t_comb)
+    step_ms = max_over_ranks(disp_ms + comb_ms, dist, dev)
+    disp_ms_max = max_over_ranks(disp_ms, dist, dev)
+    comb_ms_max = max_over_ranks(comb_ms, dist, dev)
+    err = ep.ep_plan_check_error(plan)
+    if err:
+        raise RuntimeError(f"device error word {err} after the timed steps")
+
+    # Algorithmic bytes from the actual routing.
+    counts = recv_count.cpu().numpy()
+    U = int(counts.sum())
+    n_routed = int((inputs["topk_idx"] >= 0).any(axis=-1).sum())
+    db, cb = dispatch_bytes(wl, U, n_routed), combine_bytes(wl, U)
+    peak, peak_src = hbm_peak()
+    d_gbs = db / (disp_ms_max * 1e-3) / 1e9
+    c_gbs = cb / (comb_ms_max * 1e-3) / 1e9
+    pair_gbs = (db + cb) / (step_ms * 1e-3) / 1e9
+    if comb_ms_max >= disp_ms_max:
+        dom = {"kernel": "ep_combine_kernel", "bytes": cb, "ms": comb_ms_max, "gbs": c_gbs}
+    else:
+        dom = {"kernel": "ep_dispatch (route_count + scatter_rows)", "bytes": db, "ms": disp_ms_max,
+               "gbs": d_gbs}
+    traffic = ncu_traffic("ep_combine_kernel" if dom["kernel"] == "ep_combine_kernel" else "ep_scatter_rows_kernel",
+                          wl.name)
+
+    # End to end: pinned host inputs -> device, both calls, result -> pinned host.
+    e2e = None
+    if not args.no_e2e:
+        x_h = torch.from_numpy(inputs["x"].view(np.int16)).pin_memory()
+        idx_h = torch.from_numpy(inputs["topk_idx"]).pin_memory()
+        w_h = torch.from_numpy(inputs["topk_w"]).pin_memory() if w is not None else None
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_h, non_blocking=True)
+            idx.copy_(idx_h, non_blocking=True)
+            if w is not None:
+                w.copy_(w_h, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, min(args.warmup, 3))):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 10))
+        e0.record(s)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
+        h2d = x_h.numel() * 2 + idx_h.numel() * 4 + (w_h.numel() * 4 if w_h is not None else 0)
+        e2e = {"value": e2e_ms * 1e3, "unit": "us", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(out_h.numel() * 2), "steps": n_e2e}
+
+    ep.ep_plan_destroy(plan)
+
+    cpu = None
+    if rank == 0 and args.gpus == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        steps_cpu = 2
+        ts = time_oracle(wl, inputs, steps_cpu)
+        cpu = {"value": statistics.mean(ts) * 1e6, "unit": "us", "cores": 1, "kind": "oracle",
+               "sample": f"the full {wl.name} workload, {steps_cpu} steps, single-threaded C oracle"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": step_ms * 1e3, "unit": "us", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {**describe(wl), "parallelism": "virtual EP ranks on each GPU; replicas across GPUs"},
+            "dispatch_us": disp_ms_max * 1e3, "combine_us": comb_ms_max * 1e3,
+            "dispatch_gbs": d_gbs, "combine_gbs": c_gbs, "pair_gbs": pair_gbs,
+            "pair_frac_of_peak": pair_gbs / peak, "recv_rows_U": U,
+            "algorithmic_bytes": {"dispatch": db, "combine": cb},
+            "roofline": {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["gbs"], "peak": peak,
+                         "peak_source": f"{peak_src} copy bandwidth", "unit": "GB/s",
+                         "frac": dom["gbs"] / peak, "traffic": traffic,
+                         "bytes_per_launch": dom["bytes"], "avg_launch_us": dom["ms"] * 1e3},
+            "roofline_all": {
+                "dispatch": {"achieved": d_gbs, "frac": d_gbs / peak, "bytes": db, "us": disp_ms_max * 1e3},
+                "combine": {"achieved": c_gbs, "frac": c_gbs / peak, "bytes": cb, "us": comb_ms_max * 1e3}},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": 3 * args.steps, "timed_wall_s": t_wall,
+            "geometry": info.as_dict(), "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    wl = get_workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,420 @@
+// ep_abi.cu -- the C ABI of include/ep.h: configuration checks, plans (device
+// scratch + launch geometry) and the dispatch / combine entry points.
+//
+// Conventions follow the "MORI JIT v2" design page §6: every entry point is
+// noexcept (no exception crosses extern "C"), errors are NULL / negative
+// returns with the reason kept in a thread-local string.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "ep.h"
+#include "ep_internal.h"
+
+struct EpPlan {
+    EpCfg cfg;
+    EpPlanInfo info;
+    int device;
+    int maxRecv;
+    int G;            // W*T
+    void* scratch;    // one allocation, carved below
+    int2* route;      // [G][W]
+    int32_t* tile_cnt;
+    int32_t* tile_base;
+    uint32_t* ticket;
+    int32_t* err;
+    size_t scatterSmem;
+    bool dispatched;
+};
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(e == cudaErrorMemoryAllocation ? EP_ERR_NOMEM : EP_ERR_CUDA, "%s: %s (%s)", what,
+                cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+int env_int(const char* name, int dflt) {
+    const char* v = std::getenv(name);
+    if (!v || !*v) return dflt;
+    char* end = nullptr;
+    long x = std::strtol(v, &end, 10);
+    return (end && *end == '\0' && x > 0 && x < (1 << 30)) ? (int)x : dflt;
+}
+
+// The validity rules of the design page §3.5 (EpCfgIsValid / MakeEpCfg) and
+// the dtype rule of §3.7, plus the int32 index range of this build.
+int check_cfg(const EpCfg* c) {
+    if (!c) return fail(EP_ERR_INVALID, "cfg is NULL");
+    if (c->worldSize < 1 || c->worldSize > ep::kMaxWorld)
+        return fail(EP_ERR_INVALID, "worldSize %d outside 1..%d (one destination per warp lane)",
+                    c->worldSize, ep::kMaxWorld);
+    if (c->numExpertPerToken < 1 || c->numExpertPerToken > ep::kMaxTopk)
+        return fail(EP_ERR_INVALID, "numExpertPerToken %d outside 1..%d (one topk entry per warp lane)",
+                    c->numExpertPerToken, ep::kMaxTopk);
+    if (c->hiddenDim < 1) return fail(EP_ERR_INVALID, "hiddenDim %d < 1", c->hiddenDim);
+    if (c->maxTokPerRank < 1) return fail(EP_ERR_INVALID, "maxTokPerRank %d < 1", c->maxTokPerRank);
+    if (c->numExpertPerRank < 1)
+        return fail(EP_ERR_INVALID, "numExpertPerRank %d < 1", c->numExpertPerRank);
+    if ((long long)c->worldSize * c->numExpertPerRank > (1LL << 30))
+        return fail(EP_ERR_INVALID, "too many experts");
+    if (c->useWeights != 0 && c->useWeights != 1)
+        return fail(EP_ERR_INVALID, "useWeights must be 0 or 1, got %d", c->useWeights);
+    if (c->dtype == EP_FP32 || c->dtype == EP_FP8 || c->dtype == EP_FP4X2)
+        return fail(EP_ERR_UNSUPPORTED, "dtype %d is not built (bf16 payloads only)", c->dtype);
+    if (c->dtype != EP_BF16) return fail(EP_ERR_INVALID, "unknown dtype %d", c->dtype);
+    const long long rowBytes = (long long)c->hiddenDim * 2;
+    if (rowBytes % 16 != 0)
+        return fail(EP_ERR_INVALID, "token bytes %lld (hiddenDim*2) not a multiple of 16", rowBytes);
+    const long long G = (long long)c->worldSize * c->maxTokPerRank;
+    if (G > (1LL << 30)) return fail(EP_ERR_INVALID, "worldSize*maxTokPerRank too large");
+    if (c->maxRecv < 0) return fail(EP_ERR_INVALID, "maxRecv %d < 0", c->maxRecv);
+    const long long maxRecv = c->maxRecv == 0 ? G : c->maxRecv;
+    if (maxRecv < G)
+        return fail(EP_ERR_INVALID,
+                    "maxRecv %lld does not cover the worst case worldSize*maxTokPerRank = %lld", maxRecv, G);
+    if ((long long)c->worldSize * maxRecv > (1LL << 31) - 1)
+        return fail(EP_ERR_INVALID, "worldSize*maxRecv exceeds the int32 flat index");
+    return EP_OK;
+}
+
+struct Geometry {
+    int chunkBytes, chunkStride, numChunks;
+    int scatterWarps, scatterStages;
+    int combineWarps;
+};
+
+// Copy engines and stages: fill about 200 KB of shared memory per SM with
+// row-sized stages (rows above 32 KB are copied in pieces of <= 16 KB).
+Geometry pick_geometry(const EpCfg* c, bool use_env) {
+    Geometry g{};
+    const long long rowBytes = (long long)c->hiddenDim * 2;
+    int chunk;
+    if (rowBytes <= 32768) {
+        chunk = (int)rowBytes;
+    } else {
+        const long long pieces = (rowBytes + 16383) / 16384;
+        chunk = (int)(((rowBytes + pieces - 1) / pieces + 15) & ~15LL);
+    }
+    if (use_env) chunk = std::min<long long>(rowBytes, env_int("EP_SCATTER_CHUNK", chunk) & ~15);
+    if (chunk < 16) chunk = 16;
+    g.chunkBytes = chunk;
+    g.chunkStride = (chunk + 127) & ~127;
+    g.numChunks = (int)((rowBytes + chunk - 1) / chunk);
+    const int budget = 200 * 1024;
+    int warps = 4;
+    int stages = budget / (warps * g.chunkStride);
+    if (stages < 2) {
+        warps = std::max(1, budget / (2 * g.chunkStride));
+        stages = 2;
+    }
+    stages = std::min(stages, 8);
+    if (use_env) {
+        warps = std::min(env_int("EP_SCATTER_WARPS", warps), ep::kMaxScatterWarps);
+        stages = std::max(2, std::min(env_int("EP_SCATTER_STAGES", stages), 16));
+    }
+    g.scatterWarps = warps;
+    g.scatterStages = stages;
+    g.combineWarps = use_env ? std::min(env_int("EP_COMBINE_WARPS", 8), ep::kMaxCombineWarps) : 8;
+    return g;
+}
+
+void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
+    std::memset(info, 0, sizeof *info);
+    const long long G = (long long)c->worldSize * c->maxTokPerRank;
+    const int maxRecv = c->maxRecv == 0 ? (int)G : c->maxRecv;
+    const int M = 3 + c->numExpertPerToken;
+    info->maxRecv = maxRecv;
+    info->metaFields = M;
+    info->rowBytes = (long long)c->hiddenDim * 2;
+    info->tokenBytes = G * info->rowBytes;
+    info->recvXBytes = (long long)c->worldSize * maxRecv * info->rowBytes;
+    info->recvMetaBytes = (long long)c->worldSize * maxRecv * M * 4;
+    info->countTile = ep::kCountTile;
+    info->numTiles = (int)((G + ep::kCountTile - 1) / ep::kCountTile);
+    info->scratchBytes = (long long)(align256(sizeof(int2) * G * c->worldSize) +
+                                     2 * align256(sizeof(int32_t) * (size_t)info->numTiles * c->worldSize) +
+                                     align256(sizeof(uint32_t)) + align256(sizeof(int32_t)));
+    info->scatterWarps = geo.scatterWarps;
+    info->scatterStages = geo.scatterStages;
+    info->scatterChunkBytes = geo.chunkBytes;
+    info->combineWarps = geo.combineWarps;
+    info->device = -1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ep_last_error(void) { return g_last_error; }
+
+int ep_cfg_check(const EpCfg* cfg) {
+    try {
+        g_last_error[0] = '\0';
+        return check_cfg(cfg);
+    } catch (...) {
+        return fail(EP_ERR_INVALID, "unexpected exception");
+    }
+}
+
+int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info) {
+    try {
+        if (!info) return fail(EP_ERR_INVALID, "info is NULL");
+        int rc = check_cfg(cfg);
+        if (rc) return rc;
+        const Geometry geo = pick_geometry(cfg, false);
+        fill_info(cfg, geo, info);
+        const int sms = 148;  // B200
+        info->scatterBlocks = sms * std::max(1, (200 * 1024) / (int)ep::scatter_smem_bytes(
+                                                                   geo.scatterWarps, geo.scatterStages,
+                                                                   geo.chunkStride));
+        info->combineBlocks = sms * 2;
+        return EP_OK;
+    } catch (...) {
+        return fail(EP_ERR_INVALID, "unexpected exception");
+    }
+}
+
+EpPlan* ep_plan_create(const EpCfg* cfg) {
+    EpPlan* plan = nullptr;
+    try {
+        if (check_cfg(cfg) != EP_OK) return nullptr;
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) {
+            cuda_fail(e, "cudaGetDevice");
+            return nullptr;
+        }
+        int sms = 0, smemOptin = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&smemOptin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+                cudaSuccess) {
+            cuda_fail(e, "cudaDeviceGetAttribute");
+            return nullptr;
+        }
+        Geometry geo = pick_geometry(cfg, true);
+        size_t smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+        while (smem > (size_t)smemOptin && geo.scatterStages > 2) {
+            --geo.scatterStages;
+            smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+        }
+        while (smem > (size_t)smemOptin && geo.scatterWarps > 1) {
+            --geo.scatterWarps;
+            smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+        }
+        if (smem > (size_t)smemOptin) {
+            fail(EP_ERR_INVALID, "row piece of %d bytes does not fit shared memory", geo.chunkBytes);
+            return nullptr;
+        }
+        if ((e = ep::scatter_set_smem(smem)) != cudaSuccess) {
+            cuda_fail(e, "cudaFuncSetAttribute(scatter smem)");
+            return nullptr;
+        }
+        int sPerSm = 0, cPerSm = 0;
+        if ((e = ep::scatter_blocks_per_sm(geo.scatterWarps, smem, &sPerSm)) != cudaSuccess ||
+            (e = ep::combine_blocks_per_sm(geo.combineWarps, &cPerSm)) != cudaSuccess) {
+            cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+            return nullptr;
+        }
+        if (sPerSm < 1 || cPerSm < 1) {
+            fail(EP_ERR_INVALID, "kernel geometry does not fit one SM");
+            return nullptr;
+        }
+
+        plan = new (std::nothrow) EpPlan();
+        if (!plan) {
+            fail(EP_ERR_NOMEM, "host allocation failed");
+            return nullptr;
+        }
+        plan->cfg = *cfg;
+        fill_info(cfg, geo, &plan->info);
+        plan->device = dev;
+        plan->info.device = dev;
+        plan->info.numSMs = sms;
+        plan->info.scatterBlocks = env_int("EP_SCATTER_BLOCKS", sms * sPerSm);
+        plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
+        plan->scatterSmem = smem;
+        plan->G = cfg->worldSize * cfg->maxTokPerRank;
+        plan->maxRecv = plan->info.maxRecv;
+
+        const int W = cfg->worldSize;
+        const size_t nRoute = align256(sizeof(int2) * (size_t)plan->G * W);
+        const size_t nTiles = align256(sizeof(int32_t) * (size_t)plan->info.numTiles * W);
+        const size_t total = (size_t)plan->info.scratchBytes;
+        if ((e = cudaMalloc(&plan->scratch, total)) != cudaSuccess) {
+            cuda_fail(e, "cudaMalloc(plan scratch)");
+            plan->scratch = nullptr;
+            ep_plan_destroy(plan);
+            return nullptr;
+        }
+        if ((e = cudaMemset(plan->scratch, 0, total)) != cudaSuccess) {
+            cuda_fail(e, "cudaMemset(plan scratch)");
+            ep_plan_destroy(plan);
+            return nullptr;
+        }
+        char* base = static_cast<char*>(plan->scratch);
+        plan->route = reinterpret_cast<int2*>(base);
+        plan->tile_cnt = reinterpret_cast<int32_t*>(base + nRoute);
+        plan->tile_base = reinterpret_cast<int32_t*>(base + nRoute + nTiles);
+        plan->ticket = reinterpret_cast<uint32_t*>(base + nRoute + 2 * nTiles);
+        plan->err = reinterpret_cast<int32_t*>(base + nRoute + 2 * nTiles + 256);
+        plan->dispatched = false;
+        g_last_error[0] = '\0';
+        return plan;
+    } catch (...) {
+        fail(EP_ERR_INVALID, "unexpected exception");
+        if (plan) ep_plan_destroy(plan);
+        return nullptr;
+    }
+}
+
+void ep_plan_destroy(EpPlan* plan) {
+    if (!plan) return;
+    if (plan->scratch) cudaFree(plan->scratch);
+    delete plan;
+}
+
+int ep_plan_info(const EpPlan* plan, EpPlanInfo* info) {
+    if (!plan || !info) return fail(EP_ERR_INVALID, "plan or info is NULL");
+    *info = plan->info;
+    return EP_OK;
+}
+
+static int check_device(const EpPlan* plan) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != plan->device)
+        return fail(EP_ERR_DEVICE, "current device %d is not the plan's device %d", dev, plan->device);
+    return EP_OK;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
+                void* recv_x, int32_t* recv_meta, int32_t* recv_count, void* stream) {
+    try {
+        if (!plan) return fail(EP_ERR_INVALID, "plan is NULL");
+        if (!x || !topk_idx || !recv_x || !recv_meta || !recv_count)
+            return fail(EP_ERR_INVALID, "a required buffer is NULL");
+        if (plan->cfg.useWeights && !topk_w)
+            return fail(EP_ERR_INVALID, "topk_w is NULL but useWeights is 1");
+        if (!aligned(x, 16) || !aligned(recv_x, 16))
+            return fail(EP_ERR_ALIGN, "x and recv_x must be 16-byte aligned");
+        if (!aligned(topk_idx, 4) || !aligned(recv_meta, 4) || !aligned(recv_count, 4) ||
+            (topk_w && !aligned(topk_w, 4)))
+            return fail(EP_ERR_ALIGN, "topk_idx, topk_w, recv_meta, recv_count must be 4-byte aligned");
+        int rc = check_device(plan);
+        if (rc) return rc;
+        const EpCfg& c = plan->cfg;
+        cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+        ep::RouteParams rp{};
+        rp.idx = topk_idx;
+        rp.w = c.useWeights ? topk_w : nullptr;
+        rp.route = plan->route;
+        rp.tile_cnt = plan->tile_cnt;
+        rp.tile_base = plan->tile_base;
+        rp.recv_count = recv_count;
+        rp.ticket = plan->ticket;
+        rp.err = plan->err;
+        rp.G = plan->G;
+        rp.W = c.worldSize;
+        rp.k = c.numExpertPerToken;
+        rp.nEpr = c.numExpertPerRank;
+        rp.E = c.worldSize * c.numExpertPerRank;
+        rp.numTiles = plan->info.numTiles;
+        rp.maxRecv = plan->maxRecv;
+        rp.useWeights = c.useWeights;
+        cudaError_t e = ep::launch_route_count(rp, s);
+        if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
+
+        ep::ScatterParams sp{};
+        sp.x = static_cast<const uint8_t*>(x);
+        sp.idx = topk_idx;
+        sp.route = plan->route;
+        sp.tile_base = plan->tile_base;
+        sp.recv_x = static_cast<uint8_t*>(recv_x);
+        sp.recv_meta = recv_meta;
+        sp.err = plan->err;
+        sp.rowBytes = plan->info.rowBytes;
+        sp.G = plan->G;
+        sp.W = c.worldSize;
+        sp.k = c.numExpertPerToken;
+        sp.nEpr = c.numExpertPerRank;
+        sp.E = c.worldSize * c.numExpertPerRank;
+        sp.T = c.maxTokPerRank;
+        sp.maxRecv = plan->maxRecv;
+        sp.M = plan->info.metaFields;
+        sp.chunkBytes = plan->info.scatterChunkBytes;
+        sp.chunkStride = (sp.chunkBytes + 127) & ~127;
+        sp.numChunks = (int)((sp.rowBytes + sp.chunkBytes - 1) / sp.chunkBytes);
+        sp.stages = plan->info.scatterStages;
+        e = ep::launch_scatter_rows(sp, plan->info.scatterBlocks, plan->info.scatterWarps,
+                                    plan->scatterSmem, s);
+        if (e != cudaSuccess) return cuda_fail(e, "launch scatter_rows");
+        plan->dispatched = true;
+        return EP_OK;
+    } catch (...) {
+        return fail(EP_ERR_INVALID, "unexpected exception");
+    }
+}
+
+int ep_combine(EpPlan* plan, const void* y, void* out, void* stream) {
+    try {
+        if (!plan) return fail(EP_ERR_INVALID, "plan is NULL");
+        if (!y || !out) return fail(EP_ERR_INVALID, "y or out is NULL");
+        if (!aligned(y, 16) || !aligned(out, 16))
+            return fail(EP_ERR_ALIGN, "y and out must be 16-byte aligned");
+        if (!plan->dispatched) return fail(EP_ERR_STATE, "combine before any dispatch on this plan");
+        int rc = check_device(plan);
+        if (rc) return rc;
+        ep::CombineParams cp{};
+        cp.y = static_cast<const uint8_t*>(y);
+        cp.route = plan->route;
+        cp.out = static_cast<uint8_t*>(out);
+        cp.rowBytes = plan->info.rowBytes;
+        cp.G = plan->G;
+        cp.W = plan->cfg.worldSize;
+        cp.maxRecv = plan->maxRecv;
+        cudaError_t e = ep::launch_combine(cp, plan->info.combineBlocks, plan->info.combineWarps,
+                                           static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "launch combine");
+        return EP_OK;
+    } catch (...) {
+        return fail(EP_ERR_INVALID, "unexpected exception");
+    }
+}
+
+int ep_plan_check_error(EpPlan* plan) {
+    if (!plan) return fail(EP_ERR_INVALID, "plan is NULL");
+    int rc = check_device(plan);
+    if (rc) return rc;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    int32_t word = 0;
+    if ((e = cudaMemcpy(&word, plan->err, sizeof word, cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpy(error word)");
+    if ((e = cudaMemset(plan->err, 0, sizeof word)) != cudaSuccess) return cuda_fail(e, "cudaMemset");
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    return word;
+}
+
+}  // extern "C"

@@ -1,0 +1,514 @@
+// ep_kernels.cu -- sm_100a kernels of MoE expert-parallel dispatch / combine
+// over W virtual ranks held in one GPU's memory.
+//
+// dispatch = route_count (one launch) + scatter_rows (one launch)
+//   route_count  one thread per token: destination mask (destPe = expert /
+//                numExpertPerRank, "MORI JIT v2" design page §8), per-destination
+//                weight sums, per-tile histogram by warp ballots, tile-local
+//                ranks; the last block to finish scans the tile histogram into
+//                per-(tile, destPe) bases and stores recv_count (mori PR #599:
+//                a stored count). Slots end up ordered by (srcRank, token).
+//   scatter_rows persistent copy engines, one per warp: each x row is read once
+//                from HBM into shared memory by a TMA bulk copy
+//                (cp.async.bulk, mbarrier completion) and written to every
+//                destination by TMA bulk stores from the same shared memory,
+//                while the warp's lanes write the meta records. The pages' copy
+//                loops (WarpCopy on gfx9xx, one TDM tile per token on gfx1250,
+//                design page §9 and PR #599) are the prior art.
+// combine = combine (one launch)
+//   combine      one warp per token: up to 8 destination rows in flight per
+//                16-byte column, float32 fma fold in destPe order, bf16 RNE out.
+//
+// No kernel traps or spins without a bound: waits on shared-memory barriers
+// give up after kWaitCycles, set EP_DEVERR_TIMEOUT and drain their copies.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep.h"
+#include "ep_internal.h"
+
+namespace ep {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// ------------------------------------------------------------- TMA / mbarrier
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitCycles) return false;
+    }
+    return true;
+}
+
+// Global -> shared bulk copy; completion is counted on the mbarrier in bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Shared -> global bulk copy, tracked by this thread's bulk async-groups.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// All but the most recent bulk group have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+// Every bulk group of this thread has completed (writes done).
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// =====================================================================
+// route_count: mask, weight sums, tile histogram, tile-local ranks; the last
+// block scans the histogram. kW = compile-time bound on W (8, 16 or 32).
+// =====================================================================
+template <int kW>
+__global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams p) {
+    __shared__ int s_wcnt[kCountWarps][kW];
+    __shared__ int s_wpre[kCountWarps][kW];
+    __shared__ int s_last;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = blockIdx.x * kCountTile + tid;
+    const int W = p.W, k = p.k;
+
+    uint32_t mask = 0;
+    bool bad = false;
+    float ws[kW];
+#pragma unroll
+    for (int pe = 0; pe < kW; ++pe) ws[pe] = 0.0f;
+
+    if (g < p.G) {
+        const int32_t* ids = p.idx + (size_t)g * k;
+        const float* wts = p.w ? p.w + (size_t)g * k : nullptr;
+        for (int j = 0; j < k; ++j) {
+            const int e = ids[j];
+            if (e < 0) continue;  // masked entry
+            if (e >= p.E) {       // contract violation: report, treat as masked
+                bad = true;
+                continue;
+            }
+            const int pe_j = e / p.nEpr;
+            mask |= 1u << pe_j;
+            if (wts) {
+                const float wj = wts[j];
+#pragma unroll
+                for (int pe = 0; pe < kW; ++pe)
+                    if (pe == pe_j) ws[pe] = ws[pe] + wj;  // fold in topk order
+            }
+        }
+    }
+    if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
+
+    // Per-warp histogram by ballot.
+#pragma unroll
+    for (int pe = 0; pe < kW; ++pe) {
+        if (pe < W) {
+            const uint32_t b = __ballot_sync(kFull, (mask >> pe) & 1u);
+            if (lane == 0) s_wcnt[warp][pe] = __popc(b);
+        }
+    }
+    __syncthreads();
+    if (tid < W) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < kCountWarps; ++w) {
+            s_wpre[w][tid] = run;
+            run += s_wcnt[w][tid];
+        }
+        p.tile_cnt[blockIdx.x * W + tid] = run;
+    }
+    __syncthreads();
+
+    // Tile-local rank of this token at each destination, and its weight sum.
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int pe = 0; pe < kW; ++pe) {
+        if (pe < W) {
+            const bool hit = (mask >> pe) & 1u;
+            const uint32_t b = __ballot_sync(kFull, hit);
+            if (g < p.G) {
+                int2 v;
+                v.x = hit ? s_wpre[warp][pe] + __popc(b & lt) : -1;
+                const float wsum = hit ? (p.useWeights ? ws[pe] : 1.0f) : 0.0f;
+                v.y = __float_as_int(wsum);
+                p.route[(size_t)g * W + pe] = v;
+            }
+        }
+    }
+
+    // Last block to finish turns the tile histogram into per-tile bases.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(p.ticket, 1u) == (unsigned)(p.numTiles - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int pe = warp; pe < W; pe += kCountWarps) {
+        int running = 0;
+        for (int t0 = 0; t0 < p.numTiles; t0 += 32) {
+            const int t = t0 + lane;
+            const int v = t < p.numTiles ? __ldcg(p.tile_cnt + (size_t)t * W + pe) : 0;
+            int incl = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int n = __shfl_up_sync(kFull, incl, off);
+                if (lane >= off) incl += n;
+            }
+            if (t < p.numTiles) p.tile_base[(size_t)t * W + pe] = running + incl - v;
+            running += __shfl_sync(kFull, incl, 31);
+        }
+        if (lane == 0) {
+            p.recv_count[pe] = running;  // stored, not accumulated
+            if (running > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+        }
+    }
+    if (tid == 0) *p.ticket = 0u;  // ready for the next call (graph replay too)
+}
+
+// =====================================================================
+// scatter_rows: persistent copy engines, one per warp.
+// Items are (present token, chunk) pairs of this engine's tokens
+// g = engine, engine + nEngines, ...; an S-stage ring keeps S-1 loads ahead.
+// =====================================================================
+__global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(ScatterParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int S = p.stages;
+
+    // Layout: [bars: nwarps*S u64][ring: nwarps*S*2 int] pad to 128 | stages
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    int* ring = reinterpret_cast<int*>(smem + (size_t)nwarps * S * sizeof(uint64_t));
+    const size_t head = ((size_t)nwarps * S * (sizeof(uint64_t) + 2 * sizeof(int)) + 127) & ~(size_t)127;
+    uint8_t* stage0 = smem + head + (size_t)warp * S * p.chunkStride;
+    const uint32_t stage0_addr = smem_addr(stage0);
+    const uint32_t bar0 = smem_addr(bars + warp * S);
+    int* item_tok = ring + warp * S * 2;
+    int* item_chunk = item_tok + S;
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1u);
+        mbar_fence_init();
+    }
+    __syncwarp();
+
+    const int W = p.W;
+    const int nEngines = gridDim.x * nwarps;
+    const int engine = blockIdx.x * nwarps + warp;
+
+    // Producer: next present token of this engine at or after g.
+    auto next_present = [&](int g) -> int {
+        for (; g < p.G; g += nEngines) {
+            const int lr = lane < W ? p.route[(size_t)g * W + lane].x : -1;
+            if (__ballot_sync(kFull, lr >= 0) != 0u) return g;
+        }
+        return p.G;
+    };
+
+    int pg = next_present(engine);  // producer token
+    int pc = 0;                     // producer chunk
+    int issued = 0, consumed = 0;
+    bool ok = true;
+
+    auto issue = [&]() {
+        const int s = issued % S;
+        if (lane == 0) {
+            const long long off = (long long)pc * p.chunkBytes;
+            const long long rem = p.rowBytes - off;
+            const uint32_t bytes = (uint32_t)(rem < p.chunkBytes ? rem : p.chunkBytes);
+            item_tok[s] = pg;
+            item_chunk[s] = pc;
+            mbar_arrive_expect_tx(bar0 + 8u * s, bytes);
+            bulk_load(stage0_addr + (uint32_t)s * p.chunkStride, p.x + (size_t)pg * p.rowBytes + off,
+                      bytes, bar0 + 8u * s);
+        }
+        ++issued;
+        if (++pc == p.numChunks) {
+            pc = 0;
+            pg = next_present(pg + nEngines);
+        }
+    };
+
+    for (int i = 0; i < S - 1 && pg < p.G; ++i) issue();
+
+    // Per-token state kept across the chunks of one token.
+    int cur_tok = -1;
+    uint32_t cur_mask = 0;
+    int my_slot = -1;  // lane pe: slot of the current token at pe
+
+    while (consumed < issued) {
+        const int s = consumed % S;
+        const uint32_t parity = (uint32_t)(consumed / S) & 1u;
+        __syncwarp();
+        const int g = item_tok[s];
+        const int c = item_chunk[s];
+
+        if (g != cur_tok) {
+            // Slots, routing update and meta records of token g.
+            cur_tok = g;
+            const int2 rr = lane < W ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
+            cur_mask = __ballot_sync(kFull, rr.x >= 0);
+            my_slot = -1;
+            if (rr.x >= 0) {
+                my_slot = p.tile_base[(size_t)(g / kCountTile) * W + lane] + rr.x;
+                p.route[(size_t)g * W + lane].x = my_slot;
+            }
+            const int r = g / p.T, t = g - r * p.T;
+            const int e = lane < p.k ? p.idx[(size_t)g * p.k + lane] : -1;
+            const int pe_e = (e >= 0 && e < p.E) ? e / p.nEpr : -1;
+            // field f of a record: 0 rank, 1 token, 2 weight bits, 3+j local id of entry j
+            const int j0 = lane - 3, j1 = lane + 29;
+            const int e0 = __shfl_sync(kFull, e, j0 & 31), q0 = __shfl_sync(kFull, pe_e, j0 & 31);
+            const int e1 = __shfl_sync(kFull, e, j1 & 31), q1 = __shfl_sync(kFull, pe_e, j1 & 31);
+            for (uint32_t m = cur_mask; m; m &= m - 1) {
+                const int pe = __ffs(m) - 1;
+                const int slot = __shfl_sync(kFull, my_slot, pe);
+                const int wb = __shfl_sync(kFull, rr.y, pe);
+                int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
+                int v0;
+                if (lane == 0) v0 = r;
+                else if (lane == 1) v0 = t;
+                else if (lane == 2) v0 = wb;
+                else v0 = (q0 == pe) ? e0 - pe * p.nEpr : -1;
+                if (lane < p.M) rec[lane] = v0;
+                if (lane + 32 < p.M) rec[lane + 32] = (q1 == pe) ? e1 - pe * p.nEpr : -1;
+            }
+        }
+
+        // Wait for the row piece, then send it to every destination.
+        bool got = true;
+        if (lane == 0) got = mbar_wait_bounded(bar0 + 8u * s, parity);
+        got = __shfl_sync(kFull, got, 0) != 0;
+        if (!got) {
+            ok = false;
+            break;
+        }
+        const long long off = (long long)c * p.chunkBytes;
+        const long long rem = p.rowBytes - off;
+        const uint32_t bytes = (uint32_t)(rem < p.chunkBytes ? rem : p.chunkBytes);
+        for (uint32_t m = cur_mask; m; m &= m - 1) {
+            const int pe = __ffs(m) - 1;
+            const int slot = __shfl_sync(kFull, my_slot, pe);
+            if (lane == 0)
+                bulk_store(p.recv_x + ((size_t)pe * p.maxRecv + slot) * p.rowBytes + off,
+                           stage0_addr + (uint32_t)s * p.chunkStride, bytes);
+        }
+        if (lane == 0) bulk_commit();
+        ++consumed;
+
+        // Refill the stage freed by the item before this one.
+        if (pg < p.G) {
+            if (lane == 0) bulk_wait_read_all_but_one();
+            __syncwarp();
+            issue();
+        }
+    }
+
+    if (!ok) {
+        // Give up: record it, then drain what this engine still has in flight.
+        if (lane == 0) {
+            atomicOr(p.err, EP_DEVERR_TIMEOUT);
+            for (int i = consumed; i < issued; ++i)
+                mbar_wait_bounded(bar0 + 8u * (i % S), (uint32_t)(i / S) & 1u);
+        }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+}
+
+// =====================================================================
+// combine: one warp per token, 16-byte columns, fma fold in destPe order.
+// =====================================================================
+constexpr int kCombineBatch = 8;  // destination rows in flight per column
+constexpr int kCombineUnroll = 2; // columns per lane per iteration
+
+__device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(u[i] << 16);
+        const float hi = __uint_as_float(u[i] & 0xffff0000u);
+        acc[2 * i] = __fmaf_rn(w, lo, acc[2 * i]);
+        acc[2 * i + 1] = __fmaf_rn(w, hi, acc[2 * i + 1]);
+    }
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float* acc) {
+    uint32_t u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = __float22bfloat162_rn(make_float2(acc[2 * i], acc[2 * i + 1]));
+        u[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+__global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(CombineParams p) {
+    __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
+    __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    const int V = (int)(p.rowBytes / 16);
+    const int W = p.W;
+
+    for (int g = blockIdx.x * (blockDim.x >> 5) + warp; g < p.G; g += nw) {
+        const int2 rr = lane < W ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
+        const uint32_t mask = __ballot_sync(kFull, rr.x >= 0);
+        uint4* orow = reinterpret_cast<uint4*>(p.out + (size_t)g * p.rowBytes);
+        if (mask == 0u) {
+            for (int v = lane; v < V; v += 32) orow[v] = make_uint4(0, 0, 0, 0);
+            continue;
+        }
+        // Present destinations in ascending order: rank of this lane's bit.
+        const int n = __popc(mask);
+        if (rr.x >= 0) {
+            const int pos = __popc(mask & lanemask_lt());
+            s_row[warp][pos] = p.y + ((size_t)lane * p.maxRecv + rr.x) * p.rowBytes;
+            s_w[warp][pos] = __int_as_float(rr.y);
+        }
+        __syncwarp();
+
+        for (int v0 = lane; v0 < V; v0 += 32 * kCombineUnroll) {
+            float acc[kCombineUnroll][8];
+#pragma unroll
+            for (int u = 0; u < kCombineUnroll; ++u)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+            for (int b = 0; b < n; b += kCombineBatch) {
+                uint4 val[kCombineUnroll][kCombineBatch];
+#pragma unroll
+                for (int i = 0; i < kCombineBatch; ++i) {
+                    if (b + i < n) {
+                        const uint8_t* row = s_row[warp][b + i];
+#pragma unroll
+                        for (int u = 0; u < kCombineUnroll; ++u) {
+                            const int v = v0 + 32 * u;
+                            if (v < V) val[u][i] = ld_stream_v4(row + (size_t)v * 16);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kCombineBatch; ++i) {
+                    if (b + i < n) {
+                        const float w = s_w[warp][b + i];
+#pragma unroll
+                        for (int u = 0; u < kCombineUnroll; ++u)
+                            if (v0 + 32 * u < V) fma_bf16x8(acc[u], w, val[u][i]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kCombineUnroll; ++u) {
+                const int v = v0 + 32 * u;
+                if (v < V) orow[v] = pack_bf16x8(acc[u]);
+            }
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------- launchers
+cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s) {
+    if (p.W <= 8)
+        ep_route_count_kernel<8><<<p.numTiles, kCountTile, 0, s>>>(p);
+    else if (p.W <= 16)
+        ep_route_count_kernel<16><<<p.numTiles, kCountTile, 0, s>>>(p);
+    else
+        ep_route_count_kernel<32><<<p.numTiles, kCountTile, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+size_t scatter_smem_bytes(int warps, int stages, int chunkStride) {
+    const size_t head =
+        ((size_t)warps * stages * (sizeof(uint64_t) + 2 * sizeof(int)) + 127) & ~(size_t)127;
+    return head + (size_t)warps * stages * (size_t)chunkStride;
+}
+
+cudaError_t scatter_set_smem(size_t bytes) {
+    return cudaFuncSetAttribute(ep_scatter_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)bytes);
+}
+
+cudaError_t scatter_blocks_per_sm(int warps, size_t smem, int* out) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_scatter_rows_kernel, warps * 32, smem);
+}
+
+cudaError_t combine_blocks_per_sm(int warps, int* out) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_combine_kernel, warps * 32, 0);
+}
+
+cudaError_t launch_scatter_rows(const ScatterParams& p, int blocks, int warps, size_t smem,
+                                cudaStream_t s) {
+    ep_scatter_rows_kernel<<<blocks, warps * 32, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineParams& p, int blocks, int warps, cudaStream_t s) {
+    ep_combine_kernel<<<blocks, warps * 32, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace ep

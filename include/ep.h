@@ -1,0 +1,185 @@
+/*
+ * ep.h -- C ABI of the B200 (sm_100a) MoE expert-parallel dispatch / combine
+ * library (libep_b200.so).
+ *
+ * What the calls compute (mori pages: the "MORI JIT v2" design page and mori
+ * PR #599 "Perf/ep disp 1250 ship"):
+ *
+ *   The W expert-parallel ranks are virtual: every rank's send rows, receive
+ *   rows and metadata are regions of one GPU's memory.
+ *
+ *   dispatch  For every source rank r and token t, every valid topk entry j
+ *             (expert id e >= 0) maps to the destination rank
+ *             destPe = e / numExpertPerRank (design page §8). The token is sent
+ *             once to each distinct destination (dedup of (token, destPe),
+ *             PR #599 "ballot dedup"). Destination pe numbers its rows by
+ *             (source rank, source token) ascending; row `slot` of pe lives at
+ *             flat index pe*maxRecv + slot (design page §3.2: maxRecv is the
+ *             stride of the flat receive index). Each row carries a meta record
+ *             (PR #599: three per-token fields, here followed by the local
+ *             expert ids). The receive count of each destination is stored,
+ *             not accumulated (PR #599, follow-up commits: the count is a store).
+ *   combine   out[r][t] = bf16_rne( fold over pe in P(r,t) ascending of
+ *             acc = fma(w(r,t,pe), float(y[pe][slot]), acc) ), acc0 = +0.0f,
+ *             with w(r,t,pe) = float32 sum, in topk order, of the token's topk
+ *             weights whose expert lives on pe (1.0f when useWeights == 0);
+ *             tokens routed nowhere get a zero row (design page §3.7: combine
+ *             reduces, dispatch only moves bytes).
+ *
+ * Conventions (design page §6): every entry point is noexcept; an error is a
+ * NULL or negative return, with a human-readable reason in ep_last_error().
+ * Only pointers and scalars cross the boundary.
+ *
+ * Readings where the pages leave a step open: slot order (the pages reserve
+ * slots with an atomic fetch_add, whose order is unspecified; here it is
+ * (source rank, source token) ascending, so results are deterministic); an
+ * expert id < 0 is a masked entry, so a token whose ids are all < 0 is absent;
+ * an expert id >= W*numExpertPerRank is a contract violation, reported through
+ * the device error word and treated as masked.
+ */
+#ifndef EP_B200_H
+#define EP_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Payload dtype tags, numbered as the design page's EpDType (§3.7). This build
+ * accepts EP_BF16 only; the others are rejected by ep_cfg_check. */
+typedef enum EpDType { EP_BF16 = 0, EP_FP32 = 1, EP_FP8 = 2, EP_FP4X2 = 3 } EpDType;
+
+/* The semantic fields of the design page's EpCfg (§3.2). Launch geometry is
+ * not part of it: the library picks it from the device. */
+typedef struct EpCfg {
+    int32_t worldSize;         /* W: virtual EP ranks, 1..32 */
+    int32_t hiddenDim;         /* h: elements per token row; h*2 must be a multiple of 16 */
+    int32_t maxTokPerRank;     /* T: token rows per source rank, >= 1 */
+    int32_t numExpertPerRank;  /* experts on each rank, >= 1; E = W*numExpertPerRank */
+    int32_t numExpertPerToken; /* k (topk), 1..32 */
+    int32_t maxRecv;           /* receive rows per destination; 0 means W*T; must be >= W*T */
+    int32_t dtype;             /* EpDType; EP_BF16 only */
+    int32_t useWeights;        /* 1: combine weights by the topk weights; 0: weight 1 */
+} EpCfg;
+
+/* What a plan resolved. Sizes are in bytes. */
+typedef struct EpPlanInfo {
+    int32_t maxRecv;          /* resolved receive capacity per destination */
+    int32_t metaFields;       /* int32 fields per meta record: 3 + k */
+    int64_t rowBytes;         /* h * 2 */
+    int64_t tokenBytes;       /* bytes of x and of out: W*T*rowBytes */
+    int64_t recvXBytes;       /* bytes of recv_x and of y: W*maxRecv*rowBytes */
+    int64_t recvMetaBytes;    /* W*maxRecv*metaFields*4 */
+    int64_t scratchBytes;     /* device scratch the plan owns */
+    int32_t countTile;        /* tokens per routing tile */
+    int32_t numTiles;         /* routing tiles: ceil(W*T / countTile) */
+    int32_t scatterBlocks;    /* grid of the row-scatter kernel */
+    int32_t scatterWarps;     /* copy engines (warps) per scatter block */
+    int32_t scatterStages;    /* shared-memory stages per copy engine */
+    int32_t scatterChunkBytes;/* bytes per staged copy (a row, or a piece of one) */
+    int32_t combineBlocks;    /* grid of the combine kernel */
+    int32_t combineWarps;     /* warps per combine block */
+    int32_t device;           /* CUDA device the plan lives on (-1 from ep_plan_query) */
+    int32_t numSMs;           /* SMs of that device (0 from ep_plan_query) */
+} EpPlanInfo;
+
+typedef struct EpPlan EpPlan;
+
+/* Return codes (negative) of the host entry points. */
+enum {
+    EP_OK = 0,
+    EP_ERR_INVALID = -1,     /* bad argument or configuration */
+    EP_ERR_UNSUPPORTED = -2, /* valid for the pages, not built here (dtype) */
+    EP_ERR_NOMEM = -3,       /* device allocation failed */
+    EP_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
+    EP_ERR_STATE = -5,       /* combine before any dispatch on this plan */
+    EP_ERR_ALIGN = -6,       /* a buffer is not aligned as documented */
+    EP_ERR_DEVICE = -7       /* the current device is not the plan's device */
+};
+
+/* Bits of the device error word (ep_plan_check_error). Kernels never trap:
+ * they record the problem here and keep going or return. */
+enum {
+    EP_DEVERR_EXPERT_RANGE = 1, /* an expert id >= E was seen; it was treated as masked */
+    EP_DEVERR_TIMEOUT = 2,      /* a bounded wait on a shared-memory barrier gave up */
+    EP_DEVERR_CAPACITY = 4      /* a destination received more than maxRecv rows */
+};
+
+/* Validate a configuration on the host (no CUDA call). Returns EP_OK, or
+ * EP_ERR_INVALID / EP_ERR_UNSUPPORTED with the reason in ep_last_error().
+ * Rules (design page §3.5, EpCfgIsValid): the row bytes must be a multiple of
+ * 16; topk and worldSize must fit one 32-lane warp; the receive capacity must
+ * cover the worst case (maxRecv >= W*T); only bf16 payloads (§3.7). */
+int ep_cfg_check(const EpCfg* cfg);
+
+/* Host-only sizing: fill *info for cfg as a plan on a generic device would
+ * resolve it (device = -1, numSMs = 0, geometry from a 148-SM B200). Lets a
+ * caller size recv_x / recv_meta before creating a plan. Returns EP_OK or a
+ * negative code. */
+int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
+
+/* Create a plan on the current CUDA device: validates cfg, picks the launch
+ * geometry, allocates and zeroes the plan's device scratch (routing table
+ * [W*T][W] of (slot, weight) pairs, per-tile counts and offsets, a tile
+ * ticket, the error word). Returns NULL on failure (ep_last_error() says why).
+ * Environment overrides, read here only (for geometry sweeps):
+ * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK,
+ * EP_COMBINE_BLOCKS, EP_COMBINE_WARPS. */
+EpPlan* ep_plan_create(const EpCfg* cfg);
+
+/* Free the plan and its scratch. NULL is a no-op. The caller must make sure no
+ * dispatch or combine of this plan is still running on the GPU. */
+void ep_plan_destroy(EpPlan* plan);
+
+/* Copy the plan's resolved sizes and geometry into *info. */
+int ep_plan_info(const EpPlan* plan, EpPlanInfo* info);
+
+/*
+ * Dispatch, enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ * stream). No host synchronisation, no allocation: capturable in a CUDA graph.
+ * All pointers are device pointers owned by the caller.
+ *   x          bf16  [W][T][h]            16-byte aligned
+ *   topk_idx   int32 [W][T][k]            expert ids; < 0 masked
+ *   topk_w     float [W][T][k]            NULL allowed when useWeights == 0
+ *   recv_x     bf16  [W][maxRecv][h]      16-byte aligned; rows >= recv_count[pe]
+ *                                         of destination pe are not written
+ *   recv_meta  int32 [W][maxRecv][3+k]    per row: source rank, source token,
+ *                                         weight sum (float32 bits), then for
+ *                                         each topk position j the local expert
+ *                                         id (e - pe*numExpertPerRank) when
+ *                                         entry j lives on pe, else -1; records
+ *                                         past recv_count are not written
+ *   recv_count int32 [W]                  rows received per destination (stored)
+ * The routing (slot and weight of every (r,t,pe)) stays in the plan for the
+ * next ep_combine. Returns EP_OK or a negative code; kernel-side contract
+ * violations go to the device error word.
+ */
+int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
+                void* recv_x, int32_t* recv_meta, int32_t* recv_count, void* stream);
+
+/*
+ * Combine, enqueued on `stream`, using the routing of the most recent
+ * ep_dispatch of this plan (stream order is the caller's: issue it on the same
+ * stream, or order the streams). No host synchronisation, no allocation.
+ *   y    bf16 [W][maxRecv][h]   expert outputs in the receive layout, 16-byte
+ *                               aligned; only rows < recv_count are read
+ *   out  bf16 [W][T][h]         16-byte aligned; every row is written
+ * Returns EP_OK, EP_ERR_STATE before any dispatch, or a negative code.
+ */
+int ep_combine(EpPlan* plan, const void* y, void* out, void* stream);
+
+/* Synchronise the device, return the device error word (a bitmask of
+ * EP_DEVERR_*, 0 when clean) and clear it; negative on a CUDA error. Meant for
+ * tests and debugging, not for the hot path. */
+int ep_plan_check_error(EpPlan* plan);
+
+/* Reason for the last failure on this thread ("" if none). */
+const char* ep_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_H */

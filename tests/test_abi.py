@@ -1,0 +1,163 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+entry point include/ep.h declares, its structs have the layout the header
+gives, configuration checks follow the validity rules, and calls that need a
+device fail with an error instead of crashing."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+import textwrap
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ep.h")
+
+
+@pytest.fixture(scope="module")
+def ep():
+    from combine_ep_dispatch_05_b200 import build
+    build.build()
+    import combine_ep_dispatch_05_b200 as mod
+    return mod
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ep_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for n in ("ep_plan_create", "ep_dispatch", "ep_combine", "ep_plan_destroy", "ep_last_error",
+              "ep_plan_info", "ep_plan_check_error", "ep_cfg_check", "ep_plan_query"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ep):
+    lib = ctypes.CDLL(ep.library_path())
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", ep.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ep_[a-z_]+)\b", out))
+    assert set(declared_functions()) <= exported
+    assert set(ep.binding.EXPORTED) == set(declared_functions())
+
+
+def test_struct_layout_matches_header(ep, tmp_path):
+    """sizeof/offsetof from a C compile of include/ep.h against the ctypes mirror."""
+    fields = {"EpCfg": [n for n, _ in ep.EpCfg._fields_],
+              "EpPlanInfo": [n for n, _ in ep.EpPlanInfo._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "ep.h"', 'int main(void) {']
+    for st, names in fields.items():
+        lines.append(f'  printf("{st} size %zu\\n", sizeof({st}));')
+        for n in names:
+            lines.append(f'  printf("{st} {n} %zu\\n", offsetof({st}, {n}));')
+    lines += ['  return 0;', '}']
+    c = tmp_path / "layout.c"
+    c.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)])
+    rows = [l.split() for l in subprocess.check_output([str(exe)], text=True).splitlines()]
+    for st, key, val in rows:
+        cls = getattr(ep, st)
+        if key == "size":
+            assert ctypes.sizeof(cls) == int(val), st
+        else:
+            assert getattr(cls, key).offset == int(val), (st, key)
+
+
+def test_header_compiles_as_plain_c_and_cpp(tmp_path):
+    """The ABI header needs no CUDA header and compiles as C and C++."""
+    for lang, comp in (("c", "gcc"), ("cpp", "g++")):
+        f = tmp_path / f"inc.{lang}"
+        f.write_text('#include "ep.h"\nint main(void){ EpCfg c = {0}; return (int)sizeof(c) - 32; }\n')
+        subprocess.check_call([comp, "-I", os.path.join(ROOT, "include"), str(f), "-o", str(tmp_path / lang)])
+        assert subprocess.run([str(tmp_path / lang)]).returncode == 0
+
+
+def _cfg(**kw):
+    c = dict(worldSize=8, hiddenDim=7168, maxTokPerRank=4096, numExpertPerRank=32,
+             numExpertPerToken=8, maxRecv=32768, dtype=0, useWeights=1)
+    c.update(kw)
+    return c
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(), 0),
+    (dict(maxRecv=0), 0),
+    (dict(hiddenDim=7), -1),              # 14 bytes: not a multiple of 16
+    (dict(hiddenDim=12), -1),             # 24 bytes
+    (dict(hiddenDim=8), 0),               # 16 bytes
+    (dict(numExpertPerToken=33), -1),     # topk must fit one warp
+    (dict(numExpertPerToken=0), -1),
+    (dict(worldSize=33), -1),             # worldSize must fit one warp
+    (dict(worldSize=0), -1),
+    (dict(maxRecv=32767), -1),            # capacity below the worst case
+    (dict(maxTokPerRank=0), -1),
+    (dict(numExpertPerRank=0), -1),
+    (dict(dtype=2), -2),                  # fp8 transport not built
+    (dict(dtype=1), -2),
+    (dict(dtype=9), -1),
+    (dict(useWeights=2), -1),
+    (dict(worldSize=32, maxTokPerRank=1 << 22, maxRecv=0), -1),  # flat index beyond int32
+])
+def test_cfg_check(ep, kw, code):
+    assert ep.ep_cfg_check(_cfg(**kw)) == code
+    if code:
+        assert ep.ep_last_error()
+
+
+def test_plan_query_sizes(ep):
+    info = ep.ep_plan_query(_cfg(maxRecv=0))
+    assert info.maxRecv == 8 * 4096
+    assert info.metaFields == 11
+    assert info.rowBytes == 14336
+    assert info.tokenBytes == 8 * 4096 * 14336
+    assert info.recvXBytes == 8 * 32768 * 14336
+    assert info.recvMetaBytes == 8 * 32768 * 11 * 4
+    assert info.numTiles == (8 * 4096 + info.countTile - 1) // info.countTile
+    assert info.scatterChunkBytes % 16 == 0 and info.scatterStages >= 2
+    big = ep.ep_plan_query(_cfg(hiddenDim=40000))
+    assert big.scatterChunkBytes < big.rowBytes and big.scatterChunkBytes % 16 == 0
+
+
+def test_entry_points_reject_without_crashing(ep):
+    b = ep.binding
+    assert b._lib.ep_dispatch(None, None, None, None, None, None, None, None) == b.EP_ERR_INVALID
+    assert b._lib.ep_combine(None, None, None, None) == b.EP_ERR_INVALID
+    assert b._lib.ep_plan_info(None, None) == b.EP_ERR_INVALID
+    assert b._lib.ep_plan_check_error(None) == b.EP_ERR_INVALID
+    b._lib.ep_plan_destroy(None)
+    with pytest.raises(ep.EpError):
+        ep.ep_plan_create(_cfg(hiddenDim=7))
+
+
+def test_plan_create_without_device_fails_cleanly(ep):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    with pytest.raises(ep.EpError) as e:
+        ep.ep_plan_create(_cfg(maxTokPerRank=8, maxRecv=0))
+    assert "cuda" in str(e.value).lower()
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """No fallback: importing the binding without the built library raises."""
+    pkg = tmp_path / "combine_ep_dispatch_05_b200"
+    pkg.mkdir()
+    src = os.path.join(ROOT, "combine_ep_dispatch_05_b200")
+    for f in ("__init__.py", "binding.py"):
+        (pkg / f).write_text(open(os.path.join(src, f)).read())
+    code = textwrap.dedent("""
+        import combine_ep_dispatch_05_b200 as ep
+        try:
+            ep.ep_dispatch
+        except ImportError as e:
+            print("IMPORTERROR", e)
+    """)
+    out = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
+    assert "IMPORTERROR" in out.stdout and "libep_b200.so" in out.stdout

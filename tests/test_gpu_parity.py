@@ -1,0 +1,188 @@
+"""CUDA path vs the CPU oracle, through the C ABI (needs a B200).
+
+Dispatch outputs (recv_x, recv_meta, recv_count) must be bit-exact; rows and
+records past recv_count must keep their canary; combine must be within
+2^-7|oracle| + 1e-3 and, with the same fold order and one rounding per term,
+bit-exact.
+"""
+import os
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU machines too
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import combine_ep_dispatch_05_b200 as ep  # noqa: E402
+import oracle  # noqa: E402
+import oracle_pins as P  # noqa: E402
+from gpu_harness import GpuRun, compare_combine, compare_dispatch, run_and_compare, to_dev  # noqa: E402
+from synth.inputs import WORKLOADS, make_inputs, workload  # noqa: E402
+
+
+def test_library_is_in_tree():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    assert ep.library_path().startswith(root)
+
+
+@pytest.mark.parametrize("name", ["tiny", "pr599", "latency1", "latency8", "main", "skewed"])
+def test_workload_parity(name):
+    wl = workload(name)
+    run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
+    run.close()
+
+
+def _small_random_cfg(rng, W, T, h, k, nEpr, use_w, max_recv=0, dup=True, oob=False):
+    E = W * nEpr
+    lo = -2 if dup else 0
+    hi = E + (3 if oob else 0)
+    idx = rng.integers(lo, hi, size=(W, T, k)).astype(np.int32)
+    xb = P.torch_bf16_bits(rng.standard_normal((W, T, h)).astype(np.float32))
+    w = rng.standard_normal((W, T, k)).astype(np.float32) if use_w else None
+    cfg = dict(worldSize=W, hiddenDim=h, maxTokPerRank=T, numExpertPerRank=nEpr,
+               numExpertPerToken=k, maxRecv=max_recv, dtype=0, useWeights=int(use_w))
+    return cfg, dict(x=xb, topk_idx=idx, topk_w=w)
+
+
+@pytest.mark.parametrize("case", [
+    # W, T, h, k, nEpr, weights, maxRecv -- several routing tiles with a ragged tail
+    (3, 300, 264, 5, 3, True, 0),       # 528-byte rows: combine column tail
+    (1, 513, 128, 4, 6, True, 0),       # single rank
+    (32, 9, 64, 32, 2, True, 0),        # max world size and max topk: 35 meta fields
+    (5, 77, 8, 7, 1, False, 500),       # 16-byte rows, maxRecv above W*T, no weights
+    (2, 40, 20000, 3, 4, True, 0),      # 40000-byte rows: copied in three pieces
+    (8, 1000, 1024, 6, 8, True, 0),     # 4 tiles, ragged
+])
+def test_random_parity(case):
+    W, T, h, k, nEpr, use_w, max_recv = case
+    rng = np.random.default_rng(hash(case) % (1 << 32))
+    cfg, inputs = _small_random_cfg(rng, W, T, h, k, nEpr, use_w, max_recv)
+    run, _ = run_and_compare(cfg, inputs)
+    run.close()
+
+
+def test_out_of_range_ids_reported_and_masked():
+    rng = np.random.default_rng(5)
+    cfg, inputs = _small_random_cfg(rng, 4, 64, 64, 4, 4, True, oob=True)
+    assert (inputs["topk_idx"] >= 16).any()
+    run, ref = run_and_compare(cfg, inputs)  # checks the error word against the oracle status
+    assert ref["status"] == oracle.STATUS_EXPERT_RANGE
+    run.close()
+
+
+def test_fma_single_rounding_case():
+    """The crafted input where fusing w*y into the add decides the bf16 result."""
+    cfg, idx, w, y = P.fma_sensitive_case()
+    inputs = dict(x=np.zeros((2, 1, 8), np.uint16), topk_idx=idx, topk_w=w)
+    run, _ = run_and_compare(cfg, inputs, y_override=y)
+    assert bool((run.out[0, 0] == 0x3F81).all())
+    run.close()
+
+
+def test_absent_tokens_and_empty_call():
+    """All ids masked: nothing received, zero counts, zero output rows."""
+    wl = workload("latency1")
+    inputs = make_inputs(wl)
+    inputs["topk_idx"][:] = -1
+    run, ref = run_and_compare(wl.cfg(), inputs)
+    assert int(ref["recv_count"].sum()) == 0
+    assert bool((run.out == 0).all())
+    run.close()
+
+
+def test_repeated_calls_and_reset():
+    """Two dispatches with different routing on one plan: counters and the
+    tile ticket reset, results follow each call."""
+    wl = workload("pr599").replace(h=512)
+    cfg = wl.cfg()
+    a = make_inputs(wl)
+    b = make_inputs(wl.replace(seed=77))
+    ref_a = oracle.dispatch(cfg, a["x"], a["topk_idx"], a["topk_w"])
+    ref_b = oracle.dispatch(cfg, b["x"], b["topk_idx"], b["topk_w"])
+    with GpuRun(cfg, a) as run:
+        run.dispatch()
+        torch.cuda.synchronize()
+        compare_dispatch(run, ref_a)
+        run.idx.copy_(to_dev(b["topk_idx"]))
+        run.w.copy_(to_dev(b["topk_w"]))
+        run.x.copy_(to_dev(b["x"].view(np.int16)))
+        run.recv_x.fill_(0xABCD - (1 << 16))
+        run.recv_meta.fill_(0x5EADBEEF)
+        run.dispatch()
+        run.combine()
+        torch.cuda.synchronize()
+        compare_dispatch(run, ref_b)
+        compare_combine(run, oracle.combine(cfg, ref_b["recv_x"], ref_b["slotmap"], ref_b["wsum"]))
+        assert run.error_word() == 0
+
+
+def test_graph_capture_replay():
+    """dispatch -> identity expert -> combine captured as one CUDA graph and
+    replayed: every replay reproduces eager bit for bit (MORI JIT v2 design
+    page §4: the graph-capture test)."""
+    wl = workload("pr599")
+    cfg = wl.cfg()
+    inputs = make_inputs(wl)
+    run, ref = run_and_compare(cfg, inputs)  # eager pass, checked against the oracle
+    eager_out = run.out.clone()
+    eager_meta = run.recv_meta.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            run.dispatch(stream=s)
+            run.combine(stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        run.out.fill_(0x7FC1)
+        run.recv_count.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(run.out, eager_out)
+        assert torch.equal(run.recv_meta, eager_meta)
+        assert np.array_equal(run.recv_count.cpu().numpy(), ref["recv_count"])
+    assert run.error_word() == 0
+    del g
+    run.close()
+
+
+@pytest.mark.parametrize("env", [
+    {"EP_SCATTER_STAGES": "2"},
+    {"EP_SCATTER_WARPS": "1", "EP_SCATTER_BLOCKS": "1"},   # one copy engine does everything
+    {"EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2", "EP_SCATTER_CHUNK": "1024"},
+    {"EP_COMBINE_WARPS": "1", "EP_COMBINE_BLOCKS": "3"},
+])
+def test_geometry_overrides(env, monkeypatch):
+    for k_, v in env.items():
+        monkeypatch.setenv(k_, v)
+    wl = workload("pr599").replace(h=1536)
+    run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
+    info = run.info
+    if "EP_SCATTER_BLOCKS" in env:
+        assert info.scatterBlocks == int(env["EP_SCATTER_BLOCKS"])
+    run.close()
+
+
+def test_host_side_rejections():
+    wl = workload("tiny")
+    with GpuRun(wl.cfg(), make_inputs(wl)) as run:
+        with pytest.raises(ep.EpError) as e:
+            run.combine()
+        assert e.value.code == ep.EP_ERR_STATE
+        with pytest.raises(ep.EpError) as e:
+            ep.ep_dispatch(run.plan, run.x.data_ptr() + 2, run.idx, run.w, run.recv_x, run.recv_meta,
+                           run.recv_count, torch.cuda.current_stream())
+        assert e.value.code == ep.EP_ERR_ALIGN
+        with pytest.raises(ep.EpError) as e:
+            ep.ep_dispatch(run.plan, run.x, run.idx, None, run.recv_x, run.recv_meta, run.recv_count,
+                           torch.cuda.current_stream())
+        assert e.value.code == ep.EP_ERR_INVALID
+        assert run.error_word() == 0
+
+
+def test_all_workloads_registered():
+    assert {"tiny", "pr599", "main", "latency1", "latency8", "skewed"} <= set(WORKLOADS)
