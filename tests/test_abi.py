@@ -161,3 +161,10 @@ def test_binding_fails_loudly_without_library(tmp_path):
     """)
     out = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
     assert "IMPORTERROR" in out.stdout and "libep_b200.so" in out.stdout
+
+
+def test_graft_entry_build():
+    """The build entry point compiles both libraries and loads the binding."""
+    sys.path.insert(0, ROOT)
+    import __graft_entry__
+    __graft_entry__.build()
