@@ -41,7 +41,8 @@ class EpPlanInfo(ctypes.Structure):
                 ("scatterWarps", ctypes.c_int32), ("scatterStages", ctypes.c_int32),
                 ("scatterChunkBytes", ctypes.c_int32), ("combineBlocks", ctypes.c_int32),
                 ("combineWarps", ctypes.c_int32), ("device", ctypes.c_int32),
-                ("numSMs", ctypes.c_int32)]
+                ("numSMs", ctypes.c_int32), ("scatterMode", ctypes.c_int32),
+                ("scatterPend", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}

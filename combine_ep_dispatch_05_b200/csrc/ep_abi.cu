@@ -97,12 +97,16 @@ int check_cfg(const EpCfg* c) {
 
 struct Geometry {
     int chunkBytes, chunkStride, numChunks;
+    int scatterMode, scatterPend;
     int scatterWarps, scatterStages;
     int combineWarps;
 };
 
-// Copy engines and stages: fill about 200 KB of shared memory per SM with
-// row-sized stages (rows above 32 KB are copied in pieces of <= 16 KB).
+// Copy engines and stages: two engines (warps) per block, each with as many
+// row-sized stages as fit in about 200 KB of shared memory (at most 8; rows
+// above 32 KB are copied in pieces of <= 16 KB). On B200 at 14 KB rows, 2
+// engines x 6 stages per SM beat 4 x 3, 3 x 4 and 6 x 2 (deeper per-engine
+// lookahead) and 1 x 12 (one issuing thread per SM is too few).
 Geometry pick_geometry(const EpCfg* c, bool use_env) {
     Geometry g{};
     const long long rowBytes = (long long)c->hiddenDim * 2;
@@ -119,7 +123,7 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
     g.chunkStride = (chunk + 127) & ~127;
     g.numChunks = (int)((rowBytes + chunk - 1) / chunk);
     const int budget = 200 * 1024;
-    int warps = 4;
+    int warps = 2;
     int stages = budget / (warps * g.chunkStride);
     if (stages < 2) {
         warps = std::max(1, budget / (2 * g.chunkStride));
@@ -130,6 +134,20 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
         warps = std::min(env_int("EP_SCATTER_WARPS", warps), ep::kMaxScatterWarps);
         stages = std::max(2, std::min(env_int("EP_SCATTER_STAGES", stages), 16));
     }
+    int pend = 1;
+    int mode = ep::kScatterTma;
+    if (use_env) {
+        pend = std::max(1, std::min(env_int("EP_SCATTER_PEND", pend), 3));
+        const char* m = std::getenv("EP_SCATTER_MODE");
+        if (m && std::strcmp(m, "regs") == 0) mode = ep::kScatterRegs;
+    }
+    stages = std::max(stages, pend + 1);
+    if (mode == ep::kScatterRegs) {
+        warps = std::min(use_env ? env_int("EP_SCATTER_WARPS", 8) : 8, 8);
+        stages = 0;
+    }
+    g.scatterMode = mode;
+    g.scatterPend = pend;
     g.scatterWarps = warps;
     g.scatterStages = stages;
     g.combineWarps = use_env ? std::min(env_int("EP_COMBINE_WARPS", 8), ep::kMaxCombineWarps) : 8;
@@ -155,6 +173,8 @@ void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
     info->scatterWarps = geo.scatterWarps;
     info->scatterStages = geo.scatterStages;
     info->scatterChunkBytes = geo.chunkBytes;
+    info->scatterMode = geo.scatterMode;
+    info->scatterPend = geo.scatterPend;
     info->combineWarps = geo.combineWarps;
     info->device = -1;
 }
@@ -183,7 +203,7 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info) {
         fill_info(cfg, geo, info);
         const int sms = 148;  // B200
         info->scatterBlocks = sms * std::max(1, (200 * 1024) / (int)ep::scatter_smem_bytes(
-                                                                   geo.scatterWarps, geo.scatterStages,
+                                                                   geo.scatterWarps, std::max(geo.scatterStages, 1),
                                                                    geo.chunkStride));
         info->combineBlocks = sms * 2;
         return EP_OK;
@@ -210,25 +230,29 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             return nullptr;
         }
         Geometry geo = pick_geometry(cfg, true);
-        size_t smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
-        while (smem > (size_t)smemOptin && geo.scatterStages > 2) {
-            --geo.scatterStages;
+        size_t smem = 0;
+        if (geo.scatterMode == ep::kScatterTma) {
             smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
-        }
-        while (smem > (size_t)smemOptin && geo.scatterWarps > 1) {
-            --geo.scatterWarps;
-            smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
-        }
-        if (smem > (size_t)smemOptin) {
-            fail(EP_ERR_INVALID, "row piece of %d bytes does not fit shared memory", geo.chunkBytes);
-            return nullptr;
-        }
-        if ((e = ep::scatter_set_smem(smem)) != cudaSuccess) {
-            cuda_fail(e, "cudaFuncSetAttribute(scatter smem)");
-            return nullptr;
+            while (smem > (size_t)smemOptin && geo.scatterStages > geo.scatterPend + 1) {
+                --geo.scatterStages;
+                smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+            }
+            while (smem > (size_t)smemOptin && geo.scatterWarps > 1) {
+                --geo.scatterWarps;
+                smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+            }
+            if (smem > (size_t)smemOptin) {
+                fail(EP_ERR_INVALID, "row piece of %d bytes does not fit shared memory", geo.chunkBytes);
+                return nullptr;
+            }
+            if ((e = ep::scatter_set_smem(geo.scatterPend, smem)) != cudaSuccess) {
+                cuda_fail(e, "cudaFuncSetAttribute(scatter smem)");
+                return nullptr;
+            }
         }
         int sPerSm = 0, cPerSm = 0;
-        if ((e = ep::scatter_blocks_per_sm(geo.scatterWarps, smem, &sPerSm)) != cudaSuccess ||
+        if ((e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps, smem,
+                                           &sPerSm)) != cudaSuccess ||
             (e = ep::combine_blocks_per_sm(geo.combineWarps, &cPerSm)) != cudaSuccess) {
             cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
             return nullptr;
@@ -367,8 +391,8 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
         sp.chunkStride = (sp.chunkBytes + 127) & ~127;
         sp.numChunks = (int)((sp.rowBytes + sp.chunkBytes - 1) / sp.chunkBytes);
         sp.stages = plan->info.scatterStages;
-        e = ep::launch_scatter_rows(sp, plan->info.scatterBlocks, plan->info.scatterWarps,
-                                    plan->scatterSmem, s);
+        e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend,
+                                    plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch scatter_rows");
         plan->dispatched = true;
         return EP_OK;

@@ -57,16 +57,21 @@ struct CombineParams {
 
 // Launchers (ep_kernels.cu). Each returns the cudaError_t of its launch.
 cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s);
-cudaError_t launch_scatter_rows(const ScatterParams& p, int blocks, int warps, size_t smem,
-                                cudaStream_t s);
+// Scatter variants: TMA bulk copies staged in shared memory (kPend = bulk
+// store groups left draining when a stage is refilled), or plain 16-byte
+// register copies (no shared memory).
+constexpr int kScatterTma = 0;
+constexpr int kScatterRegs = 1;
+cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
+                                size_t smem, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, int blocks, int warps, cudaStream_t s);
 
 // Shared-memory bytes the scatter kernel needs for a geometry.
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride);
-// Opt the scatter kernel in to `bytes` of dynamic shared memory.
-cudaError_t scatter_set_smem(size_t bytes);
+// Opt the TMA scatter kernel in to `bytes` of dynamic shared memory.
+cudaError_t scatter_set_smem(int pend, size_t bytes);
 // Blocks of each kernel that fit on one SM (occupancy calculator).
-cudaError_t scatter_blocks_per_sm(int warps, size_t smem, int* out);
+cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out);
 cudaError_t combine_blocks_per_sm(int warps, int* out);
 
 }  // namespace ep

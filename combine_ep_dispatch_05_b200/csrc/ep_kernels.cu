@@ -100,11 +100,6 @@ __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-// All but the most recent bulk group have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_read_all_but_one() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-
 // Every bulk group of this thread has completed (writes done).
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -227,15 +222,81 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
 }
 
 // =====================================================================
-// scatter_rows: persistent copy engines, one per warp.
-// Items are (present token, chunk) pairs of this engine's tokens
-// g = engine, engine + nEngines, ...; an S-stage ring keeps S-1 loads ahead.
+// Per-token bookkeeping of the scatter, done by one warp. The three global
+// reads it needs (the routing row, the tile bases, the topk ids) do not depend
+// on one another; TokenInputs holds them so that a warp can issue them for its
+// next token before it works on the current one.
 // =====================================================================
+struct TokenInputs {
+    int g;     // token, or -1 when nothing is loaded
+    int2 rr;   // lane < W: (tile-local rank or -1, weight bits)
+    int base;  // lane < W: base of the token's tile at destination lane
+    int e;     // lane < k: topk id
+};
+
+__device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p, int g, int lane) {
+    TokenInputs in;
+    in.g = g;
+    const int W = p.W;
+    in.rr = lane < W ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
+    in.base = lane < W ? p.tile_base[(size_t)(g / kCountTile) * W + lane] : 0;
+    in.e = lane < p.k ? p.idx[(size_t)g * p.k + lane] : -1;
+    return in;
+}
+
+// Turn the tile-local ranks of the token into slots (lane pe holds the slot
+// at pe), write them back into the routing table for combine, and write the
+// token's meta record at every destination. Returns the destination mask.
+__device__ __forceinline__ uint32_t token_slots_and_meta(const ScatterParams& p, const TokenInputs& in,
+                                                         int lane, int& my_slot) {
+    const int W = p.W, g = in.g;
+    const int2 rr = in.rr;
+    const uint32_t mask = __ballot_sync(kFull, rr.x >= 0);
+    my_slot = -1;
+    if (rr.x >= 0) {
+        my_slot = in.base + rr.x;
+        p.route[(size_t)g * W + lane].x = my_slot;
+    }
+    const int r = g / p.T, t = g - r * p.T;
+    const int e = in.e;
+    const int pe_e = (e >= 0 && e < p.E) ? e / p.nEpr : -1;
+    // field f of a record: 0 rank, 1 token, 2 weight bits, 3+j local id of entry j
+    const int j0 = lane - 3, j1 = lane + 29;
+    const int e0 = __shfl_sync(kFull, e, j0 & 31), q0 = __shfl_sync(kFull, pe_e, j0 & 31);
+    const int e1 = __shfl_sync(kFull, e, j1 & 31), q1 = __shfl_sync(kFull, pe_e, j1 & 31);
+    for (uint32_t m = mask; m; m &= m - 1) {
+        const int pe = __ffs(m) - 1;
+        const int slot = __shfl_sync(kFull, my_slot, pe);
+        const int wb = __shfl_sync(kFull, rr.y, pe);
+        int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
+        int v0;
+        if (lane == 0) v0 = r;
+        else if (lane == 1) v0 = t;
+        else if (lane == 2) v0 = wb;
+        else v0 = (q0 == pe) ? e0 - pe * p.nEpr : -1;
+        if (lane < p.M) rec[lane] = v0;
+        if (lane + 32 < p.M) rec[lane + 32] = (q1 == pe) ? e1 - pe * p.nEpr : -1;
+    }
+    return mask;
+}
+
+// =====================================================================
+// scatter_rows (TMA): persistent copy engines, one per warp.
+// Items are (present token, chunk) pairs of this engine's tokens
+// g = engine, engine + nEngines, ...; an S-stage ring keeps S - kPend loads
+// ahead and lets kPend items' bulk stores drain while the next load starts.
+// =====================================================================
+template <int kPend>
+__device__ __forceinline__ void bulk_wait_read_pend() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kPend) : "memory");
+}
+
+template <int kPend>
 __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(ScatterParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
-    const int S = p.stages;
+    const int S = p.stages;  // > kPend (checked on the host)
 
     // Layout: [bars: nwarps*S u64][ring: nwarps*S*2 int] pad to 128 | stages
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
@@ -290,9 +351,12 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
         }
     };
 
-    for (int i = 0; i < S - 1 && pg < p.G; ++i) issue();
+    const int lookahead = S - kPend;
+    for (int i = 0; i < lookahead && pg < p.G; ++i) issue();
 
     // Per-token state kept across the chunks of one token.
+    TokenInputs pre;
+    pre.g = -1;
     int cur_tok = -1;
     uint32_t cur_mask = 0;
     int my_slot = -1;  // lane pe: slot of the current token at pe
@@ -305,35 +369,13 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
         const int c = item_chunk[s];
 
         if (g != cur_tok) {
-            // Slots, routing update and meta records of token g.
             cur_tok = g;
-            const int2 rr = lane < W ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
-            cur_mask = __ballot_sync(kFull, rr.x >= 0);
-            my_slot = -1;
-            if (rr.x >= 0) {
-                my_slot = p.tile_base[(size_t)(g / kCountTile) * W + lane] + rr.x;
-                p.route[(size_t)g * W + lane].x = my_slot;
-            }
-            const int r = g / p.T, t = g - r * p.T;
-            const int e = lane < p.k ? p.idx[(size_t)g * p.k + lane] : -1;
-            const int pe_e = (e >= 0 && e < p.E) ? e / p.nEpr : -1;
-            // field f of a record: 0 rank, 1 token, 2 weight bits, 3+j local id of entry j
-            const int j0 = lane - 3, j1 = lane + 29;
-            const int e0 = __shfl_sync(kFull, e, j0 & 31), q0 = __shfl_sync(kFull, pe_e, j0 & 31);
-            const int e1 = __shfl_sync(kFull, e, j1 & 31), q1 = __shfl_sync(kFull, pe_e, j1 & 31);
-            for (uint32_t m = cur_mask; m; m &= m - 1) {
-                const int pe = __ffs(m) - 1;
-                const int slot = __shfl_sync(kFull, my_slot, pe);
-                const int wb = __shfl_sync(kFull, rr.y, pe);
-                int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
-                int v0;
-                if (lane == 0) v0 = r;
-                else if (lane == 1) v0 = t;
-                else if (lane == 2) v0 = wb;
-                else v0 = (q0 == pe) ? e0 - pe * p.nEpr : -1;
-                if (lane < p.M) rec[lane] = v0;
-                if (lane + 32 < p.M) rec[lane + 32] = (q1 == pe) ? e1 - pe * p.nEpr : -1;
-            }
+            const TokenInputs in = (pre.g == g) ? pre : load_token_inputs(p, g, lane);
+            // Prefetch the next token in the ring before working on this one.
+            pre.g = -1;
+            const int nxt = consumed + p.numChunks - c;
+            if (nxt < issued) pre = load_token_inputs(p, item_tok[nxt % S], lane);
+            cur_mask = token_slots_and_meta(p, in, lane, my_slot);
         }
 
         // Wait for the row piece, then send it to every destination.
@@ -357,9 +399,9 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
         if (lane == 0) bulk_commit();
         ++consumed;
 
-        // Refill the stage freed by the item before this one.
+        // Refill the stage whose stores (kPend items back) have been read out.
         if (pg < p.G) {
-            if (lane == 0) bulk_wait_read_all_but_one();
+            if (lane == 0) bulk_wait_read_pend<kPend>();
             __syncwarp();
             issue();
         }
@@ -375,6 +417,50 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
+}
+
+// =====================================================================
+// scatter_rows (registers): one warp per token, no shared-memory staging.
+// The warp loads a piece of the row (32 lanes x kVec 16-byte vectors) into
+// registers once and stores it to every destination; loads stream past L1.
+// =====================================================================
+constexpr int kRegVec = 28;  // 16-byte vectors per lane per piece: 14336-byte pieces
+
+__device__ __forceinline__ void st_v4(void* p, const uint4& v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(256) ep_scatter_rows_regs_kernel(ScatterParams p) {
+    const int lane = threadIdx.x & 31;
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    const long long V = p.rowBytes / 16;
+    for (int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < p.G; g += nw) {
+        const int lr = lane < p.W ? p.route[(size_t)g * p.W + lane].x : -1;
+        if (__ballot_sync(kFull, lr >= 0) == 0u) continue;
+        int my_slot;
+        const uint32_t mask = token_slots_and_meta(p, load_token_inputs(p, g, lane), lane, my_slot);
+        const uint8_t* src = p.x + (size_t)g * p.rowBytes;
+        for (long long v0 = 0; v0 < V; v0 += 32LL * kRegVec) {
+            uint4 buf[kRegVec];
+#pragma unroll
+            for (int i = 0; i < kRegVec; ++i) {
+                const long long v = v0 + lane + 32LL * i;
+                if (v < V) buf[i] = ld_stream_v4(src + v * 16);
+            }
+            for (uint32_t m = mask; m; m &= m - 1) {
+                const int pe = __ffs(m) - 1;
+                const int slot = __shfl_sync(kFull, my_slot, pe);
+                uint8_t* dst = p.recv_x + ((size_t)pe * p.maxRecv + slot) * p.rowBytes;
+#pragma unroll
+                for (int i = 0; i < kRegVec; ++i) {
+                    const long long v = v0 + lane + 32LL * i;
+                    if (v < V) st_v4(dst + v * 16, buf[i]);
+                }
+            }
+        }
+    }
 }
 
 // =====================================================================
@@ -487,22 +573,47 @@ size_t scatter_smem_bytes(int warps, int stages, int chunkStride) {
     return head + (size_t)warps * stages * (size_t)chunkStride;
 }
 
-cudaError_t scatter_set_smem(size_t bytes) {
-    return cudaFuncSetAttribute(ep_scatter_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)bytes);
+namespace {
+template <typename F>
+cudaError_t for_pend(int pend, F&& f) {
+    switch (pend) {
+        case 1: return f(ep_scatter_rows_kernel<1>);
+        case 2: return f(ep_scatter_rows_kernel<2>);
+        case 3: return f(ep_scatter_rows_kernel<3>);
+        default: return cudaErrorInvalidValue;
+    }
+}
+}  // namespace
+
+cudaError_t scatter_set_smem(int pend, size_t bytes) {
+    return for_pend(pend, [&](auto k) {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    });
 }
 
-cudaError_t scatter_blocks_per_sm(int warps, size_t smem, int* out) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_scatter_rows_kernel, warps * 32, smem);
+cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out) {
+    if (mode == kScatterRegs)
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_scatter_rows_regs_kernel, warps * 32, 0);
+    return for_pend(pend, [&](auto k) {
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, warps * 32, smem);
+    });
 }
 
 cudaError_t combine_blocks_per_sm(int warps, int* out) {
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_combine_kernel, warps * 32, 0);
 }
 
-cudaError_t launch_scatter_rows(const ScatterParams& p, int blocks, int warps, size_t smem,
-                                cudaStream_t s) {
-    ep_scatter_rows_kernel<<<blocks, warps * 32, smem, s>>>(p);
+cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
+                                size_t smem, cudaStream_t s) {
+    if (mode == kScatterRegs) {
+        ep_scatter_rows_regs_kernel<<<blocks, warps * 32, 0, s>>>(p);
+        return cudaGetLastError();
+    }
+    cudaError_t e = for_pend(pend, [&](auto k) {
+        k<<<blocks, warps * 32, smem, s>>>(p);
+        return cudaSuccess;
+    });
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

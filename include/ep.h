@@ -83,6 +83,8 @@ typedef struct EpPlanInfo {
     int32_t combineWarps;     /* warps per combine block */
     int32_t device;           /* CUDA device the plan lives on (-1 from ep_plan_query) */
     int32_t numSMs;           /* SMs of that device (0 from ep_plan_query) */
+    int32_t scatterMode;      /* 0: TMA bulk copies staged in shared memory; 1: register copies */
+    int32_t scatterPend;      /* TMA mode: bulk-store groups left draining when a stage refills */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
@@ -126,7 +128,8 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * ticket, the error word). Returns NULL on failure (ep_last_error() says why).
  * Environment overrides, read here only (for geometry sweeps):
  * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK,
- * EP_COMBINE_BLOCKS, EP_COMBINE_WARPS. */
+ * EP_SCATTER_PEND (1..3), EP_SCATTER_MODE ("tma" or "regs"), EP_COMBINE_BLOCKS,
+ * EP_COMBINE_WARPS. */
 EpPlan* ep_plan_create(const EpCfg* cfg);
 
 /* Free the plan and its scratch. NULL is a no-op. The caller must make sure no

@@ -155,6 +155,10 @@ def test_graph_capture_replay():
     {"EP_SCATTER_WARPS": "1", "EP_SCATTER_BLOCKS": "1"},   # one copy engine does everything
     {"EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2", "EP_SCATTER_CHUNK": "1024"},
     {"EP_COMBINE_WARPS": "1", "EP_COMBINE_BLOCKS": "3"},
+    {"EP_SCATTER_PEND": "2", "EP_SCATTER_STAGES": "4"},
+    {"EP_SCATTER_PEND": "3", "EP_SCATTER_STAGES": "4", "EP_SCATTER_CHUNK": "4096"},
+    {"EP_SCATTER_MODE": "regs"},
+    {"EP_SCATTER_MODE": "regs", "EP_SCATTER_WARPS": "2", "EP_SCATTER_BLOCKS": "5"},
 ])
 def test_geometry_overrides(env, monkeypatch):
     for k_, v in env.items():
