@@ -22,7 +22,8 @@ EP_ERR_STATE, EP_ERR_ALIGN, EP_ERR_DEVICE = -5, -6, -7
 EP_DEVERR_EXPERT_RANGE, EP_DEVERR_TIMEOUT, EP_DEVERR_CAPACITY = 1, 2, 4
 
 EXPORTED = ("ep_cfg_check", "ep_plan_query", "ep_plan_create", "ep_plan_destroy", "ep_plan_info",
-            "ep_dispatch", "ep_combine", "ep_plan_check_error", "ep_last_error")
+            "ep_dispatch", "ep_combine", "ep_plan_check_error", "ep_last_error", "ep_dispatch_noalloc")
+EP_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
 class EpCfg(ctypes.Structure):
@@ -71,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "ep_combine": ([P, P, P, P], I32),
         "ep_plan_check_error": ([P], I32),
         "ep_last_error": ([], ctypes.c_char_p),
+        "ep_dispatch_noalloc": ([cfgp, P, P, P, P, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -149,6 +151,15 @@ def ep_dispatch(plan: int, x, topk_idx, topk_w, recv_x, recv_meta, recv_count, s
 
 def ep_combine(plan: int, y, out, stream=None) -> int:
     return _check(_lib.ep_combine(plan, _addr(y), _addr(out), _stream(stream)), "ep_combine")
+
+
+def ep_dispatch_noalloc(cfg, x, topk_idx, topk_w, recv_x, recv_meta, recv_count, stream=None) -> int:
+    """Plan-free dispatch whose scratch is a fixed device array (no allocation);
+    see include/ep.h for its limit and its sharing rules."""
+    return _check(_lib.ep_dispatch_noalloc(ctypes.byref(_cfg(cfg)), _addr(x), _addr(topk_idx),
+                                           _addr(topk_w), _addr(recv_x), _addr(recv_meta),
+                                           _addr(recv_count), _stream(stream)),
+                  "ep_dispatch_noalloc")
 
 
 def ep_plan_check_error(plan: int) -> int:

@@ -181,6 +181,10 @@ void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
 
 }  // namespace
 
+namespace ep {
+void set_last_error(const char* msg) { std::snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+}  // namespace ep
+
 extern "C" {
 
 const char* ep_last_error(void) { return g_last_error; }

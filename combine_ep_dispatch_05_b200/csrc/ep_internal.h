@@ -73,5 +73,9 @@ cudaError_t scatter_set_smem(int pend, size_t bytes);
 // Blocks of each kernel that fit on one SM (occupancy calculator).
 cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out);
 cudaError_t combine_blocks_per_sm(int warps, int* out);
+// Current dynamic shared-memory limit of the TMA scatter kernel.
+cudaError_t scatter_get_smem(int pend, int* bytes);
+// Replace this thread's ep_last_error() text.
+void set_last_error(const char* msg);
 
 }  // namespace ep

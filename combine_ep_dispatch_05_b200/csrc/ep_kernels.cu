@@ -591,6 +591,15 @@ cudaError_t scatter_set_smem(int pend, size_t bytes) {
     });
 }
 
+cudaError_t scatter_get_smem(int pend, int* bytes) {
+    return for_pend(pend, [&](auto k) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, k);
+        *bytes = fa.maxDynamicSharedSizeBytes;
+        return e;
+    });
+}
+
 cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out) {
     if (mode == kScatterRegs)
         return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_scatter_rows_regs_kernel, warps * 32, 0);

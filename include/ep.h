@@ -181,6 +181,43 @@ int ep_plan_check_error(EpPlan* plan);
 /* Reason for the last failure on this thread ("" if none). */
 const char* ep_last_error(void);
 
+/* Bytes of device scratch that ep_dispatch_noalloc has on each device. */
+#define EP_NOALLOC_SCRATCH_BYTES (4 * 1024 * 1024)
+
+/*
+ * ep_dispatch_noalloc -- dispatch without a plan and without allocating.
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot allocate device memory where they dispatch: a serving loop whose
+ * memory pool must not grow, code running inside an allocator or driver
+ * callback (allocating there would re-enter the allocator), or an embedder
+ * whose runtime owns every device allocation.
+ *
+ * Same arguments, layouts and results as ep_dispatch (it runs the same
+ * kernels), with the configuration passed directly instead of a plan. It
+ * calls no cudaMalloc, cudaFree or other allocating routine: its scratch (the
+ * routing table, per-tile counts and bases, tile ticket, error word) is one
+ * file-scope __device__ array of EP_NOALLOC_SCRATCH_BYTES bytes, which every
+ * device that loads the library holds until the process exits.
+ *   - Limit: the configuration's scratch (about W*W*maxTokPerRank*8 bytes for
+ *     the routing table plus the tile tables) must fit the array; larger
+ *     configurations return EP_ERR_INVALID with the sizes in ep_last_error().
+ *   - The first call on a device looks up the array's device address and the
+ *     device limits (a one-time set-up, with that device current); make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; each call clears what must start at zero (tile ticket, error
+ *     word) on `stream`. Calls whose executions overlap on the GPU (other
+ *     streams, other host threads) race on the array and give wrong results:
+ *     serialise them.
+ *   - The routing table it leaves is not a plan's, so ep_combine cannot follow
+ *     it; device-side contract violations (ids >= E) are masked but not
+ *     reported (there is no plan error word to read).
+ * Returns EP_OK or a negative code (reason in ep_last_error()).
+ */
+int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_t* topk_idx,
+                        const float* topk_w, void* recv_x, int32_t* recv_meta,
+                        int32_t* recv_count, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
