@@ -24,9 +24,13 @@ struct EpPlan {
     int G;            // W*T
     void* scratch;    // one allocation, carved below
     int2* route;      // [G][W]
+    uint32_t* tok_mask;  // [G]
     int32_t* tile_cnt;
     int32_t* tile_base;
     uint32_t* ticket;
+    int32_t* work;
+    int32_t* cwork;
+    uint32_t* cdone;
     int32_t* err;
     size_t scatterSmem;
     bool dispatched;
@@ -48,8 +52,6 @@ int cuda_fail(cudaError_t e, const char* what) {
     return fail(e == cudaErrorMemoryAllocation ? EP_ERR_NOMEM : EP_ERR_CUDA, "%s: %s (%s)", what,
                 cudaGetErrorName(e), cudaGetErrorString(e));
 }
-
-size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 
 int env_int(const char* name, int dflt) {
     const char* v = std::getenv(name);
@@ -167,9 +169,7 @@ void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
     info->recvMetaBytes = (long long)c->worldSize * maxRecv * M * 4;
     info->countTile = ep::kCountTile;
     info->numTiles = (int)((G + ep::kCountTile - 1) / ep::kCountTile);
-    info->scratchBytes = (long long)(align256(sizeof(int2) * G * c->worldSize) +
-                                     2 * align256(sizeof(int32_t) * (size_t)info->numTiles * c->worldSize) +
-                                     align256(sizeof(uint32_t)) + align256(sizeof(int32_t)));
+    info->scratchBytes = (long long)ep::scratch_layout(G, c->worldSize, info->numTiles).total;
     info->scatterWarps = geo.scatterWarps;
     info->scatterStages = geo.scatterStages;
     info->scatterChunkBytes = geo.chunkBytes;
@@ -282,10 +282,8 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
         plan->maxRecv = plan->info.maxRecv;
 
-        const int W = cfg->worldSize;
-        const size_t nRoute = align256(sizeof(int2) * (size_t)plan->G * W);
-        const size_t nTiles = align256(sizeof(int32_t) * (size_t)plan->info.numTiles * W);
-        const size_t total = (size_t)plan->info.scratchBytes;
+        const ep::ScratchLayout L = ep::scratch_layout(plan->G, cfg->worldSize, plan->info.numTiles);
+        const size_t total = L.total;
         if ((e = cudaMalloc(&plan->scratch, total)) != cudaSuccess) {
             cuda_fail(e, "cudaMalloc(plan scratch)");
             plan->scratch = nullptr;
@@ -298,11 +296,15 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             return nullptr;
         }
         char* base = static_cast<char*>(plan->scratch);
-        plan->route = reinterpret_cast<int2*>(base);
-        plan->tile_cnt = reinterpret_cast<int32_t*>(base + nRoute);
-        plan->tile_base = reinterpret_cast<int32_t*>(base + nRoute + nTiles);
-        plan->ticket = reinterpret_cast<uint32_t*>(base + nRoute + 2 * nTiles);
-        plan->err = reinterpret_cast<int32_t*>(base + nRoute + 2 * nTiles + 256);
+        plan->route = reinterpret_cast<int2*>(base + L.route);
+        plan->tok_mask = reinterpret_cast<uint32_t*>(base + L.tok_mask);
+        plan->tile_cnt = reinterpret_cast<int32_t*>(base + L.tile_cnt);
+        plan->tile_base = reinterpret_cast<int32_t*>(base + L.tile_base);
+        plan->ticket = reinterpret_cast<uint32_t*>(base + L.ticket);
+        plan->work = reinterpret_cast<int32_t*>(base + L.work);
+        plan->cwork = reinterpret_cast<int32_t*>(base + L.cwork);
+        plan->cdone = reinterpret_cast<uint32_t*>(base + L.cdone);
+        plan->err = reinterpret_cast<int32_t*>(base + L.err);
         plan->dispatched = false;
         g_last_error[0] = '\0';
         return plan;
@@ -358,10 +360,12 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
         rp.idx = topk_idx;
         rp.w = c.useWeights ? topk_w : nullptr;
         rp.route = plan->route;
+        rp.tok_mask = plan->tok_mask;
         rp.tile_cnt = plan->tile_cnt;
         rp.tile_base = plan->tile_base;
         rp.recv_count = recv_count;
         rp.ticket = plan->ticket;
+        rp.work = plan->work;
         rp.err = plan->err;
         rp.G = plan->G;
         rp.W = c.worldSize;
@@ -378,7 +382,9 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
         sp.x = static_cast<const uint8_t*>(x);
         sp.idx = topk_idx;
         sp.route = plan->route;
+        sp.tok_mask = plan->tok_mask;
         sp.tile_base = plan->tile_base;
+        sp.work = plan->work;
         sp.recv_x = static_cast<uint8_t*>(recv_x);
         sp.recv_meta = recv_meta;
         sp.err = plan->err;
@@ -418,6 +424,8 @@ int ep_combine(EpPlan* plan, const void* y, void* out, void* stream) {
         cp.y = static_cast<const uint8_t*>(y);
         cp.route = plan->route;
         cp.out = static_cast<uint8_t*>(out);
+        cp.work = plan->cwork;
+        cp.done = plan->cdone;
         cp.rowBytes = plan->info.rowBytes;
         cp.G = plan->G;
         cp.W = plan->cfg.worldSize;

@@ -23,10 +23,12 @@ struct RouteParams {
     const int32_t* idx;     // [G][k]
     const float* w;         // [G][k] or nullptr (useWeights == 0)
     int2* route;            // [G][W]: (tile-local rank or -1, weight-sum bits)
+    uint32_t* tok_mask;     // [G]: destination mask of each token
     int32_t* tile_cnt;      // [numTiles][W]
     int32_t* tile_base;     // [numTiles][W], written by the last block
     int32_t* recv_count;    // [W]
     uint32_t* ticket;       // blocks finished this call; the last block resets it
+    int32_t* work;          // scatter token counter; the last block resets it
     int32_t* err;           // device error word
     int G, W, k, nEpr, E, numTiles, maxRecv, useWeights;
 };
@@ -35,7 +37,9 @@ struct ScatterParams {
     const uint8_t* x;          // [G][rowBytes]
     const int32_t* idx;        // [G][k]
     int2* route;               // [G][W]: in: tile-local rank; out: slot
+    const uint32_t* tok_mask;  // [G]: destination mask of each token
     const int32_t* tile_base;  // [numTiles][W]
+    int32_t* work;             // next token to hand out (starts at 0 each call)
     uint8_t* recv_x;           // [W][maxRecv][rowBytes]
     int32_t* recv_meta;        // [W][maxRecv][M]
     int32_t* err;
@@ -51,9 +55,35 @@ struct CombineParams {
     const uint8_t* y;      // [W][maxRecv][rowBytes]
     const int2* route;     // [G][W]: (slot or -1, weight bits)
     uint8_t* out;          // [G][rowBytes]
+    int32_t* work;         // next token to hand out (0 at the start of each call)
+    uint32_t* done;        // blocks finished; the last one resets work and done
     long long rowBytes;
     int G, W, maxRecv;
 };
+
+// Byte offsets of the dispatch scratch regions (each 256-byte aligned):
+// routing table, token masks, tile counts, tile bases, the counters (one
+// 256-byte region: tile ticket, scatter token counter, combine token counter,
+// combine blocks done), error word.
+struct ScratchLayout {
+    size_t route, tok_mask, tile_cnt, tile_base, ticket, work, cwork, cdone, err, total;
+};
+
+inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
+    auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
+    ScratchLayout L;
+    L.route = 0;
+    L.tok_mask = L.route + up(sizeof(int2) * (size_t)G * W);
+    L.tile_cnt = L.tok_mask + up(sizeof(uint32_t) * (size_t)G);
+    L.tile_base = L.tile_cnt + up(sizeof(int32_t) * (size_t)numTiles * W);
+    L.ticket = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * W);
+    L.work = L.ticket + 4;
+    L.cwork = L.ticket + 8;
+    L.cdone = L.ticket + 12;
+    L.err = L.ticket + 256;
+    L.total = L.err + 256;
+    return L;
+}
 
 // Launchers (ep_kernels.cu). Each returns the cudaError_t of its launch.
 cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s);

@@ -175,6 +175,8 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     }
     __syncthreads();
 
+    if (g < p.G) p.tok_mask[g] = mask;
+
     // Tile-local rank of this token at each destination, and its weight sum.
     const uint32_t lt = lanemask_lt();
 #pragma unroll
@@ -218,7 +220,10 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
             if (running > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
         }
     }
-    if (tid == 0) *p.ticket = 0u;  // ready for the next call (graph replay too)
+    if (tid == 0) {  // ready for the scatter and for the next call (graph replay too)
+        *p.work = 0;
+        *p.ticket = 0u;
+    }
 }
 
 // =====================================================================
@@ -282,9 +287,9 @@ __device__ __forceinline__ uint32_t token_slots_and_meta(const ScatterParams& p,
 
 // =====================================================================
 // scatter_rows (TMA): persistent copy engines, one per warp.
-// Items are (present token, chunk) pairs of this engine's tokens
-// g = engine, engine + nEngines, ...; an S-stage ring keeps S - kPend loads
-// ahead and lets kPend items' bulk stores drain while the next load starts.
+// Items are (present token, chunk) pairs of the tokens this engine is handed
+// by a global counter; an S-stage ring keeps S - kPend loads ahead and lets
+// kPend items' bulk stores drain while the next load starts.
 // =====================================================================
 template <int kPend>
 __device__ __forceinline__ void bulk_wait_read_pend() {
@@ -314,21 +319,43 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     }
     __syncwarp();
 
-    const int W = p.W;
-    const int nEngines = gridDim.x * nwarps;
-    const int engine = blockIdx.x * nwarps + warp;
 
-    // Producer: next present token of this engine at or after g.
-    auto next_present = [&](int g) -> int {
-        for (; g < p.G; g += nEngines) {
-            const int lr = lane < W ? p.route[(size_t)g * W + lane].x : -1;
-            if (__ballot_sync(kFull, lr >= 0) != 0u) return g;
+    // Producer (lane 0): tokens are handed out one at a time by a global
+    // counter, so that engines finish together whatever each token's fan-out.
+    // Two candidates are kept in flight ahead (the counter's answer and then
+    // the token's destination mask), so the hand-out costs no latency on the
+    // copy path.
+    int tA = p.G, tB = p.G, tC = p.G;  // candidates, in the order handed out
+    uint32_t mA = 0, mB = 0;           // masks of A and B
+    if (lane == 0) {
+        tA = atomicAdd(p.work, 1);
+        tB = atomicAdd(p.work, 1);
+        mA = tA < p.G ? __ldcg(p.tok_mask + tA) : 0u;
+        tC = atomicAdd(p.work, 1);
+        mB = tB < p.G ? __ldcg(p.tok_mask + tB) : 0u;
+    }
+    auto next_present = [&]() -> int {
+        int found = p.G;
+        if (lane == 0) {
+            while (tA < p.G) {
+                const int t = tA;
+                const uint32_t m = mA;
+                tA = tB;
+                mA = mB;
+                tB = tC;
+                mB = tC < p.G ? __ldcg(p.tok_mask + tC) : 0u;
+                tC = tC < p.G ? atomicAdd(p.work, 1) : p.G;
+                if (m != 0u) {
+                    found = t;
+                    break;
+                }
+            }
         }
-        return p.G;
+        return __shfl_sync(kFull, found, 0);
     };
 
-    int pg = next_present(engine);  // producer token
-    int pc = 0;                     // producer chunk
+    int pg = next_present();  // producer token
+    int pc = 0;               // producer chunk
     int issued = 0, consumed = 0;
     bool ok = true;
 
@@ -347,7 +374,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
         ++issued;
         if (++pc == p.numChunks) {
             pc = 0;
-            pg = next_present(pg + nEngines);
+            pg = next_present();
         }
     };
 
@@ -494,16 +521,27 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(Combi
     __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
     __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nw = gridDim.x * (blockDim.x >> 5);
     const int V = (int)(p.rowBytes / 16);
     const int W = p.W;
 
-    for (int g = blockIdx.x * (blockDim.x >> 5) + warp; g < p.G; g += nw) {
-        const int2 rr = lane < W ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
+    // Tokens are handed out one at a time by a global counter (their cost
+    // grows with the number of destinations, so a static split would leave a
+    // tail); the next token and its routing row are fetched one token ahead.
+    int next = 0;
+    if (lane == 0) next = atomicAdd(p.work, 1);
+    int g = __shfl_sync(kFull, next, 0);
+    int2 rr_next = (g < p.G && lane < W) ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
+    while (g < p.G) {
+        const int2 rr = rr_next;
+        if (lane == 0) next = atomicAdd(p.work, 1);
+        const int g_next = __shfl_sync(kFull, next, 0);
+        rr_next = (g_next < p.G && lane < W) ? p.route[(size_t)g_next * W + lane] : make_int2(-1, 0);
+
         const uint32_t mask = __ballot_sync(kFull, rr.x >= 0);
         uint4* orow = reinterpret_cast<uint4*>(p.out + (size_t)g * p.rowBytes);
         if (mask == 0u) {
             for (int v = lane; v < V; v += 32) orow[v] = make_uint4(0, 0, 0, 0);
+            g = g_next;
             continue;
         }
         // Present destinations in ascending order: rank of this lane's bit.
@@ -551,6 +589,18 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(Combi
             }
         }
         __syncwarp();
+        g = g_next;
+    }
+
+    // The last block to finish resets the counter for the next combine.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+            *p.work = 0;
+            *p.done = 0u;
+            __threadfence();
+        }
     }
 }
 

@@ -53,8 +53,6 @@ int noalloc_fail(int code, const char* fmt, ...) {
     return code;
 }
 
-size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
-
 // Once per device, with that device current: the device address of the
 // scratch array (the host-side symbol is only a stand-in for it) and the
 // device limits the launch geometry needs.
@@ -100,14 +98,13 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         if ((rc = ep_plan_query(cfg, &info)) != EP_OK) return noalloc_fail(rc, "%s", ep_last_error());
         const int W = cfg->worldSize;
         const long long G = (long long)W * cfg->maxTokPerRank;
-        const size_t nRoute = round256(sizeof(int2) * (size_t)G * W);
-        const size_t nTiles = round256(sizeof(int32_t) * (size_t)info.numTiles * W);
-        const size_t need = nRoute + 2 * nTiles + 256 + 256;
+        const ep::ScratchLayout L = ep::scratch_layout(G, W, info.numTiles);
+        const size_t need = L.total;
         if (need > (size_t)EP_NOALLOC_SCRATCH_BYTES)
             return noalloc_fail(EP_ERR_INVALID,
                                 "configuration needs %zu bytes of scratch; ep_dispatch_noalloc has %d "
-                                "(worldSize^2 * maxTokPerRank * 8 bytes must stay under about %d)",
-                                need, (int)EP_NOALLOC_SCRATCH_BYTES, (int)EP_NOALLOC_SCRATCH_BYTES);
+                                "(the routing table alone is worldSize^2 * maxTokPerRank * 8 bytes)",
+                                need, (int)EP_NOALLOC_SCRATCH_BYTES);
 
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
@@ -116,15 +113,17 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         if ((rc = setup_device(dev, &ds)) != EP_OK) return rc;
 
         unsigned char* base = ds.scratch;
-        int2* route = reinterpret_cast<int2*>(base);
-        int32_t* tile_cnt = reinterpret_cast<int32_t*>(base + nRoute);
-        int32_t* tile_base = reinterpret_cast<int32_t*>(base + nRoute + nTiles);
-        uint32_t* ticket = reinterpret_cast<uint32_t*>(base + nRoute + 2 * nTiles);
-        int32_t* err = reinterpret_cast<int32_t*>(base + nRoute + 2 * nTiles + 256);
+        int2* route = reinterpret_cast<int2*>(base + L.route);
+        uint32_t* tok_mask = reinterpret_cast<uint32_t*>(base + L.tok_mask);
+        int32_t* tile_cnt = reinterpret_cast<int32_t*>(base + L.tile_cnt);
+        int32_t* tile_base = reinterpret_cast<int32_t*>(base + L.tile_base);
+        uint32_t* ticket = reinterpret_cast<uint32_t*>(base + L.ticket);
+        int32_t* work = reinterpret_cast<int32_t*>(base + L.work);
+        int32_t* err = reinterpret_cast<int32_t*>(base + L.err);
         cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-        // The scratch keeps whatever the previous call left: the tile ticket
-        // and the error word must start at zero.
+        // The scratch keeps whatever the previous call left: the tile ticket,
+        // the scatter's token counter and the error word must start at zero.
         if ((e = cudaMemsetAsync(ticket, 0, 512, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
 
@@ -153,10 +152,12 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         rp.idx = topk_idx;
         rp.w = cfg->useWeights ? topk_w : nullptr;
         rp.route = route;
+        rp.tok_mask = tok_mask;
         rp.tile_cnt = tile_cnt;
         rp.tile_base = tile_base;
         rp.recv_count = recv_count;
         rp.ticket = ticket;
+        rp.work = work;
         rp.err = err;
         rp.G = (int)G;
         rp.W = W;
@@ -173,7 +174,9 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         sp.x = static_cast<const uint8_t*>(x);
         sp.idx = topk_idx;
         sp.route = route;
+        sp.tok_mask = tok_mask;
         sp.tile_base = tile_base;
+        sp.work = work;
         sp.recv_x = static_cast<uint8_t*>(recv_x);
         sp.recv_meta = recv_meta;
         sp.err = err;

@@ -166,6 +166,9 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
  * Combine, enqueued on `stream`, using the routing of the most recent
  * ep_dispatch of this plan (stream order is the caller's: issue it on the same
  * stream, or order the streams). No host synchronisation, no allocation.
+ * A combine may be repeated on the same routing (e.g. for several expert
+ * outputs). Calls on one plan share its scratch, so the executions of a
+ * plan's dispatches and combines must not overlap on the GPU.
  *   y    bf16 [W][maxRecv][h]   expert outputs in the receive layout, 16-byte
  *                               aligned; only rows < recv_count are read
  *   out  bf16 [W][T][h]         16-byte aligned; every row is written

@@ -119,6 +119,24 @@ def test_repeated_calls_and_reset():
         assert run.error_word() == 0
 
 
+def test_combine_repeated_on_one_routing():
+    """Several combines after one dispatch (e.g. for several expert outputs):
+    each follows the same routing; the token counter resets between calls."""
+    wl = workload("pr599").replace(h=1024)
+    cfg = wl.cfg()
+    inputs = make_inputs(wl)
+    run, ref = run_and_compare(cfg, inputs)
+    rng = np.random.default_rng(3)
+    for _ in range(3):
+        y = rng.integers(0, 1 << 16, size=(wl.W, wl.max_recv, wl.h)).astype(np.uint16)
+        y = np.where((y & 0x7F80) == 0x7F80, y & 0x807F, y).astype(np.uint16)
+        run.combine(y=to_dev(y.view(np.int16)))
+        torch.cuda.synchronize()
+        compare_combine(run, oracle.combine(cfg, y, ref["slotmap"], ref["wsum"]))
+    assert run.error_word() == 0
+    run.close()
+
+
 def test_graph_capture_replay():
     """dispatch -> identity expert -> combine captured as one CUDA graph and
     replayed: every replay reproduces eager bit for bit (MORI JIT v2 design
