@@ -114,6 +114,45 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
 }
 
 // =====================================================================
+// Token hand-out shared by the scatter engines and the combine warps. Worker w
+// of nU takes tokens w, w + nU, ... for R rounds (no coordination), then the
+// rest, about the last eighth of the tokens, one at a time from a global
+// counter, so that workers whose tokens had more destinations do not leave a
+// tail (the spread of a worker's total over ~100 tokens is a few percent).
+// With fewer than two tokens per worker the split is static only (no counter
+// traffic at all).
+// =====================================================================
+struct TokenSource {
+    int w, nU, R, G, i;
+    bool dyn;
+    int32_t* ctr;
+};
+
+__device__ __forceinline__ TokenSource make_source(int w, int nU, int G, int32_t* ctr) {
+    TokenSource s;
+    s.w = w;
+    s.nU = nU;
+    s.G = G;
+    s.i = 0;
+    s.ctr = ctr;
+    s.dyn = G >= 2 * nU;
+    s.R = s.dyn ? max(0, (int)((7LL * G) / (8LL * nU)) - 1) : (G + nU - 1) / nU;
+    return s;
+}
+
+// Next token of this worker, or G when it has none left.
+__device__ __forceinline__ int source_next(TokenSource& s) {
+    if (s.i < s.R) {
+        const int t = s.w + (s.i++) * s.nU;
+        if (t < s.G) return t;
+        s.i = s.R;
+    }
+    if (!s.dyn) return s.G;
+    const int t = s.R * s.nU + atomicAdd(s.ctr, 1);
+    return t < s.G ? t : s.G;
+}
+
+// =====================================================================
 // route_count: mask, weight sums, tile histogram, tile-local ranks; the last
 // block scans the histogram. kW = compile-time bound on W (8, 16 or 32).
 // =====================================================================
@@ -320,18 +359,18 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     __syncwarp();
 
 
-    // Producer (lane 0): tokens are handed out one at a time by a global
-    // counter, so that engines finish together whatever each token's fan-out.
-    // Two candidates are kept in flight ahead (the counter's answer and then
-    // the token's destination mask), so the hand-out costs no latency on the
-    // copy path.
+    // Producer (lane 0): tokens come from the shared hand-out (static rounds,
+    // then a global counter). Two candidates are kept in flight ahead (the
+    // hand-out's answer and then the token's destination mask), so finding the
+    // next present token costs no latency on the copy path.
+    TokenSource src = make_source(blockIdx.x * nwarps + warp, gridDim.x * nwarps, p.G, p.work);
     int tA = p.G, tB = p.G, tC = p.G;  // candidates, in the order handed out
     uint32_t mA = 0, mB = 0;           // masks of A and B
     if (lane == 0) {
-        tA = atomicAdd(p.work, 1);
-        tB = atomicAdd(p.work, 1);
+        tA = source_next(src);
+        tB = source_next(src);
         mA = tA < p.G ? __ldcg(p.tok_mask + tA) : 0u;
-        tC = atomicAdd(p.work, 1);
+        tC = source_next(src);
         mB = tB < p.G ? __ldcg(p.tok_mask + tB) : 0u;
     }
     auto next_present = [&]() -> int {
@@ -344,7 +383,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
                 mA = mB;
                 tB = tC;
                 mB = tC < p.G ? __ldcg(p.tok_mask + tC) : 0u;
-                tC = tC < p.G ? atomicAdd(p.work, 1) : p.G;
+                tC = tC < p.G ? source_next(src) : p.G;
                 if (m != 0u) {
                     found = t;
                     break;
@@ -524,16 +563,18 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(Combi
     const int V = (int)(p.rowBytes / 16);
     const int W = p.W;
 
-    // Tokens are handed out one at a time by a global counter (their cost
-    // grows with the number of destinations, so a static split would leave a
-    // tail); the next token and its routing row are fetched one token ahead.
+    // Tokens come from the shared hand-out (a token's cost grows with its
+    // number of destinations, so a purely static split would leave a tail);
+    // the next token and its routing row are fetched one token ahead.
+    TokenSource src = make_source(blockIdx.x * (blockDim.x >> 5) + warp, gridDim.x * (blockDim.x >> 5),
+                                  p.G, p.work);
     int next = 0;
-    if (lane == 0) next = atomicAdd(p.work, 1);
+    if (lane == 0) next = source_next(src);
     int g = __shfl_sync(kFull, next, 0);
     int2 rr_next = (g < p.G && lane < W) ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
     while (g < p.G) {
         const int2 rr = rr_next;
-        if (lane == 0) next = atomicAdd(p.work, 1);
+        if (lane == 0) next = source_next(src);
         const int g_next = __shfl_sync(kFull, next, 0);
         rr_next = (g_next < p.G && lane < W) ? p.route[(size_t)g_next * W + lane] : make_int2(-1, 0);
 
