@@ -6,8 +6,9 @@ ep_combine over W=8 virtual EP ranks on one B200, through the C ABI.
 
 Prints one JSON line (rank 0). Timing: W untimed warm-up steps, then K steps,
 each bracketed by CUDA events on the launching stream (dispatch and combine
-separately); a 256 MB buffer is rewritten between steps outside the events
-(L2 flush; the main workload's inputs are larger than L2 as well). Barrier +
+separately); L2 is flushed between steps outside the events by reading a
+256 MB buffer (``--flush write`` rewrites it instead; the main workload's
+inputs are larger than L2 as well). Barrier +
 synchronize on both sides; the reported time is the max over ranks. N > 1
 runs N independent replicas, one per GPU (each GPU holds all W virtual ranks).
 
@@ -50,6 +51,9 @@ def parse():
     ap.add_argument("--workload", default="main")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--flush", default="read", choices=["read", "write"],
+                    help="L2 flush between timed steps: read a 256 MB buffer (leaves L2 clean) "
+                         "or write it (leaves L2 full of dirty lines)")
     return ap.parse_args()
 
 
@@ -65,7 +69,8 @@ def describe(wl) -> dict:
             "world_size": wl.W, "tokens_per_rank": wl.ct, "max_tok_per_rank": wl.max_tok,
             "hidden": wl.h, "topk": wl.k, "experts": wl.E, "max_recv": wl.max_recv,
             "use_weights": wl.use_weights,
-            "l2": "256 MB buffer rewritten between steps outside the events; inputs larger than L2"}
+            "l2": "L2 flushed between steps outside the events (256 MB buffer, see flush); "
+                  "inputs larger than L2"}
 
 
 def dispatch_bytes(wl, U, n_routed):
@@ -272,15 +277,22 @@ def run_ours(args, wl):
     recv_meta = torch.empty((W, R, 3 + k), dtype=torch.int32, device=dev)
     recv_count = torch.empty((W,), dtype=torch.int32, device=dev)
     out = torch.empty((W, T, h), dtype=torch.int16, device=dev)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_out = torch.empty(1, dtype=torch.int32, device=dev)
     s = torch.cuda.current_stream(dev)
+
+    def flush_l2(i):
+        if args.flush == "write":
+            flush.fill_(i)
+        else:  # read it: evicts L2 and leaves only clean lines behind
+            torch.amax(flush, dim=0, out=flush_out.view(()))
 
     def step():
         ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, s)
         ep.ep_combine(plan, recv_x, out, s)  # identity expert: y = recv_x
 
     for i in range(max(args.warmup, 0)):
-        flush.fill_(i)
+        flush_l2(i)
         step()
     torch.cuda.synchronize(dev)
     err = ep.ep_plan_check_error(plan)
@@ -295,7 +307,7 @@ def run_ours(args, wl):
     sampler.start()
     t_wall = time.perf_counter()
     for i in range(args.steps):
-        flush.fill_(i + 1)
+        flush_l2(i + 1)
         evs[i][0].record(s)
         ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, s)
         evs[i][1].record(s)
@@ -334,39 +346,68 @@ def run_ours(args, wl):
     traffic = ncu_traffic("ep_combine_kernel" if dom["kernel"] == "ep_combine_kernel" else "ep_scatter_rows_kernel",
                           wl.name)
 
-    # End to end: pinned host inputs -> device, both calls, result -> pinned host.
+    # End to end: every step copies its inputs from pinned host memory to the
+    # device, runs dispatch and combine, and copies its result back to pinned
+    # host memory. Steps are double-buffered on three streams (host->device,
+    # compute, device->host) so that one step's upload overlaps the previous
+    # step's download, as a serving loop would run them.
     e2e = None
     if not args.no_e2e:
         x_h = torch.from_numpy(inputs["x"].view(np.int16)).pin_memory()
         idx_h = torch.from_numpy(inputs["topk_idx"]).pin_memory()
         w_h = torch.from_numpy(inputs["topk_w"]).pin_memory() if w is not None else None
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        xs, idxs, ws = [x, torch.empty_like(x)], [idx, torch.empty_like(idx)], [w, None if w is None else torch.empty_like(w)]
+        outs = [out, torch.empty_like(out)]
+        s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_free = [torch.cuda.Event() for _ in range(2)]    # compute finished with input set b
+        in_ready = [torch.cuda.Event() for _ in range(2)]   # upload of input set b finished
+        out_ready = [torch.cuda.Event() for _ in range(2)]  # combine wrote out set b
+        out_free = [torch.cuda.Event() for _ in range(2)]   # download of out set b finished
+        for b in range(2):
+            in_free[b].record(s)
+            out_free[b].record(s)
 
-        def e2e_step():
-            x.copy_(x_h, non_blocking=True)
-            idx.copy_(idx_h, non_blocking=True)
-            if w is not None:
-                w.copy_(w_h, non_blocking=True)
-            step()
-            out_h.copy_(out, non_blocking=True)
+        def e2e_step(i):
+            b = i & 1
+            with torch.cuda.stream(s_up):
+                s_up.wait_event(in_free[b])
+                xs[b].copy_(x_h, non_blocking=True)
+                idxs[b].copy_(idx_h, non_blocking=True)
+                if w_h is not None:
+                    ws[b].copy_(w_h, non_blocking=True)
+                in_ready[b].record(s_up)
+            s.wait_event(in_ready[b])
+            ep.ep_dispatch(plan, xs[b], idxs[b], ws[b], recv_x, recv_meta, recv_count, s)
+            in_free[b].record(s)
+            s.wait_event(out_free[b])
+            ep.ep_combine(plan, recv_x, outs[b], s)
+            out_ready[b].record(s)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(out_ready[b])
+                out_h[b].copy_(outs[b], non_blocking=True)
+                out_free[b].record(s_down)
 
-        for _ in range(max(1, min(args.warmup, 3))):
-            e2e_step()
+        for i in range(max(1, min(args.warmup, 3))):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         if dist is not None:
             dist.barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        n_e2e = max(1, min(args.steps, 10))
-        e0.record(s)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(s)
+        n_e2e = max(2, min(args.steps, 10))
+        e0.record(s_up)
+        for i in range(n_e2e):
+            e2e_step(i)
+        e1.record(s_down)  # after the last download, which follows everything else
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
+        # the result of the last step is the device result, byte for byte
+        assert torch.equal(out_h[(n_e2e - 1) & 1], outs[(n_e2e - 1) & 1].cpu())
         h2d = x_h.numel() * 2 + idx_h.numel() * 4 + (w_h.numel() * 4 if w_h is not None else 0)
         e2e = {"value": e2e_ms * 1e3, "unit": "us", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(out_h.numel() * 2), "steps": n_e2e}
+               "d2h_bytes_per_step": int(out_h[0].numel() * 2), "steps": n_e2e,
+               "pipeline": "double-buffered: upload of step i overlaps download of step i-1"}
 
     ep.ep_plan_destroy(plan)
 
@@ -385,7 +426,8 @@ def run_ours(args, wl):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {**describe(wl), "parallelism": "virtual EP ranks on each GPU; replicas across GPUs"},
+            "config": {**describe(wl), "flush": args.flush,
+                       "parallelism": "virtual EP ranks on each GPU; replicas across GPUs"},
             "dispatch_us": disp_ms_max * 1e3, "combine_us": comb_ms_max * 1e3,
             "dispatch_gbs": d_gbs, "combine_gbs": c_gbs, "pair_gbs": pair_gbs,
             "pair_frac_of_peak": pair_gbs / peak, "recv_rows_U": U,
