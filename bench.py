@@ -343,8 +343,7 @@ def run_ours(args, wl):
     else:
         dom = {"kernel": "ep_dispatch (route_count + scatter_rows)", "bytes": db, "ms": disp_ms_max,
                "gbs": d_gbs}
-    traffic = ncu_traffic("ep_combine_kernel" if dom["kernel"] == "ep_combine_kernel" else "ep_scatter_rows_kernel",
-                          wl.name)
+    traffic = ncu_traffic("ep_combine_kernel" if dom["kernel"] == "ep_combine_kernel" else "ep_dispatch", wl.name)
 
     # End to end: every step copies its inputs from pinned host memory to the
     # device, runs dispatch and combine, and copies its result back to pinned
