@@ -1,0 +1,77 @@
+"""The bench's multi-process host logic on CPU: two gloo ranks.
+
+With N GPUs the bench runs N replicas (each GPU holds all W virtual ranks). The
+host side of that path is the rank setup from the launcher's environment and
+the max-over-ranks reduction of the timings; the reference arm runs on rank 0
+only. These need no GPU and run here with the gloo backend.
+"""
+import json
+import os
+import socket
+import sys
+from datetime import timedelta
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import bench
+        r, w, local, d = bench.dist_setup(world)
+        got = bench.max_over_ranks(1.5 * (rank + 1), d, "cpu")
+        q.put((rank, r, w, local, got))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_max_over_ranks():
+    import torch.multiprocessing as tmp
+    ctx = tmp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [o[0] for o in out] == [0, 1]
+    for rank, r, w, local, got in out:
+        assert (r, w, local) == (rank, 2, rank)
+        assert got == pytest.approx(3.0)  # every rank sees the slowest rank's time
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    import argparse
+
+    import bench
+    wl = bench.get_workload("tiny")
+    args = argparse.Namespace(gpus=2, steps=1, warmup=0, impl="reference", workload="tiny")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    assert bench.run_reference(args, wl) == 0
+    assert capsys.readouterr().out == ""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("LOCAL_RANK", "0")
+    assert bench.run_reference(args, wl) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "us" and line["higher_is_better"] is False
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
