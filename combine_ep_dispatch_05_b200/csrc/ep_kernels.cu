@@ -105,6 +105,14 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of the stream finishes;
+// pdl_wait() blocks until that kernel has completed and its writes are
+// visible (a no-op without the launch attribute). pdl_trigger() lets the next
+// kernel of the stream start its launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     uint4 v;
     asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -161,6 +169,9 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     __shared__ int s_wcnt[kCountWarps][kW];
     __shared__ int s_wpre[kCountWarps][kW];
     __shared__ int s_last;
+
+    pdl_wait();     // the ids may come from the previous kernel of the stream
+    pdl_trigger();  // let the scatter's launch and prologue overlap this kernel
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = blockIdx.x * kCountTile + tid;
@@ -357,7 +368,8 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
         mbar_fence_init();
     }
     __syncwarp();
-
+    pdl_wait();     // routing written by route_count is visible from here on
+    pdl_trigger();
 
     // Producer (lane 0): tokens come from the shared hand-out (static rounds,
     // then a global counter). Two candidates are kept in flight ahead (the
@@ -499,6 +511,8 @@ __device__ __forceinline__ void st_v4(void* p, const uint4& v) {
 }
 
 __global__ void __launch_bounds__(256) ep_scatter_rows_regs_kernel(ScatterParams p) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int nw = gridDim.x * (blockDim.x >> 5);
     const long long V = p.rowBytes / 16;
@@ -559,6 +573,8 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* acc) {
 __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(CombineParams p) {
     __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
     __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
+    pdl_wait();  // y and the routing of the dispatch are visible from here on
+    pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int V = (int)(p.rowBytes / 16);
     const int W = p.W;
@@ -648,14 +664,33 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(Combi
 }  // namespace
 
 // ------------------------------------------------------------- launchers
+namespace {
+// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger).
+template <typename P>
+cudaError_t launch_pdl(void (*kernel)(P), int grid, int block, size_t smem, cudaStream_t s, const P& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+}  // namespace
+
 cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s) {
+    cudaError_t e;
     if (p.W <= 8)
-        ep_route_count_kernel<8><<<p.numTiles, kCountTile, 0, s>>>(p);
+        e = launch_pdl(ep_route_count_kernel<8>, p.numTiles, kCountTile, 0, s, p);
     else if (p.W <= 16)
-        ep_route_count_kernel<16><<<p.numTiles, kCountTile, 0, s>>>(p);
+        e = launch_pdl(ep_route_count_kernel<16>, p.numTiles, kCountTile, 0, s, p);
     else
-        ep_route_count_kernel<32><<<p.numTiles, kCountTile, 0, s>>>(p);
-    return cudaGetLastError();
+        e = launch_pdl(ep_route_count_kernel<32>, p.numTiles, kCountTile, 0, s, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride) {
@@ -706,19 +741,16 @@ cudaError_t combine_blocks_per_sm(int warps, int* out) {
 cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
                                 size_t smem, cudaStream_t s) {
     if (mode == kScatterRegs) {
-        ep_scatter_rows_regs_kernel<<<blocks, warps * 32, 0, s>>>(p);
-        return cudaGetLastError();
+        cudaError_t e = launch_pdl(ep_scatter_rows_regs_kernel, blocks, warps * 32, 0, s, p);
+        return e != cudaSuccess ? e : cudaGetLastError();
     }
-    cudaError_t e = for_pend(pend, [&](auto k) {
-        k<<<blocks, warps * 32, smem, s>>>(p);
-        return cudaSuccess;
-    });
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    cudaError_t e = for_pend(pend, [&](auto k) { return launch_pdl(k, blocks, warps * 32, smem, s, p); });
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_combine(const CombineParams& p, int blocks, int warps, cudaStream_t s) {
-    ep_combine_kernel<<<blocks, warps * 32, 0, s>>>(p);
+    cudaError_t e = launch_pdl(ep_combine_kernel, blocks, warps * 32, 0, s, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
