@@ -86,6 +86,26 @@ def recv_capacity(cfg: dict) -> int:
     return int(cfg["maxRecv"]) or int(cfg["worldSize"]) * int(cfg["maxTokPerRank"])
 
 
+# Payload dtypes (numbering of the design page's EpDType): the numpy type in
+# which tests hold one dispatched element, and its size in bytes.
+PAYLOAD_NP = {0: np.uint16, 1: np.float32, 2: np.uint8, 3: np.uint8}
+
+
+def payload_np(cfg: dict):
+    return PAYLOAD_NP[int(cfg["dtype"])]
+
+
+def combine_hidden(cfg: dict) -> int:
+    """Elements of a combine row: 2 * hiddenDim for fp4x2 (packed pairs)."""
+    h = int(cfg["hiddenDim"])
+    return 2 * h if int(cfg["dtype"]) == 3 else h
+
+
+def combine_np(cfg: dict):
+    """float32 for an fp32 plan; bf16 bits (uint16) otherwise."""
+    return np.float32 if int(cfg["dtype"]) == 1 else np.uint16
+
+
 def dispatch(cfg: dict, x: np.ndarray, topk_idx: np.ndarray, topk_w, recv_x=None, recv_meta=None,
              lib=None):
     """Run the oracle dispatch. Returns a dict with recv_x, recv_meta,
@@ -98,14 +118,16 @@ def dispatch(cfg: dict, x: np.ndarray, topk_idx: np.ndarray, topk_w, recv_x=None
     c = _cfg(cfg)
     W, T, h, k = c.worldSize, c.maxTokPerRank, c.hiddenDim, c.numExpertPerToken
     R = recv_capacity(cfg)
-    x = np.ascontiguousarray(x, dtype=np.uint16).reshape(W, T, h)
+    pt = payload_np(cfg)
+    x = np.ascontiguousarray(x).view(pt).reshape(W, T, h)
     idx = np.ascontiguousarray(topk_idx, dtype=np.int32).reshape(W, T, k)
     w = None if topk_w is None else np.ascontiguousarray(topk_w, dtype=np.float32).reshape(W, T, k)
     if recv_x is None:
-        recv_x = np.zeros((W, R, h), dtype=np.uint16)
+        recv_x = np.zeros((W, R, h), dtype=pt)
     if recv_meta is None:
         recv_meta = np.zeros((W, R, 3 + k), dtype=np.int32)
-    assert recv_x.shape == (W, R, h) and recv_x.dtype == np.uint16 and recv_x.flags.c_contiguous
+    recv_x = recv_x.view(pt)
+    assert recv_x.shape == (W, R, h) and recv_x.flags.c_contiguous
     assert recv_meta.shape == (W, R, 3 + k) and recv_meta.dtype == np.int32
     recv_count = np.zeros(W, dtype=np.int32)
     slotmap = np.empty((W, T, W), dtype=np.int32)
@@ -119,15 +141,18 @@ def dispatch(cfg: dict, x: np.ndarray, topk_idx: np.ndarray, topk_w, recv_x=None
 
 
 def combine(cfg: dict, y: np.ndarray, slotmap: np.ndarray, wsum: np.ndarray, lib=None) -> np.ndarray:
-    """Run the oracle combine; returns out as uint16 bf16 bits, shape (W, T, h)."""
+    """Run the oracle combine; returns out, shape (W, T, combine_hidden): bf16
+    bits (uint16), or float32 for an fp32 plan."""
     lib = lib or _load()
     c = _cfg(cfg)
-    W, T, h = c.worldSize, c.maxTokPerRank, c.hiddenDim
+    W, T = c.worldSize, c.maxTokPerRank
+    h = combine_hidden(cfg)
     R = recv_capacity(cfg)
-    y = np.ascontiguousarray(y, dtype=np.uint16).reshape(W, R, h)
+    ct = combine_np(cfg)
+    y = np.ascontiguousarray(y).view(ct).reshape(W, R, h)
     slotmap = np.ascontiguousarray(slotmap, dtype=np.int32).reshape(W, T, W)
     wsum = np.ascontiguousarray(wsum, dtype=np.float32).reshape(W, T, W)
-    out = np.empty((W, T, h), dtype=np.uint16)
+    out = np.empty((W, T, h), dtype=ct)
     rc = lib.oracle_combine(ctypes.byref(c), _ptr(y), _ptr(slotmap), _ptr(wsum), _ptr(out))
     if rc < 0:
         raise ValueError(f"oracle_combine rejected its arguments (rc={rc})")

@@ -37,6 +37,15 @@
  *     acc = fmaf(w(r,t,pe), y[pe][slot], acc) ), acc0 = +0.0f; a token with an
  *     empty P gets a zero row.
  *   - Receive rows and meta past recv_count[pe] are not written.
+ *   - Payload dtype (design page §3.7: the dtype is a property of the
+ *     transport; dispatch never computes on elements): bf16 2 bytes, fp32 4,
+ *     fp8 1, fp4x2 1 byte per element, where an fp4x2 element is a packed pair
+ *     of e2m1 values and hiddenDim counts bytes. Dispatch copies rows of
+ *     hiddenDim * size bytes. The combine leg reduces, so it takes no byte
+ *     type: it is float32 (in and out, no final rounding) for an fp32 plan and
+ *     bfloat16 otherwise, with hiddenDim elements, or 2 * hiddenDim for fp4x2
+ *     (the unpacked element count) -- the pages pair fp8/fp4 dispatch with a
+ *     bf16 combine.
  *
  * Floating point: the pages fix float32 accumulation with bfloat16 output, so
  * the oracle computes in float32 with one fused multiply-add per term (C99
@@ -91,13 +100,27 @@ static uint16_t f32_to_bf16_rne(float f)
     return (uint16_t)upper;
 }
 
+enum { DT_BF16 = 0, DT_FP32 = 1, DT_FP8 = 2, DT_FP4X2 = 3 };
+
 static int cfg_ok(const OracleCfg *c)
 {
     if (!c) return 0;
     if (c->worldSize <= 0 || c->hiddenDim <= 0 || c->maxTokPerRank <= 0) return 0;
     if (c->numExpertPerRank <= 0 || c->numExpertPerToken <= 0) return 0;
-    if (c->dtype != 0) return 0; /* bf16 only */
+    if (c->dtype < DT_BF16 || c->dtype > DT_FP4X2) return 0;
     return 1;
+}
+
+/* Bytes of one dispatched element. */
+static int64_t payload_size(const OracleCfg *c)
+{
+    return c->dtype == DT_FP32 ? 4 : c->dtype == DT_BF16 ? 2 : 1;
+}
+
+/* Elements of one combine row. */
+static int64_t combine_hidden(const OracleCfg *c)
+{
+    return c->dtype == DT_FP4X2 ? 2 * (int64_t)c->hiddenDim : c->hiddenDim;
 }
 
 static int64_t recv_cap(const OracleCfg *c)
@@ -111,11 +134,11 @@ int oracle_recv_capacity(const OracleCfg *c)
 }
 
 /*
- * Dispatch. Shapes (all row-major, C order):
- *   x          uint16 [W][T][h]          bf16 bits
+ * Dispatch. Shapes (all row-major, C order); a row is h * payload_size bytes:
+ *   x          bytes  [W][T][row]        the payload, moved bit for bit
  *   topk_idx   int32  [W][T][k]
  *   topk_w     float  [W][T][k]          may be NULL when useWeights == 0
- *   recv_x     uint16 [W][R][h]          R = maxRecv (or W*T)
+ *   recv_x     bytes  [W][R][row]        R = maxRecv (or W*T)
  *   recv_meta  int32  [W][R][3+k]
  *   recv_count int32  [W]
  *   slotmap    int32  [W][T][W]          slot of (r,t) at pe, or -1
@@ -123,8 +146,8 @@ int oracle_recv_capacity(const OracleCfg *c)
  * Returns 0, ORACLE_STATUS_EXPERT_RANGE when an id >= E was masked, or a
  * negative error.
  */
-int oracle_dispatch(const OracleCfg *c, const uint16_t *x, const int32_t *topk_idx,
-                    const float *topk_w, uint16_t *recv_x, int32_t *recv_meta,
+int oracle_dispatch(const OracleCfg *c, const uint8_t *x, const int32_t *topk_idx,
+                    const float *topk_w, uint8_t *recv_x, int32_t *recv_meta,
                     int32_t *recv_count, int32_t *slotmap, float *wsum)
 {
     if (!cfg_ok(c) || !x || !topk_idx || !recv_x || !recv_meta || !recv_count ||
@@ -132,7 +155,8 @@ int oracle_dispatch(const OracleCfg *c, const uint16_t *x, const int32_t *topk_i
         return ORACLE_ERR_ARG;
     if (c->useWeights && !topk_w) return ORACLE_ERR_ARG;
 
-    const int64_t W = c->worldSize, T = c->maxTokPerRank, h = c->hiddenDim;
+    const int64_t W = c->worldSize, T = c->maxTokPerRank;
+    const int64_t row = (int64_t)c->hiddenDim * payload_size(c);
     const int64_t nEpr = c->numExpertPerRank, k = c->numExpertPerToken;
     const int64_t E = W * nEpr, R = recv_cap(c), M = 3 + k;
     int status = ORACLE_OK;
@@ -165,7 +189,7 @@ int oracle_dispatch(const OracleCfg *c, const uint16_t *x, const int32_t *topk_i
                 }
                 if (next[pe] >= R) { free(next); return ORACLE_ERR_ARG; }
                 const int64_t slot = next[pe]++;
-                memcpy(recv_x + (pe * R + slot) * h, x + g * h, (size_t)h * sizeof(uint16_t));
+                memcpy(recv_x + (pe * R + slot) * row, x + g * row, (size_t)row);
                 int32_t *meta = recv_meta + (pe * R + slot) * M;
                 meta[0] = (int32_t)r;
                 meta[1] = (int32_t)t;
@@ -185,15 +209,21 @@ int oracle_dispatch(const OracleCfg *c, const uint16_t *x, const int32_t *topk_i
 }
 
 /*
- * Combine. y has recv_x's layout; slotmap and wsum are what oracle_dispatch
- * wrote; out is uint16 [W][T][h] bf16 bits.
+ * Combine. y is [W][R][hc] and out [W][T][hc], hc = combine_hidden: float32
+ * for an fp32 plan, bf16 bits (uint16) otherwise; slotmap and wsum are what
+ * oracle_dispatch wrote.
  */
-int oracle_combine(const OracleCfg *c, const uint16_t *y, const int32_t *slotmap,
-                   const float *wsum, uint16_t *out)
+int oracle_combine(const OracleCfg *c, const void *y_, const int32_t *slotmap,
+                   const float *wsum, void *out_)
 {
-    if (!cfg_ok(c) || !y || !slotmap || !wsum || !out) return ORACLE_ERR_ARG;
-    const int64_t W = c->worldSize, T = c->maxTokPerRank, h = c->hiddenDim;
+    if (!cfg_ok(c) || !y_ || !slotmap || !wsum || !out_) return ORACLE_ERR_ARG;
+    const int64_t W = c->worldSize, T = c->maxTokPerRank, h = combine_hidden(c);
     const int64_t R = recv_cap(c);
+    const int fp32 = c->dtype == DT_FP32;
+    const uint16_t *y = (const uint16_t *)y_;
+    const float *yf = (const float *)y_;
+    uint16_t *out = (uint16_t *)out_;
+    float *outf = (float *)out_;
     float *acc = (float *)malloc((size_t)h * sizeof *acc);
     if (!acc) return ORACLE_ERR_NOMEM;
 
@@ -203,10 +233,18 @@ int oracle_combine(const OracleCfg *c, const uint16_t *y, const int32_t *slotmap
             const int32_t slot = slotmap[g * W + pe];
             if (slot < 0) continue;
             const float w = wsum[g * W + pe];
-            const uint16_t *row = y + (pe * R + slot) * h;
-            for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, bf16_to_f32(row[i]), acc[i]);
+            if (fp32) {
+                const float *rowf = yf + (pe * R + slot) * h;
+                for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, rowf[i], acc[i]);
+            } else {
+                const uint16_t *row = y + (pe * R + slot) * h;
+                for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, bf16_to_f32(row[i]), acc[i]);
+            }
         }
-        for (int64_t i = 0; i < h; ++i) out[g * h + i] = f32_to_bf16_rne(acc[i]);
+        if (fp32)
+            for (int64_t i = 0; i < h; ++i) outf[g * h + i] = acc[i];
+        else
+            for (int64_t i = 0; i < h; ++i) out[g * h + i] = f32_to_bf16_rne(acc[i]);
     }
     free(acc);
     return ORACLE_OK;

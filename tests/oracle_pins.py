@@ -55,24 +55,35 @@ def torch_bf16_bits(f32):
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
-def random_small_case(rng, W=None):
+def random_payload(rng, shape, dtype):
+    """Random payload bits of a dispatch dtype (0 bf16, 1 fp32, 2 fp8, 3 fp4x2).
+    bf16 values stay finite and far from overflow (combine sums them); the
+    other payloads are arbitrary bit patterns (dispatch only moves them)."""
+    if dtype == 0:
+        xb = rng.integers(0, 1 << 16, size=shape).astype(np.uint16)
+        # exponents >= 2^113 lose their top exponent bit
+        return np.where((xb & 0x7F80) >= 0x7880, xb & 0xBFFF, xb).astype(np.uint16)
+    if dtype == 1:
+        return rng.integers(0, 1 << 32, size=shape, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    return rng.integers(0, 256, size=shape).astype(np.uint8)
+
+
+def random_small_case(rng, W=None, dtype=0):
     """A tiny random problem with masked entries, duplicate expert ids,
     occasional out-of-range-free ids and arbitrary-sign weights."""
     W = W or int(rng.integers(1, 6))
     T = int(rng.integers(1, 7))
     nEpr = int(rng.integers(1, 5))
     k = int(rng.integers(1, 6))
-    h = 8 * int(rng.integers(1, 4))
+    h = {0: 8, 1: 4, 2: 16, 3: 16}[dtype] * int(rng.integers(1, 4))  # rows of 16-byte multiples
     E = W * nEpr
     idx = rng.integers(-2, E, size=(W, T, k)).astype(np.int32)  # with replacement: duplicates
     w = rng.standard_normal((W, T, k)).astype(np.float32)
     use_w = int(rng.integers(0, 2))
     maxRecv = [0, W * T, W * T + 3][int(rng.integers(0, 3))]
-    xb = rng.integers(0, 1 << 16, size=(W, T, h)).astype(np.uint16)
-    # keep x finite and far from overflow: exponents >= 2^113 lose their top exponent bit
-    xb = np.where((xb & 0x7F80) >= 0x7880, xb & 0xBFFF, xb).astype(np.uint16)
+    xb = random_payload(rng, (W, T, h), dtype)
     cfg = dict(worldSize=W, hiddenDim=h, maxTokPerRank=T, numExpertPerRank=nEpr,
-               numExpertPerToken=k, maxRecv=maxRecv, dtype=0, useWeights=use_w)
+               numExpertPerToken=k, maxRecv=maxRecv, dtype=dtype, useWeights=use_w)
     return cfg, xb, idx, (w if use_w else None)
 
 
@@ -100,12 +111,13 @@ def brute_routes(cfg, idx):
 # ---------------------------------------------------------------- pins
 def pin_bruteforce_dispatch(lib=None, n_cases=40, seed=11):
     rng = np.random.default_rng(seed)
-    for _ in range(n_cases):
-        cfg, xb, idx, w = random_small_case(rng)
+    for case in range(n_cases):
+        cfg, xb, idx, w = random_small_case(rng, dtype=case % 4)
         W, T, k, nEpr, h = (cfg[n] for n in ("worldSize", "maxTokPerRank", "numExpertPerToken",
                                              "numExpertPerRank", "hiddenDim"))
         R = oracle.recv_capacity(cfg)
-        canary_x = np.full((W, R, h), 0xABCD, dtype=np.uint16)
+        row_bytes = xb[0, 0].nbytes
+        canary_x = np.full((W, R, row_bytes), 0xAB, dtype=np.uint8)
         canary_m = np.full((W, R, 3 + k), 0x5EADBEEF, dtype=np.int32)
         res = oracle.dispatch(cfg, xb, idx, w, recv_x=canary_x, recv_meta=canary_m, lib=lib)
         slot, count = brute_routes(cfg, idx)
@@ -118,7 +130,7 @@ def pin_bruteforce_dispatch(lib=None, n_cases=40, seed=11):
                     if s < 0:
                         assert res["wsum"][r, t, pe] == 0.0
                         continue
-                    assert np.array_equal(res["recv_x"][pe, s], xb[r, t])
+                    assert res["recv_x"][pe, s].tobytes() == xb[r, t].tobytes()  # bit for bit
                     meta = res["recv_meta"][pe, s]
                     assert meta[0] == r and meta[1] == t
                     # local expert ids: the position-j id, reduced modulo nEpr, where it lives on pe
@@ -142,7 +154,7 @@ def pin_bruteforce_dispatch(lib=None, n_cases=40, seed=11):
         # untouched past recv_count
         for pe in range(W):
             n = count[pe]
-            assert np.all(res["recv_x"][pe, n:] == 0xABCD)
+            assert np.all(res["recv_x"][pe, n:].view(np.uint8) == 0xAB)
             assert np.all(res["recv_meta"][pe, n:] == 0x5EADBEEF)
 
 
@@ -263,6 +275,51 @@ def pin_combine_single_rounding_case(lib=None):
     assert want == 1 + Fraction(1, 128)
     assert np.all(out[0, 0] == 0x3F81), out[0, 0]
     assert np.all(out[1, 0] == 0)
+
+
+def pin_combine_fp32_exact_fma(lib=None, seed=8):
+    """fp32 plan: combine is the float32 fold acc = RNE32(w*y + acc) over pe
+    ascending with no final rounding, evaluated here with exact rationals."""
+    rng = np.random.default_rng(seed)
+    cfg = dict(worldSize=3, hiddenDim=8, maxTokPerRank=5, numExpertPerRank=2,
+               numExpertPerToken=3, maxRecv=0, dtype=1, useWeights=1)
+    idx = rng.integers(-1, 6, size=(3, 5, 3)).astype(np.int32)
+    w = rng.standard_normal((3, 5, 3)).astype(np.float32)
+    x = rng.standard_normal((3, 5, 8)).astype(np.float32)
+    res = oracle.dispatch(cfg, x, idx, w, lib=lib)
+    y = (rng.standard_normal(res["recv_x"].shape) * np.exp2(rng.integers(-20, 20, size=res["recv_x"].shape))
+         ).astype(np.float32)
+    out = oracle.combine(cfg, y, res["slotmap"], res["wsum"], lib=lib)
+    assert out.dtype == np.float32 and out.shape == (3, 5, 8)
+    for r in range(3):
+        for t in range(5):
+            for i in range(8):
+                acc = Fraction(0)
+                for pe in range(3):
+                    s = int(res["slotmap"][r, t, pe])
+                    if s >= 0:
+                        acc = round_fraction_to_f32(Fraction(float(res["wsum"][r, t, pe])) *
+                                                    Fraction(float(y[pe, s, i])) + acc)
+                assert Fraction(float(out[r, t, i])) == acc, (r, t, i)
+
+
+def pin_fp4x2_combine_width(lib=None):
+    """fp4x2 plan: hiddenDim counts bytes of packed pairs; the bf16 combine leg
+    has 2 * hiddenDim elements per row. With one destination and weight 1 the
+    combine returns its input row, all 2 * hiddenDim elements of it."""
+    h = 16
+    cfg = dict(worldSize=2, hiddenDim=h, maxTokPerRank=2, numExpertPerRank=1,
+               numExpertPerToken=1, maxRecv=0, dtype=3, useWeights=0)
+    idx = np.array([[[1], [-1]], [[0], [1]]], dtype=np.int32)
+    x = np.arange(2 * 2 * h, dtype=np.uint8).reshape(2, 2, h)
+    res = oracle.dispatch(cfg, x, idx, None, lib=lib)
+    assert res["recv_x"].dtype == np.uint8 and res["recv_x"].shape[-1] == h
+    assert res["recv_x"][1, 0].tobytes() == x[0, 0].tobytes()
+    rng = np.random.default_rng(2)
+    y = torch_bf16_bits(rng.standard_normal((2, 4, 2 * h)).astype(np.float32))
+    out = oracle.combine(cfg, y, res["slotmap"], res["wsum"], lib=lib)
+    assert out.shape == (2, 2, 2 * h) and out.dtype == np.uint16
+    assert np.array_equal(out[0, 0], y[1, 0]) and np.all(out[0, 1] == 0)
 
 
 def pin_combine_fp64_bound(lib=None, seed=7):
@@ -498,6 +555,8 @@ ALL_PINS = [
     pin_bruteforce_weight_sum_order,
     pin_combine_exact_fma,
     pin_combine_single_rounding_case,
+    pin_combine_fp32_exact_fma,
+    pin_fp4x2_combine_width,
     pin_combine_fp64_bound,
     pin_roundtrip_unweighted_exact,
     pin_roundtrip_weighted,

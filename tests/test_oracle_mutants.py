@@ -36,6 +36,12 @@ MUTANTS = {
     "round_truncate": ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))",
                        "if (0)"),
     "bf16_widen_shift": ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = (uint32_t)b << 15;"),
+    "fp32_payload_two_bytes": ("return c->dtype == DT_FP32 ? 4 : c->dtype == DT_BF16 ? 2 : 1;",
+                               "return c->dtype == DT_FP32 ? 2 : c->dtype == DT_BF16 ? 2 : 1;"),
+    "fp4x2_combine_not_unpacked": ("return c->dtype == DT_FP4X2 ? 2 * (int64_t)c->hiddenDim : c->hiddenDim;",
+                                   "return c->hiddenDim;"),
+    "fp32_combine_rounded_to_bf16": ("for (int64_t i = 0; i < h; ++i) outf[g * h + i] = acc[i];",
+                                     "for (int64_t i = 0; i < h; ++i) outf[g * h + i] = bf16_to_f32(f32_to_bf16_rne(acc[i]));"),
     "count_not_stored": ("recv_count[pe] = (int32_t)next[pe];", "recv_count[pe] = (int32_t)next[pe] - (pe == 0);"),
 }
 
