@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="main")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp32", "fp8", "fp4x2"],
+                    help="dispatch payload type (the combine leg is fp32 for fp32, bf16 otherwise); "
+                         "fp4x2 halves hiddenDim, which then counts bytes of packed pairs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--flush", default="read", choices=["read", "write"],
@@ -57,10 +60,28 @@ def parse():
     return ap.parse_args()
 
 
-def get_workload(name):
+DTYPES = {"bf16": 0, "fp32": 1, "fp8": 2, "fp4x2": 3}
+
+
+def get_workload(name, dtype="bf16"):
     if name == "mid":  # the main shape at 1024 tokens/rank: the small ncu case
-        return workload("main").replace(name="mid", max_tok=1024, ct=1024, max_recv=8192)
-    return workload(name)
+        wl = workload("main").replace(name="mid", max_tok=1024, ct=1024, max_recv=8192)
+    else:
+        wl = workload(name)
+    dt = DTYPES[dtype]
+    if dt == 0:
+        return wl
+    # fp4x2: the same element count, in hiddenDim bytes of packed pairs
+    return wl.replace(name=f"{wl.name}_{dtype}", dtype=dt, h=wl.h // 2 if dt == 3 else wl.h)
+
+
+def payload_bytes(wl) -> int:
+    return wl.h * {0: 2, 1: 4, 2: 1, 3: 1}[wl.dtype]
+
+
+def combine_row_bytes(wl) -> int:
+    hc = 2 * wl.h if wl.dtype == 3 else wl.h
+    return hc * (4 if wl.dtype == 1 else 2)
 
 
 def describe(wl) -> dict:
@@ -69,12 +90,14 @@ def describe(wl) -> dict:
             "world_size": wl.W, "tokens_per_rank": wl.ct, "max_tok_per_rank": wl.max_tok,
             "hidden": wl.h, "topk": wl.k, "experts": wl.E, "max_recv": wl.max_recv,
             "use_weights": wl.use_weights,
+            "payload_dtype": {0: "bf16", 1: "fp32", 2: "fp8", 3: "fp4x2"}[wl.dtype],
+            "combine_dtype": "fp32" if wl.dtype == 1 else "bf16",
             "l2": "L2 flushed between steps outside the events (256 MB buffer, see flush); "
                   "inputs larger than L2"}
 
 
 def dispatch_bytes(wl, U, n_routed):
-    row, G, k, W = wl.h * 2, wl.W * wl.max_tok, wl.k, wl.W
+    row, G, k, W = payload_bytes(wl), wl.W * wl.max_tok, wl.k, wl.W
     return (n_routed * row                    # read each routed x row once
             + U * row                         # write every received row
             + G * k * 4 * (1 + int(wl.use_weights))  # topk ids (+ weights)
@@ -83,7 +106,7 @@ def dispatch_bytes(wl, U, n_routed):
 
 
 def combine_bytes(wl, U):
-    row, G = wl.h * 2, wl.W * wl.max_tok
+    row, G = combine_row_bytes(wl), wl.W * wl.max_tok
     return (U * row       # read every received row of y
             + G * row     # write every out row
             + U * 8)      # (slot, weight) of each received row
@@ -213,14 +236,19 @@ def time_oracle(wl, inputs, steps, scale=1.0):
     import oracle
     cfg = wl.cfg()
     R = oracle.recv_capacity(cfg)
-    recv_x = np.zeros((wl.W, R, wl.h), dtype=np.uint16)
+    recv_x = np.zeros((wl.W, R, wl.h), dtype=oracle.payload_np(cfg))
     recv_meta = np.zeros((wl.W, R, 3 + wl.k), dtype=np.int32)
     idx = inputs["topk_idx"]
+    y = None
+    if wl.dtype in (2, 3):  # one-byte payloads: the expert hands back bf16 rows
+        rng = np.random.default_rng(wl.seed)
+        y = rng.integers(0x3C00, 0x4000, size=(wl.W, R, oracle.combine_hidden(cfg)), dtype=np.uint16)
+        y |= (rng.integers(0, 2, size=y.shape, dtype=np.uint16) << 15)
     ts = []
     for _ in range(steps):
         t0 = time.perf_counter()
         r = oracle.dispatch(cfg, inputs["x"], idx, inputs["topk_w"], recv_x=recv_x, recv_meta=recv_meta)
-        oracle.combine(cfg, r["recv_x"], r["slotmap"], r["wsum"])
+        oracle.combine(cfg, r["recv_x"] if y is None else y, r["slotmap"], r["wsum"])
         ts.append((time.perf_counter() - t0) * scale)
     return ts
 
@@ -239,7 +267,8 @@ def run_reference(args, wl):
     cores = 1
     line = {"metric": METRIC, "value": us, "unit": "us", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": {0: "bf16", 1: "f32", 2: "fp8", 3: "fp4x2"}[wl.dtype], "data": "synthetic",
             "config": describe(wl), "impl": "reference",
             "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -270,13 +299,21 @@ def run_ours(args, wl):
     plan = ep.ep_plan_create(cfg)
     info = ep.ep_plan_info(plan)
     W, T, h, k, R = wl.W, wl.max_tok, wl.h, wl.k, info.maxRecv
-    x = torch.from_numpy(inputs["x"].view(np.int16)).to(dev)
+    x = torch.from_numpy(inputs["x"].view(np.uint8).reshape(W, T, -1)).to(dev)
     idx = torch.from_numpy(inputs["topk_idx"]).to(dev)
     w = torch.from_numpy(inputs["topk_w"]).to(dev) if inputs["topk_w"] is not None else None
-    recv_x = torch.empty((W, R, h), dtype=torch.int16, device=dev)
+    recv_x = torch.empty((W, R, info.rowBytes), dtype=torch.uint8, device=dev)
     recv_meta = torch.empty((W, R, 3 + k), dtype=torch.int32, device=dev)
     recv_count = torch.empty((W,), dtype=torch.int32, device=dev)
-    out = torch.empty((W, T, h), dtype=torch.int16, device=dev)
+    cdt = torch.float32 if wl.dtype == 1 else torch.bfloat16
+    out = torch.empty((W, T, info.combineHidden), dtype=cdt, device=dev)
+    if wl.dtype in (0, 1):
+        y = recv_x.view(cdt).view(W, R, info.combineHidden)  # identity expert: y = recv_x
+    else:
+        # one-byte payloads: the expert hands back bf16 rows (seeded, made on the device)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(wl.seed)
+        y = torch.randn((W, R, info.combineHidden), generator=gen, device=dev).to(cdt)
     flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     flush_out = torch.empty(1, dtype=torch.int32, device=dev)
     s = torch.cuda.current_stream(dev)
@@ -289,7 +326,7 @@ def run_ours(args, wl):
 
     def step():
         ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, s)
-        ep.ep_combine(plan, recv_x, out, s)  # identity expert: y = recv_x
+        ep.ep_combine(plan, y, out, s)
 
     for i in range(max(args.warmup, 0)):
         flush_l2(i)
@@ -311,7 +348,7 @@ def run_ours(args, wl):
         evs[i][0].record(s)
         ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, s)
         evs[i][1].record(s)
-        ep.ep_combine(plan, recv_x, out, s)
+        ep.ep_combine(plan, y, out, s)
         evs[i][2].record(s)
     torch.cuda.synchronize(dev)
     t_wall = time.perf_counter() - t_wall
@@ -352,7 +389,7 @@ def run_ours(args, wl):
     # step's download, as a serving loop would run them.
     e2e = None
     if not args.no_e2e:
-        x_h = torch.from_numpy(inputs["x"].view(np.int16)).pin_memory()
+        x_h = torch.from_numpy(inputs["x"].view(np.uint8).reshape(W, T, -1)).pin_memory()
         idx_h = torch.from_numpy(inputs["topk_idx"]).pin_memory()
         w_h = torch.from_numpy(inputs["topk_w"]).pin_memory() if w is not None else None
         out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
@@ -380,7 +417,7 @@ def run_ours(args, wl):
             ep.ep_dispatch(plan, xs[b], idxs[b], ws[b], recv_x, recv_meta, recv_count, s)
             in_free[b].record(s)
             s.wait_event(out_free[b])
-            ep.ep_combine(plan, recv_x, outs[b], s)
+            ep.ep_combine(plan, y, outs[b], s)
             out_ready[b].record(s)
             with torch.cuda.stream(s_down):
                 s_down.wait_event(out_ready[b])
@@ -403,15 +440,15 @@ def run_ours(args, wl):
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
         # the result of the last step is the device result, byte for byte
         assert torch.equal(out_h[(n_e2e - 1) & 1], outs[(n_e2e - 1) & 1].cpu())
-        h2d = x_h.numel() * 2 + idx_h.numel() * 4 + (w_h.numel() * 4 if w_h is not None else 0)
+        h2d = x_h.numel() + idx_h.numel() * 4 + (w_h.numel() * 4 if w_h is not None else 0)
         e2e = {"value": e2e_ms * 1e3, "unit": "us", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(out_h[0].numel() * 2), "steps": n_e2e,
+               "d2h_bytes_per_step": int(out_h[0].numel() * out_h[0].element_size()), "steps": n_e2e,
                "pipeline": "double-buffered: upload of step i overlaps download of step i-1"}
 
     ep.ep_plan_destroy(plan)
 
     cpu = None
-    if rank == 0 and args.gpus == 1 and not args.no_cpu_baseline:
+    if rank == 0 and args.gpus == 1 and not args.no_cpu_baseline and wl.dtype in (0, 1):
         import oracle
         oracle.build()
         steps_cpu = 2
@@ -423,7 +460,8 @@ def run_ours(args, wl):
         line = {
             "metric": METRIC, "value": step_ms * 1e3, "unit": "us", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": {0: "bf16", 1: "f32", 2: "fp8", 3: "fp4x2"}[wl.dtype],
             "data": "synthetic",
             "config": {**describe(wl), "flush": args.flush,
                        "parallelism": "virtual EP ranks on each GPU; replicas across GPUs"},
@@ -451,7 +489,7 @@ def run_ours(args, wl):
 
 def main():
     args = parse()
-    wl = get_workload(args.workload)
+    wl = get_workload(args.workload, args.dtype)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

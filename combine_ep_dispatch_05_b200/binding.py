@@ -43,7 +43,9 @@ class EpPlanInfo(ctypes.Structure):
                 ("scatterChunkBytes", ctypes.c_int32), ("combineBlocks", ctypes.c_int32),
                 ("combineWarps", ctypes.c_int32), ("device", ctypes.c_int32),
                 ("numSMs", ctypes.c_int32), ("scatterMode", ctypes.c_int32),
-                ("scatterPend", ctypes.c_int32)]
+                ("scatterPend", ctypes.c_int32), ("combineDtype", ctypes.c_int32),
+                ("combineHidden", ctypes.c_int32), ("combineRowBytes", ctypes.c_int64),
+                ("yBytes", ctypes.c_int64), ("outBytes", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}

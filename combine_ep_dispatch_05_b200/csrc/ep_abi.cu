@@ -61,6 +61,18 @@ int env_int(const char* name, int dflt) {
     return (end && *end == '\0' && x > 0 && x < (1 << 30)) ? (int)x : dflt;
 }
 
+// Bytes of one dispatched element (design page §3.7: the dtype is a property of
+// the transport; fp8 and fp4x2 are both one byte, fp4x2 holding a packed pair).
+int payload_size(int dtype) { return dtype == EP_FP32 ? 4 : dtype == EP_BF16 ? 2 : 1; }
+
+// The combine leg reduces, so it takes no byte type: float32 for an fp32 plan,
+// bf16 otherwise, with 2 * hiddenDim elements for fp4x2 (the unpacked count).
+int combine_dtype(int dtype) { return dtype == EP_FP32 ? EP_FP32 : EP_BF16; }
+long long combine_hidden(const EpCfg* c) { return c->dtype == EP_FP4X2 ? 2LL * c->hiddenDim : c->hiddenDim; }
+long long combine_row_bytes(const EpCfg* c) {
+    return combine_hidden(c) * (combine_dtype(c->dtype) == EP_FP32 ? 4 : 2);
+}
+
 // The validity rules of the design page §3.5 (EpCfgIsValid / MakeEpCfg) and
 // the dtype rule of §3.7, plus the int32 index range of this build.
 int check_cfg(const EpCfg* c) {
@@ -79,12 +91,11 @@ int check_cfg(const EpCfg* c) {
         return fail(EP_ERR_INVALID, "too many experts");
     if (c->useWeights != 0 && c->useWeights != 1)
         return fail(EP_ERR_INVALID, "useWeights must be 0 or 1, got %d", c->useWeights);
-    if (c->dtype == EP_FP32 || c->dtype == EP_FP8 || c->dtype == EP_FP4X2)
-        return fail(EP_ERR_UNSUPPORTED, "dtype %d is not built (bf16 payloads only)", c->dtype);
-    if (c->dtype != EP_BF16) return fail(EP_ERR_INVALID, "unknown dtype %d", c->dtype);
-    const long long rowBytes = (long long)c->hiddenDim * 2;
+    if (c->dtype < EP_BF16 || c->dtype > EP_FP4X2) return fail(EP_ERR_INVALID, "unknown dtype %d", c->dtype);
+    const long long rowBytes = (long long)c->hiddenDim * payload_size(c->dtype);
     if (rowBytes % 16 != 0)
-        return fail(EP_ERR_INVALID, "token bytes %lld (hiddenDim*2) not a multiple of 16", rowBytes);
+        return fail(EP_ERR_INVALID, "token bytes %lld (hiddenDim * %d) not a multiple of 16", rowBytes,
+                    payload_size(c->dtype));
     const long long G = (long long)c->worldSize * c->maxTokPerRank;
     if (G > (1LL << 30)) return fail(EP_ERR_INVALID, "worldSize*maxTokPerRank too large");
     if (c->maxRecv < 0) return fail(EP_ERR_INVALID, "maxRecv %d < 0", c->maxRecv);
@@ -111,7 +122,7 @@ struct Geometry {
 // lookahead) and 1 x 12 (one issuing thread per SM is too few).
 Geometry pick_geometry(const EpCfg* c, bool use_env) {
     Geometry g{};
-    const long long rowBytes = (long long)c->hiddenDim * 2;
+    const long long rowBytes = (long long)c->hiddenDim * payload_size(c->dtype);
     int chunk;
     if (rowBytes <= 32768) {
         chunk = (int)rowBytes;
@@ -163,9 +174,14 @@ void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
     const int M = 3 + c->numExpertPerToken;
     info->maxRecv = maxRecv;
     info->metaFields = M;
-    info->rowBytes = (long long)c->hiddenDim * 2;
+    info->rowBytes = (long long)c->hiddenDim * payload_size(c->dtype);
     info->tokenBytes = G * info->rowBytes;
     info->recvXBytes = (long long)c->worldSize * maxRecv * info->rowBytes;
+    info->combineDtype = combine_dtype(c->dtype);
+    info->combineHidden = (int32_t)combine_hidden(c);
+    info->combineRowBytes = combine_row_bytes(c);
+    info->yBytes = (long long)c->worldSize * maxRecv * info->combineRowBytes;
+    info->outBytes = G * info->combineRowBytes;
     info->recvMetaBytes = (long long)c->worldSize * maxRecv * M * 4;
     info->countTile = ep::kCountTile;
     info->numTiles = (int)((G + ep::kCountTile - 1) / ep::kCountTile);
@@ -257,7 +273,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         int sPerSm = 0, cPerSm = 0;
         if ((e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps, smem,
                                            &sPerSm)) != cudaSuccess ||
-            (e = ep::combine_blocks_per_sm(geo.combineWarps, &cPerSm)) != cudaSuccess) {
+            (e = ep::combine_blocks_per_sm(geo.combineWarps, cfg->dtype == EP_FP32, &cPerSm)) != cudaSuccess) {
             cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
             return nullptr;
         }
@@ -426,12 +442,12 @@ int ep_combine(EpPlan* plan, const void* y, void* out, void* stream) {
         cp.out = static_cast<uint8_t*>(out);
         cp.work = plan->cwork;
         cp.done = plan->cdone;
-        cp.rowBytes = plan->info.rowBytes;
+        cp.rowBytes = plan->info.combineRowBytes;
         cp.G = plan->G;
         cp.W = plan->cfg.worldSize;
         cp.maxRecv = plan->maxRecv;
-        cudaError_t e = ep::launch_combine(cp, plan->info.combineBlocks, plan->info.combineWarps,
-                                           static_cast<cudaStream_t>(stream));
+        cudaError_t e = ep::launch_combine(cp, plan->info.combineDtype == EP_FP32, plan->info.combineBlocks,
+                                           plan->info.combineWarps, static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_fail(e, "launch combine");
         return EP_OK;
     } catch (...) {

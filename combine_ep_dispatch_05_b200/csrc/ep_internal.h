@@ -57,7 +57,7 @@ struct CombineParams {
     uint8_t* out;          // [G][rowBytes]
     int32_t* work;         // next token to hand out (0 at the start of each call)
     uint32_t* done;        // blocks finished; the last one resets work and done
-    long long rowBytes;
+    long long rowBytes;    // bytes of a y / out row (the combine leg's row)
     int G, W, maxRecv;
 };
 
@@ -94,7 +94,8 @@ constexpr int kScatterTma = 0;
 constexpr int kScatterRegs = 1;
 cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
                                 size_t smem, cudaStream_t s);
-cudaError_t launch_combine(const CombineParams& p, int blocks, int warps, cudaStream_t s);
+// fp32: float32 combine leg (an fp32 plan); bf16 otherwise.
+cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s);
 
 // Shared-memory bytes the scatter kernel needs for a geometry.
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride);
@@ -102,7 +103,7 @@ size_t scatter_smem_bytes(int warps, int stages, int chunkStride);
 cudaError_t scatter_set_smem(int pend, size_t bytes);
 // Blocks of each kernel that fit on one SM (occupancy calculator).
 cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out);
-cudaError_t combine_blocks_per_sm(int warps, int* out);
+cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out);
 // Current dynamic shared-memory limit of the TMA scatter kernel.
 cudaError_t scatter_get_smem(int pend, int* bytes);
 // Replace this thread's ep_last_error() text.

@@ -17,7 +17,8 @@
 //                design page §9 and PR #599) are the prior art.
 // combine = combine (one launch)
 //   combine      one warp per token: up to 8 destination rows in flight per
-//                16-byte column, float32 fma fold in destPe order, bf16 RNE out.
+//                16-byte column, float32 fma fold in destPe order; bf16 RNE out
+//                (float32 out, unrounded, for a float32 plan).
 //
 // No kernel traps or spins without a bound: waits on shared-memory barriers
 // give up after kWaitCycles, set EP_DEVERR_TIMEOUT and drain their copies.
@@ -570,6 +571,29 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* acc) {
     return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
+// Element types of the combine leg: bf16 in and out (float32 fold, RNE at the
+// end), or float32 in and out (float32 fold, no final rounding).
+struct CombineBf16 {
+    static constexpr int kPer = 8;  // elements per 16-byte vector
+    static __device__ __forceinline__ void fma(float* acc, float w, const uint4& v) { fma_bf16x8(acc, w, v); }
+    static __device__ __forceinline__ uint4 pack(const float* acc) { return pack_bf16x8(acc); }
+};
+
+struct CombineF32 {
+    static constexpr int kPer = 4;
+    static __device__ __forceinline__ void fma(float* acc, float w, const uint4& v) {
+        acc[0] = __fmaf_rn(w, __uint_as_float(v.x), acc[0]);
+        acc[1] = __fmaf_rn(w, __uint_as_float(v.y), acc[1]);
+        acc[2] = __fmaf_rn(w, __uint_as_float(v.z), acc[2]);
+        acc[3] = __fmaf_rn(w, __uint_as_float(v.w), acc[3]);
+    }
+    static __device__ __forceinline__ uint4 pack(const float* acc) {
+        return make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                          __float_as_uint(acc[3]));
+    }
+};
+
+template <class Elem>
 __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(CombineParams p) {
     __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
     __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
@@ -611,11 +635,11 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(Combi
         __syncwarp();
 
         for (int v0 = lane; v0 < V; v0 += 32 * kCombineUnroll) {
-            float acc[kCombineUnroll][8];
+            float acc[kCombineUnroll][Elem::kPer];
 #pragma unroll
             for (int u = 0; u < kCombineUnroll; ++u)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+                for (int i = 0; i < Elem::kPer; ++i) acc[u][i] = 0.0f;
             for (int b = 0; b < n; b += kCombineBatch) {
                 uint4 val[kCombineUnroll][kCombineBatch];
 #pragma unroll
@@ -635,14 +659,14 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(Combi
                         const float w = s_w[warp][b + i];
 #pragma unroll
                         for (int u = 0; u < kCombineUnroll; ++u)
-                            if (v0 + 32 * u < V) fma_bf16x8(acc[u], w, val[u][i]);
+                            if (v0 + 32 * u < V) Elem::fma(acc[u], w, val[u][i]);
                     }
                 }
             }
 #pragma unroll
             for (int u = 0; u < kCombineUnroll; ++u) {
                 const int v = v0 + 32 * u;
-                if (v < V) orow[v] = pack_bf16x8(acc[u]);
+                if (v < V) orow[v] = Elem::pack(acc[u]);
             }
         }
         __syncwarp();
@@ -734,8 +758,10 @@ cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, in
     });
 }
 
-cudaError_t combine_blocks_per_sm(int warps, int* out) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_combine_kernel, warps * 32, 0);
+cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out) {
+    if (fp32)
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_combine_kernel<CombineF32>, warps * 32, 0);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_combine_kernel<CombineBf16>, warps * 32, 0);
 }
 
 cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
@@ -748,8 +774,9 @@ cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int 
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_combine(const CombineParams& p, int blocks, int warps, cudaStream_t s) {
-    cudaError_t e = launch_pdl(ep_combine_kernel, blocks, warps * 32, 0, s, p);
+cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s) {
+    cudaError_t e = fp32 ? launch_pdl(ep_combine_kernel<CombineF32>, blocks, warps * 32, 0, s, p)
+                         : launch_pdl(ep_combine_kernel<CombineBf16>, blocks, warps * 32, 0, s, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

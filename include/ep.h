@@ -47,20 +47,26 @@
 extern "C" {
 #endif
 
-/* Payload dtype tags, numbered as the design page's EpDType (§3.7). This build
- * accepts EP_BF16 only; the others are rejected by ep_cfg_check. */
+/* Payload dtype tags, numbered as the design page's EpDType (§3.7). The dtype is
+ * a property of the transport: dispatch moves hiddenDim elements per row bit for
+ * bit and never computes on them (bf16 2 bytes, fp32 4, fp8 1, fp4x2 1 byte
+ * holding a packed pair of e2m1 values, so hiddenDim counts bytes). The combine
+ * leg reduces, so it takes no byte type: it is float32 (in and out, no final
+ * rounding) for an EP_FP32 plan and bfloat16 otherwise, with hiddenDim
+ * elements per row, or 2 * hiddenDim for EP_FP4X2 (the unpacked count) -- the
+ * pages pair fp8/fp4 dispatch with a bf16 combine. */
 typedef enum EpDType { EP_BF16 = 0, EP_FP32 = 1, EP_FP8 = 2, EP_FP4X2 = 3 } EpDType;
 
 /* The semantic fields of the design page's EpCfg (§3.2). Launch geometry is
  * not part of it: the library picks it from the device. */
 typedef struct EpCfg {
     int32_t worldSize;         /* W: virtual EP ranks, 1..32 */
-    int32_t hiddenDim;         /* h: elements per token row; h*2 must be a multiple of 16 */
+    int32_t hiddenDim;         /* h: payload elements per token row; its bytes must be a multiple of 16 */
     int32_t maxTokPerRank;     /* T: token rows per source rank, >= 1 */
     int32_t numExpertPerRank;  /* experts on each rank, >= 1; E = W*numExpertPerRank */
     int32_t numExpertPerToken; /* k (topk), 1..32 */
     int32_t maxRecv;           /* receive rows per destination; 0 means W*T; must be >= W*T */
-    int32_t dtype;             /* EpDType; EP_BF16 only */
+    int32_t dtype;             /* EpDType of the dispatch payload (see above) */
     int32_t useWeights;        /* 1: combine weights by the topk weights; 0: weight 1 */
 } EpCfg;
 
@@ -68,9 +74,9 @@ typedef struct EpCfg {
 typedef struct EpPlanInfo {
     int32_t maxRecv;          /* resolved receive capacity per destination */
     int32_t metaFields;       /* int32 fields per meta record: 3 + k */
-    int64_t rowBytes;         /* h * 2 */
-    int64_t tokenBytes;       /* bytes of x and of out: W*T*rowBytes */
-    int64_t recvXBytes;       /* bytes of recv_x and of y: W*maxRecv*rowBytes */
+    int64_t rowBytes;         /* bytes of a dispatched row: h * element size */
+    int64_t tokenBytes;       /* bytes of x: W*T*rowBytes */
+    int64_t recvXBytes;       /* bytes of recv_x: W*maxRecv*rowBytes */
     int64_t recvMetaBytes;    /* W*maxRecv*metaFields*4 */
     int64_t scratchBytes;     /* device scratch the plan owns */
     int32_t countTile;        /* tokens per routing tile */
@@ -85,6 +91,11 @@ typedef struct EpPlanInfo {
     int32_t numSMs;           /* SMs of that device (0 from ep_plan_query) */
     int32_t scatterMode;      /* 0: TMA bulk copies staged in shared memory; 1: register copies */
     int32_t scatterPend;      /* TMA mode: bulk-store groups left draining when a stage refills */
+    int32_t combineDtype;     /* EP_FP32 for an fp32 plan, else EP_BF16 */
+    int32_t combineHidden;    /* elements of a y / out row: h, or 2*h for EP_FP4X2 */
+    int64_t combineRowBytes;  /* bytes of a y / out row */
+    int64_t yBytes;           /* bytes of y: W*maxRecv*combineRowBytes */
+    int64_t outBytes;         /* bytes of out: W*T*combineRowBytes */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
@@ -93,7 +104,7 @@ typedef struct EpPlan EpPlan;
 enum {
     EP_OK = 0,
     EP_ERR_INVALID = -1,     /* bad argument or configuration */
-    EP_ERR_UNSUPPORTED = -2, /* valid for the pages, not built here (dtype) */
+    EP_ERR_UNSUPPORTED = -2, /* valid for the pages, not built here */
     EP_ERR_NOMEM = -3,       /* device allocation failed */
     EP_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
     EP_ERR_STATE = -5,       /* combine before any dispatch on this plan */
@@ -113,7 +124,7 @@ enum {
  * EP_ERR_INVALID / EP_ERR_UNSUPPORTED with the reason in ep_last_error().
  * Rules (design page §3.5, EpCfgIsValid): the row bytes must be a multiple of
  * 16; topk and worldSize must fit one 32-lane warp; the receive capacity must
- * cover the worst case (maxRecv >= W*T); only bf16 payloads (§3.7). */
+ * cover the worst case (maxRecv >= W*T); dtype one of EpDType (§3.7). */
 int ep_cfg_check(const EpCfg* cfg);
 
 /* Host-only sizing: fill *info for cfg as a plan on a generic device would
@@ -143,10 +154,10 @@ int ep_plan_info(const EpPlan* plan, EpPlanInfo* info);
  * Dispatch, enqueued on `stream` (a cudaStream_t; NULL = the legacy default
  * stream). No host synchronisation, no allocation: capturable in a CUDA graph.
  * All pointers are device pointers owned by the caller.
- *   x          bf16  [W][T][h]            16-byte aligned
+ *   x          dtype [W][T][h]            16-byte aligned
  *   topk_idx   int32 [W][T][k]            expert ids; < 0 masked
  *   topk_w     float [W][T][k]            NULL allowed when useWeights == 0
- *   recv_x     bf16  [W][maxRecv][h]      16-byte aligned; rows >= recv_count[pe]
+ *   recv_x     dtype [W][maxRecv][h]      16-byte aligned; rows >= recv_count[pe]
  *                                         of destination pe are not written
  *   recv_meta  int32 [W][maxRecv][3+k]    per row: source rank, source token,
  *                                         weight sum (float32 bits), then for
@@ -169,9 +180,11 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
  * A combine may be repeated on the same routing (e.g. for several expert
  * outputs). Calls on one plan share its scratch, so the executions of a
  * plan's dispatches and combines must not overlap on the GPU.
- *   y    bf16 [W][maxRecv][h]   expert outputs in the receive layout, 16-byte
- *                               aligned; only rows < recv_count are read
- *   out  bf16 [W][T][h]         16-byte aligned; every row is written
+ *   y    [W][maxRecv][hc]  expert outputs in the receive layout, 16-byte
+ *                          aligned; only rows < recv_count are read
+ *   out  [W][T][hc]        16-byte aligned; every row is written
+ * Both are float32 for an EP_FP32 plan and bfloat16 otherwise; hc =
+ * combineHidden of ep_plan_info (2*h for EP_FP4X2, else h).
  * Returns EP_OK, EP_ERR_STATE before any dispatch, or a negative code.
  */
 int ep_combine(EpPlan* plan, const void* y, void* out, void* stream);

@@ -33,6 +33,11 @@ topk expert ids, then gating logits, then the hidden rows ``x``.
   torch's dtype conversion); returned as the raw uint16 bit patterns.
 * Rows ``t >= ct`` carry expert id -1 in every topk position (absent tokens) and
   weight 0.
+* Payload dtype (``dtype``, numbered as the design page's EpDType): 0 bf16 as
+  above; 1 fp32 N(0,1); 2 fp8 e4m3 (N(0,1) converted by torch's float8_e4m3fn);
+  3 fp4x2: N(0,1) rounded to the nearest e2m1 value (magnitudes 0, 0.5, 1, 1.5,
+  2, 3, 4, 6 and a sign bit), two 4-bit codes per byte, the first element in
+  the low nibble; ``h`` then counts bytes (2*h elements).
 """
 from __future__ import annotations
 
@@ -57,6 +62,7 @@ class Workload:
     use_weights: bool
     max_recv: int     # per-destination receive capacity (0 means W*max_tok)
     seed: int
+    dtype: int = 0    # payload: 0 bf16, 1 fp32, 2 fp8 (e4m3), 3 fp4x2 (h counts bytes)
 
     @property
     def E(self) -> int:
@@ -66,7 +72,7 @@ class Workload:
         """EpCfg field values (dtype 0 = bf16)."""
         return dict(worldSize=self.W, hiddenDim=self.h, maxTokPerRank=self.max_tok,
                     numExpertPerRank=self.n_epr, numExpertPerToken=self.k,
-                    maxRecv=self.max_recv, dtype=0, useWeights=int(self.use_weights))
+                    maxRecv=self.max_recv, dtype=self.dtype, useWeights=int(self.use_weights))
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -127,10 +133,42 @@ def bf16_bits_from_f32(a: np.ndarray) -> np.ndarray:
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
+_E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float32)
+
+
+_E2M1_MID = (_E2M1[1:] + _E2M1[:-1]) / 2  # decision points between neighbours
+
+
+def _e2m1_codes(v: np.ndarray) -> np.ndarray:
+    """4-bit e2m1 codes (sign in bit 3) of the values nearest to v (a value
+    exactly between two neighbours takes the smaller magnitude)."""
+    code = np.searchsorted(_E2M1_MID, np.abs(v), side="left").astype(np.uint8)
+    return code | (np.signbit(v).astype(np.uint8) << 3)
+
+
+def payload_from_f32(xf: np.ndarray, dtype: int) -> np.ndarray:
+    """The payload of float32 values in a dispatch dtype: uint16 bf16 bits,
+    float32, uint8 e4m3 bytes, or uint8 bytes of packed e2m1 pairs (the last
+    axis halves)."""
+    if dtype == 0:
+        return bf16_bits_from_f32(xf)
+    if dtype == 1:
+        return np.ascontiguousarray(xf, dtype=np.float32)
+    if dtype == 2:
+        import torch
+        t = torch.from_numpy(np.ascontiguousarray(xf, dtype=np.float32)).to(torch.float8_e4m3fn)
+        return t.view(torch.uint8).numpy()
+    if dtype == 3:
+        c = _e2m1_codes(xf)
+        return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+    raise ValueError(f"unknown dtype {dtype}")
+
+
 def make_inputs(wl: Workload, with_x: bool = True, x_rows: Optional[int] = None) -> dict:
     """Return the seeded inputs of one call.
 
-    Keys: ``x`` (uint16 bf16 bits, (W, max_tok, h)) unless ``with_x`` is False,
+    Keys: ``x`` (the payload, (W, max_tok, h): uint16 bf16 bits, float32, or
+    uint8 bytes for fp8 / fp4x2) unless ``with_x`` is False,
     ``topk_idx`` (int32, (W, max_tok, k)), ``topk_w`` (float32, same shape, or
     None when the workload runs without weights).
     """
@@ -144,8 +182,10 @@ def make_inputs(wl: Workload, with_x: bool = True, x_rows: Optional[int] = None)
     out = {"topk_idx": idx, "topk_w": w if wl.use_weights else None}
     if with_x:
         rows = T if x_rows is None else x_rows
-        xf = rng.standard_normal((W, rows, wl.h), dtype=np.float32)
-        x = np.zeros((W, T, wl.h), dtype=np.uint16)
-        x[:, :rows, :] = bf16_bits_from_f32(xf)
+        n_el = 2 * wl.h if wl.dtype == 3 else wl.h  # fp4x2: h bytes hold 2*h elements
+        xf = rng.standard_normal((W, rows, n_el), dtype=np.float32)
+        pay = payload_from_f32(xf, wl.dtype)
+        x = np.zeros((W, T, wl.h), dtype=pay.dtype)
+        x[:, :rows, :] = pay
         out["x"] = x
     return out

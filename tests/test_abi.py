@@ -99,9 +99,14 @@ def _cfg(**kw):
     (dict(maxRecv=32767), -1),            # capacity below the worst case
     (dict(maxTokPerRank=0), -1),
     (dict(numExpertPerRank=0), -1),
-    (dict(dtype=2), -2),                  # fp8 transport not built
-    (dict(dtype=1), -2),
+    (dict(dtype=2), 0),                   # fp8 transport: 7168-byte rows
+    (dict(dtype=1), 0),                   # fp32 transport
+    (dict(dtype=3, hiddenDim=3584), 0),   # fp4x2: hiddenDim counts bytes
+    (dict(dtype=2, hiddenDim=8), -1),     # 8-byte fp8 rows: not a multiple of 16
+    (dict(dtype=3, hiddenDim=24), -1),
+    (dict(dtype=1, hiddenDim=4), 0),      # 16-byte fp32 rows
     (dict(dtype=9), -1),
+    (dict(dtype=-1), -1),
     (dict(useWeights=2), -1),
     (dict(worldSize=32, maxTokPerRank=1 << 22, maxRecv=0), -1),  # flat index beyond int32
 ])
@@ -123,6 +128,22 @@ def test_plan_query_sizes(ep):
     assert info.scatterChunkBytes % 16 == 0 and info.scatterStages >= 2
     big = ep.ep_plan_query(_cfg(hiddenDim=40000))
     assert big.scatterChunkBytes < big.rowBytes and big.scatterChunkBytes % 16 == 0
+    assert (info.combineDtype, info.combineHidden, info.combineRowBytes) == (0, 7168, 14336)
+    assert info.yBytes == info.recvXBytes and info.outBytes == info.tokenBytes
+
+
+@pytest.mark.parametrize("dtype,h,row,chid,crow,cdt", [
+    (0, 7168, 14336, 7168, 14336, 0),   # bf16 in, bf16 out
+    (1, 7168, 28672, 7168, 28672, 1),   # fp32 in, fp32 out
+    (2, 7168, 7168, 7168, 14336, 0),    # fp8 in, bf16 out
+    (3, 3584, 3584, 7168, 14336, 0),    # fp4x2 in (h counts bytes), bf16 out over 2h
+])
+def test_plan_query_dtype_legs(ep, dtype, h, row, chid, crow, cdt):
+    info = ep.ep_plan_query(_cfg(dtype=dtype, hiddenDim=h))
+    assert info.rowBytes == row and info.tokenBytes == 8 * 4096 * row
+    assert info.recvXBytes == 8 * 32768 * row
+    assert (info.combineHidden, info.combineRowBytes, info.combineDtype) == (chid, crow, cdt)
+    assert info.yBytes == 8 * 32768 * crow and info.outBytes == 8 * 4096 * crow
 
 
 def test_entry_points_reject_without_crashing(ep):

@@ -64,6 +64,42 @@ def test_random_parity(case):
     run.close()
 
 
+@pytest.mark.parametrize("dtype,h", [(1, 1024), (2, 1024), (3, 512)], ids=["fp32", "fp8", "fp4x2"])
+def test_dtype_parity(dtype, h):
+    """Narrow and wide payloads (design page §3.7): dispatch moves the payload
+    bit for bit; the combine leg is fp32 for fp32 plans and bf16 otherwise (over
+    2*h elements for fp4x2), here on a seeded expert output."""
+    wl = workload("pr599").replace(dtype=dtype, h=h)
+    run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
+    assert run.info.rowBytes == h * {1: 4, 2: 1, 3: 1}[dtype]
+    run.close()
+
+
+@pytest.mark.parametrize("dtype", [0, 1, 2, 3], ids=["bf16", "fp32", "fp8", "fp4x2"])
+def test_dtype_random_small(dtype):
+    """Arbitrary payload bits (NaN and inf patterns included for fp32), duplicate
+    ids, masked entries, maxRecv above W*T."""
+    rng = np.random.default_rng(100 + dtype)
+    for _ in range(6):
+        cfg, xb, idx, w = P.random_small_case(rng, dtype=dtype)
+        run, _ = run_and_compare(cfg, dict(x=xb, topk_idx=idx, topk_w=w))
+        run.close()
+
+
+@pytest.mark.parametrize("dtype,h", [(2, 7168), (3, 3584)], ids=["fp8", "fp4x2"])
+def test_dtype_main_dispatch(dtype, h):
+    """The main workload with a one-byte payload, at full size: dispatch
+    bit-exact against the oracle."""
+    wl = workload("main").replace(dtype=dtype, h=h)
+    inputs = make_inputs(wl)
+    ref = oracle.dispatch(wl.cfg(), inputs["x"], inputs["topk_idx"], inputs["topk_w"])
+    with GpuRun(wl.cfg(), inputs) as run:
+        run.dispatch()
+        torch.cuda.synchronize()
+        compare_dispatch(run, ref)
+        assert run.error_word() == 0
+
+
 def test_out_of_range_ids_reported_and_masked():
     rng = np.random.default_rng(5)
     cfg, inputs = _small_random_cfg(rng, 4, 64, 64, 4, 4, True, oob=True)
@@ -106,11 +142,8 @@ def test_repeated_calls_and_reset():
         run.dispatch()
         torch.cuda.synchronize()
         compare_dispatch(run, ref_a)
-        run.idx.copy_(to_dev(b["topk_idx"]))
-        run.w.copy_(to_dev(b["topk_w"]))
-        run.x.copy_(to_dev(b["x"].view(np.int16)))
-        run.recv_x.fill_(0xABCD - (1 << 16))
-        run.recv_meta.fill_(0x5EADBEEF)
+        run.load_inputs(b)
+        run.reset_canaries()
         run.dispatch()
         run.combine()
         torch.cuda.synchronize()
