@@ -31,8 +31,13 @@ struct EpPlan {
     int32_t* work;
     int32_t* cwork;
     uint32_t* cdone;
+    int32_t* chunk_cnt;   // fused dispatch: [ceil(G/32)][W]
+    int32_t* chunk_base;
+    uint32_t* fbar;
+    uint32_t* fdone;
     int32_t* err;
     size_t scatterSmem;
+    bool fused;           // route + scan + scatter in one cooperative launch
     bool dispatched;
 };
 
@@ -293,6 +298,31 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->info.device = dev;
         plan->info.numSMs = sms;
         plan->info.scatterBlocks = env_int("EP_SCATTER_BLOCKS", sms * sPerSm);
+        // Dispatch in one cooperative launch (route + scan + scatter) only on
+        // request (EP_DISPATCH_FUSED=1): on B200 the two launches of
+        // route_count + scatter_rows measured faster at every size (main
+        // workload 476 vs 500 us, ct=1 workload 17.4 vs 20.5 us).
+        bool fused = false;
+        if (const char* f = std::getenv("EP_DISPATCH_FUSED"))
+            fused = geo.scatterMode == ep::kScatterTma && std::strcmp(f, "1") == 0;
+        int coop = 0;
+        if (fused && (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop))
+            fused = false;
+        if (fused) {
+            int fPerSm = 0;
+            if ((e = ep::fused_set_smem(cfg->worldSize, smem)) != cudaSuccess ||
+                (e = ep::fused_blocks_per_sm(cfg->worldSize, geo.scatterWarps, smem, &fPerSm)) != cudaSuccess) {
+                cuda_fail(e, "fused dispatch set-up");
+                delete plan;
+                return nullptr;
+            }
+            if (fPerSm < 1)
+                fused = false;
+            else  // a cooperative launch needs every block resident at once
+                plan->info.scatterBlocks = std::min(plan->info.scatterBlocks, sms * fPerSm);
+        }
+        plan->fused = fused;
+        plan->info.dispatchFused = fused ? 1 : 0;
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
@@ -320,6 +350,10 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->work = reinterpret_cast<int32_t*>(base + L.work);
         plan->cwork = reinterpret_cast<int32_t*>(base + L.cwork);
         plan->cdone = reinterpret_cast<uint32_t*>(base + L.cdone);
+        plan->chunk_cnt = reinterpret_cast<int32_t*>(base + L.chunk_cnt);
+        plan->chunk_base = reinterpret_cast<int32_t*>(base + L.chunk_base);
+        plan->fbar = reinterpret_cast<uint32_t*>(base + L.fbar);
+        plan->fdone = reinterpret_cast<uint32_t*>(base + L.fdone);
         plan->err = reinterpret_cast<int32_t*>(base + L.err);
         plan->dispatched = false;
         g_last_error[0] = '\0';
@@ -391,8 +425,11 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
         rp.numTiles = plan->info.numTiles;
         rp.maxRecv = plan->maxRecv;
         rp.useWeights = c.useWeights;
-        cudaError_t e = ep::launch_route_count(rp, s);
-        if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
+        cudaError_t e = cudaSuccess;
+        if (!plan->fused) {
+            e = ep::launch_route_count(rp, s);
+            if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
+        }
 
         ep::ScatterParams sp{};
         sp.x = static_cast<const uint8_t*>(x);
@@ -417,6 +454,25 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
         sp.chunkStride = (sp.chunkBytes + 127) & ~127;
         sp.numChunks = (int)((sp.rowBytes + sp.chunkBytes - 1) / sp.chunkBytes);
         sp.stages = plan->info.scatterStages;
+        if (plan->fused) {
+            // One cooperative launch: routing phase, chunk scan, copy engines.
+            sp.baseShift = 5;
+            sp.tile_base = plan->chunk_base;
+            sp.w = c.useWeights ? topk_w : nullptr;
+            sp.tok_mask_w = plan->tok_mask;
+            sp.chunk_cnt = plan->chunk_cnt;
+            sp.chunk_base_w = plan->chunk_base;
+            sp.recv_count = recv_count;
+            sp.bar = plan->fbar;
+            sp.done = plan->fdone;
+            sp.numChunks32 = (plan->G + 31) / 32;
+            sp.useWeights = c.useWeights;
+            e = ep::launch_dispatch_fused(sp, plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
+            if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_fused");
+            plan->dispatched = true;
+            return EP_OK;
+        }
+        sp.baseShift = 8;  // route_count's 256-token tiles
         e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend,
                                     plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch scatter_rows");

@@ -49,6 +49,17 @@ struct ScatterParams {
     int chunkStride;  // shared-memory bytes per stage, multiple of 128
     int numChunks;    // ceil(rowBytes / chunkBytes)
     int stages;       // stages per copy engine (>= 2)
+    int baseShift;    // tile_base has one row per 2^baseShift tokens (8: route_count tiles; 5: fused chunks)
+    // Only the fused dispatch (route + scan + scatter in one launch) uses these:
+    const float* w;          // [G][k] or nullptr
+    uint32_t* tok_mask_w;    // = tok_mask, written by the routing phase
+    int32_t* chunk_cnt;      // [numChunks32][W]
+    int32_t* chunk_base_w;   // = tile_base, written by the scan phase
+    int32_t* recv_count;     // [W]
+    unsigned* bar;           // grid-barrier counter
+    unsigned* done;          // blocks finished; the last one resets bar, work, done
+    int numChunks32;         // ceil(G / 32)
+    int useWeights;
 };
 
 struct CombineParams {
@@ -62,24 +73,32 @@ struct CombineParams {
 };
 
 // Byte offsets of the dispatch scratch regions (each 256-byte aligned):
-// routing table, token masks, tile counts, tile bases, the counters (one
-// 256-byte region: tile ticket, scatter token counter, combine token counter,
-// combine blocks done), error word.
+// routing table, token masks, tile counts, tile bases (256-token tiles of the
+// split dispatch), chunk counts and bases (32-token chunks of the fused
+// dispatch), the counters (one 256-byte region: tile ticket, scatter token
+// counter, combine token counter, combine blocks done, fused grid barrier,
+// fused blocks done), error word.
 struct ScratchLayout {
-    size_t route, tok_mask, tile_cnt, tile_base, ticket, work, cwork, cdone, err, total;
+    size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base;
+    size_t ticket, work, cwork, cdone, fbar, fdone, err, total;
 };
 
 inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
     auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
+    const size_t numChunks32 = (size_t)((G + 31) / 32);
     ScratchLayout L;
     L.route = 0;
     L.tok_mask = L.route + up(sizeof(int2) * (size_t)G * W);
     L.tile_cnt = L.tok_mask + up(sizeof(uint32_t) * (size_t)G);
     L.tile_base = L.tile_cnt + up(sizeof(int32_t) * (size_t)numTiles * W);
-    L.ticket = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * W);
+    L.chunk_cnt = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * W);
+    L.chunk_base = L.chunk_cnt + up(sizeof(int32_t) * numChunks32 * W);
+    L.ticket = L.chunk_base + up(sizeof(int32_t) * numChunks32 * W);
     L.work = L.ticket + 4;
     L.cwork = L.ticket + 8;
     L.cdone = L.ticket + 12;
+    L.fbar = L.ticket + 16;
+    L.fdone = L.ticket + 20;
     L.err = L.ticket + 256;
     L.total = L.err + 256;
     return L;
@@ -96,6 +115,11 @@ cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int 
                                 size_t smem, cudaStream_t s);
 // fp32: float32 combine leg (an fp32 plan); bf16 otherwise.
 cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s);
+// Fused dispatch (route + scan + scatter), a cooperative launch: blocks must
+// not exceed the co-resident capacity (fused_blocks_per_sm * SMs).
+cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s);
+cudaError_t fused_set_smem(int W, size_t bytes);
+cudaError_t fused_blocks_per_sm(int W, int warps, size_t smem, int* out);
 
 // Shared-memory bytes the scatter kernel needs for a geometry.
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride);

@@ -165,6 +165,35 @@ __device__ __forceinline__ int source_next(TokenSource& s) {
 // route_count: mask, weight sums, tile histogram, tile-local ranks; the last
 // block scans the histogram. kW = compile-time bound on W (8, 16 or 32).
 // =====================================================================
+// Destination mask and per-destination weight sums of token g (float32 fold
+// in topk order); ids < 0 are masked, ids >= E are reported and masked.
+template <int kW>
+__device__ __forceinline__ uint32_t route_token(const int32_t* idx, const float* w, int g, int k, int nEpr,
+                                                int E, float (&ws)[kW], bool& bad) {
+    uint32_t mask = 0;
+#pragma unroll
+    for (int pe = 0; pe < kW; ++pe) ws[pe] = 0.0f;
+    const int32_t* ids = idx + (size_t)g * k;
+    const float* wts = w ? w + (size_t)g * k : nullptr;
+    for (int j = 0; j < k; ++j) {
+        const int e = ids[j];
+        if (e < 0) continue;  // masked entry
+        if (e >= E) {         // contract violation: report, treat as masked
+            bad = true;
+            continue;
+        }
+        const int pe_j = e / nEpr;
+        mask |= 1u << pe_j;
+        if (wts) {
+            const float wj = wts[j];
+#pragma unroll
+            for (int pe = 0; pe < kW; ++pe)
+                if (pe == pe_j) ws[pe] = ws[pe] + wj;  // fold in topk order
+        }
+    }
+    return mask;
+}
+
 template <int kW>
 __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams p) {
     __shared__ int s_wcnt[kCountWarps][kW];
@@ -181,29 +210,7 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     uint32_t mask = 0;
     bool bad = false;
     float ws[kW];
-#pragma unroll
-    for (int pe = 0; pe < kW; ++pe) ws[pe] = 0.0f;
-
-    if (g < p.G) {
-        const int32_t* ids = p.idx + (size_t)g * k;
-        const float* wts = p.w ? p.w + (size_t)g * k : nullptr;
-        for (int j = 0; j < k; ++j) {
-            const int e = ids[j];
-            if (e < 0) continue;  // masked entry
-            if (e >= p.E) {       // contract violation: report, treat as masked
-                bad = true;
-                continue;
-            }
-            const int pe_j = e / p.nEpr;
-            mask |= 1u << pe_j;
-            if (wts) {
-                const float wj = wts[j];
-#pragma unroll
-                for (int pe = 0; pe < kW; ++pe)
-                    if (pe == pe_j) ws[pe] = ws[pe] + wj;  // fold in topk order
-            }
-        }
-    }
+    if (g < p.G) mask = route_token<kW>(p.idx, p.w, g, k, p.nEpr, p.E, ws, bad);
     if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
 
     // Per-warp histogram by ballot.
@@ -294,8 +301,9 @@ __device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p,
     TokenInputs in;
     in.g = g;
     const int W = p.W;
-    in.rr = lane < W ? p.route[(size_t)g * W + lane] : make_int2(-1, 0);
-    in.base = lane < W ? p.tile_base[(size_t)(g / kCountTile) * W + lane] : 0;
+    // routing data written by other blocks (or the previous kernel): read through L2
+    in.rr = lane < W ? __ldcg(p.route + (size_t)g * W + lane) : make_int2(-1, 0);
+    in.base = lane < W ? __ldcg(p.tile_base + (size_t)(g >> p.baseShift) * W + lane) : 0;
     in.e = lane < p.k ? p.idx[(size_t)g * p.k + lane] : -1;
     return in;
 }
@@ -307,12 +315,15 @@ __device__ __forceinline__ uint32_t token_slots_and_meta(const ScatterParams& p,
                                                          int lane, int& my_slot) {
     const int W = p.W, g = in.g;
     const int2 rr = in.rr;
-    const uint32_t mask = __ballot_sync(kFull, rr.x >= 0);
     my_slot = -1;
+    bool ok = false;
     if (rr.x >= 0) {
         my_slot = in.base + rr.x;
-        p.route[(size_t)g * W + lane].x = my_slot;
+        ok = my_slot < p.maxRecv;  // always, unless the counts were corrupted
+        if (!ok) atomicOr(p.err, EP_DEVERR_CAPACITY);
+        p.route[(size_t)g * W + lane].x = ok ? my_slot : -1;
     }
+    const uint32_t mask = __ballot_sync(kFull, ok);
     const int r = g / p.T, t = g - r * p.T;
     const int e = in.e;
     const int pe_e = (e >= 0 && e < p.E) ? e / p.nEpr : -1;
@@ -347,30 +358,44 @@ __device__ __forceinline__ void bulk_wait_read_pend() {
     asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kPend) : "memory");
 }
 
-template <int kPend>
-__global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(ScatterParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    const int S = p.stages;  // > kPend (checked on the host)
+// Shared memory of the copy engines of one block, carved from the dynamic
+// shared memory: [mbarriers: nwarps*S][ring: nwarps*S*2 int] pad 128 | stages.
+struct EngineSmem {
+    uint32_t stage0_addr;  // this warp's first stage
+    uint32_t bar0;         // this warp's first mbarrier
+    int* item_tok;         // [S] token of the item in each stage
+    int* item_chunk;       // [S] row piece of the item in each stage
+};
 
-    // Layout: [bars: nwarps*S u64][ring: nwarps*S*2 int] pad to 128 | stages
+__device__ __forceinline__ EngineSmem engine_smem_init(uint8_t* smem, const ScatterParams& p, int warp,
+                                                       int nwarps, int lane) {
+    const int S = p.stages;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
     int* ring = reinterpret_cast<int*>(smem + (size_t)nwarps * S * sizeof(uint64_t));
     const size_t head = ((size_t)nwarps * S * (sizeof(uint64_t) + 2 * sizeof(int)) + 127) & ~(size_t)127;
-    uint8_t* stage0 = smem + head + (size_t)warp * S * p.chunkStride;
-    const uint32_t stage0_addr = smem_addr(stage0);
-    const uint32_t bar0 = smem_addr(bars + warp * S);
-    int* item_tok = ring + warp * S * 2;
-    int* item_chunk = item_tok + S;
-
+    EngineSmem es;
+    es.stage0_addr = smem_addr(smem + head + (size_t)warp * S * p.chunkStride);
+    es.bar0 = smem_addr(bars + warp * S);
+    es.item_tok = ring + warp * S * 2;
+    es.item_chunk = es.item_tok + S;
     if (lane == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1u);
+        for (int s = 0; s < S; ++s) mbar_init(es.bar0 + 8u * s, 1u);
         mbar_fence_init();
     }
     __syncwarp();
-    pdl_wait();     // routing written by route_count is visible from here on
-    pdl_trigger();
+    return es;
+}
+
+// One copy engine (a warp): the present tokens it is handed are copied row
+// piece by row piece through an S-stage shared-memory ring, S - kPend loads
+// ahead, with kPend items' bulk stores left draining when a stage is refilled.
+template <int kPend>
+__device__ __forceinline__ void copy_engine(const ScatterParams& p, const EngineSmem& es, int lane, int warp,
+                                            int nwarps) {
+    const int S = p.stages;  // > kPend (checked on the host)
+    const uint32_t stage0_addr = es.stage0_addr, bar0 = es.bar0;
+    int* item_tok = es.item_tok;
+    int* item_chunk = es.item_chunk;
 
     // Producer (lane 0): tokens come from the shared hand-out (static rounds,
     // then a global counter). Two candidates are kept in flight ahead (the
@@ -496,6 +521,132 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
+}
+
+
+template <int kPend>
+__global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(ScatterParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
+    pdl_wait();     // routing written by route_count is visible from here on
+    pdl_trigger();
+    copy_engine<kPend>(p, es, lane, warp, nwarps);
+}
+
+// =====================================================================
+// dispatch_fused: route, scan and scatter in one cooperative launch (an
+// option, EP_DISPATCH_FUSED=1: on B200 it measured slower than route_count +
+// scatter_rows, since ~300 copy-engine warps route the tokens instead of
+// route_count's thousand, and two grid barriers and a one-warp-per-destination
+// scan cost more than the launch they save).
+//   1. every warp routes 32-token chunks: destination masks, weight sums,
+//      chunk-local ranks and chunk counts by ballot;
+//   2. grid barrier; warps scan the chunk counts, one destination each, into
+//      chunk bases and store recv_count;
+//   3. grid barrier; the copy engines run as in scatter_rows.
+// The barriers spin on a global counter with a bound; a cooperative launch
+// keeps every block resident, so they complete. The last block to finish
+// resets the counters for the next call.
+// =====================================================================
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned target) {
+    __threadfence();  // every thread's writes of this phase, before the arrival
+    __syncthreads();
+    int ok = 1;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(bar, 1u);
+        const long long t0 = clock64();
+        for (;;) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+            if (v >= target) break;
+            if (clock64() - t0 > kWaitCycles) {
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+    }
+    return __syncthreads_and(ok) != 0;
+}
+
+template <int kW>
+__global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kernel(ScatterParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int gw = blockIdx.x * nwarps + warp, nW = gridDim.x * nwarps;
+    const int W = p.W;
+    const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
+    pdl_wait();  // the ids may come from the previous kernel of the stream
+
+    // 1. route 32-token chunks
+    const uint32_t lt = lanemask_lt();
+    for (int c = gw; c < p.numChunks32; c += nW) {
+        const int g = c * 32 + lane;
+        uint32_t mask = 0;
+        bool bad = false;
+        float ws[kW];
+        if (g < p.G) mask = route_token<kW>(p.idx, p.w, g, p.k, p.nEpr, p.E, ws, bad);
+        if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
+        if (g < p.G) p.tok_mask_w[g] = mask;
+        int my_cnt = 0;
+#pragma unroll
+        for (int pe = 0; pe < kW; ++pe) {
+            if (pe < W) {
+                const bool hit = (mask >> pe) & 1u;
+                const uint32_t b = __ballot_sync(kFull, hit);
+                if (lane == pe) my_cnt = __popc(b);
+                if (g < p.G) {
+                    const float wsum = hit ? (p.useWeights ? ws[pe] : 1.0f) : 0.0f;
+                    p.route[(size_t)g * W + pe] = make_int2(hit ? __popc(b & lt) : -1, __float_as_int(wsum));
+                }
+            }
+        }
+        if (lane < W) p.chunk_cnt[(size_t)c * W + lane] = my_cnt;
+    }
+
+    bool ok = grid_barrier(p.bar, gridDim.x);
+
+    // 2. one warp per destination scans the chunk counts
+    for (int pe = gw; ok && pe < W; pe += nW) {
+        int running = 0;
+        for (int c0 = 0; c0 < p.numChunks32; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = c < p.numChunks32 ? __ldcg(p.chunk_cnt + (size_t)c * W + pe) : 0;
+            int incl = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int n = __shfl_up_sync(kFull, incl, off);
+                if (lane >= off) incl += n;
+            }
+            if (c < p.numChunks32) p.chunk_base_w[(size_t)c * W + pe] = running + incl - v;
+            running += __shfl_sync(kFull, incl, 31);
+        }
+        if (lane == 0) {
+            p.recv_count[pe] = running;  // stored, not accumulated
+            if (running > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+        }
+    }
+
+    ok = ok && grid_barrier(p.bar, 2u * gridDim.x);
+
+    // 3. copy engines
+    if (ok) copy_engine<1>(p, es, lane, warp, nwarps);
+    else if (threadIdx.x == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
+
+    // The last block to finish resets the counters for the next call.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+            *p.bar = 0u;
+            *p.work = 0;
+            *p.done = 0u;
+            __threadfence();
+        }
+    }
 }
 
 // =====================================================================
@@ -771,6 +922,44 @@ cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int 
         return e != cudaSuccess ? e : cudaGetLastError();
     }
     cudaError_t e = for_pend(pend, [&](auto k) { return launch_pdl(k, blocks, warps * 32, smem, s, p); });
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+namespace {
+template <typename F>
+cudaError_t for_world(int W, F&& f) {
+    if (W <= 8) return f(ep_dispatch_fused_kernel<8>);
+    if (W <= 16) return f(ep_dispatch_fused_kernel<16>);
+    return f(ep_dispatch_fused_kernel<32>);
+}
+}  // namespace
+
+cudaError_t fused_set_smem(int W, size_t bytes) {
+    return for_world(W, [&](auto k) {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    });
+}
+
+cudaError_t fused_blocks_per_sm(int W, int warps, size_t smem, int* out) {
+    return for_world(W, [&](auto k) {
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, warps * 32, smem);
+    });
+}
+
+cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s) {
+    cudaError_t e = for_world(p.W, [&](auto k) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(blocks);
+        cfg.blockDim = dim3(warps * 32);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, k, p);
+    });
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -96,6 +96,9 @@ typedef struct EpPlanInfo {
     int64_t combineRowBytes;  /* bytes of a y / out row */
     int64_t yBytes;           /* bytes of y: W*maxRecv*combineRowBytes */
     int64_t outBytes;         /* bytes of out: W*T*combineRowBytes */
+    int32_t dispatchFused;    /* 1: dispatch is one cooperative launch (route, scan, scatter);
+                                 0: two launches (route_count, scatter_rows) */
+    int32_t reserved0;
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
@@ -140,7 +143,7 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * Environment overrides, read here only (for geometry sweeps):
  * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK,
  * EP_SCATTER_PEND (1..3), EP_SCATTER_MODE ("tma" or "regs"), EP_COMBINE_BLOCKS,
- * EP_COMBINE_WARPS. */
+ * EP_COMBINE_WARPS, EP_DISPATCH_FUSED (0: two launches instead of one). */
 EpPlan* ep_plan_create(const EpCfg* cfg);
 
 /* Free the plan and its scratch. NULL is a no-op. The caller must make sure no

@@ -35,6 +35,16 @@ def test_workload_parity(name):
     run.close()
 
 
+@pytest.mark.parametrize("fused", ["0", "1"])
+@pytest.mark.parametrize("name", ["main", "latency8"])
+def test_workload_parity_both_dispatch_modes(name, fused, monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
+    wl = workload(name)
+    run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
+    assert run.info.dispatchFused == int(fused)
+    run.close()
+
+
 def _small_random_cfg(rng, W, T, h, k, nEpr, use_w, max_recv=0, dup=True, oob=False):
     E = W * nEpr
     lo = -2 if dup else 0
@@ -210,6 +220,10 @@ def test_graph_capture_replay():
     {"EP_SCATTER_PEND": "3", "EP_SCATTER_STAGES": "4", "EP_SCATTER_CHUNK": "4096"},
     {"EP_SCATTER_MODE": "regs"},
     {"EP_SCATTER_MODE": "regs", "EP_SCATTER_WARPS": "2", "EP_SCATTER_BLOCKS": "5"},
+    {"EP_DISPATCH_FUSED": "0"},                              # two launches: route_count + scatter_rows
+    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_BLOCKS": "3"},    # fused, few blocks: long chunk loops
+    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "8", "EP_SCATTER_STAGES": "2", "EP_SCATTER_CHUNK": "1024"},
+    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "1", "EP_SCATTER_BLOCKS": "1"},  # fewer warps than W
 ])
 def test_geometry_overrides(env, monkeypatch):
     for k_, v in env.items():
@@ -219,6 +233,8 @@ def test_geometry_overrides(env, monkeypatch):
     info = run.info
     if "EP_SCATTER_BLOCKS" in env:
         assert info.scatterBlocks == int(env["EP_SCATTER_BLOCKS"])
+    if "EP_DISPATCH_FUSED" in env:
+        assert info.dispatchFused == int(env["EP_DISPATCH_FUSED"])
     run.close()
 
 
