@@ -47,6 +47,8 @@ def _bind(lib):
     cfgp = ctypes.POINTER(OracleCfg)
     lib.oracle_dispatch.argtypes = [cfgp, P, P, P, P, P, P, P, P]
     lib.oracle_dispatch.restype = ctypes.c_int
+    lib.oracle_dispatch_scaled.argtypes = [cfgp, P, P, P, P, ctypes.c_int64, P, P, P, P, P, P]
+    lib.oracle_dispatch_scaled.restype = ctypes.c_int
     lib.oracle_combine.argtypes = [cfgp, P, P, P, P]
     lib.oracle_combine.restype = ctypes.c_int
     lib.oracle_recv_capacity.argtypes = [cfgp]
@@ -107,7 +109,7 @@ def combine_np(cfg: dict):
 
 
 def dispatch(cfg: dict, x: np.ndarray, topk_idx: np.ndarray, topk_w, recv_x=None, recv_meta=None,
-             lib=None):
+             lib=None, scales=None, recv_scales=None):
     """Run the oracle dispatch. Returns a dict with recv_x, recv_meta,
     recv_count, slotmap, wsum and status (0, or STATUS_EXPERT_RANGE).
 
@@ -132,12 +134,22 @@ def dispatch(cfg: dict, x: np.ndarray, topk_idx: np.ndarray, topk_w, recv_x=None
     recv_count = np.zeros(W, dtype=np.int32)
     slotmap = np.empty((W, T, W), dtype=np.int32)
     wsum = np.empty((W, T, W), dtype=np.float32)
-    rc = lib.oracle_dispatch(ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(w), _ptr(recv_x),
-                             _ptr(recv_meta), _ptr(recv_count), _ptr(slotmap), _ptr(wsum))
+    if scales is None:
+        rc = lib.oracle_dispatch(ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(w), _ptr(recv_x),
+                                 _ptr(recv_meta), _ptr(recv_count), _ptr(slotmap), _ptr(wsum))
+    else:
+        sw = np.ascontiguousarray(scales).view(np.uint32).reshape(W, T, -1)
+        if recv_scales is None:
+            recv_scales = np.zeros((W, R, sw.shape[-1]), dtype=np.uint32)
+        recv_scales = recv_scales.view(np.uint32)
+        assert recv_scales.shape == (W, R, sw.shape[-1]) and recv_scales.flags.c_contiguous
+        rc = lib.oracle_dispatch_scaled(ctypes.byref(c), _ptr(x), _ptr(idx), _ptr(w), _ptr(sw),
+                                        sw.shape[-1], _ptr(recv_x), _ptr(recv_meta), _ptr(recv_scales),
+                                        _ptr(recv_count), _ptr(slotmap), _ptr(wsum))
     if rc < 0:
         raise ValueError(f"oracle_dispatch rejected its arguments (rc={rc})")
     return dict(recv_x=recv_x, recv_meta=recv_meta, recv_count=recv_count,
-                slotmap=slotmap, wsum=wsum, status=rc)
+                slotmap=slotmap, wsum=wsum, status=rc, recv_scales=recv_scales)
 
 
 def combine(cfg: dict, y: np.ndarray, slotmap: np.ndarray, wsum: np.ndarray, lib=None) -> np.ndarray:

@@ -146,9 +146,40 @@ int oracle_recv_capacity(const OracleCfg *c)
  * Returns 0, ORACLE_STATUS_EXPERT_RANGE when an id >= E was masked, or a
  * negative error.
  */
+static int dispatch_impl(const OracleCfg *c, const uint8_t *x, const int32_t *topk_idx,
+                         const float *topk_w, const uint32_t *scales, int64_t scale_words,
+                         uint8_t *recv_x, int32_t *recv_meta, uint32_t *recv_scales,
+                         int32_t *recv_count, int32_t *slotmap, float *wsum);
+
 int oracle_dispatch(const OracleCfg *c, const uint8_t *x, const int32_t *topk_idx,
                     const float *topk_w, uint8_t *recv_x, int32_t *recv_meta,
                     int32_t *recv_count, int32_t *slotmap, float *wsum)
+{
+    return dispatch_impl(c, x, topk_idx, topk_w, NULL, 0, recv_x, recv_meta, NULL, recv_count,
+                         slotmap, wsum);
+}
+
+/*
+ * Dispatch with a per-token scale row (mori PR #599, its follow-up commits: the
+ * scale transport -- a fourth per-token field and the scale row carried with
+ * the payload). scales is [W][T][scale_words] 4-byte words; every received row
+ * gets its token's scale row at recv_scales [W][R][scale_words], bit for bit,
+ * like the payload. Rows past recv_count are not written.
+ */
+int oracle_dispatch_scaled(const OracleCfg *c, const uint8_t *x, const int32_t *topk_idx,
+                           const float *topk_w, const uint32_t *scales, int64_t scale_words,
+                           uint8_t *recv_x, int32_t *recv_meta, uint32_t *recv_scales,
+                           int32_t *recv_count, int32_t *slotmap, float *wsum)
+{
+    if (scale_words <= 0 || !scales || !recv_scales) return ORACLE_ERR_ARG;
+    return dispatch_impl(c, x, topk_idx, topk_w, scales, scale_words, recv_x, recv_meta,
+                         recv_scales, recv_count, slotmap, wsum);
+}
+
+static int dispatch_impl(const OracleCfg *c, const uint8_t *x, const int32_t *topk_idx,
+                         const float *topk_w, const uint32_t *scales, int64_t scale_words,
+                         uint8_t *recv_x, int32_t *recv_meta, uint32_t *recv_scales,
+                         int32_t *recv_count, int32_t *slotmap, float *wsum)
 {
     if (!cfg_ok(c) || !x || !topk_idx || !recv_x || !recv_meta || !recv_count ||
         !slotmap || !wsum)
@@ -190,6 +221,9 @@ int oracle_dispatch(const OracleCfg *c, const uint8_t *x, const int32_t *topk_id
                 if (next[pe] >= R) { free(next); return ORACLE_ERR_ARG; }
                 const int64_t slot = next[pe]++;
                 memcpy(recv_x + (pe * R + slot) * row, x + g * row, (size_t)row);
+                if (scales)
+                    memcpy(recv_scales + (pe * R + slot) * scale_words, scales + g * scale_words,
+                           (size_t)scale_words * sizeof(uint32_t));
                 int32_t *meta = recv_meta + (pe * R + slot) * M;
                 meta[0] = (int32_t)r;
                 meta[1] = (int32_t)t;

@@ -158,6 +158,30 @@ def pin_bruteforce_dispatch(lib=None, n_cases=40, seed=11):
             assert np.all(res["recv_meta"][pe, n:] == 0x5EADBEEF)
 
 
+def pin_bruteforce_scale_rows(lib=None, n_cases=16, seed=21):
+    """The scale row of a token travels with it: every received row's scale
+    row equals its source token's, bit for bit; rows past the count keep the
+    canary; the payload outputs equal the unscaled dispatch's."""
+    rng = np.random.default_rng(seed)
+    for case in range(n_cases):
+        cfg, xb, idx, w = random_small_case(rng, dtype=case % 4)
+        W, T = cfg["worldSize"], cfg["maxTokPerRank"]
+        R = oracle.recv_capacity(cfg)
+        sw = int(rng.integers(1, 70))
+        scales = rng.integers(0, 1 << 32, size=(W, T, sw), dtype=np.uint64).astype(np.uint32)
+        canary = np.full((W, R, sw), 0xC0FFEE, dtype=np.uint32)
+        res = oracle.dispatch(cfg, xb, idx, w, lib=lib, scales=scales, recv_scales=canary)
+        plain = oracle.dispatch(cfg, xb, idx, w, lib=lib)
+        for key in ("recv_count", "slotmap", "wsum", "recv_meta"):
+            assert np.array_equal(res[key], plain[key]), key
+        assert res["recv_x"].tobytes() == plain["recv_x"].tobytes()
+        slot, count = brute_routes(cfg, idx)
+        for (pe, r, t), sl in slot.items():
+            assert np.array_equal(res["recv_scales"][pe, sl], scales[r, t])
+        for pe in range(W):
+            assert np.all(res["recv_scales"][pe, count[pe]:] == 0xC0FFEE)
+
+
 def pin_bruteforce_weight_sum_order(lib=None):
     """The weight sum is the float32 fold in topk order, s0=+0: with three
     weights whose float32 sum depends on the order, the oracle must return the
@@ -553,6 +577,7 @@ def pin_out_of_range_ids(lib=None):
 ALL_PINS = [
     pin_bruteforce_dispatch,
     pin_bruteforce_weight_sum_order,
+    pin_bruteforce_scale_rows,
     pin_combine_exact_fma,
     pin_combine_single_rounding_case,
     pin_combine_fp32_exact_fma,

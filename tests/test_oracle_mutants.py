@@ -42,6 +42,8 @@ MUTANTS = {
                                    "return c->hiddenDim;"),
     "fp32_combine_rounded_to_bf16": ("for (int64_t i = 0; i < h; ++i) outf[g * h + i] = acc[i];",
                                      "for (int64_t i = 0; i < h; ++i) outf[g * h + i] = bf16_to_f32(f32_to_bf16_rne(acc[i]));"),
+    "scale_row_of_wrong_token": ("memcpy(recv_scales + (pe * R + slot) * scale_words, scales + g * scale_words,",
+                                 "memcpy(recv_scales + (pe * R + slot) * scale_words, scales + t * scale_words,"),
     "count_not_stored": ("recv_count[pe] = (int32_t)next[pe];", "recv_count[pe] = (int32_t)next[pe] - (pe == 0);"),
 }
 
