@@ -22,7 +22,9 @@ EP_ERR_STATE, EP_ERR_ALIGN, EP_ERR_DEVICE = -5, -6, -7
 EP_DEVERR_EXPERT_RANGE, EP_DEVERR_TIMEOUT, EP_DEVERR_CAPACITY = 1, 2, 4
 
 EXPORTED = ("ep_cfg_check", "ep_plan_query", "ep_plan_create", "ep_plan_destroy", "ep_plan_info",
-            "ep_dispatch", "ep_combine", "ep_plan_check_error", "ep_last_error", "ep_dispatch_noalloc")
+            "ep_dispatch", "ep_combine", "ep_plan_check_error", "ep_last_error", "ep_dispatch_noalloc",
+            "ep_dispatch_scaled")
+EP_MAX_SCALE_WORDS = 4096
 EP_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
@@ -76,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "ep_plan_check_error": ([P], I32),
         "ep_last_error": ([], ctypes.c_char_p),
         "ep_dispatch_noalloc": ([cfgp, P, P, P, P, P, P, P], I32),
+        "ep_dispatch_scaled": ([P, P, P, P, P, ctypes.c_int32, P, P, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -150,6 +153,14 @@ def ep_dispatch(plan: int, x, topk_idx, topk_w, recv_x, recv_meta, recv_count, s
     return _check(_lib.ep_dispatch(plan, _addr(x), _addr(topk_idx), _addr(topk_w), _addr(recv_x),
                                    _addr(recv_meta), _addr(recv_count), _stream(stream)),
                   "ep_dispatch")
+
+
+def ep_dispatch_scaled(plan: int, x, topk_idx, topk_w, scales, scale_words: int, recv_x, recv_meta,
+                       recv_scales, recv_count, stream=None) -> int:
+    return _check(_lib.ep_dispatch_scaled(plan, _addr(x), _addr(topk_idx), _addr(topk_w), _addr(scales),
+                                          int(scale_words), _addr(recv_x), _addr(recv_meta),
+                                          _addr(recv_scales), _addr(recv_count), _stream(stream)),
+                  "ep_dispatch_scaled")
 
 
 def ep_combine(plan: int, y, out, stream=None) -> int:

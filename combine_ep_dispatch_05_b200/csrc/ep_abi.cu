@@ -388,8 +388,31 @@ static int check_device(const EpPlan* plan) {
 
 static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
+                         const void* scales, int32_t scaleWords, void* recv_x, int32_t* recv_meta,
+                         void* recv_scales, int32_t* recv_count, void* stream);
+
 int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
                 void* recv_x, int32_t* recv_meta, int32_t* recv_count, void* stream) {
+    return dispatch_impl(plan, x, topk_idx, topk_w, nullptr, 0, recv_x, recv_meta, nullptr, recv_count,
+                         stream);
+}
+
+int ep_dispatch_scaled(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
+                       const void* scales, int32_t scaleWords, void* recv_x, int32_t* recv_meta,
+                       void* recv_scales, int32_t* recv_count, void* stream) {
+    if (scaleWords < 1 || scaleWords > EP_MAX_SCALE_WORDS)
+        return fail(EP_ERR_INVALID, "scaleWords %d outside 1..%d", scaleWords, EP_MAX_SCALE_WORDS);
+    if (!scales || !recv_scales) return fail(EP_ERR_INVALID, "scales or recv_scales is NULL");
+    if (!aligned(scales, 4) || !aligned(recv_scales, 4))
+        return fail(EP_ERR_ALIGN, "scales and recv_scales must be 4-byte aligned");
+    return dispatch_impl(plan, x, topk_idx, topk_w, scales, scaleWords, recv_x, recv_meta, recv_scales,
+                         recv_count, stream);
+}
+
+static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
+                         const void* scales, int32_t scaleWords, void* recv_x, int32_t* recv_meta,
+                         void* recv_scales, int32_t* recv_count, void* stream) {
     try {
         if (!plan) return fail(EP_ERR_INVALID, "plan is NULL");
         if (!x || !topk_idx || !recv_x || !recv_meta || !recv_count)
@@ -454,6 +477,9 @@ int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const floa
         sp.chunkStride = (sp.chunkBytes + 127) & ~127;
         sp.numChunks = (int)((sp.rowBytes + sp.chunkBytes - 1) / sp.chunkBytes);
         sp.stages = plan->info.scatterStages;
+        sp.scales = static_cast<const uint32_t*>(scales);
+        sp.recv_scales = static_cast<uint32_t*>(recv_scales);
+        sp.scaleWords = scaleWords;
         if (plan->fused) {
             // One cooperative launch: routing phase, chunk scan, copy engines.
             sp.baseShift = 5;

@@ -50,6 +50,9 @@ struct ScatterParams {
     int numChunks;    // ceil(rowBytes / chunkBytes)
     int stages;       // stages per copy engine (>= 2)
     int baseShift;    // tile_base has one row per 2^baseShift tokens (8: route_count tiles; 5: fused chunks)
+    const uint32_t* scales;  // [G][scaleWords] per-token scale rows, or nullptr
+    uint32_t* recv_scales;   // [W][maxRecv][scaleWords]
+    int scaleWords;          // 0: no scale rows
     // Only the fused dispatch (route + scan + scatter in one launch) uses these:
     const float* w;          // [G][k] or nullptr
     uint32_t* tok_mask_w;    // = tok_mask, written by the routing phase

@@ -344,6 +344,19 @@ __device__ __forceinline__ uint32_t token_slots_and_meta(const ScatterParams& p,
         if (lane < p.M) rec[lane] = v0;
         if (lane + 32 < p.M) rec[lane + 32] = (q1 == pe) ? e1 - pe * p.nEpr : -1;
     }
+    // The token's scale row travels with it to every destination.
+    if (p.scaleWords > 0) {
+        const uint32_t* src = p.scales + (size_t)g * p.scaleWords;
+        for (int w0 = 0; w0 < p.scaleWords; w0 += 32) {
+            const int wi = w0 + lane;
+            const uint32_t v = wi < p.scaleWords ? src[wi] : 0u;
+            for (uint32_t m = mask; m; m &= m - 1) {
+                const int pe = __ffs(m) - 1;
+                const int slot = __shfl_sync(kFull, my_slot, pe);
+                if (wi < p.scaleWords) p.recv_scales[((size_t)pe * p.maxRecv + slot) * p.scaleWords + wi] = v;
+            }
+        }
+    }
     return mask;
 }
 

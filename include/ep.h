@@ -176,6 +176,25 @@ int ep_plan_info(const EpPlan* plan, EpPlanInfo* info);
 int ep_dispatch(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
                 void* recv_x, int32_t* recv_meta, int32_t* recv_count, void* stream);
 
+/* Largest scale row of ep_dispatch_scaled, in 4-byte words. */
+#define EP_MAX_SCALE_WORDS 4096
+
+/*
+ * Dispatch with a per-token scale row (mori PR #599, its follow-up commits:
+ * the scale transport, a fourth per-token field carried with the payload, as
+ * quantized payloads need). Same as ep_dispatch, plus:
+ *   scales       [W][T][scaleWords]        4-byte words (e.g. float32 scales),
+ *                                          4-byte aligned; moved bit for bit
+ *   scaleWords   1..EP_MAX_SCALE_WORDS     (1: one scale per token; h/128 for
+ *                                          per-128-element block scales)
+ *   recv_scales  [W][maxRecv][scaleWords]  every received row gets its token's
+ *                                          scale row; rows past recv_count[pe]
+ *                                          are not written
+ */
+int ep_dispatch_scaled(EpPlan* plan, const void* x, const int32_t* topk_idx, const float* topk_w,
+                       const void* scales, int32_t scaleWords, void* recv_x, int32_t* recv_meta,
+                       void* recv_scales, int32_t* recv_count, void* stream);
+
 /*
  * Combine, enqueued on `stream`, using the routing of the most recent
  * ep_dispatch of this plan (stream order is the caller's: issue it on the same

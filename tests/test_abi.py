@@ -152,6 +152,9 @@ def test_entry_points_reject_without_crashing(ep):
     assert b._lib.ep_combine(None, None, None, None) == b.EP_ERR_INVALID
     assert b._lib.ep_plan_info(None, None) == b.EP_ERR_INVALID
     assert b._lib.ep_plan_check_error(None) == b.EP_ERR_INVALID
+    for words in (0, -1, b.EP_MAX_SCALE_WORDS + 1):
+        assert b._lib.ep_dispatch_scaled(None, None, None, None, None, words, None, None, None, None,
+                                         None) == b.EP_ERR_INVALID
     b._lib.ep_plan_destroy(None)
     with pytest.raises(ep.EpError):
         ep.ep_plan_create(_cfg(hiddenDim=7))

@@ -110,6 +110,43 @@ def test_dtype_main_dispatch(dtype, h):
         assert run.error_word() == 0
 
 
+def _check_scaled(cfg, inputs, sw, seed=7):
+    rng = np.random.default_rng(seed)
+    W, T = cfg["worldSize"], cfg["maxTokPerRank"]
+    scales = rng.standard_normal((W, T, sw)).astype(np.float32)
+    ref = oracle.dispatch(cfg, inputs["x"], inputs["topk_idx"], inputs.get("topk_w"), scales=scales)
+    with GpuRun(cfg, inputs) as run:
+        R = run.info.maxRecv
+        rs = torch.full((W, R, sw), 0x0C0FFEE, dtype=torch.int32, device="cuda")
+        ep.ep_dispatch_scaled(run.plan, run.x, run.idx, run.w, to_dev(scales), sw, run.recv_x,
+                              run.recv_meta, rs, run.recv_count, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        compare_dispatch(run, ref)
+        ref_s = torch.from_numpy(ref["recv_scales"].view(np.int32)).to("cuda")
+        for pe in range(W):
+            n = int(ref["recv_count"][pe])
+            assert torch.equal(rs[pe, :n], ref_s[pe, :n]), f"scale rows differ at pe {pe}"
+            assert bool((rs[pe, n:] == 0x0C0FFEE).all()), f"scale rows written past count at pe {pe}"
+        assert run.error_word() == 0
+
+
+@pytest.mark.parametrize("fused", ["0", "1"])
+@pytest.mark.parametrize("dtype,h,sw", [(2, 7168, 56), (0, 1024, 1), (3, 512, 33)],
+                         ids=["fp8-block-scales", "bf16-one-scale", "fp4x2-33-words"])
+def test_dispatch_scaled(dtype, h, sw, fused, monkeypatch):
+    """Per-token scale rows travel with the payload to every destination."""
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
+    wl = workload("pr599").replace(dtype=dtype, h=h)
+    _check_scaled(wl.cfg(), make_inputs(wl), sw)
+
+
+def test_dispatch_scaled_random_small():
+    rng = np.random.default_rng(31)
+    for case in range(6):
+        cfg, xb, idx, w = P.random_small_case(rng, dtype=case % 4)
+        _check_scaled(cfg, dict(x=xb, topk_idx=idx, topk_w=w), int(rng.integers(1, 80)), seed=case)
+
+
 def test_out_of_range_ids_reported_and_masked():
     rng = np.random.default_rng(5)
     cfg, inputs = _small_random_cfg(rng, 4, 64, 64, 4, 4, True, oob=True)
