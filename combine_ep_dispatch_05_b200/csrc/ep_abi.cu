@@ -310,8 +310,9 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             fused = false;
         if (fused) {
             int fPerSm = 0;
-            if ((e = ep::fused_set_smem(cfg->worldSize, smem)) != cudaSuccess ||
-                (e = ep::fused_blocks_per_sm(cfg->worldSize, geo.scatterWarps, smem, &fPerSm)) != cudaSuccess) {
+            if ((e = ep::fused_set_smem(cfg->worldSize, cfg->numExpertPerToken, smem)) != cudaSuccess ||
+                (e = ep::fused_blocks_per_sm(cfg->worldSize, cfg->numExpertPerToken, geo.scatterWarps, smem,
+                                             &fPerSm)) != cudaSuccess) {
                 cuda_fail(e, "fused dispatch set-up");
                 delete plan;
                 return nullptr;

@@ -121,8 +121,8 @@ cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int wa
 // Fused dispatch (route + scan + scatter), a cooperative launch: blocks must
 // not exceed the co-resident capacity (fused_blocks_per_sm * SMs).
 cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s);
-cudaError_t fused_set_smem(int W, size_t bytes);
-cudaError_t fused_blocks_per_sm(int W, int warps, size_t smem, int* out);
+cudaError_t fused_set_smem(int W, int topk, size_t bytes);
+cudaError_t fused_blocks_per_sm(int W, int topk, int warps, size_t smem, int* out);
 
 // Shared-memory bytes the scatter kernel needs for a geometry.
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride);

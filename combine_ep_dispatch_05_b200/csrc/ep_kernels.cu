@@ -166,8 +166,10 @@ __device__ __forceinline__ int source_next(TokenSource& s) {
 // block scans the histogram. kW = compile-time bound on W (8, 16 or 32).
 // =====================================================================
 // Destination mask and per-destination weight sums of token g (float32 fold
-// in topk order); ids < 0 are masked, ids >= E are reported and masked.
-template <int kW>
+// in topk order); ids < 0 are masked, ids >= E are reported and masked. kK
+// bounds k: all k ids and weights are loaded into registers first, so their
+// loads are in flight together.
+template <int kW, int kK>
 __device__ __forceinline__ uint32_t route_token(const int32_t* idx, const float* w, int g, int k, int nEpr,
                                                 int E, float (&ws)[kW], bool& bad) {
     uint32_t mask = 0;
@@ -175,9 +177,17 @@ __device__ __forceinline__ uint32_t route_token(const int32_t* idx, const float*
     for (int pe = 0; pe < kW; ++pe) ws[pe] = 0.0f;
     const int32_t* ids = idx + (size_t)g * k;
     const float* wts = w ? w + (size_t)g * k : nullptr;
-    for (int j = 0; j < k; ++j) {
-        const int e = ids[j];
-        if (e < 0) continue;  // masked entry
+    int e_j[kK];
+    float w_j[kK];
+#pragma unroll
+    for (int j = 0; j < kK; ++j) {
+        e_j[j] = j < k ? ids[j] : -1;
+        w_j[j] = (wts && j < k) ? wts[j] : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kK; ++j) {
+        const int e = e_j[j];
+        if (e < 0) continue;  // masked entry (or j >= k)
         if (e >= E) {         // contract violation: report, treat as masked
             bad = true;
             continue;
@@ -185,16 +195,15 @@ __device__ __forceinline__ uint32_t route_token(const int32_t* idx, const float*
         const int pe_j = e / nEpr;
         mask |= 1u << pe_j;
         if (wts) {
-            const float wj = wts[j];
 #pragma unroll
             for (int pe = 0; pe < kW; ++pe)
-                if (pe == pe_j) ws[pe] = ws[pe] + wj;  // fold in topk order
+                if (pe == pe_j) ws[pe] = ws[pe] + w_j[j];  // fold in topk order
         }
     }
     return mask;
 }
 
-template <int kW>
+template <int kW, int kK>
 __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams p) {
     __shared__ int s_wcnt[kCountWarps][kW];
     __shared__ int s_wpre[kCountWarps][kW];
@@ -210,7 +219,7 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     uint32_t mask = 0;
     bool bad = false;
     float ws[kW];
-    if (g < p.G) mask = route_token<kW>(p.idx, p.w, g, k, p.nEpr, p.E, ws, bad);
+    if (g < p.G) mask = route_token<kW, kK>(p.idx, p.w, g, k, p.nEpr, p.E, ws, bad);
     if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
 
     // Per-warp histogram by ballot.
@@ -261,17 +270,25 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     __threadfence();
     for (int pe = warp; pe < W; pe += kCountWarps) {
         int running = 0;
-        for (int t0 = 0; t0 < p.numTiles; t0 += 32) {
-            const int t = t0 + lane;
-            const int v = t < p.numTiles ? __ldcg(p.tile_cnt + (size_t)t * W + pe) : 0;
-            int incl = v;
+        for (int t0 = 0; t0 < p.numTiles; t0 += 32 * 8) {
+            int v[8];  // 8 rows of 32 tiles: all loads in flight before the scans
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int n = __shfl_up_sync(kFull, incl, off);
-                if (lane >= off) incl += n;
+            for (int u = 0; u < 8; ++u) {
+                const int t = t0 + 32 * u + lane;
+                v[u] = t < p.numTiles ? __ldcg(p.tile_cnt + (size_t)t * W + pe) : 0;
             }
-            if (t < p.numTiles) p.tile_base[(size_t)t * W + pe] = running + incl - v;
-            running += __shfl_sync(kFull, incl, 31);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int t = t0 + 32 * u + lane;
+                int incl = v[u];
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int n = __shfl_up_sync(kFull, incl, off);
+                    if (lane >= off) incl += n;
+                }
+                if (t < p.numTiles) p.tile_base[(size_t)t * W + pe] = running + incl - v[u];
+                running += __shfl_sync(kFull, incl, 31);
+            }
         }
         if (lane == 0) {
             p.recv_count[pe] = running;  // stored, not accumulated
@@ -585,7 +602,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned target) {
     return __syncthreads_and(ok) != 0;
 }
 
-template <int kW>
+template <int kW, int kK>
 __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kernel(ScatterParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -601,7 +618,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kerne
         uint32_t mask = 0;
         bool bad = false;
         float ws[kW];
-        if (g < p.G) mask = route_token<kW>(p.idx, p.w, g, p.k, p.nEpr, p.E, ws, bad);
+        if (g < p.G) mask = route_token<kW, kK>(p.idx, p.w, g, p.k, p.nEpr, p.E, ws, bad);
         if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
         if (g < p.G) p.tok_mask_w[g] = mask;
         int my_cnt = 0;
@@ -870,14 +887,19 @@ cudaError_t launch_pdl(void (*kernel)(P), int grid, int block, size_t smem, cuda
 }
 }  // namespace
 
+// Instances by bounds on W and k (8, 16 or 32 each).
 cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s) {
+    auto go = [&](auto kernel) { return launch_pdl(kernel, p.numTiles, kCountTile, 0, s, p); };
     cudaError_t e;
     if (p.W <= 8)
-        e = launch_pdl(ep_route_count_kernel<8>, p.numTiles, kCountTile, 0, s, p);
+        e = p.k <= 8 ? go(ep_route_count_kernel<8, 8>) : p.k <= 16 ? go(ep_route_count_kernel<8, 16>)
+                                                                : go(ep_route_count_kernel<8, 32>);
     else if (p.W <= 16)
-        e = launch_pdl(ep_route_count_kernel<16>, p.numTiles, kCountTile, 0, s, p);
+        e = p.k <= 8 ? go(ep_route_count_kernel<16, 8>) : p.k <= 16 ? go(ep_route_count_kernel<16, 16>)
+                                                                 : go(ep_route_count_kernel<16, 32>);
     else
-        e = launch_pdl(ep_route_count_kernel<32>, p.numTiles, kCountTile, 0, s, p);
+        e = p.k <= 8 ? go(ep_route_count_kernel<32, 8>) : p.k <= 16 ? go(ep_route_count_kernel<32, 16>)
+                                                                 : go(ep_route_count_kernel<32, 32>);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -940,27 +962,32 @@ cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int 
 
 namespace {
 template <typename F>
-cudaError_t for_world(int W, F&& f) {
-    if (W <= 8) return f(ep_dispatch_fused_kernel<8>);
-    if (W <= 16) return f(ep_dispatch_fused_kernel<16>);
-    return f(ep_dispatch_fused_kernel<32>);
+cudaError_t for_world(int W, int k, F&& f) {
+    if (W <= 8)
+        return k <= 8 ? f(ep_dispatch_fused_kernel<8, 8>) : k <= 16 ? f(ep_dispatch_fused_kernel<8, 16>)
+                                                             : f(ep_dispatch_fused_kernel<8, 32>);
+    if (W <= 16)
+        return k <= 8 ? f(ep_dispatch_fused_kernel<16, 8>) : k <= 16 ? f(ep_dispatch_fused_kernel<16, 16>)
+                                                              : f(ep_dispatch_fused_kernel<16, 32>);
+    return k <= 8 ? f(ep_dispatch_fused_kernel<32, 8>) : k <= 16 ? f(ep_dispatch_fused_kernel<32, 16>)
+                                                          : f(ep_dispatch_fused_kernel<32, 32>);
 }
 }  // namespace
 
-cudaError_t fused_set_smem(int W, size_t bytes) {
-    return for_world(W, [&](auto k) {
+cudaError_t fused_set_smem(int W, int topk, size_t bytes) {
+    return for_world(W, topk, [&](auto k) {
         return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     });
 }
 
-cudaError_t fused_blocks_per_sm(int W, int warps, size_t smem, int* out) {
-    return for_world(W, [&](auto k) {
+cudaError_t fused_blocks_per_sm(int W, int topk, int warps, size_t smem, int* out) {
+    return for_world(W, topk, [&](auto k) {
         return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, warps * 32, smem);
     });
 }
 
 cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s) {
-    cudaError_t e = for_world(p.W, [&](auto k) {
+    cudaError_t e = for_world(p.W, p.k, [&](auto k) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(blocks);
         cfg.blockDim = dim3(warps * 32);
