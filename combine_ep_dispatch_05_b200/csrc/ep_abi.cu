@@ -38,6 +38,7 @@ struct EpPlan {
     int32_t* err;
     size_t scatterSmem;
     bool fused;           // route + scan + scatter in one cooperative launch
+    unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
     bool dispatched;
 };
 
@@ -324,6 +325,11 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         }
         plan->fused = fused;
         plan->info.dispatchFused = fused ? 1 : 0;
+        // Test hook for the failure path: the fused dispatch's grid barrier can
+        // never complete, so every block gives up after its bounded wait and
+        // reports EP_DEVERR_TIMEOUT (no copy is issued).
+        if (const char* t = std::getenv("EP_TEST_UNREACHABLE_BARRIER"))
+            plan->barrierSlack = std::strcmp(t, "1") == 0 ? 1u : 0u;
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
@@ -494,6 +500,7 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
             sp.done = plan->fdone;
             sp.numChunks32 = (plan->G + 31) / 32;
             sp.useWeights = c.useWeights;
+            sp.barrierSlack = plan->barrierSlack;
             e = ep::launch_dispatch_fused(sp, plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
             if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_fused");
             plan->dispatched = true;

@@ -63,6 +63,7 @@ struct ScatterParams {
     unsigned* done;          // blocks finished; the last one resets bar, work, done
     int numChunks32;         // ceil(G / 32)
     int useWeights;
+    unsigned barrierSlack;   // 0; 1 makes the first grid barrier unreachable (tests of the timeout path)
 };
 
 struct CombineParams {

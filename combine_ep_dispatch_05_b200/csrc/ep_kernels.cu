@@ -637,7 +637,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kerne
         if (lane < W) p.chunk_cnt[(size_t)c * W + lane] = my_cnt;
     }
 
-    bool ok = grid_barrier(p.bar, gridDim.x);
+    bool ok = grid_barrier(p.bar, gridDim.x + p.barrierSlack);
 
     // 2. one warp per destination scans the chunk counts
     for (int pe = gw; ok && pe < W; pe += nW) {
@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kerne
         }
     }
 
-    ok = ok && grid_barrier(p.bar, 2u * gridDim.x);
+    ok = ok && grid_barrier(p.bar, 2u * gridDim.x + p.barrierSlack);
 
     // 3. copy engines
     if (ok) copy_engine<1>(p, es, lane, warp, nwarps);

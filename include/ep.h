@@ -143,7 +143,11 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * Environment overrides, read here only (for geometry sweeps):
  * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK,
  * EP_SCATTER_PEND (1..3), EP_SCATTER_MODE ("tma" or "regs"), EP_COMBINE_BLOCKS,
- * EP_COMBINE_WARPS, EP_DISPATCH_FUSED (0: two launches instead of one). */
+ * EP_COMBINE_WARPS, EP_DISPATCH_FUSED (1: one cooperative launch instead of
+ * two). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 (with EP_DISPATCH_FUSED=1)
+ * makes the fused dispatch's grid barrier unreachable, so that its bounded
+ * wait runs out: every block reports EP_DEVERR_TIMEOUT, issues no copy and
+ * returns about one second later, and the context stays usable. */
 EpPlan* ep_plan_create(const EpCfg* cfg);
 
 /* Free the plan and its scratch. NULL is a no-op. The caller must make sure no

@@ -275,6 +275,26 @@ def test_geometry_overrides(env, monkeypatch):
     run.close()
 
 
+def test_bounded_wait_runs_out_and_reports(monkeypatch):
+    """Failure detection without a GPU fault: a grid barrier that nothing can
+    complete (test hook) makes every block give up after its bounded wait;
+    the host reads EP_DEVERR_TIMEOUT from the error word, and the context and
+    a fresh plan keep working."""
+    monkeypatch.setenv("EP_DISPATCH_FUSED", "1")
+    monkeypatch.setenv("EP_TEST_UNREACHABLE_BARRIER", "1")
+    wl = workload("latency8")
+    inputs = make_inputs(wl)
+    with GpuRun(wl.cfg(), inputs) as run:
+        assert run.info.dispatchFused == 1
+        run.dispatch()
+        err = run.error_word()  # synchronises: the kernel has returned
+        assert err & ep.EP_DEVERR_TIMEOUT
+        assert bool((run.recv_x == 0xAB).all())  # no copy was issued
+    monkeypatch.delenv("EP_TEST_UNREACHABLE_BARRIER")
+    run, _ = run_and_compare(wl.cfg(), inputs)  # the device is healthy
+    run.close()
+
+
 def test_host_side_rejections():
     wl = workload("tiny")
     with GpuRun(wl.cfg(), make_inputs(wl)) as run:
