@@ -39,6 +39,7 @@ struct EpPlan {
     size_t scatterSmem;
     bool fused;           // route + scan + scatter in one cooperative launch
     unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
+    int fanoutSwitch;       // x100, see ScatterParams
     bool dispatched;
 };
 
@@ -121,11 +122,13 @@ struct Geometry {
     int combineWarps;
 };
 
-// Copy engines and stages: two engines (warps) per block, each with as many
-// row-sized stages as fit in about 200 KB of shared memory (at most 8; rows
-// above 32 KB are copied in pieces of <= 16 KB). On B200 at 14 KB rows, 2
-// engines x 6 stages per SM beat 4 x 3, 3 x 4 and 6 x 2 (deeper per-engine
-// lookahead) and 1 x 12 (one issuing thread per SM is too few).
+// Copy engines and stages: three engines (warps) per block for rows of 8 KB
+// and more, two otherwise, each with as many row-sized stages as fit in about
+// 215 KB of shared memory (at most 8; two engines when fewer than 4 stages
+// would fit; rows above 32 KB are copied in pieces of <= 16 KB). On B200 at
+// 14 KB rows, 3 x 5 with one engine sitting out at a high fan-out matches 2 x 7
+// on uniform routing (472 us) and beats it by 12% on skewed routing (295 vs
+// 335 us); 1 x 14 is far slower (one issuing thread per SM).
 Geometry pick_geometry(const EpCfg* c, bool use_env) {
     Geometry g{};
     const long long rowBytes = (long long)c->hiddenDim * payload_size(c->dtype);
@@ -141,9 +144,15 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
     g.chunkBytes = chunk;
     g.chunkStride = (chunk + 127) & ~127;
     g.numChunks = (int)((rowBytes + chunk - 1) / chunk);
-    const int budget = 200 * 1024;
-    int warps = 2;
+    const int budget = 215 * 1024;
+    // Rows of 8 KB and more: a third engine, which sits out at a high fan-out
+    // (see copy_engine). Smaller rows already give several blocks per SM.
+    int warps = g.chunkStride >= 8192 ? 3 : 2;
     int stages = budget / (warps * g.chunkStride);
+    if (stages < 4) {
+        warps = 2;
+        stages = budget / (warps * g.chunkStride);
+    }
     if (stages < 2) {
         warps = std::max(1, budget / (2 * g.chunkStride));
         stages = 2;
@@ -325,6 +334,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         }
         plan->fused = fused;
         plan->info.dispatchFused = fused ? 1 : 0;
+        plan->fanoutSwitch = env_int("EP_SCATTER_FANOUT_SWITCH", 375);
         // Test hook for the failure path: the fused dispatch's grid barrier can
         // never complete, so every block gives up after its bounded wait and
         // reports EP_DEVERR_TIMEOUT (no copy is issued).
@@ -484,6 +494,8 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         sp.chunkStride = (sp.chunkBytes + 127) & ~127;
         sp.numChunks = (int)((sp.rowBytes + sp.chunkBytes - 1) / sp.chunkBytes);
         sp.stages = plan->info.scatterStages;
+        sp.recv_count = recv_count;
+        sp.fanoutSwitch = plan->fanoutSwitch;
         sp.scales = static_cast<const uint32_t*>(scales);
         sp.recv_scales = static_cast<uint32_t*>(recv_scales);
         sp.scaleWords = scaleWords;

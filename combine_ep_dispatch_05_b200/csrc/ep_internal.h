@@ -50,6 +50,7 @@ struct ScatterParams {
     int numChunks;    // ceil(rowBytes / chunkBytes)
     int stages;       // stages per copy engine (>= 2)
     int baseShift;    // tile_base has one row per 2^baseShift tokens (8: route_count tiles; 5: fused chunks)
+    int fanoutSwitch;        // x100: above this mean fan-out (rows per token) one engine per block sits out (0: never)
     const uint32_t* scales;  // [G][scaleWords] per-token scale rows, or nullptr
     uint32_t* recv_scales;   // [W][maxRecv][scaleWords]
     int scaleWords;          // 0: no scale rows
