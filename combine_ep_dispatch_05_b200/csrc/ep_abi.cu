@@ -40,6 +40,7 @@ struct EpPlan {
     bool fused;           // route + scan + scatter in one cooperative launch
     unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
     int fanoutSwitch;       // x100, see ScatterParams
+    int combineTile;        // combine kernel instance
     bool dispatched;
 };
 
@@ -119,7 +120,7 @@ struct Geometry {
     int chunkBytes, chunkStride, numChunks;
     int scatterMode, scatterPend;
     int scatterWarps, scatterStages;
-    int combineWarps;
+    int combineWarps, combineTile;
 };
 
 // Copy engines and stages: three engines (warps) per block for rows of 8 KB
@@ -179,6 +180,9 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
     g.scatterWarps = warps;
     g.scatterStages = stages;
     g.combineWarps = use_env ? std::min(env_int("EP_COMBINE_WARPS", 8), ep::kMaxCombineWarps) : 8;
+    g.combineTile = 0;
+    if (use_env)
+        if (const char* t = std::getenv("EP_COMBINE_TILE")) g.combineTile = std::max(0, std::min(std::atoi(t), 3));
     return g;
 }
 
@@ -288,7 +292,8 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         int sPerSm = 0, cPerSm = 0;
         if ((e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps, smem,
                                            &sPerSm)) != cudaSuccess ||
-            (e = ep::combine_blocks_per_sm(geo.combineWarps, cfg->dtype == EP_FP32, &cPerSm)) != cudaSuccess) {
+            (e = ep::combine_blocks_per_sm(geo.combineWarps, cfg->dtype == EP_FP32, geo.combineTile, &cPerSm)) !=
+                cudaSuccess) {
             cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
             return nullptr;
         }
@@ -335,6 +340,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->fused = fused;
         plan->info.dispatchFused = fused ? 1 : 0;
         plan->fanoutSwitch = env_int("EP_SCATTER_FANOUT_SWITCH", 375);
+        plan->combineTile = geo.combineTile;
         // Test hook for the failure path: the fused dispatch's grid barrier can
         // never complete, so every block gives up after its bounded wait and
         // reports EP_DEVERR_TIMEOUT (no copy is issued).
@@ -548,8 +554,9 @@ int ep_combine(EpPlan* plan, const void* y, void* out, void* stream) {
         cp.G = plan->G;
         cp.W = plan->cfg.worldSize;
         cp.maxRecv = plan->maxRecv;
-        cudaError_t e = ep::launch_combine(cp, plan->info.combineDtype == EP_FP32, plan->info.combineBlocks,
-                                           plan->info.combineWarps, static_cast<cudaStream_t>(stream));
+        cudaError_t e = ep::launch_combine(cp, plan->info.combineDtype == EP_FP32, plan->combineTile,
+                                           plan->info.combineBlocks, plan->info.combineWarps,
+                                           static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_fail(e, "launch combine");
         return EP_OK;
     } catch (...) {

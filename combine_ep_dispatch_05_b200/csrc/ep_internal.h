@@ -15,7 +15,7 @@ constexpr int kCountWarps = kCountTile / 32;
 constexpr int kMaxWorld = 32;   // one destination bit per lane of a 32-bit mask
 constexpr int kMaxTopk = 32;    // one topk entry per lane
 constexpr int kMaxScatterWarps = 16;
-constexpr int kMaxCombineWarps = 16;
+constexpr int kMaxCombineWarps = 8;
 // Bounded waits give up after this many SM clock cycles (about 1 s at 1.9 GHz).
 constexpr long long kWaitCycles = 2000000000LL;
 
@@ -119,7 +119,8 @@ constexpr int kScatterRegs = 1;
 cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
                                 size_t smem, cudaStream_t s);
 // fp32: float32 combine leg (an fp32 plan); bf16 otherwise.
-cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s);
+// tile: combine kernel instance (columns x rows per pass, blocks per SM), see ep_kernels.cu.
+cudaError_t launch_combine(const CombineParams& p, bool fp32, int tile, int blocks, int warps, cudaStream_t s);
 // Fused dispatch (route + scan + scatter), a cooperative launch: blocks must
 // not exceed the co-resident capacity (fused_blocks_per_sm * SMs).
 cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s);
@@ -132,7 +133,7 @@ size_t scatter_smem_bytes(int warps, int stages, int chunkStride);
 cudaError_t scatter_set_smem(int pend, size_t bytes);
 // Blocks of each kernel that fit on one SM (occupancy calculator).
 cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out);
-cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out);
+cudaError_t combine_blocks_per_sm(int warps, bool fp32, int tile, int* out);
 // Current dynamic shared-memory limit of the TMA scatter kernel.
 cudaError_t scatter_get_smem(int pend, int* bytes);
 // Replace this thread's ep_last_error() text.

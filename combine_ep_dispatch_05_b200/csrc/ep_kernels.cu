@@ -128,8 +128,8 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
 // rest, about the last eighth of the tokens, one at a time from a global
 // counter, so that workers whose tokens had more destinations do not leave a
 // tail (the spread of a worker's total over ~100 tokens is a few percent).
-// With fewer than two tokens per worker the split is static only (no counter
-// traffic at all).
+// With fewer than eight tokens per worker the split is static only: the
+// counter would put thousands of atomics on one address for little balance.
 // =====================================================================
 struct TokenSource {
     int w, nU, R, G, i;
@@ -144,7 +144,7 @@ __device__ __forceinline__ TokenSource make_source(int w, int nU, int G, int32_t
     s.G = G;
     s.i = 0;
     s.ctr = ctr;
-    s.dyn = G >= 2 * nU;
+    s.dyn = G >= 8 * nU;
     s.R = s.dyn ? max(0, (int)((7LL * G) / (8LL * nU)) - 1) : (G + nU - 1) / nU;
     return s;
 }
@@ -742,8 +742,6 @@ __global__ void __launch_bounds__(256) ep_scatter_rows_regs_kernel(ScatterParams
 // =====================================================================
 // combine: one warp per token, 16-byte columns, fma fold in destPe order.
 // =====================================================================
-constexpr int kCombineBatch = 8;  // destination rows in flight per column
-constexpr int kCombineUnroll = 2; // columns per lane per iteration
 
 __device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) {
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -788,8 +786,53 @@ struct CombineF32 {
     }
 };
 
-template <class Elem>
-__global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(CombineParams p) {
+// One token's output row: for each group of kU 16-byte columns per lane, the
+// loads of up to kB destination rows are issued together, then folded in
+// destination order (so the result does not depend on kU or kB).
+template <class Elem, int kU, int kB>
+__device__ __forceinline__ void combine_columns(const uint8_t* const* rows, const float* wts, int n, uint4* orow,
+                                                int V, int lane) {
+    for (int v0 = lane; v0 < V; v0 += 32 * kU) {
+        float acc[kU][Elem::kPer];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+#pragma unroll
+            for (int i = 0; i < Elem::kPer; ++i) acc[u][i] = 0.0f;
+        for (int b = 0; b < n; b += kB) {
+            uint4 val[kU][kB];
+#pragma unroll
+            for (int i = 0; i < kB; ++i) {
+                if (b + i < n) {
+                    const uint8_t* row = rows[b + i];
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        const int v = v0 + 32 * u;
+                        if (v < V) val[u][i] = ld_stream_v4(row + (size_t)v * 16);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kB; ++i) {
+                if (b + i < n) {
+                    const float w = wts[b + i];
+#pragma unroll
+                    for (int u = 0; u < kU; ++u)
+                        if (v0 + 32 * u < V) Elem::fma(acc[u], w, val[u][i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < V) orow[v] = Elem::pack(acc[u]);
+        }
+    }
+}
+
+// kCols x kRows loads in flight per lane and pass; kMinBlocks blocks of 256
+// threads per SM bound the registers (65536 / (256 * kMinBlocks)).
+template <class Elem, int kCols, int kRows, int kMinBlocks>
+__global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_kernel(CombineParams p) {
     __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
     __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
     pdl_wait();  // y and the routing of the dispatch are visible from here on
@@ -829,46 +872,14 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32) ep_combine_kernel(Combi
         }
         __syncwarp();
 
-        for (int v0 = lane; v0 < V; v0 += 32 * kCombineUnroll) {
-            float acc[kCombineUnroll][Elem::kPer];
-#pragma unroll
-            for (int u = 0; u < kCombineUnroll; ++u)
-#pragma unroll
-                for (int i = 0; i < Elem::kPer; ++i) acc[u][i] = 0.0f;
-            for (int b = 0; b < n; b += kCombineBatch) {
-                uint4 val[kCombineUnroll][kCombineBatch];
-#pragma unroll
-                for (int i = 0; i < kCombineBatch; ++i) {
-                    if (b + i < n) {
-                        const uint8_t* row = s_row[warp][b + i];
-#pragma unroll
-                        for (int u = 0; u < kCombineUnroll; ++u) {
-                            const int v = v0 + 32 * u;
-                            if (v < V) val[u][i] = ld_stream_v4(row + (size_t)v * 16);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < kCombineBatch; ++i) {
-                    if (b + i < n) {
-                        const float w = s_w[warp][b + i];
-#pragma unroll
-                        for (int u = 0; u < kCombineUnroll; ++u)
-                            if (v0 + 32 * u < V) Elem::fma(acc[u], w, val[u][i]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kCombineUnroll; ++u) {
-                const int v = v0 + 32 * u;
-                if (v < V) orow[v] = Elem::pack(acc[u]);
-            }
-        }
+        combine_columns<Elem, kCols, kRows>(s_row[warp], s_w[warp], n, orow, V, lane);
         __syncwarp();
         g = g_next;
     }
 
-    // The last block to finish resets the counter for the next combine.
+    // The last block to finish resets the counter for the next combine (only
+    // needed when the hand-out used it: the same for every block of a launch).
+    if (!src.dyn) return;
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -958,10 +969,23 @@ cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, in
     });
 }
 
-cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out) {
-    if (fp32)
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_combine_kernel<CombineF32>, warps * 32, 0);
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_combine_kernel<CombineBf16>, warps * 32, 0);
+namespace {
+// Combine kernel instances: tile 0 = 2 columns x 8 rows (2 blocks/SM),
+// 1 = 2 x 4 (4 blocks/SM), 2 = 1 x 8 (4 blocks/SM), 3 = 2 x 4 (3 blocks/SM).
+template <class Elem, typename F>
+cudaError_t for_tile(int tile, F&& f) {
+    switch (tile) {
+        case 1: return f(ep_combine_kernel<Elem, 2, 4, 4>);
+        case 2: return f(ep_combine_kernel<Elem, 1, 8, 4>);
+        case 3: return f(ep_combine_kernel<Elem, 2, 4, 3>);
+        default: return f(ep_combine_kernel<Elem, 2, 8, 2>);
+    }
+}
+}  // namespace
+
+cudaError_t combine_blocks_per_sm(int warps, bool fp32, int tile, int* out) {
+    auto occ = [&](auto k) { return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, warps * 32, 0); };
+    return fp32 ? for_tile<CombineF32>(tile, occ) : for_tile<CombineBf16>(tile, occ);
 }
 
 cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
@@ -1017,9 +1041,9 @@ cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps,
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s) {
-    cudaError_t e = fp32 ? launch_pdl(ep_combine_kernel<CombineF32>, blocks, warps * 32, 0, s, p)
-                         : launch_pdl(ep_combine_kernel<CombineBf16>, blocks, warps * 32, 0, s, p);
+cudaError_t launch_combine(const CombineParams& p, bool fp32, int tile, int blocks, int warps, cudaStream_t s) {
+    auto go = [&](auto k) { return launch_pdl(k, blocks, warps * 32, 0, s, p); };
+    cudaError_t e = fp32 ? for_tile<CombineF32>(tile, go) : for_tile<CombineBf16>(tile, go);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
