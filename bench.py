@@ -54,6 +54,8 @@ def parse():
                          "fp4x2 halves hiddenDim, which then counts bytes of packed pairs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the hot-L2 timing of back-to-back calls in CUDA graphs")
     ap.add_argument("--flush", default="read", choices=["read", "write"],
                     help="L2 flush between timed steps: read a 256 MB buffer (leaves L2 clean) "
                          "or write it (leaves L2 full of dirty lines)")
@@ -278,6 +280,65 @@ def run_reference(args, wl):
 
 
 # ------------------------------------------------------------------ our arm
+def dispatch_kernels(info) -> str:
+    """The kernels one dispatch of this plan launches."""
+    if info.dispatchLowLatency:
+        return "ep_dispatch_ll (one launch)"
+    if info.dispatchFused:
+        return "ep_dispatch_fused (one cooperative launch)"
+    return "ep_dispatch (route_count + scatter_rows)"
+
+
+def dispatch_launches(info) -> int:
+    return 1 if (info.dispatchLowLatency or info.dispatchFused) else 2
+
+
+GRAPH_CALLS = 20   # calls captured back to back in one CUDA graph
+GRAPH_ROUNDS = 10  # timed replays of each graph, interleaved
+
+
+def time_graphs(calls: dict, dev, dist) -> dict:
+    """Hot-L2 device time per call. Each entry of ``calls`` (a function of the
+    stream) is captured GRAPH_CALLS times back to back in one CUDA graph. The
+    graphs are replayed in turn, GRAPH_ROUNDS timed rounds after two untimed
+    ones, each replay bracketed by CUDA events on its stream; the result is the
+    median replay ÷ GRAPH_CALLS (max over ranks). Launch overhead is left out
+    and consecutive calls may overlap through programmatic dependent launch,
+    so this is the per-call cost of a steady stream of calls."""
+    import torch
+    cs = torch.cuda.Stream(dev)
+    cs.wait_stream(torch.cuda.current_stream(dev))
+    graphs = {}
+    for name, fn in calls.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cs):
+            with torch.cuda.graph(g, stream=cs):
+                for _ in range(GRAPH_CALLS):
+                    fn(cs)
+        graphs[name] = g
+    times = {name: [] for name in graphs}
+    with torch.cuda.stream(cs):
+        for r in range(GRAPH_ROUNDS + 2):
+            for name, g in graphs.items():
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(cs)
+                g.replay()
+                e1.record(cs)
+                if r >= 2:
+                    times[name].append((e0, e1))
+    torch.cuda.synchronize(dev)
+    res = {}
+    for name, evs in times.items():
+        med = statistics.median(a.elapsed_time(b) for a, b in evs) / GRAPH_CALLS
+        res[name + "_us"] = max_over_ranks(med, dist, dev) * 1e3
+    for g in graphs.values():
+        del g
+    graphs.clear()
+    res.update({"calls_per_graph": GRAPH_CALLS, "rounds": GRAPH_ROUNDS, "l2": "hot (no flush)",
+                "statistic": "median replay / calls"})
+    return res
+
+
 def run_ours(args, wl):
     import torch
     rank, world, local, dist = dist_setup(args.gpus)
@@ -366,6 +427,18 @@ def run_ours(args, wl):
     if err:
         raise RuntimeError(f"device error word {err} after the timed steps")
 
+    graph = None
+    if not args.no_graph:
+        graph = time_graphs({
+            "dispatch": lambda st: ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, st),
+            "combine": lambda st: ep.ep_combine(plan, y, out, st),
+            "pair": lambda st: (ep.ep_dispatch(plan, x, idx, w, recv_x, recv_meta, recv_count, st),
+                                ep.ep_combine(plan, y, out, st)),
+        }, dev, dist)
+        err = ep.ep_plan_check_error(plan)
+        if err:
+            raise RuntimeError(f"device error word {err} after the graph timing")
+
     # Algorithmic bytes from the actual routing.
     counts = recv_count.cpu().numpy()
     U = int(counts.sum())
@@ -378,8 +451,7 @@ def run_ours(args, wl):
     if comb_ms_max >= disp_ms_max:
         dom = {"kernel": "ep_combine_kernel", "bytes": cb, "ms": comb_ms_max, "gbs": c_gbs}
     else:
-        dom = {"kernel": "ep_dispatch (route_count + scatter_rows)", "bytes": db, "ms": disp_ms_max,
-               "gbs": d_gbs}
+        dom = {"kernel": dispatch_kernels(info), "bytes": db, "ms": disp_ms_max, "gbs": d_gbs}
     traffic = ncu_traffic("ep_combine_kernel" if dom["kernel"] == "ep_combine_kernel" else "ep_dispatch", wl.name)
 
     # End to end: every step copies its inputs from pinned host memory to the
@@ -476,8 +548,9 @@ def run_ours(args, wl):
             "roofline_all": {
                 "dispatch": {"achieved": d_gbs, "frac": d_gbs / peak, "bytes": db, "us": disp_ms_max * 1e3},
                 "combine": {"achieved": c_gbs, "frac": c_gbs / peak, "bytes": cb, "us": comb_ms_max * 1e3}},
+            "graph_hot": graph,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
-            "gpu_launches": 3 * args.steps, "timed_wall_s": t_wall,
+            "gpu_launches": (dispatch_launches(info) + 1) * args.steps, "timed_wall_s": t_wall,
             "geometry": info.as_dict(), "impl": "ours",
         }
         print(json.dumps(line), flush=True)

@@ -38,6 +38,16 @@ struct EpPlan {
     int32_t* err;
     size_t scatterSmem;
     bool fused;           // route + scan + scatter in one cooperative launch
+    bool ll;              // small-batch single launch (dispatch_ll)
+    size_t llSmem;        // its dynamic shared memory
+    int llTile;           // its tokens per block
+    unsigned* ll_status;  // its scratch: tile status words, tile counts, present list, counters
+    int32_t* ll_agg;
+    int32_t* ll_plist;
+    unsigned long long* ll_ptotal;
+    int32_t* ll_ticket;
+    unsigned* ll_done;
+    unsigned* ll_epoch;
     unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
     int fanoutSwitch;       // x100, see ScatterParams
     int combineTile;        // combine kernel instance
@@ -61,12 +71,13 @@ int cuda_fail(cudaError_t e, const char* what) {
                 cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-int env_int(const char* name, int dflt) {
+// An integer from the environment in [lo, 2^30), else dflt.
+int env_int(const char* name, int dflt, int lo = 1) {
     const char* v = std::getenv(name);
     if (!v || !*v) return dflt;
     char* end = nullptr;
     long x = std::strtol(v, &end, 10);
-    return (end && *end == '\0' && x > 0 && x < (1 << 30)) ? (int)x : dflt;
+    return (end && *end == '\0' && x >= lo && x < (1 << 30)) ? (int)x : dflt;
 }
 
 // Bytes of one dispatched element (design page §3.7: the dtype is a property of
@@ -186,6 +197,35 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
     return g;
 }
 
+// Plans of at most EP_LL_MAX_TOKENS tokens per rank (the design page's
+// internode dispatch switches to its low-latency family at 512 tokens a
+// launch) may take the single-launch low-latency dispatch (dispatch_ll); a
+// tile (a block's tokens) must fit one block's threads. It is off by default
+// (kLlDefaultMaxTokens = 0): on B200 it measured no faster than route_count +
+// scatter_rows, whose launch boundary programmatic dependent launch already
+// hides (ct = 1 workload: 19.5 vs 17.4 us; the 512-token workload: 32.9 vs
+// 33.8 us), since its own handoffs cost as many dependent memory round trips.
+constexpr int kLlDefaultMaxTokens = 0;
+
+// Returns the stages per copy engine of the low-latency dispatch that fit
+// `smemOptin` (the shared memory in *smem, the tile in *tile), or 0 when the
+// plan does not take it.
+int ll_stages(const EpCfg* c, const Geometry& geo, bool fused, int blocks, size_t smemOptin, size_t* smem,
+              int* tile) {
+    const long long G = (long long)c->worldSize * c->maxTokPerRank;
+    const int llMax = env_int("EP_LL_MAX_TOKENS", kLlDefaultMaxTokens, 0);
+    if (fused || geo.scatterMode != ep::kScatterTma || geo.scatterPend != 1 || geo.scatterWarps > ep::kLlWarps ||
+        c->maxTokPerRank > llMax || blocks < 1)
+        return 0;
+    *tile = ep::ll_tile_tokens(G, blocks);
+    if (*tile > ep::kLlThreads) return 0;
+    for (int st = geo.scatterStages; st >= 2; --st) {
+        *smem = ep::ll_smem_bytes(*tile, c->worldSize, geo.scatterWarps, st, geo.chunkStride);
+        if (*smem <= smemOptin) return st;
+    }
+    return 0;
+}
+
 void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
     std::memset(info, 0, sizeof *info);
     const long long G = (long long)c->worldSize * c->maxTokPerRank;
@@ -245,6 +285,15 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info) {
                                                                    geo.scatterWarps, std::max(geo.scatterStages, 1),
                                                                    geo.chunkStride));
         info->combineBlocks = sms * 2;
+        size_t llSmem = 0;
+        int llTile = 0;
+        const int llStages = ll_stages(cfg, geo, false, sms, 227 * 1024 - 4096, &llSmem, &llTile);
+        if (llStages > 0) {
+            const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
+            info->dispatchLowLatency = 1;
+            info->scatterBlocks = (int)((G + llTile - 1) / llTile);
+            info->scatterStages = llStages;
+        }
         return EP_OK;
     } catch (...) {
         return fail(EP_ERR_INVALID, "unexpected exception");
@@ -339,11 +388,43 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         }
         plan->fused = fused;
         plan->info.dispatchFused = fused ? 1 : 0;
-        plan->fanoutSwitch = env_int("EP_SCATTER_FANOUT_SWITCH", 375);
+        // Small batches: the single-launch low-latency dispatch (ll_stages).
+        // The kernel's static shared memory (under 4 KB) comes on top.
+        plan->ll = false;
+        plan->llSmem = 0;
+        plan->llTile = 0;
+        {
+            const int llBlocks = std::max(1, env_int("EP_SCATTER_BLOCKS", sms));
+            size_t llSmem = 0;
+            int llTile = 0;
+            const int llStages =
+                ll_stages(cfg, geo, fused, llBlocks, (size_t)smemOptin - 4096, &llSmem, &llTile);
+            if (llStages > 0) {
+                int per = 0;
+                if ((e = ep::ll_set_smem(cfg->worldSize, cfg->numExpertPerToken, llSmem)) != cudaSuccess ||
+                    (e = ep::ll_blocks_per_sm(cfg->worldSize, cfg->numExpertPerToken, llSmem, &per)) !=
+                        cudaSuccess) {
+                    cuda_fail(e, "low-latency dispatch set-up");
+                    delete plan;
+                    return nullptr;
+                }
+                if (per >= 1) {
+                    const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
+                    plan->ll = true;
+                    plan->llSmem = llSmem;
+                    plan->llTile = llTile;
+                    plan->info.scatterBlocks = (int)((G + llTile - 1) / llTile);
+                    plan->info.scatterStages = llStages;
+                }
+            }
+        }
+        plan->info.dispatchLowLatency = plan->ll ? 1 : 0;
+        plan->fanoutSwitch = env_int("EP_SCATTER_FANOUT_SWITCH", 375, 0);
         plan->combineTile = geo.combineTile;
-        // Test hook for the failure path: the fused dispatch's grid barrier can
-        // never complete, so every block gives up after its bounded wait and
-        // reports EP_DEVERR_TIMEOUT (no copy is issued).
+        // Test hook for the failure path: the fused dispatch's grid barrier,
+        // or the low-latency dispatch's wait for earlier tiles, can never
+        // complete, so the blocks give up after their bounded wait and report
+        // EP_DEVERR_TIMEOUT.
         if (const char* t = std::getenv("EP_TEST_UNREACHABLE_BARRIER"))
             plan->barrierSlack = std::strcmp(t, "1") == 0 ? 1u : 0u;
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
@@ -378,6 +459,13 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->fbar = reinterpret_cast<uint32_t*>(base + L.fbar);
         plan->fdone = reinterpret_cast<uint32_t*>(base + L.fdone);
         plan->err = reinterpret_cast<int32_t*>(base + L.err);
+        plan->ll_status = reinterpret_cast<unsigned*>(base + L.ll_status);
+        plan->ll_agg = reinterpret_cast<int32_t*>(base + L.ll_agg);
+        plan->ll_plist = reinterpret_cast<int32_t*>(base + L.ll_plist);
+        plan->ll_ptotal = reinterpret_cast<unsigned long long*>(base + L.ll_ptotal);
+        plan->ll_ticket = reinterpret_cast<int32_t*>(base + L.ll_ticket);
+        plan->ll_done = reinterpret_cast<unsigned*>(base + L.ll_done);
+        plan->ll_epoch = reinterpret_cast<unsigned*>(base + L.ll_epoch);
         plan->dispatched = false;
         g_last_error[0] = '\0';
         return plan;
@@ -472,10 +560,6 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         rp.maxRecv = plan->maxRecv;
         rp.useWeights = c.useWeights;
         cudaError_t e = cudaSuccess;
-        if (!plan->fused) {
-            e = ep::launch_route_count(rp, s);
-            if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
-        }
 
         ep::ScatterParams sp{};
         sp.x = static_cast<const uint8_t*>(x);
@@ -505,6 +589,27 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         sp.scales = static_cast<const uint32_t*>(scales);
         sp.recv_scales = static_cast<uint32_t*>(recv_scales);
         sp.scaleWords = scaleWords;
+        if (plan->ll) {
+            // One launch: every block routes and scans the batch, then copies its share.
+            const int nEpr = c.numExpertPerRank;
+            sp.w = c.useWeights ? topk_w : nullptr;
+            sp.useWeights = c.useWeights;
+            sp.nEprShift = (nEpr & (nEpr - 1)) == 0 ? __builtin_ctz((unsigned)nEpr) : -1;
+            sp.llListCap = plan->llTile;
+            sp.llEngines = plan->info.scatterWarps;
+            sp.ll_status = plan->ll_status;
+            sp.ll_agg = plan->ll_agg;
+            sp.ll_plist = plan->ll_plist;
+            sp.ll_ptotal = plan->ll_ptotal;
+            sp.ll_ticket = plan->ll_ticket;
+            sp.ll_done = plan->ll_done;
+            sp.ll_epoch = plan->ll_epoch;
+            sp.barrierSlack = plan->barrierSlack;
+            e = ep::launch_dispatch_ll(sp, plan->info.scatterBlocks, plan->llSmem, s);
+            if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_ll");
+            plan->dispatched = true;
+            return EP_OK;
+        }
         if (plan->fused) {
             // One cooperative launch: routing phase, chunk scan, copy engines.
             sp.baseShift = 5;
@@ -524,6 +629,8 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
             plan->dispatched = true;
             return EP_OK;
         }
+        e = ep::launch_route_count(rp, s);
+        if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
         sp.baseShift = 8;  // route_count's 256-token tiles
         e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend,
                                     plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);

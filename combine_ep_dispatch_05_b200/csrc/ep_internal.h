@@ -16,6 +16,12 @@ constexpr int kMaxWorld = 32;   // one destination bit per lane of a 32-bit mask
 constexpr int kMaxTopk = 32;    // one topk entry per lane
 constexpr int kMaxScatterWarps = 16;
 constexpr int kMaxCombineWarps = 8;
+// Threads of a low-latency dispatch block (its first warps are the copy
+// engines); a block routes a tile of at most kLlThreads tokens, and a launch
+// has at most kLlMaxTiles tiles.
+constexpr int kLlThreads = 512;
+constexpr int kLlWarps = kLlThreads / 32;
+constexpr int kLlMaxTiles = 256;
 // Bounded waits give up after this many SM clock cycles (about 1 s at 1.9 GHz).
 constexpr long long kWaitCycles = 2000000000LL;
 
@@ -65,6 +71,17 @@ struct ScatterParams {
     int numChunks32;         // ceil(G / 32)
     int useWeights;
     unsigned barrierSlack;   // 0; 1 makes the first grid barrier unreachable (tests of the timeout path)
+    // Only the low-latency dispatch uses these (and w, recv_count, useWeights):
+    int nEprShift;           // log2(nEpr) when nEpr is a power of two, else -1
+    int llListCap;           // tokens per tile (<= kLlThreads); gridDim.x = ceil(G / llListCap)
+    int llEngines;           // copy-engine warps per block (<= kLlWarps)
+    unsigned* ll_status;     // [kLlMaxTiles]: (epoch << 1) | 1 once the tile's counts are published
+    int32_t* ll_agg;         // [kLlMaxTiles][W + 1]: rows of each tile at each destination, present tokens
+    int32_t* ll_plist;       // [G][W + 2]: present token q: tag, token, slot at each destination
+    unsigned long long* ll_ptotal;  // (tag << 32) | present tokens of the call, from the last tile
+    int32_t* ll_ticket;      // next tile to hand out (0 at the start of each call)
+    unsigned* ll_done;       // blocks past the hand-out; the last one resets ticket and done
+    unsigned* ll_epoch;      // calls so far (tags the status words of this call)
 };
 
 struct CombineParams {
@@ -80,12 +97,14 @@ struct CombineParams {
 // Byte offsets of the dispatch scratch regions (each 256-byte aligned):
 // routing table, token masks, tile counts, tile bases (256-token tiles of the
 // split dispatch), chunk counts and bases (32-token chunks of the fused
-// dispatch), the counters (one 256-byte region: tile ticket, scatter token
-// counter, combine token counter, combine blocks done, fused grid barrier,
-// fused blocks done), error word.
+// dispatch), the low-latency dispatch's tile status words, tile counts and
+// present-token list, the counters (one 256-byte region: tile ticket, scatter
+// token counter, combine token counter, combine blocks done, fused grid
+// barrier, fused blocks done, low-latency tile ticket, blocks done, call epoch
+// and present total), error word.
 struct ScratchLayout {
-    size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base;
-    size_t ticket, work, cwork, cdone, fbar, fdone, err, total;
+    size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base, ll_status, ll_agg, ll_plist;
+    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, err, total;
 };
 
 inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
@@ -98,12 +117,20 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
     L.tile_base = L.tile_cnt + up(sizeof(int32_t) * (size_t)numTiles * W);
     L.chunk_cnt = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * W);
     L.chunk_base = L.chunk_cnt + up(sizeof(int32_t) * numChunks32 * W);
-    L.ticket = L.chunk_base + up(sizeof(int32_t) * numChunks32 * W);
+    const size_t llTiles = (size_t)(G < kLlMaxTiles ? G : kLlMaxTiles);
+    L.ll_status = L.chunk_base + up(sizeof(int32_t) * numChunks32 * W);
+    L.ll_agg = L.ll_status + up(sizeof(uint32_t) * llTiles);
+    L.ll_plist = L.ll_agg + up(sizeof(int32_t) * llTiles * (W + 1));
+    L.ticket = L.ll_plist + up(sizeof(int32_t) * (size_t)G * (W + 2));
     L.work = L.ticket + 4;
     L.cwork = L.ticket + 8;
     L.cdone = L.ticket + 12;
     L.fbar = L.ticket + 16;
     L.fdone = L.ticket + 20;
+    L.ll_ticket = L.ticket + 24;
+    L.ll_done = L.ticket + 28;
+    L.ll_epoch = L.ticket + 32;
+    L.ll_ptotal = L.ticket + 40;
     L.err = L.ticket + 256;
     L.total = L.err + 256;
     return L;
@@ -126,6 +153,14 @@ cudaError_t launch_combine(const CombineParams& p, bool fp32, int tile, int bloc
 cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s);
 cudaError_t fused_set_smem(int W, int topk, size_t bytes);
 cudaError_t fused_blocks_per_sm(int W, int topk, int warps, size_t smem, int* out);
+// Low-latency dispatch (one launch, no dependency between blocks) for small
+// batches: shared memory it needs, opt-in, occupancy, launch (kLlThreads
+// threads per block).
+int ll_tile_tokens(long long G, int blocks);
+size_t ll_smem_bytes(int tileTokens, int W, int warps, int stages, int chunkStride);
+cudaError_t ll_set_smem(int W, int topk, size_t bytes);
+cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out);
+cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s);
 
 // Shared-memory bytes the scatter kernel needs for a geometry.
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride);

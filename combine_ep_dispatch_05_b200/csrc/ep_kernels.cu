@@ -308,21 +308,67 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
 // next token before it works on the current one.
 // =====================================================================
 struct TokenInputs {
-    int g;     // token, or -1 when nothing is loaded
-    int2 rr;   // lane < W: (tile-local rank or -1, weight bits)
+    int h;     // the feed's handle of the token, or -1 when nothing is loaded
+    int g;     // token
+    int2 rr;   // lane < W: (tile-local rank or -1, weight bits); list feed: (slot or -1, -)
     int base;  // lane < W: base of the token's tile at destination lane
     int e;     // lane < k: topk id
+    float wt;  // lane < k: topk weight (list feed only)
 };
 
 __device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p, int g, int lane) {
     TokenInputs in;
+    in.h = g;
     in.g = g;
+    in.wt = 0.0f;
     const int W = p.W;
     // routing data written by other blocks (or the previous kernel): read through L2
     in.rr = lane < W ? __ldcg(p.route + (size_t)g * W + lane) : make_int2(-1, 0);
     in.base = lane < W ? __ldcg(p.tile_base + (size_t)(g >> p.baseShift) * W + lane) : 0;
     in.e = lane < p.k ? p.idx[(size_t)g * p.k + lane] : -1;
     return in;
+}
+
+// The scale row of token g travels with it to every destination in `mask`
+// (lane pe holds the slot at pe).
+__device__ __forceinline__ void write_scales(const ScatterParams& p, int g, uint32_t mask, int my_slot, int lane) {
+    const uint32_t* src = p.scales + (size_t)g * p.scaleWords;
+    for (int w0 = 0; w0 < p.scaleWords; w0 += 32) {
+        const int wi = w0 + lane;
+        const uint32_t v = wi < p.scaleWords ? src[wi] : 0u;
+        for (uint32_t m = mask; m; m &= m - 1) {
+            const int pe = __ffs(m) - 1;
+            const int slot = __shfl_sync(kFull, my_slot, pe);
+            if (wi < p.scaleWords) p.recv_scales[((size_t)pe * p.maxRecv + slot) * p.scaleWords + wi] = v;
+        }
+    }
+}
+
+// Meta records and scale rows of token g at every destination in `mask`.
+// Lane pe holds the token's slot at pe (my_slot) and its weight-sum bits
+// (wb_lane); lane j < k holds topk id e of entry j.
+__device__ __forceinline__ void write_records(const ScatterParams& p, int g, uint32_t mask, int my_slot,
+                                              int wb_lane, int e, int lane) {
+    const int r = g / p.T, t = g - r * p.T;
+    const int pe_e = (e >= 0 && e < p.E) ? e / p.nEpr : -1;
+    // field f of a record: 0 rank, 1 token, 2 weight bits, 3+j local id of entry j
+    const int j0 = lane - 3, j1 = lane + 29;
+    const int e0 = __shfl_sync(kFull, e, j0 & 31), q0 = __shfl_sync(kFull, pe_e, j0 & 31);
+    const int e1 = __shfl_sync(kFull, e, j1 & 31), q1 = __shfl_sync(kFull, pe_e, j1 & 31);
+    for (uint32_t m = mask; m; m &= m - 1) {
+        const int pe = __ffs(m) - 1;
+        const int slot = __shfl_sync(kFull, my_slot, pe);
+        const int wb = __shfl_sync(kFull, wb_lane, pe);
+        int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
+        int v0;
+        if (lane == 0) v0 = r;
+        else if (lane == 1) v0 = t;
+        else if (lane == 2) v0 = wb;
+        else v0 = (q0 == pe) ? e0 - pe * p.nEpr : -1;
+        if (lane < p.M) rec[lane] = v0;
+        if (lane + 32 < p.M) rec[lane + 32] = (q1 == pe) ? e1 - pe * p.nEpr : -1;
+    }
+    if (p.scaleWords > 0) write_scales(p, g, mask, my_slot, lane);
 }
 
 // Turn the tile-local ranks of the token into slots (lane pe holds the slot
@@ -341,39 +387,7 @@ __device__ __forceinline__ uint32_t token_slots_and_meta(const ScatterParams& p,
         p.route[(size_t)g * W + lane].x = ok ? my_slot : -1;
     }
     const uint32_t mask = __ballot_sync(kFull, ok);
-    const int r = g / p.T, t = g - r * p.T;
-    const int e = in.e;
-    const int pe_e = (e >= 0 && e < p.E) ? e / p.nEpr : -1;
-    // field f of a record: 0 rank, 1 token, 2 weight bits, 3+j local id of entry j
-    const int j0 = lane - 3, j1 = lane + 29;
-    const int e0 = __shfl_sync(kFull, e, j0 & 31), q0 = __shfl_sync(kFull, pe_e, j0 & 31);
-    const int e1 = __shfl_sync(kFull, e, j1 & 31), q1 = __shfl_sync(kFull, pe_e, j1 & 31);
-    for (uint32_t m = mask; m; m &= m - 1) {
-        const int pe = __ffs(m) - 1;
-        const int slot = __shfl_sync(kFull, my_slot, pe);
-        const int wb = __shfl_sync(kFull, rr.y, pe);
-        int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
-        int v0;
-        if (lane == 0) v0 = r;
-        else if (lane == 1) v0 = t;
-        else if (lane == 2) v0 = wb;
-        else v0 = (q0 == pe) ? e0 - pe * p.nEpr : -1;
-        if (lane < p.M) rec[lane] = v0;
-        if (lane + 32 < p.M) rec[lane + 32] = (q1 == pe) ? e1 - pe * p.nEpr : -1;
-    }
-    // The token's scale row travels with it to every destination.
-    if (p.scaleWords > 0) {
-        const uint32_t* src = p.scales + (size_t)g * p.scaleWords;
-        for (int w0 = 0; w0 < p.scaleWords; w0 += 32) {
-            const int wi = w0 + lane;
-            const uint32_t v = wi < p.scaleWords ? src[wi] : 0u;
-            for (uint32_t m = mask; m; m &= m - 1) {
-                const int pe = __ffs(m) - 1;
-                const int slot = __shfl_sync(kFull, my_slot, pe);
-                if (wi < p.scaleWords) p.recv_scales[((size_t)pe * p.maxRecv + slot) * p.scaleWords + wi] = v;
-            }
-        }
-    }
+    write_records(p, g, mask, my_slot, rr.y, in.e, lane);
     return mask;
 }
 
@@ -416,46 +430,49 @@ __device__ __forceinline__ EngineSmem engine_smem_init(uint8_t* smem, const Scat
     return es;
 }
 
-// One copy engine (a warp): the present tokens it is handed are copied row
-// piece by row piece through an S-stage shared-memory ring, S - kPend loads
-// ahead, with kPend items' bulk stores left draining when a stage is refilled.
-template <int kPend>
-__device__ __forceinline__ void copy_engine(const ScatterParams& p, const EngineSmem& es, int lane, int warp,
-                                            int nwarps) {
-    const int S = p.stages;  // > kPend (checked on the host)
-
-    // Engines per block: at a high mean fan-out the copies are bandwidth-bound
-    // and one engine fewer per SM writes faster (B200: 472 vs 503 us at fan-out
-    // 5.3); at a low fan-out the per-token latency chain dominates and every
-    // engine helps (skewed routing, fan-out 2.9: 302 vs 335 us). The counts of
-    // this dispatch decide.
-    if (p.fanoutSwitch > 0 && nwarps > 2) {
-        const int cnt = lane < p.W ? __ldcg(p.recv_count + lane) : 0;
-        int rows = cnt;
+// Engines per block: at a high mean fan-out the copies are bandwidth-bound
+// and one engine fewer per SM writes faster (B200: 472 vs 503 us at fan-out
+// 5.3); at a low fan-out the per-token latency chain dominates and every
+// engine helps (skewed routing, fan-out 2.9: 302 vs 335 us). The counts of
+// this dispatch (recv_count, complete before the call) decide.
+__device__ __forceinline__ int active_engines(const ScatterParams& p, int nwarps, int lane) {
+    if (p.fanoutSwitch <= 0 || nwarps <= 2) return nwarps;
+    const int cnt = lane < p.W ? __ldcg(p.recv_count + lane) : 0;
+    int rows = cnt;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) rows += __shfl_xor_sync(kFull, rows, off);
-        if ((long long)rows * 100 > (long long)p.fanoutSwitch * p.G) nwarps -= 1;
-        if (warp >= nwarps) return;  // this engine's stages stay unused
-    }
-    const uint32_t stage0_addr = es.stage0_addr, bar0 = es.bar0;
-    int* item_tok = es.item_tok;
-    int* item_chunk = es.item_chunk;
+    for (int off = 16; off > 0; off >>= 1) rows += __shfl_xor_sync(kFull, rows, off);
+    return (long long)rows * 100 > (long long)p.fanoutSwitch * p.G ? nwarps - 1 : nwarps;
+}
 
-    // Producer (lane 0): tokens come from the shared hand-out (static rounds,
-    // then a global counter). Two candidates are kept in flight ahead (the
-    // hand-out's answer and then the token's destination mask), so finding the
-    // next present token costs no latency on the copy path.
-    TokenSource src = make_source(blockIdx.x * nwarps + warp, gridDim.x * nwarps, p.G, p.work);
-    int tA = p.G, tB = p.G, tC = p.G;  // candidates, in the order handed out
-    uint32_t mA = 0, mB = 0;           // masks of A and B
-    if (lane == 0) {
-        tA = source_next(src);
-        tB = source_next(src);
-        mA = tA < p.G ? __ldcg(p.tok_mask + tA) : 0u;
-        tC = source_next(src);
-        mB = tB < p.G ? __ldcg(p.tok_mask + tB) : 0u;
+// Token feeds of a copy engine. A feed hands out token handles (p.G: none
+// left), maps a handle to the token's row, issues the global loads of a
+// token's inputs (so that the engine can prefetch them one token ahead), and
+// prepares a token: its slots, routing-table entries and meta records.
+
+// Split dispatch: tokens from the shared hand-out (static rounds, then a
+// global counter); route_count's tile-local ranks plus the tile's base give
+// the slots. Two candidates are kept in flight ahead (the hand-out's answer
+// and then the token's destination mask), so finding the next present token
+// costs no latency on the copy path.
+struct GlobalFeed {
+    TokenSource src;
+    int tA, tB, tC;  // candidates, in the order handed out (lane 0)
+    uint32_t mA, mB;  // masks of A and B
+
+    __device__ __forceinline__ void init(const ScatterParams& p, int worker, int nWorkers, int lane) {
+        src = make_source(worker, nWorkers, p.G, p.work);
+        tA = tB = tC = p.G;
+        mA = mB = 0u;
+        if (lane == 0) {
+            tA = source_next(src);
+            tB = source_next(src);
+            mA = tA < p.G ? __ldcg(p.tok_mask + tA) : 0u;
+            tC = source_next(src);
+            mB = tB < p.G ? __ldcg(p.tok_mask + tB) : 0u;
+        }
     }
-    auto next_present = [&]() -> int {
+    // Next present token (warp-uniform), or p.G.
+    __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
         int found = p.G;
         if (lane == 0) {
             while (tA < p.G) {
@@ -473,10 +490,99 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
             }
         }
         return __shfl_sync(kFull, found, 0);
-    };
+    }
+    __device__ __forceinline__ int row(const ScatterParams&, int h) const { return h; }
+    __device__ __forceinline__ TokenInputs load(const ScatterParams& p, int h, int lane) const {
+        return load_token_inputs(p, h, lane);
+    }
+    __device__ __forceinline__ uint32_t prepare(const ScatterParams& p, const TokenInputs& in, int lane,
+                                                int& my_slot) const {
+        return token_slots_and_meta(p, in, lane, my_slot);
+    }
+};
 
-    int pg = next_present();  // producer token
-    int pc = 0;               // producer chunk
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait (bounded) until *p == want; false when the wait gave up.
+__device__ __forceinline__ bool wait_tag(const unsigned* p, unsigned want) {
+    if (ld_acquire_u32(p) == want) return true;
+    const long long t0 = clock64();
+    while (ld_acquire_u32(p) != want) {
+        if (clock64() - t0 > kWaitCycles) return false;
+        __nanosleep(32);
+    }
+    return true;
+}
+
+// Single-launch small-batch dispatch: the call's present tokens are a list
+// in global memory (entry q: tag, token, slot at each destination), written
+// by the blocks that routed them; this block copies entries b, b + nb, ...
+// (handle i = entry b + i*nb). The routing rows and meta records are already
+// written; the engine copies the rows (and the scale rows, when the call has
+// them).
+struct PlistFeed {
+    const int32_t* plist;  // [P][W + 2]
+    int b, nb, n, i, step;
+    unsigned tag;
+
+    __device__ __forceinline__ const int32_t* entry(const ScatterParams& p, int h) const {
+        return plist + (size_t)(b + (size_t)h * nb) * (p.W + 2);
+    }
+    // Next handle, once its entry is published (lane 0 waits, bounded).
+    __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
+        int h = p.G;
+        if (i < n) {
+            h = i;
+            i += step;
+            int ok = 1;
+            if (lane == 0) ok = wait_tag(reinterpret_cast<const unsigned*>(entry(p, h)), tag);
+            __syncwarp();
+            if (!__shfl_sync(kFull, ok, 0)) {
+                if (lane == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
+                n = 0;  // copy nothing more
+                h = p.G;
+            }
+        }
+        return h;
+    }
+    __device__ __forceinline__ int row(const ScatterParams& p, int h) const { return __ldcg(entry(p, h) + 1); }
+    __device__ __forceinline__ TokenInputs load(const ScatterParams& p, int h, int lane) const {
+        const int32_t* e = entry(p, h);
+        TokenInputs in;
+        in.h = h;
+        in.g = __ldcg(e + 1);
+        in.rr = make_int2(lane < p.W ? __ldcg(e + 2 + lane) : -1, 0);
+        in.base = 0;
+        in.e = -1;
+        in.wt = 0.0f;
+        return in;
+    }
+    __device__ __forceinline__ uint32_t prepare(const ScatterParams& p, const TokenInputs& in, int lane,
+                                                int& my_slot) const {
+        my_slot = in.rr.x;
+        const uint32_t mask = __ballot_sync(kFull, my_slot >= 0);
+        if (p.scaleWords > 0) write_scales(p, in.g, mask, my_slot, lane);
+        return mask;
+    }
+};
+
+// One copy engine (a warp): the present tokens its feed hands out are copied
+// row piece by row piece through an S-stage shared-memory ring, S - kPend
+// loads ahead, with kPend items' bulk stores left draining when a stage is
+// refilled.
+template <int kPend, class Feed>
+__device__ __forceinline__ void copy_engine(const ScatterParams& p, const EngineSmem& es, int lane, Feed& feed) {
+    const int S = p.stages;  // > kPend (checked on the host)
+    const uint32_t stage0_addr = es.stage0_addr, bar0 = es.bar0;
+    int* item_tok = es.item_tok;
+    int* item_chunk = es.item_chunk;
+
+    int pg = feed.next(p, lane);  // producer token (handle)
+    int pc = 0;                   // producer chunk
     int issued = 0, consumed = 0;
     bool ok = true;
 
@@ -489,13 +595,13 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
             item_tok[s] = pg;
             item_chunk[s] = pc;
             mbar_arrive_expect_tx(bar0 + 8u * s, bytes);
-            bulk_load(stage0_addr + (uint32_t)s * p.chunkStride, p.x + (size_t)pg * p.rowBytes + off,
+            bulk_load(stage0_addr + (uint32_t)s * p.chunkStride, p.x + (size_t)feed.row(p, pg) * p.rowBytes + off,
                       bytes, bar0 + 8u * s);
         }
         ++issued;
         if (++pc == p.numChunks) {
             pc = 0;
-            pg = next_present();
+            pg = feed.next(p, lane);
         }
     };
 
@@ -504,7 +610,7 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
 
     // Per-token state kept across the chunks of one token.
     TokenInputs pre;
-    pre.g = -1;
+    pre.h = -1;
     int cur_tok = -1;
     uint32_t cur_mask = 0;
     int my_slot = -1;  // lane pe: slot of the current token at pe
@@ -513,17 +619,17 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
         const int s = consumed % S;
         const uint32_t parity = (uint32_t)(consumed / S) & 1u;
         __syncwarp();
-        const int g = item_tok[s];
+        const int h = item_tok[s];
         const int c = item_chunk[s];
 
-        if (g != cur_tok) {
-            cur_tok = g;
-            const TokenInputs in = (pre.g == g) ? pre : load_token_inputs(p, g, lane);
+        if (h != cur_tok) {
+            cur_tok = h;
+            const TokenInputs in = (pre.h == h) ? pre : feed.load(p, h, lane);
             // Prefetch the next token in the ring before working on this one.
-            pre.g = -1;
+            pre.h = -1;
             const int nxt = consumed + p.numChunks - c;
-            if (nxt < issued) pre = load_token_inputs(p, item_tok[nxt % S], lane);
-            cur_mask = token_slots_and_meta(p, in, lane, my_slot);
+            if (nxt < issued) pre = feed.load(p, item_tok[nxt % S], lane);
+            cur_mask = feed.prepare(p, in, lane, my_slot);
         }
 
         // Wait for the row piece, then send it to every destination.
@@ -567,6 +673,17 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
     __syncwarp();
 }
 
+// Split-dispatch copy engines: the engines of this block that the fan-out
+// leaves active take tokens from the shared hand-out.
+template <int kPend>
+__device__ __forceinline__ void global_copy_engines(const ScatterParams& p, const EngineSmem& es, int lane,
+                                                    int warp, int nwarps) {
+    const int engines = active_engines(p, nwarps, lane);
+    if (warp >= engines) return;  // this engine's stages stay unused
+    GlobalFeed feed;
+    feed.init(p, blockIdx.x * engines + warp, gridDim.x * engines, lane);
+    copy_engine<kPend>(p, es, lane, feed);
+}
 
 template <int kPend>
 __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(ScatterParams p) {
@@ -575,7 +692,233 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
     pdl_wait();     // routing written by route_count is visible from here on
     pdl_trigger();
-    copy_engine<kPend>(p, es, lane, warp, nwarps);
+    global_copy_engines<kPend>(p, es, lane, warp, nwarps);
+}
+
+// =====================================================================
+// dispatch_ll: the whole dispatch of a small batch in one launch (the
+// low-latency family; the pages switch to theirs at 512 tokens a launch).
+// Block = tile of up to kLlThreads consecutive tokens, one thread per token:
+//   1. the block takes the next tile from a ticket, routes its tokens
+//      (destination masks; counts per 32-token chunk by ballot) and publishes
+//      the tile's count at every destination and of present tokens, then a
+//      status word tagged with this call's epoch;
+//   2. it adds up the counts of all earlier tiles, each loaded as soon as its
+//      status is published (a bounded wait). Tiles are handed out in order,
+//      so a block only waits on blocks that are already running, and no
+//      block waits before publishing: the waits end. The last tile stores
+//      recv_count and publishes the number of present tokens P;
+//   3. each thread of a present token computes its slots (tile base + chunk
+//      base + rank in the chunk), writes the token's routing row and meta
+//      records, and publishes the token as entry q of the present list (q =
+//      its number among the call's present tokens, in (srcRank, token)
+//      order); absent tokens get their routing rows;
+//   4. the block's copy engines copy entries b, b + nb, ... (b = its tile),
+//      each once it is published: the copies spread over all blocks however
+//      the present tokens cluster.
+// Shared memory: [slots of the tile's present tokens: T x W], then the copy
+// engines' barriers and stages.
+// =====================================================================
+__device__ __forceinline__ int dest_pe(int e, int nEpr, int shift) { return shift >= 0 ? e >> shift : e / nEpr; }
+
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+template <int kW, int kK>
+__global__ void __launch_bounds__(kLlThreads, 1) ep_dispatch_ll_kernel(ScatterParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_cnt[kLlWarps][kW + 1];  // per chunk: rows at each destination, present tokens
+    __shared__ int s_base[kW + 1];           // the same for all earlier tiles
+    __shared__ int s_agg[kW + 1];            // the same for this tile
+    __shared__ int s_tile, s_present, s_ok;
+    __shared__ unsigned s_tag;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = p.G, W = p.W, k = p.k, C = W + 1;
+    const int TT = p.llListCap;
+    int* tile_slot = reinterpret_cast<int*>(smem);  // [TT][W]
+    uint8_t* area = smem + (((size_t)TT * W * sizeof(int) + 127) & ~(size_t)127);
+
+    pdl_wait();  // the ids and the counters of the previous call are visible from here on
+    pdl_trigger();
+    if (tid == 0) {
+        s_tile = atomicAdd(p.ll_ticket, 1);
+        s_tag = (__ldcg(p.ll_epoch) << 1) | 1u;
+    }
+    if (tid <= kW) s_base[tid] = 0;
+    __syncthreads();
+    const int t = s_tile;
+    const unsigned tag = s_tag;
+    // Every block has its tile: the last one to get here resets the hand-out
+    // for the next call and advances the epoch (the blocks of this call keep
+    // the tag they read).
+    if (tid == 0 && atomicAdd(p.ll_done, 1u) == gridDim.x - 1) {
+        *p.ll_ticket = 0;
+        *p.ll_done = 0u;
+        atomicAdd(p.ll_epoch, 1u);
+    }
+
+    // 1. Route this tile: thread i takes token t*TT + i. Its ids (entries
+    // that are masked or out of range become -1) and weights stay in
+    // registers for step 3.
+    const int g = t * TT + tid;
+    const bool live = tid < TT && g < G;
+    uint32_t mask = 0;
+    bool bad = false;
+    int e[kK];
+    float wj[kK];
+#pragma unroll
+    for (int j = 0; j < kK; ++j) {
+        e[j] = (live && j < k) ? p.idx[(size_t)g * k + j] : -1;
+        wj[j] = (live && j < k && p.w != nullptr) ? p.w[(size_t)g * k + j] : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kK; ++j) {
+        if (e[j] >= p.E) {  // contract violation: report, treat as masked
+            bad = true;
+            e[j] = -1;
+        }
+        if (e[j] >= 0) mask |= 1u << dest_pe(e[j], p.nEpr, p.nEprShift);
+    }
+    if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
+    int cnt = 0;
+#pragma unroll
+    for (int pe = 0; pe < kW; ++pe) {
+        if (pe < W) {
+            const uint32_t bb = __ballot_sync(kFull, (mask >> pe) & 1u);
+            if (lane == pe) cnt = __popc(bb);
+        }
+    }
+    const uint32_t bp = __ballot_sync(kFull, mask != 0u);
+    if (lane < W) s_cnt[warp][lane] = cnt;
+    if (lane == 0) s_cnt[warp][W] = __popc(bp);
+    __syncthreads();
+    // Chunk bases within the tile (in place) and the tile's counts; publish.
+    if (warp == 0) {
+        for (int col = lane; col < C; col += 32) {  // 33 columns when W = 32
+            int run = 0;
+            for (int w = 0; w < kLlWarps; ++w) {
+                const int c = s_cnt[w][col];
+                s_cnt[w][col] = run;
+                run += c;
+            }
+            s_agg[col] = run;
+            p.ll_agg[(size_t)t * C + col] = run;
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release_u32(p.ll_status + t, tag);
+    }
+
+    // 2. Counts of the earlier tiles. (barrierSlack, a test hook, 0
+    // otherwise, makes the awaited tag one that no block writes.)
+    const unsigned want = tag + (p.barrierSlack << 1);
+    int ok = 1;
+    for (int i = tid; i < t; i += kLlThreads) {
+        if (!wait_tag(p.ll_status + i, want)) {
+            ok = 0;
+            break;
+        }
+        for (int c = 0; c < C; ++c) atomicAdd(&s_base[c], __ldcg(p.ll_agg + (size_t)i * C + c));
+    }
+    if (!__syncthreads_and(ok)) {
+        if (tid == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
+        return;  // nothing copied: the counts are unknown
+    }
+    if (t == (int)gridDim.x - 1) {
+        if (tid < W) {
+            const int total = s_base[tid] + s_agg[tid];
+            p.recv_count[tid] = total;  // stored, not accumulated
+            if (total > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+        }
+        if (tid == 0)
+            st_release_u64(p.ll_ptotal, ((unsigned long long)tag << 32) | (unsigned)(s_base[W] + s_agg[W]));
+    }
+
+    // 3. Slots, routing rows, meta records and present-list entries of this
+    // tile's tokens.
+    const uint32_t lt = lanemask_lt();
+    const int li = s_cnt[warp][W] + __popc(bp & lt);  // present token number within the tile
+#pragma unroll
+    for (int pe = 0; pe < kW; ++pe) {
+        if (pe < W) {
+            const bool hit = (mask >> pe) & 1u;
+            const uint32_t bb = __ballot_sync(kFull, hit);
+            if (live && mask != 0u) {
+                int slot = hit ? s_base[pe] + s_cnt[warp][pe] + __popc(bb & lt) : -1;
+                if (slot >= p.maxRecv) {  // only when the counts were corrupted
+                    atomicOr(p.err, EP_DEVERR_CAPACITY);
+                    slot = -1;
+                }
+                tile_slot[li * W + pe] = slot;
+            }
+        }
+    }
+    if (live) {
+        const int r = g / p.T, tok = g - r * p.T;
+        int32_t* ent = p.ll_plist + (size_t)(s_base[W] + li) * (W + 2);
+        if (mask != 0u) ent[1] = g;
+        for (int pe = 0; pe < W; ++pe) {
+            const int slot = mask != 0u ? tile_slot[li * W + pe] : -1;
+            if (mask != 0u) ent[2 + pe] = slot;
+            if (slot < 0) {
+                p.route[(size_t)g * W + pe] = make_int2(-1, 0);
+                continue;
+            }
+            float ws = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kK; ++j)
+                if (e[j] >= 0 && dest_pe(e[j], p.nEpr, p.nEprShift) == pe) ws = ws + wj[j];
+            const int wb = __float_as_int(p.useWeights ? ws : 1.0f);
+            p.route[(size_t)g * W + pe] = make_int2(slot, wb);
+            int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
+            rec[0] = r;
+            rec[1] = tok;
+            rec[2] = wb;
+#pragma unroll
+            for (int j = 0; j < kK; ++j)
+                if (j < k) rec[3 + j] = (e[j] >= 0 && dest_pe(e[j], p.nEpr, p.nEprShift) == pe) ? e[j] - pe * p.nEpr : -1;
+        }
+        if (mask != 0u) st_release_u32(reinterpret_cast<unsigned*>(ent), tag);  // after the entry's fields
+    }
+
+    // 4. Copy engines, once the number of present tokens is known.
+    if (tid == 0) {
+        const unsigned long long wantP = (unsigned long long)want;
+        unsigned long long v = ld_acquire_u64(p.ll_ptotal);
+        const long long t0 = clock64();
+        while ((v >> 32) != wantP && clock64() - t0 <= kWaitCycles) {
+            __nanosleep(32);
+            v = ld_acquire_u64(p.ll_ptotal);
+        }
+        s_ok = (v >> 32) == wantP;
+        s_present = (int)(v & 0xffffffffu);
+        if (!s_ok) atomicOr(p.err, EP_DEVERR_TIMEOUT);
+    }
+    __syncthreads();
+    const int engines = p.llEngines;
+    if (!s_ok || warp >= engines) return;
+    const int present = s_present, nb = gridDim.x;
+    const EngineSmem es = engine_smem_init(area, p, warp, engines, lane);
+    PlistFeed feed;
+    feed.plist = p.ll_plist;
+    feed.b = t;
+    feed.nb = nb;
+    feed.n = present > t ? (present - 1 - t) / nb + 1 : 0;
+    feed.i = warp;
+    feed.step = engines;
+    feed.tag = tag;
+    copy_engine<1>(p, es, lane, feed);
 }
 
 // =====================================================================
@@ -677,7 +1020,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kerne
     ok = ok && grid_barrier(p.bar, 2u * gridDim.x + p.barrierSlack);
 
     // 3. copy engines
-    if (ok) copy_engine<1>(p, es, lane, warp, nwarps);
+    if (ok) global_copy_engines<1>(p, es, lane, warp, nwarps);
     else if (threadIdx.x == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
 
     // The last block to finish resets the counters for the next call.
@@ -1038,6 +1381,52 @@ cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps,
         cfg.numAttrs = 1;
         return cudaLaunchKernelEx(&cfg, k, p);
     });
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+namespace {
+template <typename F>
+cudaError_t for_world_ll(int W, int k, F&& f) {
+    if (W <= 8)
+        return k <= 8 ? f(ep_dispatch_ll_kernel<8, 8>) : k <= 16 ? f(ep_dispatch_ll_kernel<8, 16>)
+                                                          : f(ep_dispatch_ll_kernel<8, 32>);
+    if (W <= 16)
+        return k <= 8 ? f(ep_dispatch_ll_kernel<16, 8>) : k <= 16 ? f(ep_dispatch_ll_kernel<16, 16>)
+                                                           : f(ep_dispatch_ll_kernel<16, 32>);
+    return k <= 8 ? f(ep_dispatch_ll_kernel<32, 8>) : k <= 16 ? f(ep_dispatch_ll_kernel<32, 16>)
+                                                       : f(ep_dispatch_ll_kernel<32, 32>);
+}
+}  // namespace
+
+int ll_tile_tokens(long long G, int blocks) {
+    // Tokens per tile: the batch spread over `blocks` blocks, at least enough
+    // that there are no more than kLlMaxTiles tiles.
+    long long tt = (G + blocks - 1) / blocks;
+    const long long minTt = (G + kLlMaxTiles - 1) / kLlMaxTiles;
+    if (tt < minTt) tt = minTt;
+    if (tt < 1) tt = 1;
+    return (int)tt;
+}
+
+size_t ll_smem_bytes(int tileTokens, int W, int warps, int stages, int chunkStride) {
+    const size_t list = ((size_t)tileTokens * (size_t)W * sizeof(int) + 127) & ~(size_t)127;
+    return list + scatter_smem_bytes(warps, stages, chunkStride);
+}
+
+cudaError_t ll_set_smem(int W, int topk, size_t bytes) {
+    return for_world_ll(W, topk, [&](auto k) {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    });
+}
+
+cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out) {
+    return for_world_ll(W, topk, [&](auto k) {
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, kLlThreads, smem);
+    });
+}
+
+cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s) {
+    cudaError_t e = for_world_ll(p.W, p.k, [&](auto k) { return launch_pdl(k, blocks, kLlThreads, smem, s, p); });
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -98,7 +98,14 @@ typedef struct EpPlanInfo {
     int64_t outBytes;         /* bytes of out: W*T*combineRowBytes */
     int32_t dispatchFused;    /* 1: dispatch is one cooperative launch (route, scan, scatter);
                                  0: two launches (route_count, scatter_rows) */
-    int32_t reserved0;
+    int32_t dispatchLowLatency; /* 1: dispatch is the small-batch single launch: each block
+                                 routes one tile of tokens (scatterBlocks tiles), adds up the
+                                 counts that earlier tiles publish, writes its tokens' slots
+                                 and records, and copies every scatterBlocks-th present token.
+                                 Taken when maxTokPerRank <= EP_LL_MAX_TOKENS (0, i.e. off,
+                                 by default; the design page's internode dispatch switches
+                                 to its low-latency family at 512 tokens a launch, §9).
+                                 Results are identical either way. */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
@@ -131,7 +138,8 @@ enum {
 int ep_cfg_check(const EpCfg* cfg);
 
 /* Host-only sizing: fill *info for cfg as a plan on a generic device would
- * resolve it (device = -1, numSMs = 0, geometry from a 148-SM B200). Lets a
+ * resolve it (device = -1, numSMs = 0, geometry from a 148-SM B200 without
+ * the geometry overrides; EP_LL_MAX_TOKENS is honoured). Lets a
  * caller size recv_x / recv_meta before creating a plan. Returns EP_OK or a
  * negative code. */
 int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
@@ -144,10 +152,16 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK,
  * EP_SCATTER_PEND (1..3), EP_SCATTER_MODE ("tma" or "regs"), EP_COMBINE_BLOCKS,
  * EP_COMBINE_WARPS, EP_DISPATCH_FUSED (1: one cooperative launch instead of
- * two). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 (with EP_DISPATCH_FUSED=1)
- * makes the fused dispatch's grid barrier unreachable, so that its bounded
- * wait runs out: every block reports EP_DEVERR_TIMEOUT, issues no copy and
- * returns about one second later, and the context stays usable. */
+ * two), EP_LL_MAX_TOKENS (largest maxTokPerRank that takes the low-latency
+ * dispatch; 0, i.e. off, by default), EP_SCATTER_FANOUT_SWITCH (100 x
+ * the mean fan-out above which one copy engine per block sits out; 375 by
+ * default, 0 never). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 makes the fused
+ * dispatch's grid barrier (with EP_DISPATCH_FUSED=1), or the low-latency
+ * dispatch's wait for the counts of earlier tiles, unreachable, so that the
+ * bounded wait runs out: the waiting blocks report EP_DEVERR_TIMEOUT, issue no
+ * copy and return about one second later (the low-latency dispatch's first
+ * tile waits on nothing and writes its meta records before it gives up), and
+ * the context stays usable. */
 EpPlan* ep_plan_create(const EpCfg* cfg);
 
 /* Free the plan and its scratch. NULL is a no-op. The caller must make sure no

@@ -146,6 +146,35 @@ def test_plan_query_dtype_legs(ep, dtype, h, row, chid, crow, cdt):
     assert info.yBytes == 8 * 32768 * crow and info.outBytes == 8 * 4096 * crow
 
 
+@pytest.mark.parametrize("kw,ll", [
+    (dict(), 0),                                                       # main shape: 4096 tokens a rank
+    (dict(maxTokPerRank=512, maxRecv=0), 1),                           # 512 tokens a rank: low latency
+    (dict(maxTokPerRank=513, maxRecv=0), 0),                           # above the switch
+    (dict(worldSize=4, maxTokPerRank=512, numExpertPerRank=8, numExpertPerToken=6, maxRecv=0), 1),
+    (dict(maxTokPerRank=512, numExpertPerToken=32, maxRecv=0), 1),     # topk 32
+    (dict(worldSize=32, maxTokPerRank=512, numExpertPerToken=8, maxRecv=0), 1),  # 16384 tokens: 111 a block
+    (dict(maxTokPerRank=1, maxRecv=0), 1),
+    (dict(maxTokPerRank=512, maxRecv=0, dtype=1), 1),                  # fp32 rows of 28672 bytes
+    (dict(maxTokPerRank=512, maxRecv=0, hiddenDim=100000), 1),         # rows copied in pieces
+])
+def test_plan_query_dispatch_family(ep, kw, ll, monkeypatch):
+    """With EP_LL_MAX_TOKENS=512, plans of at most 512 tokens a rank take the
+    single-launch low-latency dispatch; the rest take route_count +
+    scatter_rows. Both give identical results. By default the low-latency
+    dispatch is off."""
+    assert ep.ep_plan_query(_cfg(**kw)).dispatchLowLatency == 0
+    monkeypatch.setenv("EP_LL_MAX_TOKENS", "512")
+    cfg = _cfg(**kw)
+    info = ep.ep_plan_query(cfg)
+    assert info.dispatchLowLatency == ll
+    assert info.dispatchFused == 0
+    if ll:
+        G = cfg["worldSize"] * cfg["maxTokPerRank"]
+        tile = -(-G // 148)
+        assert info.scatterBlocks == -(-G // tile) <= 148
+        assert info.scatterStages >= 2
+
+
 def test_entry_points_reject_without_crashing(ep):
     b = ep.binding
     assert b._lib.ep_dispatch(None, None, None, None, None, None, None, None) == b.EP_ERR_INVALID
