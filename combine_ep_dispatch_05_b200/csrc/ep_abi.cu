@@ -29,6 +29,8 @@ struct EpPlan {
     int32_t* tile_base;
     uint32_t* ticket;
     int32_t* work;
+    int32_t* pacc;        // route_count's present-token sum and the call's total
+    int32_t* ptotal;
     int32_t* cwork;
     uint32_t* cdone;
     int32_t* chunk_cnt;   // fused dispatch: [ceil(G/32)][W]
@@ -452,6 +454,8 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->tile_base = reinterpret_cast<int32_t*>(base + L.tile_base);
         plan->ticket = reinterpret_cast<uint32_t*>(base + L.ticket);
         plan->work = reinterpret_cast<int32_t*>(base + L.work);
+        plan->pacc = reinterpret_cast<int32_t*>(base + L.pacc);
+        plan->ptotal = reinterpret_cast<int32_t*>(base + L.ptotal);
         plan->cwork = reinterpret_cast<int32_t*>(base + L.cwork);
         plan->cdone = reinterpret_cast<uint32_t*>(base + L.cdone);
         plan->chunk_cnt = reinterpret_cast<int32_t*>(base + L.chunk_cnt);
@@ -550,6 +554,8 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         rp.recv_count = recv_count;
         rp.ticket = plan->ticket;
         rp.work = plan->work;
+        rp.pacc = plan->pacc;
+        rp.ptotal = plan->ptotal;
         rp.err = plan->err;
         rp.G = plan->G;
         rp.W = c.worldSize;
@@ -632,6 +638,7 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         e = ep::launch_route_count(rp, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
         sp.baseShift = 8;  // route_count's 256-token tiles
+        sp.ptotal = plan->ptotal;
         e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend,
                                     plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch scatter_rows");

@@ -35,6 +35,8 @@ struct RouteParams {
     int32_t* recv_count;    // [W]
     uint32_t* ticket;       // blocks finished this call; the last block resets it
     int32_t* work;          // scatter token counter; the last block resets it
+    int32_t* pacc;          // present tokens, summed over the blocks (the last block resets it)
+    int32_t* ptotal;        // present tokens of the call, stored by the last block
     int32_t* err;           // device error word
     int G, W, k, nEpr, E, numTiles, maxRecv, useWeights;
 };
@@ -46,6 +48,7 @@ struct ScatterParams {
     const uint32_t* tok_mask;  // [G]: destination mask of each token
     const int32_t* tile_base;  // [numTiles][W]
     int32_t* work;             // next token to hand out (starts at 0 each call)
+    const int32_t* ptotal;     // present tokens of the call (route_count), or nullptr: unknown
     uint8_t* recv_x;           // [W][maxRecv][rowBytes]
     int32_t* recv_meta;        // [W][maxRecv][M]
     int32_t* err;
@@ -101,10 +104,11 @@ struct CombineParams {
 // present-token list, the counters (one 256-byte region: tile ticket, scatter
 // token counter, combine token counter, combine blocks done, fused grid
 // barrier, fused blocks done, low-latency tile ticket, blocks done, call epoch
-// and present total), error word.
+// and present total, route_count's present-token sum and total), error word.
 struct ScratchLayout {
     size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base, ll_status, ll_agg, ll_plist;
-    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, err, total;
+    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, pacc, ptotal, err,
+        total;
 };
 
 inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
@@ -131,6 +135,8 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
     L.ll_done = L.ticket + 28;
     L.ll_epoch = L.ticket + 32;
     L.ll_ptotal = L.ticket + 40;
+    L.pacc = L.ticket + 48;
+    L.ptotal = L.ticket + 52;
     L.err = L.ticket + 256;
     L.total = L.err + 256;
     return L;

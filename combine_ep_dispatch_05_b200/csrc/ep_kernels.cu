@@ -137,14 +137,16 @@ struct TokenSource {
     int32_t* ctr;
 };
 
-__device__ __forceinline__ TokenSource make_source(int w, int nU, int G, int32_t* ctr) {
+// P: the tokens that carry work (present tokens when the caller knows them,
+// else G); the counter is used only when there are 8 of them per worker.
+__device__ __forceinline__ TokenSource make_source(int w, int nU, int G, int32_t* ctr, int P) {
     TokenSource s;
     s.w = w;
     s.nU = nU;
     s.G = G;
     s.i = 0;
     s.ctr = ctr;
-    s.dyn = G >= 8 * nU;
+    s.dyn = G >= 8 * nU && P >= 8 * nU;
     s.R = s.dyn ? max(0, (int)((7LL * G) / (8LL * nU)) - 1) : (G + nU - 1) / nU;
     return s;
 }
@@ -261,6 +263,10 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
         }
     }
 
+    // Present tokens of the block, into the call's accumulator.
+    const int present = __syncthreads_count(g < p.G && mask != 0u);
+    if (tid == 0 && present > 0) atomicAdd(p.pacc, present);
+
     // Last block to finish turns the tile histogram into per-tile bases.
     __threadfence();
     __syncthreads();
@@ -268,6 +274,7 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    if (tid == 0) *p.ptotal = atomicExch(p.pacc, 0);  // present tokens of the call; reset for the next
     for (int pe = warp; pe < W; pe += kCountWarps) {
         int running = 0;
         for (int t0 = 0; t0 < p.numTiles; t0 += 32 * 8) {
@@ -456,13 +463,30 @@ __device__ __forceinline__ int active_engines(const ScatterParams& p, int nwarps
 // costs no latency on the copy path.
 struct GlobalFeed {
     TokenSource src;
-    int tA, tB, tC;  // candidates, in the order handed out (lane 0)
+    int tA, tB, tC;  // dynamic hand-out: candidates, in the order handed out (lane 0)
     uint32_t mA, mB;  // masks of A and B
+    // Static hand-out only (fewer than 8 present tokens per worker): the
+    // worker's rounds are scanned 32 at a time, lane l loading the mask of
+    // round i0 + l; the next 32 masks are loaded while these are used.
+    int i0;
+    uint32_t pm;     // present rounds of [i0, i0 + 32) not yet handed out
+    uint32_t mnext;  // this lane's mask in the next 32 rounds
 
-    __device__ __forceinline__ void init(const ScatterParams& p, int worker, int nWorkers, int lane) {
-        src = make_source(worker, nWorkers, p.G, p.work);
+    __device__ __forceinline__ uint32_t round_mask(const ScatterParams& p, int i) const {
+        const long long t = src.w + (long long)i * src.nU;
+        return (i < src.R && t < p.G) ? __ldcg(p.tok_mask + t) : 0u;
+    }
+    __device__ __forceinline__ void init(const ScatterParams& p, int worker, int nWorkers, int P, int lane) {
+        src = make_source(worker, nWorkers, p.G, p.work, P);
         tA = tB = tC = p.G;
         mA = mB = 0u;
+        if (!src.dyn) {
+            i0 = 0;
+            const uint32_t m0 = round_mask(p, lane);
+            mnext = round_mask(p, 32 + lane);
+            pm = __ballot_sync(kFull, m0 != 0u);
+            return;
+        }
         if (lane == 0) {
             tA = source_next(src);
             tB = source_next(src);
@@ -473,6 +497,17 @@ struct GlobalFeed {
     }
     // Next present token (warp-uniform), or p.G.
     __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
+        if (!src.dyn) {
+            while (pm == 0u) {
+                i0 += 32;
+                if (i0 >= src.R) return p.G;
+                pm = __ballot_sync(kFull, mnext != 0u);
+                mnext = round_mask(p, i0 + 32 + lane);
+            }
+            const int l = __ffs(pm) - 1;
+            pm &= pm - 1;
+            return src.w + (i0 + l) * src.nU;
+        }
         int found = p.G;
         if (lane == 0) {
             while (tA < p.G) {
@@ -678,10 +713,11 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
 template <int kPend>
 __device__ __forceinline__ void global_copy_engines(const ScatterParams& p, const EngineSmem& es, int lane,
                                                     int warp, int nwarps) {
+    const int P = p.ptotal != nullptr ? __ldcg(p.ptotal) : p.G;  // present tokens of the call
     const int engines = active_engines(p, nwarps, lane);
     if (warp >= engines) return;  // this engine's stages stay unused
     GlobalFeed feed;
-    feed.init(p, blockIdx.x * engines + warp, gridDim.x * engines, lane);
+    feed.init(p, blockIdx.x * engines + warp, gridDim.x * engines, P, lane);
     copy_engine<kPend>(p, es, lane, feed);
 }
 
@@ -1188,7 +1224,7 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
     // number of destinations, so a purely static split would leave a tail);
     // the next token and its routing row are fetched one token ahead.
     TokenSource src = make_source(blockIdx.x * (blockDim.x >> 5) + warp, gridDim.x * (blockDim.x >> 5),
-                                  p.G, p.work);
+                                  p.G, p.work, p.G);
     int next = 0;
     if (lane == 0) next = source_next(src);
     int g = __shfl_sync(kFull, next, 0);

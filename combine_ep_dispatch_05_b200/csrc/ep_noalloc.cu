@@ -119,11 +119,14 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         int32_t* tile_base = reinterpret_cast<int32_t*>(base + L.tile_base);
         uint32_t* ticket = reinterpret_cast<uint32_t*>(base + L.ticket);
         int32_t* work = reinterpret_cast<int32_t*>(base + L.work);
+        int32_t* pacc = reinterpret_cast<int32_t*>(base + L.pacc);
+        int32_t* ptotal = reinterpret_cast<int32_t*>(base + L.ptotal);
         int32_t* err = reinterpret_cast<int32_t*>(base + L.err);
         cudaStream_t s = static_cast<cudaStream_t>(stream);
 
         // The scratch keeps whatever the previous call left: the tile ticket,
-        // the scatter's token counter and the error word must start at zero.
+        // the scatter's token counter, the present-token sum and the error
+        // word must start at zero.
         if ((e = cudaMemsetAsync(ticket, 0, 512, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
 
@@ -158,6 +161,8 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         rp.recv_count = recv_count;
         rp.ticket = ticket;
         rp.work = work;
+        rp.pacc = pacc;
+        rp.ptotal = ptotal;
         rp.err = err;
         rp.G = (int)G;
         rp.W = W;
@@ -177,6 +182,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         sp.tok_mask = tok_mask;
         sp.tile_base = tile_base;
         sp.work = work;
+        sp.ptotal = ptotal;
         sp.recv_x = static_cast<uint8_t*>(recv_x);
         sp.recv_meta = recv_meta;
         sp.err = err;
