@@ -29,8 +29,7 @@ struct EpPlan {
     int32_t* tile_base;
     uint32_t* ticket;
     int32_t* work;
-    int32_t* pacc;        // route_count's present-token sum and the call's total
-    int32_t* ptotal;
+    int32_t* ptotal;      // route_count's present-token total (last-block scan)
     int32_t* cwork;
     uint32_t* cdone;
     int32_t* chunk_cnt;   // fused dispatch: [ceil(G/32)][W]
@@ -39,6 +38,7 @@ struct EpPlan {
     uint32_t* fdone;
     int32_t* err;
     size_t scatterSmem;
+    size_t baseSmem;      // > 0: the scatter scans the tile counts into this much shared memory
     bool fused;           // route + scan + scatter in one cooperative launch
     bool ll;              // small-batch single launch (dispatch_ll)
     size_t llSmem;        // its dynamic shared memory
@@ -320,18 +320,33 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             return nullptr;
         }
         Geometry geo = pick_geometry(cfg, true);
-        size_t smem = 0;
+        size_t smem = 0, baseSmem = 0;
+        const char* fusedEnv = std::getenv("EP_DISPATCH_FUSED");
+        const bool wantFused = fusedEnv && std::strcmp(fusedEnv, "1") == 0;
         if (geo.scatterMode == ep::kScatterTma) {
-            smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
-            while (smem > (size_t)smemOptin && geo.scatterStages > geo.scatterPend + 1) {
+            // The TMA scatter scans route_count's tile counts itself when
+            // they fit a few KB of shared memory (route_count then ends
+            // without a last-block scan); the fused dispatch has its own.
+            const int numTiles =
+                (int)(((long long)cfg->worldSize * cfg->maxTokPerRank + ep::kCountTile - 1) / ep::kCountTile);
+            const size_t bs = ep::scatter_base_smem_bytes(numTiles, cfg->worldSize);
+            const char* scanEnv = std::getenv("EP_SCATTER_SCAN");
+            const bool scanInRoute = scanEnv && std::strcmp(scanEnv, "route") == 0;
+            if (!wantFused && !scanInRoute && bs <= ep::kMaxBaseSmemBytes) baseSmem = bs;
+            const size_t limit = (size_t)smemOptin - 1024;  // the kernels' static shared memory
+            auto total = [&]() {
+                return baseSmem + ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+            };
+            smem = total();
+            while (smem > limit && geo.scatterStages > geo.scatterPend + 1) {
                 --geo.scatterStages;
-                smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+                smem = total();
             }
-            while (smem > (size_t)smemOptin && geo.scatterWarps > 1) {
+            while (smem > limit && geo.scatterWarps > 1) {
                 --geo.scatterWarps;
-                smem = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+                smem = total();
             }
-            if (smem > (size_t)smemOptin) {
+            if (smem > limit) {
                 fail(EP_ERR_INVALID, "row piece of %d bytes does not fit shared memory", geo.chunkBytes);
                 return nullptr;
             }
@@ -368,9 +383,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         // request (EP_DISPATCH_FUSED=1): on B200 the two launches of
         // route_count + scatter_rows measured faster at every size (main
         // workload 476 vs 500 us, ct=1 workload 17.4 vs 20.5 us).
-        bool fused = false;
-        if (const char* f = std::getenv("EP_DISPATCH_FUSED"))
-            fused = geo.scatterMode == ep::kScatterTma && std::strcmp(f, "1") == 0;
+        bool fused = wantFused && geo.scatterMode == ep::kScatterTma;
         int coop = 0;
         if (fused && (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop))
             fused = false;
@@ -431,6 +444,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             plan->barrierSlack = std::strcmp(t, "1") == 0 ? 1u : 0u;
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
+        plan->baseSmem = fused ? 0 : baseSmem;
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
         plan->maxRecv = plan->info.maxRecv;
 
@@ -454,7 +468,6 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->tile_base = reinterpret_cast<int32_t*>(base + L.tile_base);
         plan->ticket = reinterpret_cast<uint32_t*>(base + L.ticket);
         plan->work = reinterpret_cast<int32_t*>(base + L.work);
-        plan->pacc = reinterpret_cast<int32_t*>(base + L.pacc);
         plan->ptotal = reinterpret_cast<int32_t*>(base + L.ptotal);
         plan->cwork = reinterpret_cast<int32_t*>(base + L.cwork);
         plan->cdone = reinterpret_cast<uint32_t*>(base + L.cdone);
@@ -554,8 +567,8 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         rp.recv_count = recv_count;
         rp.ticket = plan->ticket;
         rp.work = plan->work;
-        rp.pacc = plan->pacc;
         rp.ptotal = plan->ptotal;
+        rp.lastScan = plan->baseSmem == 0 ? 1 : 0;
         rp.err = plan->err;
         rp.G = plan->G;
         rp.W = c.worldSize;
@@ -619,6 +632,7 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         if (plan->fused) {
             // One cooperative launch: routing phase, chunk scan, copy engines.
             sp.baseShift = 5;
+            sp.baseStride = c.worldSize;
             sp.tile_base = plan->chunk_base;
             sp.w = c.useWeights ? topk_w : nullptr;
             sp.tok_mask_w = plan->tok_mask;
@@ -638,6 +652,10 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         e = ep::launch_route_count(rp, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
         sp.baseShift = 8;  // route_count's 256-token tiles
+        sp.baseStride = c.worldSize + 1;
+        sp.tile_cnt = plan->tile_cnt;
+        sp.numTiles = plan->info.numTiles;
+        sp.baseSmemBytes = (int)plan->baseSmem;
         sp.ptotal = plan->ptotal;
         e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend,
                                     plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);

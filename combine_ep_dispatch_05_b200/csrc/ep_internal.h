@@ -30,15 +30,15 @@ struct RouteParams {
     const float* w;         // [G][k] or nullptr (useWeights == 0)
     int2* route;            // [G][W]: (tile-local rank or -1, weight-sum bits)
     uint32_t* tok_mask;     // [G]: destination mask of each token
-    int32_t* tile_cnt;      // [numTiles][W]
-    int32_t* tile_base;     // [numTiles][W], written by the last block
-    int32_t* recv_count;    // [W]
+    int32_t* tile_cnt;      // [numTiles][W + 1]: rows at each destination, present tokens
+    int32_t* tile_base;     // [numTiles][W + 1], written by the last block (lastScan)
+    int32_t* recv_count;    // [W], stored by the last block (lastScan)
     uint32_t* ticket;       // blocks finished this call; the last block resets it
-    int32_t* work;          // scatter token counter; the last block resets it
-    int32_t* pacc;          // present tokens, summed over the blocks (the last block resets it)
-    int32_t* ptotal;        // present tokens of the call, stored by the last block
+    int32_t* work;          // scatter token counter; block 0 resets it
+    int32_t* ptotal;        // present tokens of the call, stored by the last block (lastScan)
     int32_t* err;           // device error word
     int G, W, k, nEpr, E, numTiles, maxRecv, useWeights;
+    int lastScan;           // 1: the last block scans the tile counts; 0: the scatter does
 };
 
 struct ScatterParams {
@@ -46,9 +46,13 @@ struct ScatterParams {
     const int32_t* idx;        // [G][k]
     int2* route;               // [G][W]: in: tile-local rank; out: slot
     const uint32_t* tok_mask;  // [G]: destination mask of each token
-    const int32_t* tile_base;  // [numTiles][W]
+    const int32_t* tile_base;  // [numTiles][baseStride]: bases computed in global memory, or
+    const int32_t* tile_cnt;   // [numTiles][W + 1]: route_count's counts, scanned by each block
+    int baseStride;            // W + 1 (route_count tiles) or W (fused chunks)
+    int baseSmemBytes;         // > 0: each block scans tile_cnt into this much shared memory
+    int numTiles;
     int32_t* work;             // next token to hand out (starts at 0 each call)
-    const int32_t* ptotal;     // present tokens of the call (route_count), or nullptr: unknown
+    const int32_t* ptotal;     // present tokens of the call (route_count's last block), or nullptr
     uint8_t* recv_x;           // [W][maxRecv][rowBytes]
     int32_t* recv_meta;        // [W][maxRecv][M]
     int32_t* err;
@@ -104,11 +108,10 @@ struct CombineParams {
 // present-token list, the counters (one 256-byte region: tile ticket, scatter
 // token counter, combine token counter, combine blocks done, fused grid
 // barrier, fused blocks done, low-latency tile ticket, blocks done, call epoch
-// and present total, route_count's present-token sum and total), error word.
+// and present total, route_count's present-token total), error word.
 struct ScratchLayout {
     size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base, ll_status, ll_agg, ll_plist;
-    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, pacc, ptotal, err,
-        total;
+    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, ptotal, err, total;
 };
 
 inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
@@ -118,8 +121,8 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
     L.route = 0;
     L.tok_mask = L.route + up(sizeof(int2) * (size_t)G * W);
     L.tile_cnt = L.tok_mask + up(sizeof(uint32_t) * (size_t)G);
-    L.tile_base = L.tile_cnt + up(sizeof(int32_t) * (size_t)numTiles * W);
-    L.chunk_cnt = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * W);
+    L.tile_base = L.tile_cnt + up(sizeof(int32_t) * (size_t)numTiles * (W + 1));
+    L.chunk_cnt = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * (W + 1));
     L.chunk_base = L.chunk_cnt + up(sizeof(int32_t) * numChunks32 * W);
     const size_t llTiles = (size_t)(G < kLlMaxTiles ? G : kLlMaxTiles);
     L.ll_status = L.chunk_base + up(sizeof(int32_t) * numChunks32 * W);
@@ -135,8 +138,7 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
     L.ll_done = L.ticket + 28;
     L.ll_epoch = L.ticket + 32;
     L.ll_ptotal = L.ticket + 40;
-    L.pacc = L.ticket + 48;
-    L.ptotal = L.ticket + 52;
+    L.ptotal = L.ticket + 48;
     L.err = L.ticket + 256;
     L.total = L.err + 256;
     return L;
@@ -170,6 +172,10 @@ cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, 
 
 // Shared-memory bytes the scatter kernel needs for a geometry.
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride);
+// Shared memory for the tile bases when the scatter scans route_count's tile
+// counts itself ([numTiles][W + 1] ints, rounded up to 128 bytes).
+size_t scatter_base_smem_bytes(int numTiles, int W);
+constexpr size_t kMaxBaseSmemBytes = 16384;
 // Opt the TMA scatter kernel in to `bytes` of dynamic shared memory.
 cudaError_t scatter_set_smem(int pend, size_t bytes);
 // Blocks of each kernel that fit on one SM (occupancy calculator).

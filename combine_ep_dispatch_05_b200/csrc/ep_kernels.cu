@@ -207,7 +207,7 @@ __device__ __forceinline__ uint32_t route_token(const int32_t* idx, const float*
 
 template <int kW, int kK>
 __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams p) {
-    __shared__ int s_wcnt[kCountWarps][kW];
+    __shared__ int s_wcnt[kCountWarps][kW + 1];
     __shared__ int s_wpre[kCountWarps][kW];
     __shared__ int s_last;
 
@@ -216,7 +216,9 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = blockIdx.x * kCountTile + tid;
-    const int W = p.W, k = p.k;
+    const int W = p.W, k = p.k, C = W + 1;
+    // The previous call's scatter has finished: its token counter restarts.
+    if (blockIdx.x == 0 && tid == 0) *p.work = 0;
 
     uint32_t mask = 0;
     bool bad = false;
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     if (g < p.G) mask = route_token<kW, kK>(p.idx, p.w, g, k, p.nEpr, p.E, ws, bad);
     if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
 
-    // Per-warp histogram by ballot.
+    // Per-warp histogram by ballot; column W counts the present tokens.
 #pragma unroll
     for (int pe = 0; pe < kW; ++pe) {
         if (pe < W) {
@@ -232,15 +234,17 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
             if (lane == 0) s_wcnt[warp][pe] = __popc(b);
         }
     }
+    const uint32_t bp = __ballot_sync(kFull, mask != 0u);
+    if (lane == 0) s_wcnt[warp][W] = __popc(bp);
     __syncthreads();
-    if (tid < W) {
+    if (tid < C) {
         int run = 0;
 #pragma unroll
         for (int w = 0; w < kCountWarps; ++w) {
-            s_wpre[w][tid] = run;
+            if (tid < W) s_wpre[w][tid] = run;
             run += s_wcnt[w][tid];
         }
-        p.tile_cnt[blockIdx.x * W + tid] = run;
+        p.tile_cnt[blockIdx.x * C + tid] = run;
     }
     __syncthreads();
 
@@ -263,26 +267,26 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
         }
     }
 
-    // Present tokens of the block, into the call's accumulator.
-    const int present = __syncthreads_count(g < p.G && mask != 0u);
-    if (tid == 0 && present > 0) atomicAdd(p.pacc, present);
+    // When the scatter scans the tile counts itself, this block is done.
+    if (!p.lastScan) return;
 
-    // Last block to finish turns the tile histogram into per-tile bases.
+    // Otherwise the last block to finish turns the tile histogram into
+    // per-tile bases (column W: present tokens before the tile), stores
+    // recv_count and the call's present-token total.
     __threadfence();
     __syncthreads();
     if (tid == 0) s_last = (atomicAdd(p.ticket, 1u) == (unsigned)(p.numTiles - 1));
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    if (tid == 0) *p.ptotal = atomicExch(p.pacc, 0);  // present tokens of the call; reset for the next
-    for (int pe = warp; pe < W; pe += kCountWarps) {
+    for (int pe = warp; pe < C; pe += kCountWarps) {
         int running = 0;
         for (int t0 = 0; t0 < p.numTiles; t0 += 32 * 8) {
             int v[8];  // 8 rows of 32 tiles: all loads in flight before the scans
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int t = t0 + 32 * u + lane;
-                v[u] = t < p.numTiles ? __ldcg(p.tile_cnt + (size_t)t * W + pe) : 0;
+                v[u] = t < p.numTiles ? __ldcg(p.tile_cnt + (size_t)t * C + pe) : 0;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -293,19 +297,73 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
                     const int n = __shfl_up_sync(kFull, incl, off);
                     if (lane >= off) incl += n;
                 }
-                if (t < p.numTiles) p.tile_base[(size_t)t * W + pe] = running + incl - v[u];
+                if (t < p.numTiles) p.tile_base[(size_t)t * C + pe] = running + incl - v[u];
                 running += __shfl_sync(kFull, incl, 31);
             }
         }
         if (lane == 0) {
-            p.recv_count[pe] = running;  // stored, not accumulated
-            if (running > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+            if (pe < W) {
+                p.recv_count[pe] = running;  // stored, not accumulated
+                if (running > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+            } else {
+                *p.ptotal = running;
+            }
         }
     }
-    if (tid == 0) {  // ready for the scatter and for the next call (graph replay too)
-        *p.work = 0;
-        *p.ticket = 0u;
+    if (tid == 0) *p.ticket = 0u;  // ready for the next call (graph replay too)
+}
+
+// The scatter's own scan of route_count's tile counts ([numTiles][W + 1]),
+// by one block into its shared memory: s_base[t][pe] = rows at pe of the
+// tiles before t (column W: present tokens). Block 0 stores recv_count.
+// Returns the call's present tokens; *rows = the rows of all destinations.
+// Returns -1 (after setting EP_DEVERR_TIMEOUT) when the copy of the counts
+// did not arrive within the bounded wait.
+__device__ int scan_tile_bases(const ScatterParams& p, int* s_base, int* rows) {
+    __shared__ int s_tot[kMaxWorld + 1];
+    __shared__ __align__(8) uint64_t s_bar;
+    const int C = p.W + 1, n = p.numTiles * C;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    // One bulk copy brings the whole table (rounded up to 16 bytes: the
+    // table's region is padded to 256) into shared memory.
+    const uint32_t bar = smem_addr(&s_bar);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1u);
+        mbar_fence_init();
+        const uint32_t bytes = ((uint32_t)n * 4u + 15u) & ~15u;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load(smem_addr(s_base), p.tile_cnt, bytes, bar);
     }
+    __syncthreads();
+    if (!__syncthreads_and(mbar_wait_bounded(bar, 0u))) {
+        if (threadIdx.x == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
+        return -1;
+    }
+    for (int col = warp; col < C; col += nwarps) {
+        int running = 0;
+        for (int t0 = 0; t0 < p.numTiles; t0 += 32) {
+            const int t = t0 + lane;
+            const int v = t < p.numTiles ? s_base[t * C + col] : 0;
+            int incl = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int m = __shfl_up_sync(kFull, incl, off);
+                if (lane >= off) incl += m;
+            }
+            if (t < p.numTiles) s_base[t * C + col] = running + incl - v;
+            running += __shfl_sync(kFull, incl, 31);
+        }
+        if (lane == 0) s_tot[col] = running;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && (int)threadIdx.x < p.W) {
+        p.recv_count[threadIdx.x] = s_tot[threadIdx.x];  // stored, not accumulated
+        if (s_tot[threadIdx.x] > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+    }
+    int r = 0;
+    for (int pe = 0; pe < p.W; ++pe) r += s_tot[pe];
+    *rows = r;
+    return s_tot[p.W];
 }
 
 // =====================================================================
@@ -323,7 +381,8 @@ struct TokenInputs {
     float wt;  // lane < k: topk weight (list feed only)
 };
 
-__device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p, int g, int lane) {
+__device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p, int g, int lane,
+                                                       const int* s_base) {
     TokenInputs in;
     in.h = g;
     in.g = g;
@@ -331,7 +390,8 @@ __device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p,
     const int W = p.W;
     // routing data written by other blocks (or the previous kernel): read through L2
     in.rr = lane < W ? __ldcg(p.route + (size_t)g * W + lane) : make_int2(-1, 0);
-    in.base = lane < W ? __ldcg(p.tile_base + (size_t)(g >> p.baseShift) * W + lane) : 0;
+    const size_t bi = (size_t)(g >> p.baseShift) * p.baseStride + lane;
+    in.base = lane < W ? (s_base != nullptr ? s_base[bi] : __ldcg(p.tile_base + bi)) : 0;
     in.e = lane < p.k ? p.idx[(size_t)g * p.k + lane] : -1;
     return in;
 }
@@ -442,12 +502,14 @@ __device__ __forceinline__ EngineSmem engine_smem_init(uint8_t* smem, const Scat
 // 5.3); at a low fan-out the per-token latency chain dominates and every
 // engine helps (skewed routing, fan-out 2.9: 302 vs 335 us). The counts of
 // this dispatch (recv_count, complete before the call) decide.
-__device__ __forceinline__ int active_engines(const ScatterParams& p, int nwarps, int lane) {
+// rows: the call's rows at all destinations, or -1: read them from recv_count.
+__device__ __forceinline__ int active_engines(const ScatterParams& p, int nwarps, int lane, int rows) {
     if (p.fanoutSwitch <= 0 || nwarps <= 2) return nwarps;
-    const int cnt = lane < p.W ? __ldcg(p.recv_count + lane) : 0;
-    int rows = cnt;
+    if (rows < 0) {
+        rows = lane < p.W ? __ldcg(p.recv_count + lane) : 0;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) rows += __shfl_xor_sync(kFull, rows, off);
+        for (int off = 16; off > 0; off >>= 1) rows += __shfl_xor_sync(kFull, rows, off);
+    }
     return (long long)rows * 100 > (long long)p.fanoutSwitch * p.G ? nwarps - 1 : nwarps;
 }
 
@@ -471,12 +533,15 @@ struct GlobalFeed {
     int i0;
     uint32_t pm;     // present rounds of [i0, i0 + 32) not yet handed out
     uint32_t mnext;  // this lane's mask in the next 32 rounds
+    const int* s_base;  // tile bases in shared memory, or nullptr: in global memory
 
     __device__ __forceinline__ uint32_t round_mask(const ScatterParams& p, int i) const {
         const long long t = src.w + (long long)i * src.nU;
         return (i < src.R && t < p.G) ? __ldcg(p.tok_mask + t) : 0u;
     }
-    __device__ __forceinline__ void init(const ScatterParams& p, int worker, int nWorkers, int P, int lane) {
+    __device__ __forceinline__ void init(const ScatterParams& p, int worker, int nWorkers, int P, int lane,
+                                         const int* bases) {
+        s_base = bases;
         src = make_source(worker, nWorkers, p.G, p.work, P);
         tA = tB = tC = p.G;
         mA = mB = 0u;
@@ -528,7 +593,7 @@ struct GlobalFeed {
     }
     __device__ __forceinline__ int row(const ScatterParams&, int h) const { return h; }
     __device__ __forceinline__ TokenInputs load(const ScatterParams& p, int h, int lane) const {
-        return load_token_inputs(p, h, lane);
+        return load_token_inputs(p, h, lane, s_base);
     }
     __device__ __forceinline__ uint32_t prepare(const ScatterParams& p, const TokenInputs& in, int lane,
                                                 int& my_slot) const {
@@ -710,25 +775,36 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
 
 // Split-dispatch copy engines: the engines of this block that the fan-out
 // leaves active take tokens from the shared hand-out.
+// P: present tokens of the call; rows: its rows at all destinations (-1:
+// read recv_count); s_base: tile bases in shared memory, or nullptr.
 template <int kPend>
 __device__ __forceinline__ void global_copy_engines(const ScatterParams& p, const EngineSmem& es, int lane,
-                                                    int warp, int nwarps) {
-    const int P = p.ptotal != nullptr ? __ldcg(p.ptotal) : p.G;  // present tokens of the call
-    const int engines = active_engines(p, nwarps, lane);
+                                                    int warp, int nwarps, int P, int rows, const int* s_base) {
+    const int engines = active_engines(p, nwarps, lane, rows);
     if (warp >= engines) return;  // this engine's stages stay unused
     GlobalFeed feed;
-    feed.init(p, blockIdx.x * engines + warp, gridDim.x * engines, P, lane);
+    feed.init(p, blockIdx.x * engines + warp, gridDim.x * engines, P, lane, s_base);
     copy_engine<kPend>(p, es, lane, feed);
 }
 
+// Shared memory: [tile bases, when the scatter scans them: baseSmemBytes]
+// [the copy engines' barriers, rings and stages].
 template <int kPend>
 __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(ScatterParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
+    int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem) : nullptr;
+    const EngineSmem es = engine_smem_init(smem + p.baseSmemBytes, p, warp, nwarps, lane);
     pdl_wait();     // routing written by route_count is visible from here on
     pdl_trigger();
-    global_copy_engines<kPend>(p, es, lane, warp, nwarps);
+    int P, rows = -1;
+    if (s_base != nullptr) {
+        P = scan_tile_bases(p, s_base, &rows);
+        if (P < 0) return;  // the counts did not arrive: nothing is copied
+    } else {
+        P = p.ptotal != nullptr ? __ldcg(p.ptotal) : p.G;
+    }
+    global_copy_engines<kPend>(p, es, lane, warp, nwarps, P, rows, s_base);
 }
 
 // =====================================================================
@@ -1056,7 +1132,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kerne
     ok = ok && grid_barrier(p.bar, 2u * gridDim.x + p.barrierSlack);
 
     // 3. copy engines
-    if (ok) global_copy_engines<1>(p, es, lane, warp, nwarps);
+    if (ok) global_copy_engines<1>(p, es, lane, warp, nwarps, p.G, -1, nullptr);
     else if (threadIdx.x == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
 
     // The last block to finish resets the counters for the next call.
@@ -1095,7 +1171,7 @@ __global__ void __launch_bounds__(256) ep_scatter_rows_regs_kernel(ScatterParams
         const int lr = lane < p.W ? p.route[(size_t)g * p.W + lane].x : -1;
         if (__ballot_sync(kFull, lr >= 0) == 0u) continue;
         int my_slot;
-        const uint32_t mask = token_slots_and_meta(p, load_token_inputs(p, g, lane), lane, my_slot);
+        const uint32_t mask = token_slots_and_meta(p, load_token_inputs(p, g, lane, nullptr), lane, my_slot);
         const uint8_t* src = p.x + (size_t)g * p.rowBytes;
         for (long long v0 = 0; v0 < V; v0 += 32LL * kRegVec) {
             uint4 buf[kRegVec];
@@ -1305,6 +1381,10 @@ cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s) {
         e = p.k <= 8 ? go(ep_route_count_kernel<32, 8>) : p.k <= 16 ? go(ep_route_count_kernel<32, 16>)
                                                                  : go(ep_route_count_kernel<32, 32>);
     return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+size_t scatter_base_smem_bytes(int numTiles, int W) {
+    return ((size_t)numTiles * (size_t)(W + 1) * sizeof(int) + 127) & ~(size_t)127;
 }
 
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride) {

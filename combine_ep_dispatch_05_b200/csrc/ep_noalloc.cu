@@ -119,14 +119,12 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         int32_t* tile_base = reinterpret_cast<int32_t*>(base + L.tile_base);
         uint32_t* ticket = reinterpret_cast<uint32_t*>(base + L.ticket);
         int32_t* work = reinterpret_cast<int32_t*>(base + L.work);
-        int32_t* pacc = reinterpret_cast<int32_t*>(base + L.pacc);
         int32_t* ptotal = reinterpret_cast<int32_t*>(base + L.ptotal);
         int32_t* err = reinterpret_cast<int32_t*>(base + L.err);
         cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-        // The scratch keeps whatever the previous call left: the tile ticket,
-        // the scatter's token counter, the present-token sum and the error
-        // word must start at zero.
+        // The scratch keeps whatever the previous call left: the tile ticket
+        // and the error word must start at zero.
         if ((e = cudaMemsetAsync(ticket, 0, 512, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
 
@@ -161,8 +159,8 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         rp.recv_count = recv_count;
         rp.ticket = ticket;
         rp.work = work;
-        rp.pacc = pacc;
         rp.ptotal = ptotal;
+        rp.lastScan = 1;  // the last block scans the tile counts
         rp.err = err;
         rp.G = (int)G;
         rp.W = W;
@@ -200,6 +198,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         sp.numChunks = (int)((sp.rowBytes + sp.chunkBytes - 1) / sp.chunkBytes);
         sp.stages = stages;
         sp.baseShift = 8;  // route_count's 256-token tiles
+        sp.baseStride = W + 1;
         if ((e = ep::launch_scatter_rows(sp, ep::kScatterTma, pend, ds.numSMs * perSm, warps, smem, s)) !=
             cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch scatter_rows: %s", cudaGetErrorString(e));
