@@ -64,6 +64,7 @@ struct ScatterParams {
     int stages;       // stages per copy engine (>= 2)
     int baseShift;    // tile_base has one row per 2^baseShift tokens (8: route_count tiles; 5: fused chunks)
     int fanoutSwitch;        // x100: above this mean fan-out (rows per token) one engine per block sits out (0: never)
+    int pdlEarly;            // 1: let the next kernel of the stream launch once this one starts copying
     const uint32_t* scales;  // [G][scaleWords] per-token scale rows, or nullptr
     uint32_t* recv_scales;   // [W][maxRecv][scaleWords]
     int scaleWords;          // 0: no scale rows
@@ -99,6 +100,7 @@ struct CombineParams {
     uint32_t* done;        // blocks finished; the last one resets work and done
     long long rowBytes;    // bytes of a y / out row (the combine leg's row)
     int G, W, maxRecv;
+    int pdlEarly;          // 1: let the next kernel of the stream launch once this one starts
 };
 
 // Byte offsets of the dispatch scratch regions (each 256-byte aligned):

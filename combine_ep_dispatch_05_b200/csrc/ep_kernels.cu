@@ -796,7 +796,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem) : nullptr;
     const EngineSmem es = engine_smem_init(smem + p.baseSmemBytes, p, warp, nwarps, lane);
     pdl_wait();     // routing written by route_count is visible from here on
-    pdl_trigger();
+    if (p.pdlEarly) pdl_trigger();  // else the next kernel launches as this one exits
     int P, rows = -1;
     if (s_base != nullptr) {
         P = scan_tile_bases(p, s_base, &rows);
@@ -1163,7 +1163,7 @@ __device__ __forceinline__ void st_v4(void* p, const uint4& v) {
 
 __global__ void __launch_bounds__(256) ep_scatter_rows_regs_kernel(ScatterParams p) {
     pdl_wait();
-    pdl_trigger();
+    if (p.pdlEarly) pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int nw = gridDim.x * (blockDim.x >> 5);
     const long long V = p.rowBytes / 16;
@@ -1291,7 +1291,7 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
     __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
     __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
     pdl_wait();  // y and the routing of the dispatch are visible from here on
-    pdl_trigger();
+    if (p.pdlEarly) pdl_trigger();  // else the next kernel launches as this one exits
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int V = (int)(p.rowBytes / 16);
     const int W = p.W;

@@ -199,6 +199,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         sp.stages = stages;
         sp.baseShift = 8;  // route_count's 256-token tiles
         sp.baseStride = W + 1;
+        sp.pdlEarly = 0;  // the next kernel launches as this one exits
         if ((e = ep::launch_scatter_rows(sp, ep::kScatterTma, pend, ds.numSMs * perSm, warps, smem, s)) !=
             cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch scatter_rows: %s", cudaGetErrorString(e));

@@ -156,7 +156,9 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * dispatch; 0, i.e. off, by default), EP_SCATTER_FANOUT_SWITCH (100 x
  * the mean fan-out above which one copy engine per block sits out; 375 by
  * default, 0 never), EP_SCATTER_SCAN ("route": route_count's last block scans
- * the tile counts even when the scatter could). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 makes the fused
+ * the tile counts even when the scatter could), EP_PDL_EARLY (1: scatter and
+ * combine let the next kernel of the stream launch when they start rather than
+ * as they exit). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 makes the fused
  * dispatch's grid barrier (with EP_DISPATCH_FUSED=1), or the low-latency
  * dispatch's wait for the counts of earlier tiles, unreachable, so that the
  * bounded wait runs out: the waiting blocks report EP_DEVERR_TIMEOUT, issue no

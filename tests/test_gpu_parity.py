@@ -287,6 +287,7 @@ def test_graph_capture_replay():
     {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "1", "EP_SCATTER_BLOCKS": "1"},  # fewer warps than W
     {"EP_LL_MAX_TOKENS": "0"},                               # split dispatch at this size
     {"EP_SCATTER_SCAN": "route"},                            # route_count's last block scans the counts
+    {"EP_PDL_EARLY": "1"},                                   # dependents launch when scatter / combine start
     {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "4"},   # four tiles of 512 tokens
     {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "7", "EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2",
      "EP_SCATTER_CHUNK": "512"},                             # many engines, rows in six pieces
