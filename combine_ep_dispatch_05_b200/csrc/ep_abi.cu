@@ -38,7 +38,10 @@ struct EpPlan {
     uint32_t* fdone;
     int32_t* err;
     size_t scatterSmem;
+    bool dense;           // large batches: route_count's earlier form, tile bases in global memory
     size_t baseSmem;      // > 0: the scatter scans the tile counts into this much shared memory
+    size_t baseOffset;    // its offset in the scatter's shared memory, and the engines'
+    size_t engineOffset;
     bool fused;           // route + scan + scatter in one cooperative launch
     bool ll;              // small-batch single launch (dispatch_ll)
     size_t llSmem;        // its dynamic shared memory
@@ -321,7 +324,17 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             return nullptr;
         }
         Geometry geo = pick_geometry(cfg, true);
-        size_t smem = 0, baseSmem = 0;
+        size_t smem = 0, baseSmem = 0, baseOffset = 0, engineOffset = 0;
+        // Batches above kDenseMinTokens tokens take route_count in its
+        // large-batch form with the dense copy path: on B200 the main
+        // workload's dispatch measured 470 us that way against 478 us with
+        // the sparse-batch machinery (present-token column, scatter-side
+        // scan), which pays off only for small batches (ct = 1: 15.3 vs
+        // 17.4 us). EP_DISPATCH_DENSE=0/1 overrides.
+        constexpr long long kDenseMinTokens = 16384;
+        const long long Gtok = (long long)cfg->worldSize * cfg->maxTokPerRank;
+        const int denseEnv = env_int("EP_DISPATCH_DENSE", -1, 0);
+        const bool dense = denseEnv >= 0 ? denseEnv != 0 : Gtok > kDenseMinTokens;
         const char* fusedEnv = std::getenv("EP_DISPATCH_FUSED");
         const bool wantFused = fusedEnv && std::strcmp(fusedEnv, "1") == 0;
         if (geo.scatterMode == ep::kScatterTma) {
@@ -333,11 +346,43 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             const size_t bs = ep::scatter_base_smem_bytes(numTiles, cfg->worldSize);
             const char* scanEnv = std::getenv("EP_SCATTER_SCAN");
             const bool scanInRoute = scanEnv && std::strcmp(scanEnv, "route") == 0;
-            if (!wantFused && !scanInRoute && bs <= ep::kMaxBaseSmemBytes) baseSmem = bs;
+            if (!wantFused && !scanInRoute && !dense && bs <= ep::kMaxBaseSmemBytes) baseSmem = bs;
             const size_t limit = (size_t)smemOptin - 1024;  // the kernels' static shared memory
+            // Layout (EP_SCATTER_LAYOUT, for sweeps): 0 tile bases first,
+            // then the engines; 1 engines first; 2 tile bases first, engines
+            // from the next 1 KB boundary.
+            const int layout = env_int("EP_SCATTER_LAYOUT", 0, 0);
             auto total = [&]() {
-                return baseSmem + ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+                const size_t eng = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+                if (baseSmem == 0) return eng;
+                if (layout == 1) return eng + baseSmem;
+                if (layout == 2) return ((baseSmem + 1023) & ~(size_t)1023) + eng;
+                return baseSmem + eng;
             };
+            auto offsets = [&](size_t* bo, size_t* eo) {
+                const size_t eng = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+                *bo = 0;
+                *eo = baseSmem;
+                if (baseSmem == 0) *eo = 0;
+                else if (layout == 1) *bo = eng, *eo = 0;
+                else if (layout == 2) *eo = (baseSmem + 1023) & ~(size_t)1023;
+            };
+            // The table must not cost a block per SM (7 KB rows: 2 blocks of
+            // 8 stages fit an SM without it, 1 with it).
+            if (baseSmem > 0) {
+                const size_t eng = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+                int with = 0, without = 0;
+                if ((e = ep::scatter_set_smem(geo.scatterPend, std::min(limit, eng + baseSmem + 1024))) !=
+                        cudaSuccess ||
+                    (e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps,
+                                                   std::min(limit, eng), &without)) != cudaSuccess ||
+                    (e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps,
+                                                   std::min(limit, eng + baseSmem), &with)) != cudaSuccess) {
+                    cuda_fail(e, "scatter occupancy");
+                    return nullptr;
+                }
+                if (with < without) baseSmem = 0;
+            }
             smem = total();
             while (smem > limit && geo.scatterStages > geo.scatterPend + 1) {
                 --geo.scatterStages;
@@ -351,6 +396,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
                 fail(EP_ERR_INVALID, "row piece of %d bytes does not fit shared memory", geo.chunkBytes);
                 return nullptr;
             }
+            offsets(&baseOffset, &engineOffset);
             if ((e = ep::scatter_set_smem(geo.scatterPend, smem)) != cudaSuccess) {
                 cuda_fail(e, "cudaFuncSetAttribute(scatter smem)");
                 return nullptr;
@@ -450,7 +496,10 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             plan->barrierSlack = std::strcmp(t, "1") == 0 ? 1u : 0u;
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
+        plan->dense = !fused && dense && geo.scatterMode == ep::kScatterTma;
         plan->baseSmem = fused ? 0 : baseSmem;
+        plan->baseOffset = fused ? 0 : baseOffset;
+        plan->engineOffset = fused ? 0 : engineOffset;
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
         plan->maxRecv = plan->info.maxRecv;
 
@@ -656,15 +705,17 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
             plan->dispatched = true;
             return EP_OK;
         }
-        e = ep::launch_route_count(rp, s);
+        e = ep::launch_route_count(rp, plan->dense, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
         sp.baseShift = 8;  // route_count's 256-token tiles
-        sp.baseStride = c.worldSize + 1;
+        sp.baseStride = plan->dense ? c.worldSize : c.worldSize + 1;
         sp.tile_cnt = plan->tile_cnt;
         sp.numTiles = plan->info.numTiles;
         sp.baseSmemBytes = (int)plan->baseSmem;
-        sp.ptotal = plan->ptotal;
-        e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend,
+        sp.baseOffset = (int)plan->baseOffset;
+        sp.engineOffset = (int)plan->engineOffset;
+        sp.ptotal = plan->dense ? nullptr : plan->ptotal;  // dense: every token counts as present
+        e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend, plan->dense,
                                     plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch scatter_rows");
         plan->dispatched = true;

@@ -50,6 +50,8 @@ struct ScatterParams {
     const int32_t* tile_cnt;   // [numTiles][W + 1]: route_count's counts, scanned by each block
     int baseStride;            // W + 1 (route_count tiles) or W (fused chunks)
     int baseSmemBytes;         // > 0: each block scans tile_cnt into this much shared memory
+    int baseOffset;            // shared-memory byte offsets of the tile bases and of the engines
+    int engineOffset;
     int numTiles;
     int32_t* work;             // next token to hand out (starts at 0 each call)
     const int32_t* ptotal;     // present tokens of the call (route_count's last block), or nullptr
@@ -147,13 +149,17 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
 }
 
 // Launchers (ep_kernels.cu). Each returns the cudaError_t of its launch.
-cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s);
+// dense: the large-batch form (tile counts at the W destinations only, last-block
+// scan, tile bases with stride W); else W + 1 columns, lastScan as set.
+cudaError_t launch_route_count(const RouteParams& p, bool dense, cudaStream_t s);
 // Scatter variants: TMA bulk copies staged in shared memory (kPend = bulk
 // store groups left draining when a stage is refilled), or plain 16-byte
 // register copies (no shared memory).
 constexpr int kScatterTma = 0;
 constexpr int kScatterRegs = 1;
-cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
+// dense: the large-batch instance (shared hand-out, tile bases in global
+// memory with stride W, no scan of its own).
+cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, bool dense, int blocks, int warps,
                                 size_t smem, cudaStream_t s);
 // fp32: float32 combine leg (an fp32 plan); bf16 otherwise.
 // tile: combine kernel instance (columns x rows per pass, blocks per SM), see ep_kernels.cu.

@@ -205,7 +205,11 @@ __device__ __forceinline__ uint32_t route_token(const int32_t* idx, const float*
     return mask;
 }
 
-template <int kW, int kK>
+// kDense: the form for large batches -- tile counts at the W destinations
+// only, scanned by the last block, which also restarts the scatter's token
+// counter. Otherwise the tile counts carry a column of present tokens (W + 1
+// columns) and the scatter may scan them itself (lastScan == 0).
+template <int kW, int kK, bool kDense>
 __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams p) {
     __shared__ int s_wcnt[kCountWarps][kW + 1];
     __shared__ int s_wpre[kCountWarps][kW];
@@ -216,9 +220,9 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = blockIdx.x * kCountTile + tid;
-    const int W = p.W, k = p.k, C = W + 1;
+    const int W = p.W, k = p.k, C = kDense ? W : W + 1;
     // The previous call's scatter has finished: its token counter restarts.
-    if (blockIdx.x == 0 && tid == 0) *p.work = 0;
+    if (!kDense && blockIdx.x == 0 && tid == 0) *p.work = 0;
 
     uint32_t mask = 0;
     bool bad = false;
@@ -234,8 +238,10 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
             if (lane == 0) s_wcnt[warp][pe] = __popc(b);
         }
     }
-    const uint32_t bp = __ballot_sync(kFull, mask != 0u);
-    if (lane == 0) s_wcnt[warp][W] = __popc(bp);
+    if (!kDense) {
+        const uint32_t bp = __ballot_sync(kFull, mask != 0u);
+        if (lane == 0) s_wcnt[warp][W] = __popc(bp);
+    }
     __syncthreads();
     if (tid < C) {
         int run = 0;
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     }
 
     // When the scatter scans the tile counts itself, this block is done.
-    if (!p.lastScan) return;
+    if (!kDense && !p.lastScan) return;
 
     // Otherwise the last block to finish turns the tile histogram into
     // per-tile bases (column W: present tokens before the tile), stores
@@ -310,7 +316,10 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
             }
         }
     }
-    if (tid == 0) *p.ticket = 0u;  // ready for the next call (graph replay too)
+    if (tid == 0) {  // ready for the scatter and for the next call (graph replay too)
+        if (kDense) *p.work = 0;
+        *p.ticket = 0u;
+    }
 }
 
 // The scatter's own scan of route_count's tile counts ([numTiles][W + 1]),
@@ -381,6 +390,8 @@ struct TokenInputs {
     float wt;  // lane < k: topk weight (list feed only)
 };
 
+// kSmemBase: the tile bases are in shared memory (s_base), else in global memory.
+template <bool kSmemBase>
 __device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p, int g, int lane,
                                                        const int* s_base) {
     TokenInputs in;
@@ -391,7 +402,8 @@ __device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p,
     // routing data written by other blocks (or the previous kernel): read through L2
     in.rr = lane < W ? __ldcg(p.route + (size_t)g * W + lane) : make_int2(-1, 0);
     const size_t bi = (size_t)(g >> p.baseShift) * p.baseStride + lane;
-    in.base = lane < W ? (s_base != nullptr ? s_base[bi] : __ldcg(p.tile_base + bi)) : 0;
+    if (kSmemBase) in.base = lane < W ? s_base[bi] : 0;
+    else in.base = lane < W ? __ldcg(p.tile_base + bi) : 0;
     in.e = lane < p.k ? p.idx[(size_t)g * p.k + lane] : -1;
     return in;
 }
@@ -518,40 +530,28 @@ __device__ __forceinline__ int active_engines(const ScatterParams& p, int nwarps
 // token's inputs (so that the engine can prefetch them one token ahead), and
 // prepares a token: its slots, routing-table entries and meta records.
 
-// Split dispatch: tokens from the shared hand-out (static rounds, then a
-// global counter); route_count's tile-local ranks plus the tile's base give
-// the slots. Two candidates are kept in flight ahead (the hand-out's answer
-// and then the token's destination mask), so finding the next present token
-// costs no latency on the copy path.
-struct GlobalFeed {
-    TokenSource src;
-    int tA, tB, tC;  // dynamic hand-out: candidates, in the order handed out (lane 0)
-    uint32_t mA, mB;  // masks of A and B
-    // Static hand-out only (fewer than 8 present tokens per worker): the
-    // worker's rounds are scanned 32 at a time, lane l loading the mask of
-    // round i0 + l; the next 32 masks are loaded while these are used.
-    int i0;
-    uint32_t pm;     // present rounds of [i0, i0 + 32) not yet handed out
-    uint32_t mnext;  // this lane's mask in the next 32 rounds
-    const int* s_base;  // tile bases in shared memory, or nullptr: in global memory
+// Split dispatch feeds: route_count's tile-local ranks plus the tile's base
+// give a token's slots. There is one feed per hand-out mode, each templated on
+// where the tile bases live, so that the per-token path has no branch on
+// either (the choice is made once per engine).
 
-    __device__ __forceinline__ uint32_t round_mask(const ScatterParams& p, int i) const {
-        const long long t = src.w + (long long)i * src.nU;
-        return (i < src.R && t < p.G) ? __ldcg(p.tok_mask + t) : 0u;
-    }
-    __device__ __forceinline__ void init(const ScatterParams& p, int worker, int nWorkers, int P, int lane,
+// Dense batches: tokens from the shared hand-out (static rounds, then a
+// global counter). Two candidates are kept in flight ahead (the hand-out's
+// answer and then the token's destination mask), so finding the next
+// present token costs no latency on the copy path.
+template <bool kSmemBase>
+struct DynFeed {
+    TokenSource src;
+    int tA, tB, tC;  // candidates, in the order handed out (lane 0)
+    uint32_t mA, mB;  // masks of A and B
+    const int* s_base;
+
+    __device__ __forceinline__ void init(const ScatterParams& p, const TokenSource& s0, int lane,
                                          const int* bases) {
+        src = s0;
         s_base = bases;
-        src = make_source(worker, nWorkers, p.G, p.work, P);
         tA = tB = tC = p.G;
         mA = mB = 0u;
-        if (!src.dyn) {
-            i0 = 0;
-            const uint32_t m0 = round_mask(p, lane);
-            mnext = round_mask(p, 32 + lane);
-            pm = __ballot_sync(kFull, m0 != 0u);
-            return;
-        }
         if (lane == 0) {
             tA = source_next(src);
             tB = source_next(src);
@@ -562,17 +562,6 @@ struct GlobalFeed {
     }
     // Next present token (warp-uniform), or p.G.
     __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
-        if (!src.dyn) {
-            while (pm == 0u) {
-                i0 += 32;
-                if (i0 >= src.R) return p.G;
-                pm = __ballot_sync(kFull, mnext != 0u);
-                mnext = round_mask(p, i0 + 32 + lane);
-            }
-            const int l = __ffs(pm) - 1;
-            pm &= pm - 1;
-            return src.w + (i0 + l) * src.nU;
-        }
         int found = p.G;
         if (lane == 0) {
             while (tA < p.G) {
@@ -593,7 +582,53 @@ struct GlobalFeed {
     }
     __device__ __forceinline__ int row(const ScatterParams&, int h) const { return h; }
     __device__ __forceinline__ TokenInputs load(const ScatterParams& p, int h, int lane) const {
-        return load_token_inputs(p, h, lane, s_base);
+        return load_token_inputs<kSmemBase>(p, h, lane, s_base);
+    }
+    __device__ __forceinline__ uint32_t prepare(const ScatterParams& p, const TokenInputs& in, int lane,
+                                                int& my_slot) const {
+        return token_slots_and_meta(p, in, lane, my_slot);
+    }
+};
+
+// Sparse batches (fewer than 8 present tokens per worker): static hand-out
+// only; the worker's rounds are scanned 32 at a time, lane l loading the
+// mask of round i0 + l, and the next 32 masks are loaded while these are
+// used.
+template <bool kSmemBase>
+struct StaticFeed {
+    TokenSource src;
+    int i0;
+    uint32_t pm;     // present rounds of [i0, i0 + 32) not yet handed out
+    uint32_t mnext;  // this lane's mask in the next 32 rounds
+    const int* s_base;
+
+    __device__ __forceinline__ uint32_t round_mask(const ScatterParams& p, int i) const {
+        const long long t = src.w + (long long)i * src.nU;
+        return (i < src.R && t < p.G) ? __ldcg(p.tok_mask + t) : 0u;
+    }
+    __device__ __forceinline__ void init(const ScatterParams& p, const TokenSource& s0, int lane,
+                                         const int* bases) {
+        src = s0;
+        s_base = bases;
+        i0 = 0;
+        const uint32_t m0 = round_mask(p, lane);
+        mnext = round_mask(p, 32 + lane);
+        pm = __ballot_sync(kFull, m0 != 0u);
+    }
+    __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
+        while (pm == 0u) {
+            i0 += 32;
+            if (i0 >= src.R) return p.G;
+            pm = __ballot_sync(kFull, mnext != 0u);
+            mnext = round_mask(p, i0 + 32 + lane);
+        }
+        const int l = __ffs(pm) - 1;
+        pm &= pm - 1;
+        return src.w + (i0 + l) * src.nU;
+    }
+    __device__ __forceinline__ int row(const ScatterParams&, int h) const { return h; }
+    __device__ __forceinline__ TokenInputs load(const ScatterParams& p, int h, int lane) const {
+        return load_token_inputs<kSmemBase>(p, h, lane, s_base);
     }
     __device__ __forceinline__ uint32_t prepare(const ScatterParams& p, const TokenInputs& in, int lane,
                                                 int& my_slot) const {
@@ -777,24 +812,54 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
 // leaves active take tokens from the shared hand-out.
 // P: present tokens of the call; rows: its rows at all destinations (-1:
 // read recv_count); s_base: tile bases in shared memory, or nullptr.
+template <int kPend, bool kSmemBase>
+__device__ __forceinline__ void run_split_engine(const ScatterParams& p, const EngineSmem& es, int lane,
+                                                 const TokenSource& src, const int* s_base) {
+    if (src.dyn) {
+        DynFeed<kSmemBase> feed;
+        feed.init(p, src, lane, s_base);
+        copy_engine<kPend>(p, es, lane, feed);
+    } else {
+        StaticFeed<kSmemBase> feed;
+        feed.init(p, src, lane, s_base);
+        copy_engine<kPend>(p, es, lane, feed);
+    }
+}
+
 template <int kPend>
 __device__ __forceinline__ void global_copy_engines(const ScatterParams& p, const EngineSmem& es, int lane,
                                                     int warp, int nwarps, int P, int rows, const int* s_base) {
     const int engines = active_engines(p, nwarps, lane, rows);
     if (warp >= engines) return;  // this engine's stages stay unused
-    GlobalFeed feed;
-    feed.init(p, blockIdx.x * engines + warp, gridDim.x * engines, P, lane, s_base);
-    copy_engine<kPend>(p, es, lane, feed);
+    const TokenSource src = make_source(blockIdx.x * engines + warp, gridDim.x * engines, p.G, p.work, P);
+    if (s_base != nullptr) run_split_engine<kPend, true>(p, es, lane, src, s_base);
+    else run_split_engine<kPend, false>(p, es, lane, src, nullptr);
 }
 
-// Shared memory: [tile bases, when the scatter scans them: baseSmemBytes]
-// [the copy engines' barriers, rings and stages].
-template <int kPend>
+// Shared memory: the copy engines' barriers, rings and stages at
+// engineOffset, and the tile bases (when the scatter scans them) at
+// baseOffset. kDense: the instance for large batches, whose copy engines only
+// take the shared hand-out with tile bases from global memory (one code path,
+// as compact as the loop allows); the other instance also has the sparse
+// hand-out and the shared-memory tile bases.
+template <int kPend, bool kDense>
 __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(ScatterParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem) : nullptr;
-    const EngineSmem es = engine_smem_init(smem + p.baseSmemBytes, p, warp, nwarps, lane);
+    if (kDense) {
+        const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
+        pdl_wait();     // routing written by route_count is visible from here on
+        if (p.pdlEarly) pdl_trigger();  // else the next kernel launches as this one exits
+        const int engines = active_engines(p, nwarps, lane, -1);
+        if (warp >= engines) return;  // this engine's stages stay unused
+        DynFeed<false> feed;
+        feed.init(p, make_source(blockIdx.x * engines + warp, gridDim.x * engines, p.G, p.work, p.G), lane,
+                  nullptr);
+        copy_engine<kPend>(p, es, lane, feed);
+        return;
+    }
+    int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem + p.baseOffset) : nullptr;
+    const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, nwarps, lane);
     pdl_wait();     // routing written by route_count is visible from here on
     if (p.pdlEarly) pdl_trigger();  // else the next kernel launches as this one exits
     int P, rows = -1;
@@ -1171,7 +1236,7 @@ __global__ void __launch_bounds__(256) ep_scatter_rows_regs_kernel(ScatterParams
         const int lr = lane < p.W ? p.route[(size_t)g * p.W + lane].x : -1;
         if (__ballot_sync(kFull, lr >= 0) == 0u) continue;
         int my_slot;
-        const uint32_t mask = token_slots_and_meta(p, load_token_inputs(p, g, lane, nullptr), lane, my_slot);
+        const uint32_t mask = token_slots_and_meta(p, load_token_inputs<false>(p, g, lane, nullptr), lane, my_slot);
         const uint8_t* src = p.x + (size_t)g * p.rowBytes;
         for (long long v0 = 0; v0 < V; v0 += 32LL * kRegVec) {
             uint4 buf[kRegVec];
@@ -1368,18 +1433,26 @@ cudaError_t launch_pdl(void (*kernel)(P), int grid, int block, size_t smem, cuda
 }  // namespace
 
 // Instances by bounds on W and k (8, 16 or 32 each).
-cudaError_t launch_route_count(const RouteParams& p, cudaStream_t s) {
+namespace {
+template <bool kDense>
+cudaError_t launch_route_count_as(const RouteParams& p, cudaStream_t s) {
     auto go = [&](auto kernel) { return launch_pdl(kernel, p.numTiles, kCountTile, 0, s, p); };
-    cudaError_t e;
     if (p.W <= 8)
-        e = p.k <= 8 ? go(ep_route_count_kernel<8, 8>) : p.k <= 16 ? go(ep_route_count_kernel<8, 16>)
-                                                                : go(ep_route_count_kernel<8, 32>);
-    else if (p.W <= 16)
-        e = p.k <= 8 ? go(ep_route_count_kernel<16, 8>) : p.k <= 16 ? go(ep_route_count_kernel<16, 16>)
-                                                                 : go(ep_route_count_kernel<16, 32>);
-    else
-        e = p.k <= 8 ? go(ep_route_count_kernel<32, 8>) : p.k <= 16 ? go(ep_route_count_kernel<32, 16>)
-                                                                 : go(ep_route_count_kernel<32, 32>);
+        return p.k <= 8    ? go(ep_route_count_kernel<8, 8, kDense>)
+               : p.k <= 16 ? go(ep_route_count_kernel<8, 16, kDense>)
+                           : go(ep_route_count_kernel<8, 32, kDense>);
+    if (p.W <= 16)
+        return p.k <= 8    ? go(ep_route_count_kernel<16, 8, kDense>)
+               : p.k <= 16 ? go(ep_route_count_kernel<16, 16, kDense>)
+                           : go(ep_route_count_kernel<16, 32, kDense>);
+    return p.k <= 8    ? go(ep_route_count_kernel<32, 8, kDense>)
+           : p.k <= 16 ? go(ep_route_count_kernel<32, 16, kDense>)
+                       : go(ep_route_count_kernel<32, 32, kDense>);
+}
+}  // namespace
+
+cudaError_t launch_route_count(const RouteParams& p, bool dense, cudaStream_t s) {
+    const cudaError_t e = dense ? launch_route_count_as<true>(p, s) : launch_route_count_as<false>(p, s);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1395,37 +1468,55 @@ size_t scatter_smem_bytes(int warps, int stages, int chunkStride) {
 
 namespace {
 template <typename F>
-cudaError_t for_pend(int pend, F&& f) {
-    switch (pend) {
-        case 1: return f(ep_scatter_rows_kernel<1>);
-        case 2: return f(ep_scatter_rows_kernel<2>);
-        case 3: return f(ep_scatter_rows_kernel<3>);
+cudaError_t for_pend(int pend, bool dense, F&& f) {
+    switch (pend * 2 + (dense ? 1 : 0)) {
+        case 2: return f(ep_scatter_rows_kernel<1, false>);
+        case 3: return f(ep_scatter_rows_kernel<1, true>);
+        case 4: return f(ep_scatter_rows_kernel<2, false>);
+        case 5: return f(ep_scatter_rows_kernel<2, true>);
+        case 6: return f(ep_scatter_rows_kernel<3, false>);
+        case 7: return f(ep_scatter_rows_kernel<3, true>);
         default: return cudaErrorInvalidValue;
     }
 }
 }  // namespace
 
 cudaError_t scatter_set_smem(int pend, size_t bytes) {
-    return for_pend(pend, [&](auto k) {
-        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    });
+    for (int d = 0; d < 2; ++d) {
+        const cudaError_t e = for_pend(pend, d != 0, [&](auto k) {
+            return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        });
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t scatter_get_smem(int pend, int* bytes) {
-    return for_pend(pend, [&](auto k) {
+    int lim = 1 << 30;
+    for (int d = 0; d < 2; ++d) {
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, k);
-        *bytes = fa.maxDynamicSharedSizeBytes;
-        return e;
-    });
+        const cudaError_t e = for_pend(pend, d != 0, [&](auto k) { return cudaFuncGetAttributes(&fa, k); });
+        if (e != cudaSuccess) return e;
+        lim = fa.maxDynamicSharedSizeBytes < lim ? fa.maxDynamicSharedSizeBytes : lim;
+    }
+    *bytes = lim;
+    return cudaSuccess;
 }
 
 cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out) {
     if (mode == kScatterRegs)
         return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_scatter_rows_regs_kernel, warps * 32, 0);
-    return for_pend(pend, [&](auto k) {
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, warps * 32, smem);
-    });
+    int lo = 1 << 30;
+    for (int d = 0; d < 2; ++d) {
+        int n = 0;
+        const cudaError_t e = for_pend(pend, d != 0, [&](auto k) {
+            return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, warps * 32, smem);
+        });
+        if (e != cudaSuccess) return e;
+        lo = n < lo ? n : lo;
+    }
+    *out = lo;
+    return cudaSuccess;
 }
 
 namespace {
@@ -1447,13 +1538,13 @@ cudaError_t combine_blocks_per_sm(int warps, bool fp32, int tile, int* out) {
     return fp32 ? for_tile<CombineF32>(tile, occ) : for_tile<CombineBf16>(tile, occ);
 }
 
-cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, int blocks, int warps,
+cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, bool dense, int blocks, int warps,
                                 size_t smem, cudaStream_t s) {
     if (mode == kScatterRegs) {
         cudaError_t e = launch_pdl(ep_scatter_rows_regs_kernel, blocks, warps * 32, 0, s, p);
         return e != cudaSuccess ? e : cudaGetLastError();
     }
-    cudaError_t e = for_pend(pend, [&](auto k) { return launch_pdl(k, blocks, warps * 32, smem, s, p); });
+    cudaError_t e = for_pend(pend, dense, [&](auto k) { return launch_pdl(k, blocks, warps * 32, smem, s, p); });
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

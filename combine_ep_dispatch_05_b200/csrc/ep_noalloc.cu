@@ -170,7 +170,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         rp.numTiles = info.numTiles;
         rp.maxRecv = info.maxRecv;
         rp.useWeights = cfg->useWeights;
-        if ((e = ep::launch_route_count(rp, s)) != cudaSuccess)
+        if ((e = ep::launch_route_count(rp, false, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch route_count: %s", cudaGetErrorString(e));
 
         ep::ScatterParams sp{};
@@ -200,7 +200,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         sp.baseShift = 8;  // route_count's 256-token tiles
         sp.baseStride = W + 1;
         sp.pdlEarly = 0;  // the next kernel launches as this one exits
-        if ((e = ep::launch_scatter_rows(sp, ep::kScatterTma, pend, ds.numSMs * perSm, warps, smem, s)) !=
+        if ((e = ep::launch_scatter_rows(sp, ep::kScatterTma, pend, false, ds.numSMs * perSm, warps, smem, s)) !=
             cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch scatter_rows: %s", cudaGetErrorString(e));
         return EP_OK;

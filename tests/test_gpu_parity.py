@@ -58,6 +58,16 @@ def test_workload_parity_dispatch_families(name, ll, monkeypatch):
     run.close()
 
 
+@pytest.mark.parametrize("name", ["main", "skewed"])
+def test_large_batch_with_sparse_machinery(name, monkeypatch):
+    """The main shapes through the small-batch form of the split dispatch
+    (present-token column, scatter-side scan of the tile counts)."""
+    monkeypatch.setenv("EP_DISPATCH_DENSE", "0")
+    wl = workload(name)
+    run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
+    run.close()
+
+
 def _small_random_cfg(rng, W, T, h, k, nEpr, use_w, max_recv=0, dup=True, oob=False):
     E = W * nEpr
     lo = -2 if dup else 0
@@ -288,6 +298,9 @@ def test_graph_capture_replay():
     {"EP_LL_MAX_TOKENS": "0"},                               # split dispatch at this size
     {"EP_SCATTER_SCAN": "route"},                            # route_count's last block scans the counts
     {"EP_PDL_EARLY": "1"},                                   # dependents launch when scatter / combine start
+    {"EP_SCATTER_LAYOUT": "1"},                              # tile bases after the engines' stages
+    {"EP_SCATTER_LAYOUT": "2"},                              # engines' stages from a 1 KB boundary
+    {"EP_DISPATCH_DENSE": "1"},                              # route_count's large-batch form
     {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "4"},   # four tiles of 512 tokens
     {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "7", "EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2",
      "EP_SCATTER_CHUNK": "512"},                             # many engines, rows in six pieces
