@@ -299,6 +299,7 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info) {
             info->dispatchLowLatency = 1;
             info->scatterBlocks = (int)((G + llTile - 1) / llTile);
             info->scatterStages = llStages;
+            info->scratchBytes = (long long)ep::scratch_layout(G, cfg->worldSize, info->numTiles, true).total;
         }
         return EP_OK;
     } catch (...) {
@@ -503,7 +504,8 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
         plan->maxRecv = plan->info.maxRecv;
 
-        const ep::ScratchLayout L = ep::scratch_layout(plan->G, cfg->worldSize, plan->info.numTiles);
+        const ep::ScratchLayout L = ep::scratch_layout(plan->G, cfg->worldSize, plan->info.numTiles, plan->ll);
+        plan->info.scratchBytes = (long long)L.total;
         const size_t total = L.total;
         if ((e = cudaMalloc(&plan->scratch, total)) != cudaSuccess) {
             cuda_fail(e, "cudaMalloc(plan scratch)");

@@ -118,7 +118,8 @@ struct ScratchLayout {
     size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, ptotal, err, total;
 };
 
-inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
+// ll: the plan takes the single-launch dispatch (its regions are empty otherwise).
+inline ScratchLayout scratch_layout(long long G, int W, int numTiles, bool ll = false) {
     auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
     const size_t numChunks32 = (size_t)((G + 31) / 32);
     ScratchLayout L;
@@ -128,11 +129,11 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles) {
     L.tile_base = L.tile_cnt + up(sizeof(int32_t) * (size_t)numTiles * (W + 1));
     L.chunk_cnt = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * (W + 1));
     L.chunk_base = L.chunk_cnt + up(sizeof(int32_t) * numChunks32 * W);
-    const size_t llTiles = (size_t)(G < kLlMaxTiles ? G : kLlMaxTiles);
+    const size_t llTiles = ll ? (size_t)(G < kLlMaxTiles ? G : kLlMaxTiles) : 0;
     L.ll_status = L.chunk_base + up(sizeof(int32_t) * numChunks32 * W);
     L.ll_agg = L.ll_status + up(sizeof(uint32_t) * llTiles);
     L.ll_plist = L.ll_agg + up(sizeof(int32_t) * llTiles * (W + 1));
-    L.ticket = L.ll_plist + up(sizeof(int32_t) * (size_t)G * (W + 2));
+    L.ticket = L.ll_plist + (ll ? up(sizeof(int32_t) * (size_t)G * (W + 2)) : 0);
     L.work = L.ticket + 4;
     L.cwork = L.ticket + 8;
     L.cdone = L.ticket + 12;

@@ -5,9 +5,11 @@
 //   route_count  one thread per token: destination mask (destPe = expert /
 //                numExpertPerRank, "MORI JIT v2" design page §8), per-destination
 //                weight sums, per-tile histogram by warp ballots, tile-local
-//                ranks; the last block to finish scans the tile histogram into
-//                per-(tile, destPe) bases and stores recv_count (mori PR #599:
-//                a stored count). Slots end up ordered by (srcRank, token).
+//                ranks. For large batches the last block to finish scans the
+//                tile histogram into per-(tile, destPe) bases and stores
+//                recv_count (mori PR #599: a stored count); for small batches
+//                every scatter block scans it in its own shared memory.
+//                Slots end up ordered by (srcRank, token).
 //   scatter_rows persistent copy engines, one per warp: each x row is read once
 //                from HBM into shared memory by a TMA bulk copy
 //                (cp.async.bulk, mbarrier completion) and written to every
@@ -19,9 +21,12 @@
 //   combine      one warp per token: up to 8 destination rows in flight per
 //                16-byte column, float32 fma fold in destPe order; bf16 RNE out
 //                (float32 out, unrounded, for a float32 plan).
+// Options: dispatch_ll (one launch; blocks publish tile counts and read their
+// predecessors') and dispatch_fused (one cooperative launch, grid barriers).
 //
-// No kernel traps or spins without a bound: waits on shared-memory barriers
-// give up after kWaitCycles, set EP_DEVERR_TIMEOUT and drain their copies.
+// No kernel traps or spins without a bound: waits on shared-memory barriers,
+// grid barriers and other blocks' published words give up after
+// kWaitCycles, set EP_DEVERR_TIMEOUT and drain their copies.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>

@@ -158,7 +158,10 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * default, 0 never), EP_SCATTER_SCAN ("route": route_count's last block scans
  * the tile counts even when the scatter could), EP_PDL_EARLY (1: scatter and
  * combine let the next kernel of the stream launch when they start rather than
- * as they exit). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 makes the fused
+ * as they exit), EP_DISPATCH_DENSE (1 / 0: the large-batch form of the split
+ * dispatch for every plan / for none; by default plans of more than 16384
+ * tokens, W*T, take it), EP_SCATTER_LAYOUT (0..2: where the scatter's tile
+ * bases sit in shared memory). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 makes the fused
  * dispatch's grid barrier (with EP_DISPATCH_FUSED=1), or the low-latency
  * dispatch's wait for the counts of earlier tiles, unreachable, so that the
  * bounded wait runs out: the waiting blocks report EP_DEVERR_TIMEOUT, issue no
