@@ -169,8 +169,9 @@ __device__ __forceinline__ int source_next(TokenSource& s) {
 }
 
 // =====================================================================
-// route_count: mask, weight sums, tile histogram, tile-local ranks; the last
-// block scans the histogram. kW = compile-time bound on W (8, 16 or 32).
+// route_count: mask, weight sums, tile histogram, tile-local ranks; for large
+// batches the last block scans the histogram, for small batches every
+// scatter block does. kW = compile-time bound on W (8, 16 or 32).
 // =====================================================================
 // Destination mask and per-destination weight sums of token g (float32 fold
 // in topk order); ids < 0 are masked, ids >= E are reported and masked. kK
@@ -477,9 +478,9 @@ __device__ __forceinline__ uint32_t token_slots_and_meta(const ScatterParams& p,
 
 // =====================================================================
 // scatter_rows (TMA): persistent copy engines, one per warp.
-// Items are (present token, chunk) pairs of the tokens this engine is handed
-// by a global counter; an S-stage ring keeps S - kPend loads ahead and lets
-// kPend items' bulk stores drain while the next load starts.
+// Items are (present token, chunk) pairs of the tokens this engine's feed
+// hands it; an S-stage ring keeps S - kPend loads ahead and lets kPend
+// items' bulk stores drain while the next load starts.
 // =====================================================================
 template <int kPend>
 __device__ __forceinline__ void bulk_wait_read_pend() {
@@ -813,10 +814,7 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
     __syncwarp();
 }
 
-// Split-dispatch copy engines: the engines of this block that the fan-out
-// leaves active take tokens from the shared hand-out.
-// P: present tokens of the call; rows: its rows at all destinations (-1:
-// read recv_count); s_base: tile bases in shared memory, or nullptr.
+// One split-dispatch copy engine, with the feed of the call's hand-out mode.
 template <int kPend, bool kSmemBase>
 __device__ __forceinline__ void run_split_engine(const ScatterParams& p, const EngineSmem& es, int lane,
                                                  const TokenSource& src, const int* s_base) {
@@ -831,6 +829,10 @@ __device__ __forceinline__ void run_split_engine(const ScatterParams& p, const E
     }
 }
 
+// Split-dispatch copy engines: the engines of this block that the fan-out
+// leaves active take tokens from the shared hand-out. P: present tokens of
+// the call; rows: its rows at all destinations (-1: read recv_count);
+// s_base: tile bases in shared memory, or nullptr.
 template <int kPend>
 __device__ __forceinline__ void global_copy_engines(const ScatterParams& p, const EngineSmem& es, int lane,
                                                     int warp, int nwarps, int P, int rows, const int* s_base) {
