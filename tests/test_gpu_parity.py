@@ -58,6 +58,24 @@ def test_workload_parity_dispatch_families(name, ll, monkeypatch):
     run.close()
 
 
+@pytest.mark.parametrize("dense", ["0", "1"], ids=["small-batch-form", "large-batch-form"])
+@pytest.mark.parametrize("ct,topk", [(512, 6), (512, 8), (1024, 6), (1024, 8), (2048, 6), (2048, 8),
+                                     (4096, 6), (4096, 8), (1, 6), (8, 6)])
+def test_pr599_correctness_matrix(ct, topk, dense, monkeypatch):
+    """The correctness matrix of mori PR #599 ("Perf/ep disp 1250 ship",
+    correctness section): tokens per rank 512..4096 at topk 6 and 8 (topk 8
+    reaches the paths with more than one entry per lane), and 1 or 8 live
+    tokens of 512 at topk 6 (idle warps), at its EP4 shape with 8 experts per
+    rank (hidden 2048 here: the row width is not what the matrix varies),
+    through both forms of the split dispatch."""
+    monkeypatch.setenv("EP_DISPATCH_DENSE", dense)
+    max_tok = max(ct, 512)
+    wl = workload("pr599").replace(h=2048, ct=ct, max_tok=max_tok, max_recv=4 * max_tok, k=topk,
+                                   seed=1000 + ct + topk)
+    run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
+    run.close()
+
+
 @pytest.mark.parametrize("name", ["main", "skewed"])
 def test_large_batch_with_sparse_machinery(name, monkeypatch):
     """The main shapes through the small-batch form of the split dispatch
