@@ -50,7 +50,7 @@ def random_combine_input(cfg, seed=12345):
     return oracle_pins.torch_bf16_bits(vals)
 
 
-class GpuRun:
+class DeviceRun:
     """One plan plus the device buffers of one workload."""
 
     def __init__(self, cfg: dict, inputs: dict):
@@ -115,7 +115,7 @@ class GpuRun:
         self.close()
 
 
-def compare_dispatch(run: GpuRun, ref: dict):
+def compare_dispatch(run: DeviceRun, ref: dict):
     """Bit-exact comparison of dispatch outputs, on the device. Rows and
     records past recv_count must still hold the canary."""
     W = run.shape[0]
@@ -132,7 +132,7 @@ def compare_dispatch(run: GpuRun, ref: dict):
         assert bool((run.recv_meta[pe, n:] == CANARY_META).all()), f"meta written past count at pe {pe}"
 
 
-def compare_combine(run: GpuRun, ref_out: np.ndarray):
+def compare_combine(run: DeviceRun, ref_out: np.ndarray):
     """Combine: the tolerance of the spec (|d| <= 2^-7 |oracle| + 1e-3), and
     bit-exactness, since both sides fold in the same order with one rounding
     per term."""
@@ -163,7 +163,7 @@ def run_and_compare(cfg: dict, inputs: dict, y_override=None):
         y_override = random_combine_input(cfg)
     y_np = ref["recv_x"] if y_override is None else y_override
     ref_out = oracle.combine(cfg, y_np, ref["slotmap"], ref["wsum"])
-    run = GpuRun(cfg, inputs)
+    run = DeviceRun(cfg, inputs)
     try:
         run.dispatch()
         if y_override is None:

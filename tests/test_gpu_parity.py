@@ -19,7 +19,7 @@ if not torch.cuda.is_available():  # pragma: no cover - collected on CPU machines t
 import combine_ep_dispatch_05_b200 as ep  # noqa: E402
 import oracle  # noqa: E402
 import oracle_pins as P  # noqa: E402
-from gpu_harness import (CANARY_META, GpuRun, compare_combine, compare_dispatch, run_and_compare,  # noqa: E402
+from gpu_harness import (CANARY_META, DeviceRun, compare_combine, compare_dispatch, run_and_compare,  # noqa: E402
                          to_dev)
 from synth.inputs import WORKLOADS, make_inputs, workload  # noqa: E402
 
@@ -149,7 +149,7 @@ def test_dtype_main_dispatch(dtype, h):
     wl = workload("main").replace(dtype=dtype, h=h)
     inputs = make_inputs(wl)
     ref = oracle.dispatch(wl.cfg(), inputs["x"], inputs["topk_idx"], inputs["topk_w"])
-    with GpuRun(wl.cfg(), inputs) as run:
+    with DeviceRun(wl.cfg(), inputs) as run:
         run.dispatch()
         torch.cuda.synchronize()
         compare_dispatch(run, ref)
@@ -161,7 +161,7 @@ def _check_scaled(cfg, inputs, sw, seed=7):
     W, T = cfg["worldSize"], cfg["maxTokPerRank"]
     scales = rng.standard_normal((W, T, sw)).astype(np.float32)
     ref = oracle.dispatch(cfg, inputs["x"], inputs["topk_idx"], inputs.get("topk_w"), scales=scales)
-    with GpuRun(cfg, inputs) as run:
+    with DeviceRun(cfg, inputs) as run:
         R = run.info.maxRecv
         rs = torch.full((W, R, sw), 0x0C0FFEE, dtype=torch.int32, device="cuda")
         ep.ep_dispatch_scaled(run.plan, run.x, run.idx, run.w, to_dev(scales), sw, run.recv_x,
@@ -237,7 +237,7 @@ def test_repeated_calls_and_reset():
     b = make_inputs(wl.replace(seed=77))
     ref_a = oracle.dispatch(cfg, a["x"], a["topk_idx"], a["topk_w"])
     ref_b = oracle.dispatch(cfg, b["x"], b["topk_idx"], b["topk_w"])
-    with GpuRun(cfg, a) as run:
+    with DeviceRun(cfg, a) as run:
         run.dispatch()
         torch.cuda.synchronize()
         compare_dispatch(run, ref_a)
@@ -356,7 +356,7 @@ def test_bounded_wait_runs_out_and_reports(family, monkeypatch):
     monkeypatch.setenv("EP_TEST_UNREACHABLE_BARRIER", "1")
     wl = workload("latency8")
     inputs = make_inputs(wl)
-    with GpuRun(wl.cfg(), inputs) as run:
+    with DeviceRun(wl.cfg(), inputs) as run:
         assert run.info.dispatchFused == (family == "fused")
         assert run.info.dispatchLowLatency == (family == "lowlat")
         run.dispatch()
@@ -389,7 +389,7 @@ def test_bounded_wait_runs_out_and_reports(family, monkeypatch):
 
 def test_host_side_rejections():
     wl = workload("tiny")
-    with GpuRun(wl.cfg(), make_inputs(wl)) as run:
+    with DeviceRun(wl.cfg(), make_inputs(wl)) as run:
         with pytest.raises(ep.EpError) as e:
             run.combine()
         assert e.value.code == ep.EP_ERR_STATE
