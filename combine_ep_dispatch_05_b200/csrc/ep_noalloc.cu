@@ -92,6 +92,10 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         if (cfg->useWeights && !topk_w) return noalloc_fail(EP_ERR_INVALID, "topk_w is NULL but useWeights is 1");
         if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(recv_x)) % 16 != 0)
             return noalloc_fail(EP_ERR_ALIGN, "x and recv_x must be 16-byte aligned");
+        // The same 4-byte rule as ep_dispatch: the kernels load and store these as int32 / float.
+        if ((reinterpret_cast<uintptr_t>(topk_idx) | reinterpret_cast<uintptr_t>(recv_meta) |
+             reinterpret_cast<uintptr_t>(recv_count) | reinterpret_cast<uintptr_t>(topk_w)) % 4 != 0)
+            return noalloc_fail(EP_ERR_ALIGN, "topk_idx, topk_w, recv_meta, recv_count must be 4-byte aligned");
 
         // Sizes and geometry of the default plan for this configuration.
         EpPlanInfo info;

@@ -221,3 +221,21 @@ def test_graft_entry_build():
     sys.path.insert(0, ROOT)
     import __graft_entry__
     __graft_entry__.build()
+
+
+@pytest.mark.parametrize("which", ["topk_idx", "topk_w", "recv_meta", "recv_count", "x", "recv_x"])
+def test_noalloc_rejects_misaligned_buffers_before_any_launch(ep, which):
+    """ep_dispatch_noalloc checks alignment as ep_dispatch does, on the host,
+    before it touches the device: a misaligned int32 / float buffer (4 bytes)
+    or payload buffer (16 bytes) gives EP_ERR_ALIGN. The addresses here are
+    never dereferenced, and on a machine without a GPU the call would fail with
+    a CUDA error instead if it had got as far as the device."""
+    from combine_ep_dispatch_05_b200 import binding as b
+    bufs = {n: 0x10000 * (i + 1) for i, n in enumerate(
+        ["x", "topk_idx", "topk_w", "recv_x", "recv_meta", "recv_count"])}
+    bufs[which] += 2 if which not in ("x", "recv_x") else 8
+    cfg = b._cfg(_cfg(maxTokPerRank=8, maxRecv=0))
+    rc = b._lib.ep_dispatch_noalloc(ctypes.byref(cfg), bufs["x"], bufs["topk_idx"], bufs["topk_w"],
+                                    bufs["recv_x"], bufs["recv_meta"], bufs["recv_count"], None)
+    assert rc == b.EP_ERR_ALIGN
+    assert "aligned" in ep.ep_last_error()

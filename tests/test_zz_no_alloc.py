@@ -70,6 +70,15 @@ def test_noalloc_matches_plan_dispatch_two_calls():
     _check_against_plan(workload("main").replace(seed=9))  # second call: other shape, other routing
 
 
+def test_noalloc_matches_plan_dispatch_on_sparse_and_unweighted_batches():
+    """The call always scans the tile counts in route_count's last block and
+    hands out tokens by the present-token total; plans take that form only
+    under overrides. Batches with absent tokens (ct = 1 and 8 of 512 tokens a
+    rank, no weights) and the tiny batch must still match a plan bit for bit."""
+    for name in ("latency1", "latency8", "tiny"):
+        _check_against_plan(workload(name))
+
+
 def test_noalloc_refuses_configurations_beyond_its_scratch():
     cfg = dict(worldSize=32, hiddenDim=64, maxTokPerRank=1024, numExpertPerRank=2,
                numExpertPerToken=4, maxRecv=0, dtype=0, useWeights=0)
