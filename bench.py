@@ -12,9 +12,9 @@ inputs are larger than L2 as well). Barrier +
 synchronize on both sides; the reported time is the max over ranks. N > 1
 runs N independent replicas, one per GPU (each GPU holds all W virtual ranks).
 
---impl reference times the CPU oracle (the plain C statement of the method)
-on this host's cores, on a bounded sample of the same workload (see
-``ref_sample``), scaled to the full step.
+--impl reference times the CPU oracle (the plain C statement of the method) on
+the full workload on this host: its OpenMP build on all cores is the value, and
+one step of its single-threaded build is reported beside it (``cpu_baseline``).
 """
 from __future__ import annotations
 
@@ -227,25 +227,34 @@ def max_over_ranks(val: float, dist, device) -> float:
 
 
 # ------------------------------------------------------------------ reference arm
-def ref_sample(wl, frac_den=8):
-    """The bounded sample the CPU oracle runs per reference step: the same
-    workload with 1/frac_den of the tokens per rank (same routing law, same
-    hidden size and capacity per token), so every per-token cost is the same;
-    the step time is scaled back by the token ratio."""
-    ct = max(1, wl.ct // frac_den)
-    mt = max(1, wl.max_tok // frac_den)
-    sample = wl.replace(ct=ct, max_tok=mt, max_recv=wl.W * mt)
-    scale = (wl.W * wl.max_tok) / (sample.W * sample.max_tok)
-    return sample, scale, (f"{wl.name} shape with {mt} of {wl.max_tok} tokens per rank "
-                           f"(maxRecv {wl.W * mt}), time x {scale:g}")
+def host_cpu() -> dict:
+    """The host's usable cores and its CPU model."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    return {"nproc": cores, "cpu_model": model}
 
 
-def time_oracle(wl, inputs, steps, scale=1.0):
+def time_oracle(wl, inputs, steps, lib=None):
+    """Seconds of (dispatch, combine) per oracle step on the full workload.
+    lib: an oracle build (None: the single-threaded one). The receive and
+    output buffers are allocated once, outside the timed calls."""
     import oracle
     cfg = wl.cfg()
     R = oracle.recv_capacity(cfg)
     recv_x = np.zeros((wl.W, R, wl.h), dtype=oracle.payload_np(cfg))
     recv_meta = np.zeros((wl.W, R, 3 + wl.k), dtype=np.int32)
+    out = np.zeros((wl.W, wl.max_tok, oracle.combine_hidden(cfg)), dtype=oracle.combine_np(cfg))
     idx = inputs["topk_idx"]
     y = None
     if wl.dtype in (2, 3):  # one-byte payloads: the expert hands back bf16 rows
@@ -255,31 +264,48 @@ def time_oracle(wl, inputs, steps, scale=1.0):
     ts = []
     for _ in range(steps):
         t0 = time.perf_counter()
-        r = oracle.dispatch(cfg, inputs["x"], idx, inputs["topk_w"], recv_x=recv_x, recv_meta=recv_meta)
-        oracle.combine(cfg, r["recv_x"] if y is None else y, r["slotmap"], r["wsum"])
-        ts.append((time.perf_counter() - t0) * scale)
+        r = oracle.dispatch(cfg, inputs["x"], idx, inputs["topk_w"], recv_x=recv_x, recv_meta=recv_meta,
+                            lib=lib)
+        t1 = time.perf_counter()
+        oracle.combine(cfg, r["recv_x"] if y is None else y, r["slotmap"], r["wsum"], lib=lib, out=out)
+        ts.append((t1 - t0, time.perf_counter() - t1))
     return ts
+
+
+def cpu_baseline(wl, inputs, steps, warmup, single_steps=1) -> dict:
+    """The oracle on this host: the OpenMP build on all cores (the value),
+    and the single-threaded build for one step beside it. Both run the full
+    workload; their results are identical."""
+    import oracle
+    oracle.build()
+    omp = oracle.load_omp()
+    threads = oracle.threads(omp)
+    time_oracle(wl, inputs, warmup, omp)
+    ts = time_oracle(wl, inputs, steps, omp)
+    one = time_oracle(wl, inputs, single_steps, None)
+    mean = lambda xs: statistics.mean(xs) * 1e6  # noqa: E731
+    return {"value": mean([d + c for d, c in ts]), "unit": "us", "cores": threads, "kind": "oracle",
+            "sample": (f"the full {wl.name} workload, {steps} steps after {warmup} warm-up, OpenMP build of "
+                       f"the C oracle on {threads} threads (dispatch shares out the {wl.W} destinations, "
+                       f"combine the tokens); single-threaded build for {single_steps} step(s) beside it"),
+            "dispatch_us": mean([d for d, _ in ts]), "combine_us": mean([c for _, c in ts]),
+            "single_core_us": mean([d + c for d, c in one]),
+            "single_core_dispatch_us": mean([d for d, _ in one]),
+            "single_core_combine_us": mean([c for _, c in one]), **host_cpu()}
 
 
 def run_reference(args, wl):
     rank, world, local, dist = dist_setup(args.gpus)
     if rank != 0:
         return 0
-    import oracle
-    oracle.build()
-    swl, scale, sample = ref_sample(wl)
-    inputs = make_inputs(swl)
-    time_oracle(swl, inputs, args.warmup, scale)
-    ts = time_oracle(swl, inputs, args.steps, scale)
-    us = statistics.mean(ts) * 1e6
-    cores = 1
+    inputs = make_inputs(wl)
+    cpu = cpu_baseline(wl, inputs, args.steps, args.warmup)
+    us = cpu["value"]
     line = {"metric": METRIC, "value": us, "unit": "us", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None,
             "dtype": {0: "bf16", 1: "f32", 2: "fp8", 3: "fp4x2"}[wl.dtype], "data": "synthetic",
-            "config": describe(wl), "impl": "reference",
-            "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "config": describe(wl), "impl": "reference", "cpu_baseline": cpu,
             "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -526,13 +552,8 @@ def run_ours(args, wl):
     ep.ep_plan_destroy(plan)
 
     cpu = None
-    if rank == 0 and args.gpus == 1 and not args.no_cpu_baseline and wl.dtype in (0, 1):
-        import oracle
-        oracle.build()
-        steps_cpu = 2
-        ts = time_oracle(wl, inputs, steps_cpu)
-        cpu = {"value": statistics.mean(ts) * 1e6, "unit": "us", "cores": 1, "kind": "oracle",
-               "sample": f"the full {wl.name} workload, {steps_cpu} steps, single-threaded C oracle"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, inputs, steps=3, warmup=1)
 
     if rank == 0:
         line = {

@@ -4,9 +4,10 @@ Only the tests, the smoke check and the CPU-baseline leg of the bench may
 import this package. The product path (the CUDA library and its binding) never
 imports, links or calls it.
 
-The arithmetic lives in ``ep_oracle.c`` (plain single-threaded C, compiled here
-with ``gcc -O2 -ffp-contract=off``); this module only builds it and marshals
-numpy arrays through ctypes.
+The arithmetic lives in ``ep_oracle.c`` (plain C, compiled here with ``gcc -O2
+-ffp-contract=off``); this module only builds it and marshals numpy arrays
+through ctypes. ``load_omp()`` gives the same source built with OpenMP, whose
+results are identical, for timing the oracle on all host cores.
 """
 from __future__ import annotations
 
@@ -32,14 +33,24 @@ class OracleCfg(ctypes.Structure):
         "numExpertPerToken", "maxRecv", "dtype", "useWeights")]
 
 
+_LIB_OMP = os.path.join(_HERE, "libep_oracle_omp.so")
+_lib_omp = None
+_FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def _compile(out: str, extra: list, force: bool) -> str:
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_FLAGS, *extra, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
-    """Compile ep_oracle.c into a shared library next to it."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
-                               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+    """Compile ep_oracle.c into shared libraries next to it: the
+    single-threaded build (returned) and the OpenMP build."""
+    _compile(_LIB_OMP, ["-fopenmp"], force)
+    return _compile(_LIB, [], force)
 
 
 def _bind(lib):
@@ -57,6 +68,8 @@ def _bind(lib):
     lib.oracle_f32_to_bf16.restype = None
     lib.oracle_bf16_to_f32.argtypes = [P, P, ctypes.c_int64]
     lib.oracle_bf16_to_f32.restype = None
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = ctypes.c_int
     return lib
 
 
@@ -66,6 +79,22 @@ def _load():
         if _lib is None:
             _lib = _bind(ctypes.CDLL(build()))
     return _lib
+
+
+def load_omp():
+    """The OpenMP build of the same source: same results, all host cores
+    (OMP_NUM_THREADS caps them). Pass it as ``lib=``."""
+    global _lib_omp
+    with _lock:
+        if _lib_omp is None:
+            build()
+            _lib_omp = _bind(ctypes.CDLL(_LIB_OMP))
+    return _lib_omp
+
+
+def threads(lib=None) -> int:
+    """Threads a call of this build may use (1 for the single-threaded one)."""
+    return int((lib or _load()).oracle_threads())
 
 
 def load_library(path: str):
@@ -152,9 +181,11 @@ def dispatch(cfg: dict, x: np.ndarray, topk_idx: np.ndarray, topk_w, recv_x=None
                 slotmap=slotmap, wsum=wsum, status=rc, recv_scales=recv_scales)
 
 
-def combine(cfg: dict, y: np.ndarray, slotmap: np.ndarray, wsum: np.ndarray, lib=None) -> np.ndarray:
+def combine(cfg: dict, y: np.ndarray, slotmap: np.ndarray, wsum: np.ndarray, lib=None,
+            out: np.ndarray = None) -> np.ndarray:
     """Run the oracle combine; returns out, shape (W, T, combine_hidden): bf16
-    bits (uint16), or float32 for an fp32 plan."""
+    bits (uint16), or float32 for an fp32 plan. ``out`` may be passed
+    pre-allocated (every row is written)."""
     lib = lib or _load()
     c = _cfg(cfg)
     W, T = c.worldSize, c.maxTokPerRank
@@ -164,7 +195,9 @@ def combine(cfg: dict, y: np.ndarray, slotmap: np.ndarray, wsum: np.ndarray, lib
     y = np.ascontiguousarray(y).view(ct).reshape(W, R, h)
     slotmap = np.ascontiguousarray(slotmap, dtype=np.int32).reshape(W, T, W)
     wsum = np.ascontiguousarray(wsum, dtype=np.float32).reshape(W, T, W)
-    out = np.empty((W, T, h), dtype=ct)
+    if out is None:
+        out = np.empty((W, T, h), dtype=ct)
+    assert out.shape == (W, T, h) and out.dtype == ct and out.flags.c_contiguous
     rc = lib.oracle_combine(ctypes.byref(c), _ptr(y), _ptr(slotmap), _ptr(wsum), _ptr(out))
     if rc < 0:
         raise ValueError(f"oracle_combine rejected its arguments (rc={rc})")

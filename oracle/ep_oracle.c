@@ -1,11 +1,17 @@
 /*
  * ep_oracle.c -- CPU oracle for MoE expert-parallel dispatch and combine.
  *
- * TEST INFRASTRUCTURE ONLY. This file is the plain, slow, single-threaded
- * statement of what the dispatch and combine calls compute. It exists so that
- * tests, the smoke check and the CPU baseline of the bench can check the CUDA
- * path against it. Nothing in the product links or calls it, and it shares no
- * header, helper, table or constant with the CUDA path.
+ * TEST INFRASTRUCTURE ONLY. This file is the plain, slow statement of what
+ * the dispatch and combine calls compute. It exists so that tests, the smoke
+ * check and the CPU baseline of the bench can check the CUDA path against it.
+ * Nothing in the product links or calls it, and it shares no header, helper,
+ * table or constant with the CUDA path.
+ *
+ * It is built twice: single-threaded, and with OpenMP (-fopenmp), where the
+ * destinations of dispatch and the tokens of combine are shared out over the
+ * host's cores. Every output element is computed by the same steps in the
+ * same order in both builds, so their results are identical; the OpenMP build
+ * only times the same definition on all cores.
  *
  * Sources (mori pages):
  *   - "MORI JIT v2" design page, §3.2 (EpCfg: worldSize, hiddenDim,
@@ -56,6 +62,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 typedef struct {
     int32_t worldSize;
@@ -191,23 +200,26 @@ static int dispatch_impl(const OracleCfg *c, const uint8_t *x, const int32_t *to
     const int64_t nEpr = c->numExpertPerRank, k = c->numExpertPerToken;
     const int64_t E = W * nEpr, R = recv_cap(c), M = 3 + k;
     int status = ORACLE_OK;
+    int overflow = 0;
 
-    int64_t *next = (int64_t *)calloc((size_t)W, sizeof *next);
-    if (!next) return ORACLE_ERR_NOMEM;
-
-    /* Tokens in (source rank, source token) ascending order; every destination
-     * hands out its slots in that order. */
-    for (int64_t r = 0; r < W; ++r) {
-        for (int64_t t = 0; t < T; ++t) {
-            const int64_t g = r * T + t;
-            const int32_t *ids = topk_idx + g * k;
-            for (int64_t pe = 0; pe < W; ++pe) {
+    /* Every destination hands out its slots in (source rank, source token)
+     * ascending order, independently of the other destinations: destination pe
+     * counts n from 0 over the tokens that reach it. Built with OpenMP, the
+     * destinations run side by side; each writes only its own slots, receive
+     * rows, meta records and slot-map column, by the same steps. */
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : status, overflow)
+    for (int64_t pe = 0; pe < W; ++pe) {
+        int64_t n = 0;
+        for (int64_t r = 0; r < W; ++r) {
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t g = r * T + t;
+                const int32_t *ids = topk_idx + g * k;
                 int hit = 0;
                 float s = 0.0f;
                 for (int64_t j = 0; j < k; ++j) {
                     int32_t e = ids[j];
                     if (e < 0) continue;
-                    if (e >= E) { status = ORACLE_STATUS_EXPERT_RANGE; continue; }
+                    if (e >= E) { status |= ORACLE_STATUS_EXPERT_RANGE; continue; }
                     if (e / nEpr != pe) continue;
                     hit = 1;
                     if (c->useWeights) s = s + topk_w[g * k + j];
@@ -218,8 +230,8 @@ static int dispatch_impl(const OracleCfg *c, const uint8_t *x, const int32_t *to
                     wsum[g * W + pe] = 0.0f;
                     continue;
                 }
-                if (next[pe] >= R) { free(next); return ORACLE_ERR_ARG; }
-                const int64_t slot = next[pe]++;
+                if (n >= R) { overflow = 1; continue; }
+                const int64_t slot = n++;
                 memcpy(recv_x + (pe * R + slot) * row, x + g * row, (size_t)row);
                 if (scales)
                     memcpy(recv_scales + (pe * R + slot) * scale_words, scales + g * scale_words,
@@ -236,9 +248,9 @@ static int dispatch_impl(const OracleCfg *c, const uint8_t *x, const int32_t *to
                 wsum[g * W + pe] = s;
             }
         }
+        recv_count[pe] = (int32_t)n;
     }
-    for (int64_t pe = 0; pe < W; ++pe) recv_count[pe] = (int32_t)next[pe];
-    free(next);
+    if (overflow) return ORACLE_ERR_ARG; /* more rows than maxRecv at some destination */
     return status;
 }
 
@@ -258,30 +270,47 @@ int oracle_combine(const OracleCfg *c, const void *y_, const int32_t *slotmap,
     const float *yf = (const float *)y_;
     uint16_t *out = (uint16_t *)out_;
     float *outf = (float *)out_;
-    float *acc = (float *)malloc((size_t)h * sizeof *acc);
-    if (!acc) return ORACLE_ERR_NOMEM;
+    int nomem = 0;
 
-    for (int64_t g = 0; g < W * T; ++g) {
-        for (int64_t i = 0; i < h; ++i) acc[i] = 0.0f;
-        for (int64_t pe = 0; pe < W; ++pe) {
-            const int32_t slot = slotmap[g * W + pe];
-            if (slot < 0) continue;
-            const float w = wsum[g * W + pe];
-            if (fp32) {
-                const float *rowf = yf + (pe * R + slot) * h;
-                for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, rowf[i], acc[i]);
-            } else {
-                const uint16_t *row = y + (pe * R + slot) * h;
-                for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, bf16_to_f32(row[i]), acc[i]);
+    /* Built with OpenMP, the tokens are spread over the host's cores; each
+     * output row is the same fold in the same order either way. */
+#pragma omp parallel
+    {
+        float *acc = (float *)malloc((size_t)h * sizeof *acc);
+#pragma omp for schedule(static) reduction(| : nomem)
+        for (int64_t g = 0; g < W * T; ++g) {
+            if (!acc) { nomem = 1; continue; }
+            for (int64_t i = 0; i < h; ++i) acc[i] = 0.0f;
+            for (int64_t pe = 0; pe < W; ++pe) {
+                const int32_t slot = slotmap[g * W + pe];
+                if (slot < 0) continue;
+                const float w = wsum[g * W + pe];
+                if (fp32) {
+                    const float *rowf = yf + (pe * R + slot) * h;
+                    for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, rowf[i], acc[i]);
+                } else {
+                    const uint16_t *row = y + (pe * R + slot) * h;
+                    for (int64_t i = 0; i < h; ++i) acc[i] = fmaf(w, bf16_to_f32(row[i]), acc[i]);
+                }
             }
+            if (fp32)
+                for (int64_t i = 0; i < h; ++i) outf[g * h + i] = acc[i];
+            else
+                for (int64_t i = 0; i < h; ++i) out[g * h + i] = f32_to_bf16_rne(acc[i]);
         }
-        if (fp32)
-            for (int64_t i = 0; i < h; ++i) outf[g * h + i] = acc[i];
-        else
-            for (int64_t i = 0; i < h; ++i) out[g * h + i] = f32_to_bf16_rne(acc[i]);
+        free(acc);
     }
-    free(acc);
-    return ORACLE_OK;
+    return nomem ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* Threads a call may use: the OpenMP build's team size, 1 otherwise. */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /* The two format conversions, exported so that tests can pin them against an

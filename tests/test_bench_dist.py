@@ -73,5 +73,8 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     assert bench.run_reference(args, wl) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "us" and line["higher_is_better"] is False
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["value"] == line["value"]
+    assert cpu["cores"] >= 1 and cpu["nproc"] >= 1 and cpu["cpu_model"]
+    assert cpu["single_core_us"] > 0 and "full tiny workload" in cpu["sample"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0

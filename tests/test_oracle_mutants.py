@@ -22,8 +22,8 @@ MUTANTS = {
     "local_id_sign": ("(int32_t)(e - pe * nEpr)", "(int32_t)(pe * nEpr - e)"),
     "masked_minus_one_routed": ("if (e < 0) continue;", "if (e < -1) continue;"),
     "slot_order_token_major": (
-        "for (int64_t r = 0; r < W; ++r) {\n        for (int64_t t = 0; t < T; ++t) {",
-        "for (int64_t t = 0; t < T; ++t) {\n        for (int64_t r = 0; r < W; ++r) {"),
+        "for (int64_t r = 0; r < W; ++r) {\n            for (int64_t t = 0; t < T; ++t) {",
+        "for (int64_t t = 0; t < T; ++t) {\n            for (int64_t r = 0; r < W; ++r) {"),
     "combine_drops_accumulator": ("acc[i] = fmaf(w, bf16_to_f32(row[i]), acc[i]);",
                                   "acc[i] = fmaf(w, bf16_to_f32(row[i]), 0.0f);"),
     "combine_unfused": ("acc[i] = fmaf(w, bf16_to_f32(row[i]), acc[i]);",
@@ -44,7 +44,7 @@ MUTANTS = {
                                      "for (int64_t i = 0; i < h; ++i) outf[g * h + i] = bf16_to_f32(f32_to_bf16_rne(acc[i]));"),
     "scale_row_of_wrong_token": ("memcpy(recv_scales + (pe * R + slot) * scale_words, scales + g * scale_words,",
                                  "memcpy(recv_scales + (pe * R + slot) * scale_words, scales + t * scale_words,"),
-    "count_not_stored": ("recv_count[pe] = (int32_t)next[pe];", "recv_count[pe] = (int32_t)next[pe] - (pe == 0);"),
+    "count_not_stored": ("recv_count[pe] = (int32_t)n;", "recv_count[pe] = (int32_t)n - (pe == 0);"),
 }
 
 
