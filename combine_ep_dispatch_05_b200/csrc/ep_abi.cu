@@ -55,8 +55,6 @@ struct EpPlan {
     unsigned* ll_epoch;
     unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
     int fanoutSwitch;       // x100, see ScatterParams
-    int combineTile;        // combine kernel instance
-    int pdlEarly;           // scatter and combine trigger the next kernel's launch at their start
     bool dispatched;
 };
 
@@ -135,9 +133,8 @@ int check_cfg(const EpCfg* c) {
 
 struct Geometry {
     int chunkBytes, chunkStride, numChunks;
-    int scatterMode, scatterPend;
     int scatterWarps, scatterStages;
-    int combineWarps, combineTile;
+    int combineWarps;
 };
 
 // Copy engines and stages: three engines (warps) per block for rows of 8 KB
@@ -180,26 +177,9 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
         warps = std::min(env_int("EP_SCATTER_WARPS", warps), ep::kMaxScatterWarps);
         stages = std::max(2, std::min(env_int("EP_SCATTER_STAGES", stages), 16));
     }
-    int pend = 1;
-    int mode = ep::kScatterTma;
-    if (use_env) {
-        pend = std::max(1, std::min(env_int("EP_SCATTER_PEND", pend), 3));
-        const char* m = std::getenv("EP_SCATTER_MODE");
-        if (m && std::strcmp(m, "regs") == 0) mode = ep::kScatterRegs;
-    }
-    stages = std::max(stages, pend + 1);
-    if (mode == ep::kScatterRegs) {
-        warps = std::min(use_env ? env_int("EP_SCATTER_WARPS", 8) : 8, 8);
-        stages = 0;
-    }
-    g.scatterMode = mode;
-    g.scatterPend = pend;
     g.scatterWarps = warps;
     g.scatterStages = stages;
     g.combineWarps = use_env ? std::min(env_int("EP_COMBINE_WARPS", 8), ep::kMaxCombineWarps) : 8;
-    g.combineTile = 0;
-    if (use_env)
-        if (const char* t = std::getenv("EP_COMBINE_TILE")) g.combineTile = std::max(0, std::min(std::atoi(t), 3));
     return g;
 }
 
@@ -220,7 +200,7 @@ int ll_stages(const EpCfg* c, const Geometry& geo, bool fused, int blocks, size_
               int* tile) {
     const long long G = (long long)c->worldSize * c->maxTokPerRank;
     const int llMax = env_int("EP_LL_MAX_TOKENS", kLlDefaultMaxTokens, 0);
-    if (fused || geo.scatterMode != ep::kScatterTma || geo.scatterPend != 1 || geo.scatterWarps > ep::kLlWarps ||
+    if (fused || geo.scatterWarps > ep::kLlWarps ||
         c->maxTokPerRank > llMax || blocks < 1)
         return 0;
     *tile = ep::ll_tile_tokens(G, blocks);
@@ -254,8 +234,8 @@ void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
     info->scatterWarps = geo.scatterWarps;
     info->scatterStages = geo.scatterStages;
     info->scatterChunkBytes = geo.chunkBytes;
-    info->scatterMode = geo.scatterMode;
-    info->scatterPend = geo.scatterPend;
+    info->scatterMode = 0;  // TMA bulk copies staged in shared memory
+    info->scatterPend = 1;  // one item's bulk stores left draining when a stage refills
     info->combineWarps = geo.combineWarps;
     info->device = -1;
 }
@@ -338,76 +318,59 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         const bool dense = denseEnv >= 0 ? denseEnv != 0 : Gtok > kDenseMinTokens;
         const char* fusedEnv = std::getenv("EP_DISPATCH_FUSED");
         const bool wantFused = fusedEnv && std::strcmp(fusedEnv, "1") == 0;
-        if (geo.scatterMode == ep::kScatterTma) {
-            // The TMA scatter scans route_count's tile counts itself when
-            // they fit a few KB of shared memory (route_count then ends
-            // without a last-block scan); the fused dispatch has its own.
+        {
+            // The scatter scans route_count's tile counts itself when they
+            // fit a few KB of shared memory (route_count then ends without a
+            // last-block scan); the fused dispatch has its own. Shared memory:
+            // the tile bases (if any) first, then the copy engines.
             const int numTiles =
                 (int)(((long long)cfg->worldSize * cfg->maxTokPerRank + ep::kCountTile - 1) / ep::kCountTile);
             const size_t bs = ep::scatter_base_smem_bytes(numTiles, cfg->worldSize);
             const char* scanEnv = std::getenv("EP_SCATTER_SCAN");
             const bool scanInRoute = scanEnv && std::strcmp(scanEnv, "route") == 0;
             if (!wantFused && !scanInRoute && !dense && bs <= ep::kMaxBaseSmemBytes) baseSmem = bs;
-            const size_t limit = (size_t)smemOptin - 1024;  // the kernels' static shared memory
-            // Layout (EP_SCATTER_LAYOUT, for sweeps): 0 tile bases first,
-            // then the engines; 1 engines first; 2 tile bases first, engines
-            // from the next 1 KB boundary.
-            const int layout = env_int("EP_SCATTER_LAYOUT", 0, 0);
-            auto total = [&]() {
-                const size_t eng = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
-                if (baseSmem == 0) return eng;
-                if (layout == 1) return eng + baseSmem;
-                if (layout == 2) return ((baseSmem + 1023) & ~(size_t)1023) + eng;
-                return baseSmem + eng;
-            };
-            auto offsets = [&](size_t* bo, size_t* eo) {
-                const size_t eng = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
-                *bo = 0;
-                *eo = baseSmem;
-                if (baseSmem == 0) *eo = 0;
-                else if (layout == 1) *bo = eng, *eo = 0;
-                else if (layout == 2) *eo = (baseSmem + 1023) & ~(size_t)1023;
+            const size_t limit = (size_t)smemOptin - ep::kStaticSmemReserve;
+            auto engines = [&]() {
+                return ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
             };
             // The table must not cost a block per SM (7 KB rows: 2 blocks of
             // 8 stages fit an SM without it, 1 with it).
             if (baseSmem > 0) {
-                const size_t eng = ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+                const size_t eng = engines();
                 int with = 0, without = 0;
-                if ((e = ep::scatter_set_smem(geo.scatterPend, std::min(limit, eng + baseSmem + 1024))) !=
+                if ((e = ep::scatter_set_smem(std::min(limit, eng + baseSmem + 1024))) != cudaSuccess ||
+                    (e = ep::scatter_blocks_per_sm(geo.scatterWarps, std::min(limit, eng), &without)) !=
                         cudaSuccess ||
-                    (e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps,
-                                                   std::min(limit, eng), &without)) != cudaSuccess ||
-                    (e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps,
-                                                   std::min(limit, eng + baseSmem), &with)) != cudaSuccess) {
+                    (e = ep::scatter_blocks_per_sm(geo.scatterWarps, std::min(limit, eng + baseSmem), &with)) !=
+                        cudaSuccess) {
                     cuda_fail(e, "scatter occupancy");
                     return nullptr;
                 }
                 if (with < without) baseSmem = 0;
             }
-            smem = total();
-            while (smem > limit && geo.scatterStages > geo.scatterPend + 1) {
+            smem = baseSmem + engines();
+            while (smem > limit && geo.scatterStages > 2) {
                 --geo.scatterStages;
-                smem = total();
+                smem = baseSmem + engines();
             }
             while (smem > limit && geo.scatterWarps > 1) {
                 --geo.scatterWarps;
-                smem = total();
+                smem = baseSmem + engines();
             }
             if (smem > limit) {
                 fail(EP_ERR_INVALID, "row piece of %d bytes does not fit shared memory", geo.chunkBytes);
                 return nullptr;
             }
-            offsets(&baseOffset, &engineOffset);
-            if ((e = ep::scatter_set_smem(geo.scatterPend, smem)) != cudaSuccess) {
+            baseOffset = 0;
+            engineOffset = baseSmem;
+            if ((e = ep::scatter_set_smem(smem)) != cudaSuccess) {
                 cuda_fail(e, "cudaFuncSetAttribute(scatter smem)");
                 return nullptr;
             }
         }
         int sPerSm = 0, cPerSm = 0;
-        if ((e = ep::scatter_blocks_per_sm(geo.scatterMode, geo.scatterPend, geo.scatterWarps, smem,
-                                           &sPerSm)) != cudaSuccess ||
-            (e = ep::combine_blocks_per_sm(geo.combineWarps, cfg->dtype == EP_FP32, geo.combineTile, &cPerSm)) !=
-                cudaSuccess) {
+        if ((e = ep::scatter_blocks_per_sm(geo.scatterWarps, smem, &sPerSm)) != cudaSuccess ||
+            (e = ep::combine_blocks_per_sm(geo.combineWarps, cfg->dtype == EP_FP32, &cPerSm)) != cudaSuccess) {
             cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
             return nullptr;
         }
@@ -431,7 +394,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         // request (EP_DISPATCH_FUSED=1): on B200 the two launches of
         // route_count + scatter_rows measured faster at every size (main
         // workload 476 vs 500 us, ct=1 workload 17.4 vs 20.5 us).
-        bool fused = wantFused && geo.scatterMode == ep::kScatterTma;
+        bool fused = wantFused;
         int coop = 0;
         if (fused && (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop))
             fused = false;
@@ -483,12 +446,6 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         }
         plan->info.dispatchLowLatency = plan->ll ? 1 : 0;
         plan->fanoutSwitch = env_int("EP_SCATTER_FANOUT_SWITCH", 375, 0);
-        // Scatter and combine let the next kernel launch only as they exit:
-        // a dependent grid launched at their start keeps a waiting block on
-        // every SM for the whole copy, and on B200 a captured dispatch +
-        // combine pair then took 997 instead of 927 us at the main workload.
-        plan->pdlEarly = env_int("EP_PDL_EARLY", 0, 0) != 0 ? 1 : 0;
-        plan->combineTile = geo.combineTile;
         // Test hook for the failure path: the fused dispatch's grid barrier,
         // or the low-latency dispatch's wait for earlier tiles, can never
         // complete, so the blocks give up after their bounded wait and report
@@ -497,7 +454,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
             plan->barrierSlack = std::strcmp(t, "1") == 0 ? 1u : 0u;
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
-        plan->dense = !fused && dense && geo.scatterMode == ep::kScatterTma;
+        plan->dense = !fused && dense;
         plan->baseSmem = fused ? 0 : baseSmem;
         plan->baseOffset = fused ? 0 : baseOffset;
         plan->engineOffset = fused ? 0 : engineOffset;
@@ -662,7 +619,6 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         sp.stages = plan->info.scatterStages;
         sp.recv_count = recv_count;
         sp.fanoutSwitch = plan->fanoutSwitch;
-        sp.pdlEarly = plan->pdlEarly;
         sp.scales = static_cast<const uint32_t*>(scales);
         sp.recv_scales = static_cast<uint32_t*>(recv_scales);
         sp.scaleWords = scaleWords;
@@ -717,8 +673,8 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         sp.baseOffset = (int)plan->baseOffset;
         sp.engineOffset = (int)plan->engineOffset;
         sp.ptotal = plan->dense ? nullptr : plan->ptotal;  // dense: every token counts as present
-        e = ep::launch_scatter_rows(sp, plan->info.scatterMode, plan->info.scatterPend, plan->dense,
-                                    plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
+        e = ep::launch_scatter_rows(sp, plan->dense, plan->info.scatterBlocks, plan->info.scatterWarps,
+                                    plan->scatterSmem, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch scatter_rows");
         plan->dispatched = true;
         return EP_OK;
@@ -746,9 +702,8 @@ int ep_combine(EpPlan* plan, const void* y, void* out, void* stream) {
         cp.G = plan->G;
         cp.W = plan->cfg.worldSize;
         cp.maxRecv = plan->maxRecv;
-        cp.pdlEarly = plan->pdlEarly;
-        cudaError_t e = ep::launch_combine(cp, plan->info.combineDtype == EP_FP32, plan->combineTile,
-                                           plan->info.combineBlocks, plan->info.combineWarps,
+        cudaError_t e = ep::launch_combine(cp, plan->info.combineDtype == EP_FP32, plan->info.combineBlocks,
+                                           plan->info.combineWarps,
                                            static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_fail(e, "launch combine");
         return EP_OK;

@@ -22,6 +22,9 @@ constexpr int kMaxCombineWarps = 8;
 constexpr int kLlThreads = 512;
 constexpr int kLlWarps = kLlThreads / 32;
 constexpr int kLlMaxTiles = 256;
+// Shared memory kept back from the dynamic budget for the kernels' static
+// shared memory.
+constexpr size_t kStaticSmemReserve = 2048;
 // Bounded waits give up after this many SM clock cycles (about 1 s at 1.9 GHz).
 constexpr long long kWaitCycles = 2000000000LL;
 
@@ -66,7 +69,6 @@ struct ScatterParams {
     int stages;       // stages per copy engine (>= 2)
     int baseShift;    // tile_base has one row per 2^baseShift tokens (8: route_count tiles; 5: fused chunks)
     int fanoutSwitch;        // x100: above this mean fan-out (rows per token) one engine per block sits out (0: never)
-    int pdlEarly;            // 1: let the next kernel of the stream launch once this one starts copying
     const uint32_t* scales;  // [G][scaleWords] per-token scale rows, or nullptr
     uint32_t* recv_scales;   // [W][maxRecv][scaleWords]
     int scaleWords;          // 0: no scale rows
@@ -102,7 +104,6 @@ struct CombineParams {
     uint32_t* done;        // blocks finished; the last one resets work and done
     long long rowBytes;    // bytes of a y / out row (the combine leg's row)
     int G, W, maxRecv;
-    int pdlEarly;          // 1: let the next kernel of the stream launch once this one starts
 };
 
 // Byte offsets of the dispatch scratch regions (each 256-byte aligned):
@@ -153,18 +154,13 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles, bool ll = 
 // dense: the large-batch form (tile counts at the W destinations only, last-block
 // scan, tile bases with stride W); else W + 1 columns, lastScan as set.
 cudaError_t launch_route_count(const RouteParams& p, bool dense, cudaStream_t s);
-// Scatter variants: TMA bulk copies staged in shared memory (kPend = bulk
-// store groups left draining when a stage is refilled), or plain 16-byte
-// register copies (no shared memory).
-constexpr int kScatterTma = 0;
-constexpr int kScatterRegs = 1;
-// dense: the large-batch instance (shared hand-out, tile bases in global
-// memory with stride W, no scan of its own).
-cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, bool dense, int blocks, int warps,
-                                size_t smem, cudaStream_t s);
+// The scatter: TMA bulk copies staged in shared memory. dense: the
+// large-batch instance (shared hand-out, tile bases in global memory with
+// stride W, no scan of its own).
+cudaError_t launch_scatter_rows(const ScatterParams& p, bool dense, int blocks, int warps, size_t smem,
+                                cudaStream_t s);
 // fp32: float32 combine leg (an fp32 plan); bf16 otherwise.
-// tile: combine kernel instance (columns x rows per pass, blocks per SM), see ep_kernels.cu.
-cudaError_t launch_combine(const CombineParams& p, bool fp32, int tile, int blocks, int warps, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s);
 // Fused dispatch (route + scan + scatter), a cooperative launch: blocks must
 // not exceed the co-resident capacity (fused_blocks_per_sm * SMs).
 cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s);
@@ -185,13 +181,13 @@ size_t scatter_smem_bytes(int warps, int stages, int chunkStride);
 // counts itself ([numTiles][W + 1] ints, rounded up to 128 bytes).
 size_t scatter_base_smem_bytes(int numTiles, int W);
 constexpr size_t kMaxBaseSmemBytes = 16384;
-// Opt the TMA scatter kernel in to `bytes` of dynamic shared memory.
-cudaError_t scatter_set_smem(int pend, size_t bytes);
+// Opt the scatter kernel in to `bytes` of dynamic shared memory.
+cudaError_t scatter_set_smem(size_t bytes);
 // Blocks of each kernel that fit on one SM (occupancy calculator).
-cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out);
-cudaError_t combine_blocks_per_sm(int warps, bool fp32, int tile, int* out);
-// Current dynamic shared-memory limit of the TMA scatter kernel.
-cudaError_t scatter_get_smem(int pend, int* bytes);
+cudaError_t scatter_blocks_per_sm(int warps, size_t smem, int* out);
+cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out);
+// Current dynamic shared-memory limit of the scatter kernel.
+cudaError_t scatter_get_smem(int* bytes);
 // Replace this thread's ep_last_error() text.
 void set_last_error(const char* msg);
 

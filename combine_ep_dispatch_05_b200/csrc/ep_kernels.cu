@@ -856,7 +856,6 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     if (kDense) {
         const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
         pdl_wait();     // routing written by route_count is visible from here on
-        if (p.pdlEarly) pdl_trigger();  // else the next kernel launches as this one exits
         const int engines = active_engines(p, nwarps, lane, -1);
         if (warp >= engines) return;  // this engine's stages stay unused
         DynFeed<false> feed;
@@ -868,7 +867,6 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem + p.baseOffset) : nullptr;
     const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, nwarps, lane);
     pdl_wait();     // routing written by route_count is visible from here on
-    if (p.pdlEarly) pdl_trigger();  // else the next kernel launches as this one exits
     int P, rows = -1;
     if (s_base != nullptr) {
         P = scan_tile_bases(p, s_base, &rows);
@@ -1221,52 +1219,6 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kerne
 }
 
 // =====================================================================
-// scatter_rows (registers): one warp per token, no shared-memory staging.
-// The warp loads a piece of the row (32 lanes x kVec 16-byte vectors) into
-// registers once and stores it to every destination; loads stream past L1.
-// =====================================================================
-constexpr int kRegVec = 28;  // 16-byte vectors per lane per piece: 14336-byte pieces
-
-__device__ __forceinline__ void st_v4(void* p, const uint4& v) {
-    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
-}
-
-__global__ void __launch_bounds__(256) ep_scatter_rows_regs_kernel(ScatterParams p) {
-    pdl_wait();
-    if (p.pdlEarly) pdl_trigger();
-    const int lane = threadIdx.x & 31;
-    const int nw = gridDim.x * (blockDim.x >> 5);
-    const long long V = p.rowBytes / 16;
-    for (int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < p.G; g += nw) {
-        const int lr = lane < p.W ? p.route[(size_t)g * p.W + lane].x : -1;
-        if (__ballot_sync(kFull, lr >= 0) == 0u) continue;
-        int my_slot;
-        const uint32_t mask = token_slots_and_meta(p, load_token_inputs<false>(p, g, lane, nullptr), lane, my_slot);
-        const uint8_t* src = p.x + (size_t)g * p.rowBytes;
-        for (long long v0 = 0; v0 < V; v0 += 32LL * kRegVec) {
-            uint4 buf[kRegVec];
-#pragma unroll
-            for (int i = 0; i < kRegVec; ++i) {
-                const long long v = v0 + lane + 32LL * i;
-                if (v < V) buf[i] = ld_stream_v4(src + v * 16);
-            }
-            for (uint32_t m = mask; m; m &= m - 1) {
-                const int pe = __ffs(m) - 1;
-                const int slot = __shfl_sync(kFull, my_slot, pe);
-                uint8_t* dst = p.recv_x + ((size_t)pe * p.maxRecv + slot) * p.rowBytes;
-#pragma unroll
-                for (int i = 0; i < kRegVec; ++i) {
-                    const long long v = v0 + lane + 32LL * i;
-                    if (v < V) st_v4(dst + v * 16, buf[i]);
-                }
-            }
-        }
-    }
-}
-
-// =====================================================================
 // combine: one warp per token, 16-byte columns, fma fold in destPe order.
 // =====================================================================
 
@@ -1363,7 +1315,6 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
     __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
     __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
     pdl_wait();  // y and the routing of the dispatch are visible from here on
-    if (p.pdlEarly) pdl_trigger();  // else the next kernel launches as this one exits
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int V = (int)(p.rowBytes / 16);
     const int W = p.W;
@@ -1475,22 +1426,14 @@ size_t scatter_smem_bytes(int warps, int stages, int chunkStride) {
 
 namespace {
 template <typename F>
-cudaError_t for_pend(int pend, bool dense, F&& f) {
-    switch (pend * 2 + (dense ? 1 : 0)) {
-        case 2: return f(ep_scatter_rows_kernel<1, false>);
-        case 3: return f(ep_scatter_rows_kernel<1, true>);
-        case 4: return f(ep_scatter_rows_kernel<2, false>);
-        case 5: return f(ep_scatter_rows_kernel<2, true>);
-        case 6: return f(ep_scatter_rows_kernel<3, false>);
-        case 7: return f(ep_scatter_rows_kernel<3, true>);
-        default: return cudaErrorInvalidValue;
-    }
+cudaError_t for_dense(bool dense, F&& f) {
+    return dense ? f(ep_scatter_rows_kernel<1, true>) : f(ep_scatter_rows_kernel<1, false>);
 }
 }  // namespace
 
-cudaError_t scatter_set_smem(int pend, size_t bytes) {
+cudaError_t scatter_set_smem(size_t bytes) {
     for (int d = 0; d < 2; ++d) {
-        const cudaError_t e = for_pend(pend, d != 0, [&](auto k) {
+        const cudaError_t e = for_dense(d != 0, [&](auto k) {
             return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         });
         if (e != cudaSuccess) return e;
@@ -1498,11 +1441,11 @@ cudaError_t scatter_set_smem(int pend, size_t bytes) {
     return cudaSuccess;
 }
 
-cudaError_t scatter_get_smem(int pend, int* bytes) {
+cudaError_t scatter_get_smem(int* bytes) {
     int lim = 1 << 30;
     for (int d = 0; d < 2; ++d) {
         cudaFuncAttributes fa;
-        const cudaError_t e = for_pend(pend, d != 0, [&](auto k) { return cudaFuncGetAttributes(&fa, k); });
+        const cudaError_t e = for_dense(d != 0, [&](auto k) { return cudaFuncGetAttributes(&fa, k); });
         if (e != cudaSuccess) return e;
         lim = fa.maxDynamicSharedSizeBytes < lim ? fa.maxDynamicSharedSizeBytes : lim;
     }
@@ -1510,13 +1453,11 @@ cudaError_t scatter_get_smem(int pend, int* bytes) {
     return cudaSuccess;
 }
 
-cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, int* out) {
-    if (mode == kScatterRegs)
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, ep_scatter_rows_regs_kernel, warps * 32, 0);
+cudaError_t scatter_blocks_per_sm(int warps, size_t smem, int* out) {
     int lo = 1 << 30;
     for (int d = 0; d < 2; ++d) {
         int n = 0;
-        const cudaError_t e = for_pend(pend, d != 0, [&](auto k) {
+        const cudaError_t e = for_dense(d != 0, [&](auto k) {
             return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, warps * 32, smem);
         });
         if (e != cudaSuccess) return e;
@@ -1527,31 +1468,22 @@ cudaError_t scatter_blocks_per_sm(int mode, int pend, int warps, size_t smem, in
 }
 
 namespace {
-// Combine kernel instances: tile 0 = 2 columns x 8 rows (2 blocks/SM),
-// 1 = 2 x 4 (4 blocks/SM), 2 = 1 x 8 (4 blocks/SM), 3 = 2 x 4 (3 blocks/SM).
-template <class Elem, typename F>
-cudaError_t for_tile(int tile, F&& f) {
-    switch (tile) {
-        case 1: return f(ep_combine_kernel<Elem, 2, 4, 4>);
-        case 2: return f(ep_combine_kernel<Elem, 1, 8, 4>);
-        case 3: return f(ep_combine_kernel<Elem, 2, 4, 3>);
-        default: return f(ep_combine_kernel<Elem, 2, 8, 2>);
-    }
-}
+// The combine instance: 2 columns x 8 rows of 16-byte loads in flight per
+// lane, 2 blocks of 256 threads per SM (B200: tiles of 2 x 4 at 4 or 3 blocks
+// per SM and 1 x 8 at 4 measured slower at the main workload and within 2% on
+// skewed routing).
+template <class Elem>
+constexpr auto combine_kernel = ep_combine_kernel<Elem, 2, 8, 2>;
 }  // namespace
 
-cudaError_t combine_blocks_per_sm(int warps, bool fp32, int tile, int* out) {
-    auto occ = [&](auto k) { return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, warps * 32, 0); };
-    return fp32 ? for_tile<CombineF32>(tile, occ) : for_tile<CombineBf16>(tile, occ);
+cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out) {
+    return fp32 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, combine_kernel<CombineF32>, warps * 32, 0)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, combine_kernel<CombineBf16>, warps * 32, 0);
 }
 
-cudaError_t launch_scatter_rows(const ScatterParams& p, int mode, int pend, bool dense, int blocks, int warps,
-                                size_t smem, cudaStream_t s) {
-    if (mode == kScatterRegs) {
-        cudaError_t e = launch_pdl(ep_scatter_rows_regs_kernel, blocks, warps * 32, 0, s, p);
-        return e != cudaSuccess ? e : cudaGetLastError();
-    }
-    cudaError_t e = for_pend(pend, dense, [&](auto k) { return launch_pdl(k, blocks, warps * 32, smem, s, p); });
+cudaError_t launch_scatter_rows(const ScatterParams& p, bool dense, int blocks, int warps, size_t smem,
+                                cudaStream_t s) {
+    cudaError_t e = for_dense(dense, [&](auto k) { return launch_pdl(k, blocks, warps * 32, smem, s, p); });
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -1644,11 +1576,10 @@ cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, 
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_combine(const CombineParams& p, bool fp32, int tile, int blocks, int warps, cudaStream_t s) {
-    auto go = [&](auto k) { return launch_pdl(k, blocks, warps * 32, 0, s, p); };
-    cudaError_t e = fp32 ? for_tile<CombineF32>(tile, go) : for_tile<CombineBf16>(tile, go);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s) {
+    const cudaError_t e = fp32 ? launch_pdl(combine_kernel<CombineF32>, blocks, warps * 32, 0, s, p)
+                               : launch_pdl(combine_kernel<CombineBf16>, blocks, warps * 32, 0, s, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace ep

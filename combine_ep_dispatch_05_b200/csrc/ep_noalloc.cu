@@ -133,24 +133,22 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
             return noalloc_fail(EP_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
 
         // Scatter geometry: the default plan's engines and stages.
-        const int pend = 1;
         const int warps = info.scatterWarps;
-        int stages = std::max(info.scatterStages, pend + 1);
+        int stages = std::max(info.scatterStages, 2);
         const int chunkStride = (info.scatterChunkBytes + 127) & ~127;
+        const size_t smemMax = (size_t)ds.smemOptin - ep::kStaticSmemReserve;
         size_t smem = ep::scatter_smem_bytes(warps, stages, chunkStride);
-        while (smem > (size_t)ds.smemOptin && stages > pend + 1)
-            smem = ep::scatter_smem_bytes(warps, --stages, chunkStride);
-        if (smem > (size_t)ds.smemOptin)
-            return noalloc_fail(EP_ERR_INVALID, "row piece does not fit shared memory");
+        while (smem > smemMax && stages > 2) smem = ep::scatter_smem_bytes(warps, --stages, chunkStride);
+        if (smem > smemMax) return noalloc_fail(EP_ERR_INVALID, "row piece does not fit shared memory");
         // Raise (never lower) the kernel's dynamic shared-memory limit, so that
         // plans created with a larger limit keep working.
         int limit = 0;
-        if ((e = ep::scatter_get_smem(pend, &limit)) != cudaSuccess)
+        if ((e = ep::scatter_get_smem(&limit)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "cudaFuncGetAttributes: %s", cudaGetErrorString(e));
-        if ((size_t)limit < smem && (e = ep::scatter_set_smem(pend, smem)) != cudaSuccess)
+        if ((size_t)limit < smem && (e = ep::scatter_set_smem(smem)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         int perSm = 0;
-        if ((e = ep::scatter_blocks_per_sm(ep::kScatterTma, pend, warps, smem, &perSm)) != cudaSuccess || perSm < 1)
+        if ((e = ep::scatter_blocks_per_sm(warps, smem, &perSm)) != cudaSuccess || perSm < 1)
             return noalloc_fail(EP_ERR_CUDA, "occupancy query failed");
 
         ep::RouteParams rp{};
@@ -203,9 +201,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         sp.stages = stages;
         sp.baseShift = 8;  // route_count's 256-token tiles
         sp.baseStride = W + 1;
-        sp.pdlEarly = 0;  // the next kernel launches as this one exits
-        if ((e = ep::launch_scatter_rows(sp, ep::kScatterTma, pend, false, ds.numSMs * perSm, warps, smem, s)) !=
-            cudaSuccess)
+        if ((e = ep::launch_scatter_rows(sp, false, ds.numSMs * perSm, warps, smem, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch scatter_rows: %s", cudaGetErrorString(e));
         return EP_OK;
     } catch (...) {

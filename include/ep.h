@@ -89,8 +89,8 @@ typedef struct EpPlanInfo {
     int32_t combineWarps;     /* warps per combine block */
     int32_t device;           /* CUDA device the plan lives on (-1 from ep_plan_query) */
     int32_t numSMs;           /* SMs of that device (0 from ep_plan_query) */
-    int32_t scatterMode;      /* 0: TMA bulk copies staged in shared memory; 1: register copies */
-    int32_t scatterPend;      /* TMA mode: bulk-store groups left draining when a stage refills */
+    int32_t scatterMode;      /* 0: TMA bulk copies staged in shared memory (the only mode) */
+    int32_t scatterPend;      /* bulk-store groups left draining when a stage refills (1) */
     int32_t combineDtype;     /* EP_FP32 for an fp32 plan, else EP_BF16 */
     int32_t combineHidden;    /* elements of a y / out row: h, or 2*h for EP_FP4X2 */
     int64_t combineRowBytes;  /* bytes of a y / out row */
@@ -149,20 +149,17 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * [W*T][W] of (slot, weight) pairs, per-tile counts and offsets, a tile
  * ticket, the error word). Returns NULL on failure (ep_last_error() says why).
  * Environment overrides, read here only (for geometry sweeps):
- * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK,
- * EP_SCATTER_PEND (1..3), EP_SCATTER_MODE ("tma" or "regs"), EP_COMBINE_BLOCKS,
+ * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK, EP_COMBINE_BLOCKS,
  * EP_COMBINE_WARPS, EP_DISPATCH_FUSED (1: one cooperative launch instead of
  * two), EP_LL_MAX_TOKENS (largest maxTokPerRank that takes the low-latency
  * dispatch; 0, i.e. off, by default), EP_SCATTER_FANOUT_SWITCH (100 x
  * the mean fan-out above which one copy engine per block sits out; 375 by
  * default, 0 never), EP_SCATTER_SCAN ("route": route_count's last block scans
- * the tile counts even when the scatter could), EP_PDL_EARLY (1: scatter and
- * combine let the next kernel of the stream launch when they start rather than
- * as they exit), EP_DISPATCH_DENSE (1 / 0: the large-batch form of the split
- * dispatch for every plan / for none; by default plans of more than 16384
- * tokens, W*T, take it), EP_SCATTER_LAYOUT (0..2: where the scatter's tile
- * bases sit in shared memory). Test hook: EP_TEST_UNREACHABLE_BARRIER=1 makes the fused
- * dispatch's grid barrier (with EP_DISPATCH_FUSED=1), or the low-latency
+ * the tile counts even when the scatter could), EP_DISPATCH_DENSE (1 / 0: the
+ * large-batch form of the split dispatch for every plan / for none; by default
+ * plans of more than 16384 tokens, W*T, take it). Test hook:
+ * EP_TEST_UNREACHABLE_BARRIER=1 makes the fused dispatch's grid barrier (with
+ * EP_DISPATCH_FUSED=1), or the low-latency
  * dispatch's wait for the counts of earlier tiles, unreachable, so that the
  * bounded wait runs out: the waiting blocks report EP_DEVERR_TIMEOUT, issue no
  * copy and return about one second later (the low-latency dispatch's first

@@ -302,22 +302,16 @@ def test_graph_capture_replay():
 
 @pytest.mark.parametrize("env", [
     {"EP_SCATTER_STAGES": "2"},
+    {"EP_SCATTER_STAGES": "4", "EP_SCATTER_CHUNK": "4096"},  # rows in pieces, a short ring
     {"EP_SCATTER_WARPS": "1", "EP_SCATTER_BLOCKS": "1"},   # one copy engine does everything
     {"EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2", "EP_SCATTER_CHUNK": "1024"},
     {"EP_COMBINE_WARPS": "1", "EP_COMBINE_BLOCKS": "3"},
-    {"EP_SCATTER_PEND": "2", "EP_SCATTER_STAGES": "4"},
-    {"EP_SCATTER_PEND": "3", "EP_SCATTER_STAGES": "4", "EP_SCATTER_CHUNK": "4096"},
-    {"EP_SCATTER_MODE": "regs"},
-    {"EP_SCATTER_MODE": "regs", "EP_SCATTER_WARPS": "2", "EP_SCATTER_BLOCKS": "5"},
     {"EP_DISPATCH_FUSED": "0"},                              # two launches: route_count + scatter_rows
     {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_BLOCKS": "3"},    # fused, few blocks: long chunk loops
     {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "8", "EP_SCATTER_STAGES": "2", "EP_SCATTER_CHUNK": "1024"},
     {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "1", "EP_SCATTER_BLOCKS": "1"},  # fewer warps than W
     {"EP_LL_MAX_TOKENS": "0"},                               # split dispatch at this size
     {"EP_SCATTER_SCAN": "route"},                            # route_count's last block scans the counts
-    {"EP_PDL_EARLY": "1"},                                   # dependents launch when scatter / combine start
-    {"EP_SCATTER_LAYOUT": "1"},                              # tile bases after the engines' stages
-    {"EP_SCATTER_LAYOUT": "2"},                              # engines' stages from a 1 KB boundary
     {"EP_DISPATCH_DENSE": "1"},                              # route_count's large-batch form
     {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "4"},   # four tiles of 512 tokens
     {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "7", "EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2",
