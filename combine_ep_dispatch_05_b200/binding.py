@@ -23,7 +23,11 @@ EP_DEVERR_EXPERT_RANGE, EP_DEVERR_TIMEOUT, EP_DEVERR_CAPACITY = 1, 2, 4
 
 EXPORTED = ("ep_cfg_check", "ep_plan_query", "ep_plan_create", "ep_plan_destroy", "ep_plan_info",
             "ep_dispatch", "ep_combine", "ep_plan_check_error", "ep_last_error", "ep_dispatch_noalloc",
-            "ep_dispatch_scaled")
+            "ep_dispatch_scaled", "ep_comm_create", "ep_comm_handle", "ep_comm_connect", "ep_comm_info",
+            "ep_comm_dispatch", "ep_comm_combine", "ep_comm_check_error", "ep_comm_destroy")
+EP_SYNC_DEVICE, EP_SYNC_HOST = 0, 1
+EP_ERR_PEER = -8
+EP_COMM_HANDLE_BYTES = 256
 EP_MAX_SCALE_WORDS = 4096
 EP_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
@@ -54,6 +58,23 @@ class EpPlanInfo(ctypes.Structure):
         return {n: getattr(self, n) for n, _ in self._fields_}
 
 
+class EpCommInfo(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_int32), ("worldSize", ctypes.c_int32), ("sync", ctypes.c_int32),
+                ("maxRecv", ctypes.c_int32), ("metaFields", ctypes.c_int32), ("maxLanding", ctypes.c_int32),
+                ("rowBytes", ctypes.c_int64), ("combineRowBytes", ctypes.c_int64),
+                ("recvX", ctypes.c_void_p), ("recvMeta", ctypes.c_void_p), ("recvCount", ctypes.c_void_p),
+                ("sharedBytes", ctypes.c_int64), ("localBytes", ctypes.c_int64),
+                ("scatterBlocks", ctypes.c_int32), ("scatterWarps", ctypes.c_int32),
+                ("scatterStages", ctypes.c_int32), ("combineBlocks", ctypes.c_int32),
+                ("combineWarps", ctypes.c_int32), ("device", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+HOST_BARRIER = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p)
+
+
 class EpError(RuntimeError):
     def __init__(self, code: int, where: str, msg: str):
         super().__init__(f"{where} failed ({code}): {msg}")
@@ -79,6 +100,14 @@ def _load() -> ctypes.CDLL:
         "ep_last_error": ([], ctypes.c_char_p),
         "ep_dispatch_noalloc": ([cfgp, P, P, P, P, P, P, P], I32),
         "ep_dispatch_scaled": ([P, P, P, P, P, ctypes.c_int32, P, P, P, P, P], I32),
+        "ep_comm_create": ([cfgp, ctypes.c_int32, ctypes.c_int32, HOST_BARRIER, P], P),
+        "ep_comm_handle": ([P, P], I32),
+        "ep_comm_connect": ([P, P], I32),
+        "ep_comm_info": ([P, ctypes.POINTER(EpCommInfo)], I32),
+        "ep_comm_dispatch": ([P, P, P, P, P], I32),
+        "ep_comm_combine": ([P, P, P, P], I32),
+        "ep_comm_check_error": ([P], I32),
+        "ep_comm_destroy": ([P], None),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -182,3 +211,68 @@ def ep_plan_check_error(plan: int) -> int:
 
 def library_path() -> str:
     return LIB_PATH
+
+
+# ------------------------------------------------------------ ranks in processes
+# The host barrier functions handed to the library must outlive the
+# communicator: they are kept here by communicator handle.
+_barriers: dict = {}
+
+
+def ep_comm_create(cfg, rank: int, sync: int = EP_SYNC_DEVICE, barrier=None) -> int:
+    """Rank `rank` of a communicator (include/ep_comm.h). barrier: for
+    EP_SYNC_HOST, a function of no arguments that returns once every rank has
+    called it and raises when that cannot happen (e.g. a torch.distributed
+    barrier with a timeout)."""
+    cb = None
+    if barrier is not None:
+        def _call(_ctx):
+            try:
+                barrier()
+                return 0
+            except Exception:  # a rank did not arrive: the library abandons the call
+                return 1
+        cb = HOST_BARRIER(_call)
+    h = _lib.ep_comm_create(ctypes.byref(_cfg(cfg)), int(rank), int(sync),
+                            cb if cb is not None else HOST_BARRIER(), None)
+    if not h:
+        raise EpError(EP_ERR_INVALID, "ep_comm_create", ep_last_error())
+    _barriers[h] = cb
+    return h
+
+
+def ep_comm_handle(comm: int) -> bytes:
+    buf = ctypes.create_string_buffer(EP_COMM_HANDLE_BYTES)
+    _check(_lib.ep_comm_handle(comm, buf), "ep_comm_handle")
+    return buf.raw
+
+
+def ep_comm_connect(comm: int, records) -> int:
+    """records: every rank's ep_comm_handle bytes, in rank order."""
+    blob = b"".join(bytes(r) for r in records)
+    buf = ctypes.create_string_buffer(blob, len(blob))
+    return _check(_lib.ep_comm_connect(comm, buf), "ep_comm_connect")
+
+
+def ep_comm_info(comm: int) -> EpCommInfo:
+    info = EpCommInfo()
+    _check(_lib.ep_comm_info(comm, ctypes.byref(info)), "ep_comm_info")
+    return info
+
+
+def ep_comm_dispatch(comm: int, x, topk_idx, topk_w, stream=None) -> int:
+    return _check(_lib.ep_comm_dispatch(comm, _addr(x), _addr(topk_idx), _addr(topk_w), _stream(stream)),
+                  "ep_comm_dispatch")
+
+
+def ep_comm_combine(comm: int, y, out, stream=None) -> int:
+    return _check(_lib.ep_comm_combine(comm, _addr(y), _addr(out), _stream(stream)), "ep_comm_combine")
+
+
+def ep_comm_check_error(comm: int) -> int:
+    return _check(_lib.ep_comm_check_error(comm), "ep_comm_check_error")
+
+
+def ep_comm_destroy(comm: int) -> None:
+    _lib.ep_comm_destroy(comm)
+    _barriers.pop(comm, None)

@@ -14,8 +14,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libep_b200.so")
 SOURCES = [os.path.join(PKG, "csrc", "ep_abi.cu"), os.path.join(PKG, "csrc", "ep_kernels.cu"),
-           os.path.join(PKG, "csrc", "ep_noalloc.cu")]
-DEPS = SOURCES + glob.glob(os.path.join(PKG, "csrc", "*.h")) + [os.path.join(ROOT, "include", "ep.h")]
+           os.path.join(PKG, "csrc", "ep_noalloc.cu"), os.path.join(PKG, "csrc", "ep_comm.cu")]
+DEPS = SOURCES + glob.glob(os.path.join(PKG, "csrc", "*.h")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared", "-I" + os.path.join(ROOT, "include")]
 

@@ -244,6 +244,48 @@ void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
 
 namespace ep {
 void set_last_error(const char* msg) { std::snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+
+int fail_code(int code, const char* msg) { return fail(code, "%s", msg); }
+
+int cfg_valid(const EpCfg* cfg) { return check_cfg(cfg); }
+
+// The split dispatch's copy geometry of a plan of cfg on the current device,
+// with route_count's last block scanning the tile counts (no tile table in
+// the scatter's shared memory), and the combine's grid.
+int copy_geometry(const EpCfg* cfg, CopyGeometry* out) {
+    int dev = 0, sms = 0, smemOptin = 0;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&smemOptin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return cuda_fail(e, "device attributes");
+    Geometry geo = pick_geometry(cfg, true);
+    const size_t limit = (size_t)smemOptin - kStaticSmemReserve;
+    size_t smem = scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+    while (smem > limit && geo.scatterStages > 2)
+        smem = scatter_smem_bytes(geo.scatterWarps, --geo.scatterStages, geo.chunkStride);
+    while (smem > limit && geo.scatterWarps > 1)
+        smem = scatter_smem_bytes(--geo.scatterWarps, geo.scatterStages, geo.chunkStride);
+    if (smem > limit) return fail(EP_ERR_INVALID, "row piece of %d bytes does not fit shared memory", geo.chunkBytes);
+    int sPerSm = 0, cPerSm = 0;
+    if ((e = scatter_set_smem(smem)) != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(scatter smem)");
+    if ((e = scatter_blocks_per_sm(geo.scatterWarps, smem, &sPerSm)) != cudaSuccess ||
+        (e = combine_blocks_per_sm(geo.combineWarps, cfg->dtype == EP_FP32, &cPerSm)) != cudaSuccess)
+        return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (sPerSm < 1 || cPerSm < 1) return fail(EP_ERR_INVALID, "kernel geometry does not fit one SM");
+    out->chunkBytes = geo.chunkBytes;
+    out->chunkStride = geo.chunkStride;
+    out->numChunks = geo.numChunks;
+    out->warps = geo.scatterWarps;
+    out->stages = geo.scatterStages;
+    out->blocks = env_int("EP_SCATTER_BLOCKS", sms * sPerSm);
+    out->smem = smem;
+    out->combineWarps = geo.combineWarps;
+    out->combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
+    out->numSMs = sms;
+    out->device = dev;
+    return EP_OK;
+}
 }  // namespace ep
 
 extern "C" {
@@ -663,6 +705,11 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
             plan->dispatched = true;
             return EP_OK;
         }
+        rp.x = static_cast<const uint8_t*>(x);
+        rp.rowBytes = plan->info.rowBytes;
+        rp.prefetchTokens = ep::prefetch_tokens(plan->G, plan->info.rowBytes,
+                                                (long long)plan->info.scatterBlocks * plan->info.scatterWarps,
+                                                plan->info.scatterStages);
         e = ep::launch_route_count(rp, plan->dense, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
         sp.baseShift = 8;  // route_count's 256-token tiles

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ep.h"
+
 namespace ep {
 
 // Tokens per routing tile: one 256-thread block counts one tile, one thread
@@ -28,6 +30,17 @@ constexpr size_t kStaticSmemReserve = 2048;
 // Bounded waits give up after this many SM clock cycles (about 1 s at 1.9 GHz).
 constexpr long long kWaitCycles = 2000000000LL;
 
+// Ranks in separate processes (one GPU each): where every rank's shared
+// buffers are mapped in this process, and this rank's copy of the count
+// table. Lives in device memory; the kernels read it through a pointer.
+struct PeerTable {
+    uint8_t* recv_x[kMaxWorld];     // rank q's receive rows [maxRecv][rowBytes]
+    int32_t* recv_meta[kMaxWorld];  // rank q's meta records [maxRecv][M]
+    uint8_t* landing[kMaxWorld];    // rank q's landing rows of the push combine [maxLanding][combine row]
+    int32_t* counts[kMaxWorld];     // rank q's count table [W][W]: row r = rows source r sends to each rank
+    unsigned* flags[kMaxWorld];     // rank q's barrier flags [W]: the last epoch each rank arrived at
+};
+
 struct RouteParams {
     const int32_t* idx;     // [G][k]
     const float* w;         // [G][k] or nullptr (useWeights == 0)
@@ -42,7 +55,22 @@ struct RouteParams {
     int32_t* err;           // device error word
     int G, W, k, nEpr, E, numTiles, maxRecv, useWeights;
     int lastScan;           // 1: the last block scans the tile counts; 0: the scatter does
+    // The rows of present tokens g < prefetchTokens are prefetched into L2:
+    // the scatter's copy engines load them first (see prefetch_tokens).
+    const uint8_t* x;       // [G][rowBytes]
+    long long rowBytes;
+    int prefetchTokens;
 };
+
+// Tokens whose rows route_count prefetches into L2 for a scatter of `engines`
+// copy engines with `stages` stages each: every engine's first stages - 1
+// tokens (the hand-out gives engine w the tokens w, w + engines, ... first),
+// or every token when the whole batch takes at most 32 MB.
+inline int prefetch_tokens(long long G, long long rowBytes, long long engines, int stages) {
+    const long long early = engines * (long long)(stages > 1 ? stages - 1 : 1);
+    if (G * rowBytes <= (32LL << 20) || early >= G) return (int)G;
+    return (int)early;
+}
 
 struct ScatterParams {
     const uint8_t* x;          // [G][rowBytes]
@@ -72,6 +100,12 @@ struct ScatterParams {
     const uint32_t* scales;  // [G][scaleWords] per-token scale rows, or nullptr
     uint32_t* recv_scales;   // [W][maxRecv][scaleWords]
     int scaleWords;          // 0: no scale rows
+    // Ranks in separate processes (nullptr: the W ranks are regions of recv_x /
+    // recv_meta on this GPU). recv_count above is then this rank's count row.
+    const PeerTable* peers;
+    int rank;                // this rank (source of every token of the call)
+    const int32_t* counts;   // this rank's count table [W][W], complete (after the exchange)
+    int32_t* recv_total;     // rows this rank receives, stored by block 0
     // Only the fused dispatch (route + scan + scatter in one launch) uses these:
     const float* w;          // [G][k] or nullptr
     uint32_t* tok_mask_w;    // = tok_mask, written by the routing phase
@@ -104,6 +138,37 @@ struct CombineParams {
     uint32_t* done;        // blocks finished; the last one resets work and done
     long long rowBytes;    // bytes of a y / out row (the combine leg's row)
     int G, W, maxRecv;
+    // Ranks in separate processes: y is this rank's landing rows, where the
+    // rows of destination pe start after those of the destinations before it
+    // (counts: this rank's count table; nullptr: one GPU, y = [W][maxRecv]).
+    const int32_t* counts;
+    int rank;
+    int32_t* err;          // the call is skipped when a barrier of it gave up (counts != nullptr)
+};
+
+// The count exchange and the barrier of ranks in separate processes (one
+// block of 32 threads).
+struct SyncParams {
+    const PeerTable* peers;
+    const int32_t* myCount;  // this rank's count row [W] (route_count's scan)
+    unsigned* epoch;         // barriers this rank has passed (its own, on the device)
+    int32_t* err;
+    int rank, W;
+    int exchange;            // 1: copy this rank's count row into row `rank` of every rank's count table
+    int barrier;             // 1: then wait until every rank has arrived at this barrier
+    unsigned slack;          // 0; test hook: 1 waits for an epoch that no rank reaches
+};
+
+// The push half of the combine of ranks in separate processes: every row
+// this rank received goes back, as its expert output, to the landing rows
+// of the rank it came from.
+struct PushParams {
+    const uint8_t* y;         // this rank's expert outputs [maxRecv][rowBytes]
+    const PeerTable* peers;
+    const int32_t* counts;    // this rank's count table [W][W]
+    int32_t* err;
+    long long rowBytes;       // bytes of a combine row
+    int rank, W, maxRecv, maxLanding;
 };
 
 // Byte offsets of the dispatch scratch regions (each 256-byte aligned):
@@ -175,20 +240,39 @@ cudaError_t ll_set_smem(int W, int topk, size_t bytes);
 cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out);
 cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s);
 
+// Ranks in separate processes: the count exchange / barrier, and the push.
+cudaError_t launch_comm_sync(const SyncParams& p, cudaStream_t s);
+cudaError_t launch_comm_push(const PushParams& p, int blocks, cudaStream_t s);
+
 // Shared-memory bytes the scatter kernel needs for a geometry.
 size_t scatter_smem_bytes(int warps, int stages, int chunkStride);
 // Shared memory for the tile bases when the scatter scans route_count's tile
 // counts itself ([numTiles][W + 1] ints, rounded up to 128 bytes).
 size_t scatter_base_smem_bytes(int numTiles, int W);
 constexpr size_t kMaxBaseSmemBytes = 16384;
-// Opt the scatter kernel in to `bytes` of dynamic shared memory.
+// Opt a kernel in to `bytes` of dynamic shared memory (these only ever raise
+// the limit, so that plans made earlier keep theirs).
 cudaError_t scatter_set_smem(size_t bytes);
 // Blocks of each kernel that fit on one SM (occupancy calculator).
 cudaError_t scatter_blocks_per_sm(int warps, size_t smem, int* out);
 cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out);
 // Current dynamic shared-memory limit of the scatter kernel.
 cudaError_t scatter_get_smem(int* bytes);
-// Replace this thread's ep_last_error() text.
+// Replace this thread's ep_last_error() text; fail_code also returns `code`.
 void set_last_error(const char* msg);
+int fail_code(int code, const char* msg);
+// ep_cfg_check's rules, without clearing the last error first.
+int cfg_valid(const EpCfg* cfg);
+
+// Copy and combine geometry of a plan on the current device (route_count's
+// last block scans the tile counts); EP_OK or a negative code.
+struct CopyGeometry {
+    int chunkBytes, chunkStride, numChunks;
+    int warps, stages, blocks;  // copy engines per block, stages per engine, scatter grid
+    size_t smem;                // the scatter's dynamic shared memory
+    int combineWarps, combineBlocks;
+    int numSMs, device;
+};
+int copy_geometry(const EpCfg* cfg, CopyGeometry* out);
 
 }  // namespace ep

@@ -102,6 +102,11 @@ __device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t byt
                  : "memory");
 }
 
+// Bring [p, p + bytes) into L2 (no completion to wait for).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -235,6 +240,14 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     float ws[kW];
     if (g < p.G) mask = route_token<kW, kK>(p.idx, p.w, g, k, p.nEpr, p.E, ws, bad);
     if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
+    // The scatter's first tokens: their rows start towards L2 now, while the
+    // tile counts are still being made, instead of after the scatter starts.
+    if (mask != 0u && g < p.prefetchTokens) {
+        const uint8_t* row = p.x + (size_t)g * p.rowBytes;
+        const long long n = p.rowBytes < (64 << 10) ? p.rowBytes : (64 << 10);
+        for (long long off = 0; off < n; off += 16384)
+            prefetch_l2(row + off, (uint32_t)(n - off < 16384 ? n - off : 16384));
+    }
 
     // Per-warp histogram by ballot; column W counts the present tokens.
 #pragma unroll
@@ -414,6 +427,57 @@ __device__ __forceinline__ TokenInputs load_token_inputs(const ScatterParams& p,
     return in;
 }
 
+// Where the rows, meta records and scale rows of each destination start, for
+// the kernels of one block: slot s of destination pe is at s_dst_x[pe] +
+// s * rowBytes (and likewise for the records and scale rows), and slots at or
+// above s_dst_cap[pe] are refused. On one GPU the destinations are regions of
+// recv_x / recv_meta / recv_scales, pe * maxRecv rows apart. With ranks in
+// separate processes each destination is another rank's receive buffer, where
+// this rank's rows start after those of the ranks before it (the count table),
+// so slots are counted from there.
+__shared__ uint8_t* s_dst_x[kMaxWorld];
+__shared__ int32_t* s_dst_meta[kMaxWorld];
+__shared__ uint32_t* s_dst_scales[kMaxWorld];
+__shared__ int s_dst_cap[kMaxWorld];
+
+// Every thread of the block calls it (it ends with __syncthreads); with
+// peers, after the count table is complete. Block 0 stores the rows this rank
+// receives. Returns false when an earlier barrier of the call gave up: then
+// nothing may be written to the other ranks.
+__device__ __forceinline__ bool dest_setup(const ScatterParams& p) {
+    const int pe = threadIdx.x;
+    if (pe < p.W) {
+        long long first;  // this source's first row in destination pe's buffers
+        uint8_t* x;
+        int32_t* meta;
+        uint32_t* sc = nullptr;
+        if (p.peers != nullptr) {
+            int before = 0;
+            for (int r = 0; r < p.rank; ++r) before += __ldcg(p.counts + r * p.W + pe);
+            first = before;
+            x = p.peers->recv_x[pe];
+            meta = p.peers->recv_meta[pe];
+        } else {
+            first = (long long)pe * p.maxRecv;
+            x = p.recv_x;
+            meta = p.recv_meta;
+            sc = p.recv_scales;
+        }
+        s_dst_x[pe] = x + first * p.rowBytes;
+        s_dst_meta[pe] = meta + first * p.M;
+        s_dst_scales[pe] = sc != nullptr ? sc + first * p.scaleWords : nullptr;
+        s_dst_cap[pe] = p.peers != nullptr ? p.maxRecv - (int)first : p.maxRecv;
+    }
+    const bool go = __syncthreads_and(p.peers == nullptr || (__ldcg(p.err) & EP_DEVERR_TIMEOUT) == 0) != 0;
+    if (go && p.peers != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        int total = 0;
+        for (int r = 0; r < p.W; ++r) total += __ldcg(p.counts + r * p.W + p.rank);
+        *p.recv_total = total;
+        if (total > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+    }
+    return go;
+}
+
 // The scale row of token g travels with it to every destination in `mask`
 // (lane pe holds the slot at pe).
 __device__ __forceinline__ void write_scales(const ScatterParams& p, int g, uint32_t mask, int my_slot, int lane) {
@@ -424,7 +488,7 @@ __device__ __forceinline__ void write_scales(const ScatterParams& p, int g, uint
         for (uint32_t m = mask; m; m &= m - 1) {
             const int pe = __ffs(m) - 1;
             const int slot = __shfl_sync(kFull, my_slot, pe);
-            if (wi < p.scaleWords) p.recv_scales[((size_t)pe * p.maxRecv + slot) * p.scaleWords + wi] = v;
+            if (wi < p.scaleWords) s_dst_scales[pe][(size_t)slot * p.scaleWords + wi] = v;
         }
     }
 }
@@ -434,7 +498,7 @@ __device__ __forceinline__ void write_scales(const ScatterParams& p, int g, uint
 // (wb_lane); lane j < k holds topk id e of entry j.
 __device__ __forceinline__ void write_records(const ScatterParams& p, int g, uint32_t mask, int my_slot,
                                               int wb_lane, int e, int lane) {
-    const int r = g / p.T, t = g - r * p.T;
+    const int r = p.peers != nullptr ? p.rank : g / p.T, t = g - (p.peers != nullptr ? 0 : r * p.T);
     const int pe_e = (e >= 0 && e < p.E) ? e / p.nEpr : -1;
     // field f of a record: 0 rank, 1 token, 2 weight bits, 3+j local id of entry j
     const int j0 = lane - 3, j1 = lane + 29;
@@ -444,7 +508,7 @@ __device__ __forceinline__ void write_records(const ScatterParams& p, int g, uin
         const int pe = __ffs(m) - 1;
         const int slot = __shfl_sync(kFull, my_slot, pe);
         const int wb = __shfl_sync(kFull, wb_lane, pe);
-        int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
+        int32_t* rec = s_dst_meta[pe] + (size_t)slot * p.M;
         int v0;
         if (lane == 0) v0 = r;
         else if (lane == 1) v0 = t;
@@ -467,7 +531,7 @@ __device__ __forceinline__ uint32_t token_slots_and_meta(const ScatterParams& p,
     bool ok = false;
     if (rr.x >= 0) {
         my_slot = in.base + rr.x;
-        ok = my_slot < p.maxRecv;  // always, unless the counts were corrupted
+        ok = my_slot < s_dst_cap[lane];  // always, unless the counts were corrupted
         if (!ok) atomicOr(p.err, EP_DEVERR_CAPACITY);
         p.route[(size_t)g * W + lane].x = ok ? my_slot : -1;
     }
@@ -788,7 +852,7 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
             const int pe = __ffs(m) - 1;
             const int slot = __shfl_sync(kFull, my_slot, pe);
             if (lane == 0)
-                bulk_store(p.recv_x + ((size_t)pe * p.maxRecv + slot) * p.rowBytes + off,
+                bulk_store(s_dst_x[pe] + (size_t)slot * p.rowBytes + off,
                            stage0_addr + (uint32_t)s * p.chunkStride, bytes);
         }
         if (lane == 0) bulk_commit();
@@ -811,6 +875,12 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
         }
     }
     if (lane == 0) bulk_wait_all();
+    // Another rank reads these rows after a barrier: make this engine's bulk
+    // stores visible beyond this GPU first.
+    if (p.peers != nullptr && lane == 0) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence_system();
+    }
     __syncwarp();
 }
 
@@ -856,6 +926,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     if (kDense) {
         const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
         pdl_wait();     // routing written by route_count is visible from here on
+        if (!dest_setup(p)) return;
         const int engines = active_engines(p, nwarps, lane, -1);
         if (warp >= engines) return;  // this engine's stages stay unused
         DynFeed<false> feed;
@@ -867,6 +938,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem + p.baseOffset) : nullptr;
     const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, nwarps, lane);
     pdl_wait();     // routing written by route_count is visible from here on
+    if (!dest_setup(p)) return;
     int P, rows = -1;
     if (s_base != nullptr) {
         P = scan_tile_bases(p, s_base, &rows);
@@ -933,6 +1005,7 @@ __global__ void __launch_bounds__(kLlThreads, 1) ep_dispatch_ll_kernel(ScatterPa
 
     pdl_wait();  // the ids and the counters of the previous call are visible from here on
     pdl_trigger();
+    dest_setup(p);
     if (tid == 0) {
         s_tile = atomicAdd(p.ll_ticket, 1);
         s_tag = (__ldcg(p.ll_epoch) << 1) | 1u;
@@ -1149,6 +1222,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kerne
     const int W = p.W;
     const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
     pdl_wait();  // the ids may come from the previous kernel of the stream
+    dest_setup(p);
 
     // 1. route 32-token chunks
     const uint32_t lt = lanemask_lt();
@@ -1319,6 +1393,24 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
     const int V = (int)(p.rowBytes / 16);
     const int W = p.W;
 
+    // Lane pe: where destination pe's rows start in y. One GPU: region pe of
+    // [W][maxRecv]. Ranks in processes: y is this rank's landing rows, in
+    // destination order (this rank's count row gives each destination's rows).
+    const uint8_t* ybase;
+    if (p.counts != nullptr) {
+        if ((__ldcg(p.err) & EP_DEVERR_TIMEOUT) != 0) return;  // a barrier of this call gave up
+        const int c = lane < W ? __ldcg(p.counts + p.rank * W + lane) : 0;
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int m = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += m;
+        }
+        ybase = p.y + (size_t)(incl - c) * p.rowBytes;
+    } else {
+        ybase = p.y + (size_t)lane * p.maxRecv * p.rowBytes;
+    }
+
     // Tokens come from the shared hand-out (a token's cost grows with its
     // number of destinations, so a purely static split would leave a tail);
     // the next token and its routing row are fetched one token ahead.
@@ -1345,7 +1437,7 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
         const int n = __popc(mask);
         if (rr.x >= 0) {
             const int pos = __popc(mask & lanemask_lt());
-            s_row[warp][pos] = p.y + ((size_t)lane * p.maxRecv + rr.x) * p.rowBytes;
+            s_row[warp][pos] = ybase + (size_t)rr.x * p.rowBytes;
             s_w[warp][pos] = __int_as_float(rr.y);
         }
         __syncwarp();
@@ -1367,6 +1459,130 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
             __threadfence();
         }
     }
+}
+
+// =====================================================================
+// Ranks in separate processes (one GPU each). Every rank maps every rank's
+// shared buffers (receive rows, meta records, landing rows, count table,
+// barrier flags); the PeerTable holds the addresses in this process.
+// =====================================================================
+__device__ __forceinline__ void st_release_sys_u32(unsigned* p, unsigned v) {
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_sys_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// The barrier of the ranks, one warp. Each rank counts its barriers (the
+// epoch lives on the device, so the replays of a captured graph stay in
+// step, as the design page's cross-device barrier does); a rank arrives by
+// storing its epoch in slot `rank` of every rank's flags, after a system-scope
+// fence so that all it wrote before is visible to them, and then waits until
+// every slot of its own flags has reached the epoch. The wait gives up after
+// kWaitCycles and reports EP_DEVERR_TIMEOUT; the epochs of the ranks are then
+// out of step and the communicator must be rebuilt.
+__device__ __forceinline__ bool comm_barrier(const SyncParams& p, int lane) {
+    unsigned e = 0;
+    if (lane == 0) e = *p.epoch + 1u;
+    e = __shfl_sync(kFull, e, 0);
+    __threadfence_system();
+    __syncwarp();
+    if (lane < p.W) st_release_sys_u32(p.peers->flags[lane] + p.rank, e);
+    bool ok = true;
+    if (lane < p.W) {
+        const unsigned* f = p.peers->flags[p.rank] + lane;
+        const unsigned want = e + p.slack;
+        if ((int)(ld_acquire_sys_u32(f) - want) < 0) {
+            const long long t0 = clock64();
+            while ((int)(ld_acquire_sys_u32(f) - want) < 0) {
+                if (clock64() - t0 > kWaitCycles) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+    }
+    ok = __all_sync(kFull, ok);
+    if (lane == 0) {
+        *p.epoch = e;
+        if (!ok) atomicOr(p.err, EP_DEVERR_TIMEOUT);
+    }
+    __threadfence_system();
+    return ok;
+}
+
+__global__ void __launch_bounds__(32) ep_comm_sync_kernel(SyncParams p) {
+    pdl_wait();  // the count row and the rows of the previous kernel are complete
+    const int lane = threadIdx.x;
+    if ((__ldcg(p.err) & EP_DEVERR_TIMEOUT) != 0) return;  // an earlier barrier gave up
+    if (p.exchange && lane < p.W) {
+        int32_t* dst = p.peers->counts[lane] + p.rank * p.W;
+        for (int pe = 0; pe < p.W; ++pe) dst[pe] = __ldcg(p.myCount + pe);
+    }
+    if (p.barrier) comm_barrier(p, lane);
+}
+
+// The push: receive slot s of this rank holds a row of source r (slots are
+// in source order, r's rows from before(r) on); its expert output goes to
+// landing row land(r) + s - before(r) of rank r, where land(r) counts the
+// rows r sent to the ranks before this one, so that r's landing rows are in
+// destination order. One warp per row, 8 16-byte loads in flight per lane.
+__global__ void __launch_bounds__(256) ep_comm_push_kernel(PushParams p) {
+    __shared__ int s_before[kMaxWorld + 1];
+    __shared__ int s_land[kMaxWorld];
+    __shared__ uint8_t* s_dst[kMaxWorld];
+    pdl_wait();  // the expert outputs and the count table are complete
+    if ((__ldcg(p.err) & EP_DEVERR_TIMEOUT) != 0) return;  // a barrier gave up: touch no other rank
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    if (warp == 0) {
+        const int c = lane < p.W ? __ldcg(p.counts + lane * p.W + p.rank) : 0;
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int m = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += m;
+        }
+        if (lane < p.W) {
+            s_before[lane] = incl - c;
+            int land = 0;
+            for (int pe = 0; pe < p.rank; ++pe) land += __ldcg(p.counts + lane * p.W + pe);
+            s_land[lane] = land;
+            s_dst[lane] = p.peers->landing[lane];
+        }
+        if (lane == 31) s_before[p.W] = incl;
+    }
+    __syncthreads();
+    const int total = s_before[p.W];
+    if (total > p.maxRecv) {  // only when the counts were corrupted
+        if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(p.err, EP_DEVERR_CAPACITY);
+        return;
+    }
+    const int V = (int)(p.rowBytes / 16);
+    for (int s = blockIdx.x * nwarps + warp; s < total; s += gridDim.x * nwarps) {
+        int r = 0;
+        while (r + 1 < p.W && s >= s_before[r + 1]) ++r;
+        const long long li = (long long)s_land[r] + (s - s_before[r]);
+        if (li >= p.maxLanding) {  // only when the counts were corrupted
+            if (lane == 0) atomicOr(p.err, EP_DEVERR_CAPACITY);
+            continue;
+        }
+        const uint8_t* src = p.y + (size_t)s * p.rowBytes;
+        uint8_t* dst = s_dst[r] + (size_t)li * p.rowBytes;
+        for (int v0 = lane; v0 < V; v0 += 32 * 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + 32 * u < V) v[u] = ld_stream_v4(src + (size_t)(v0 + 32 * u) * 16);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + 32 * u < V) *reinterpret_cast<uint4*>(dst + (size_t)(v0 + 32 * u) * 16) = v[u];
+        }
+    }
+    __threadfence_system();  // the rows are read by rank r after the next barrier
 }
 
 }  // namespace
@@ -1429,13 +1645,22 @@ template <typename F>
 cudaError_t for_dense(bool dense, F&& f) {
     return dense ? f(ep_scatter_rows_kernel<1, true>) : f(ep_scatter_rows_kernel<1, false>);
 }
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` (never lower it:
+// plans and calls made earlier may rely on a larger limit).
+template <typename K>
+cudaError_t raise_smem(K kernel, size_t bytes) {
+    cudaFuncAttributes fa;
+    const cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    if ((size_t)fa.maxDynamicSharedSizeBytes >= bytes) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
 }  // namespace
 
 cudaError_t scatter_set_smem(size_t bytes) {
     for (int d = 0; d < 2; ++d) {
-        const cudaError_t e = for_dense(d != 0, [&](auto k) {
-            return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-        });
+        const cudaError_t e = for_dense(d != 0, [&](auto k) { return raise_smem(k, bytes); });
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -1502,9 +1727,7 @@ cudaError_t for_world(int W, int k, F&& f) {
 }  // namespace
 
 cudaError_t fused_set_smem(int W, int topk, size_t bytes) {
-    return for_world(W, topk, [&](auto k) {
-        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    });
+    return for_world(W, topk, [&](auto k) { return raise_smem(k, bytes); });
 }
 
 cudaError_t fused_blocks_per_sm(int W, int topk, int warps, size_t smem, int* out) {
@@ -1560,9 +1783,7 @@ size_t ll_smem_bytes(int tileTokens, int W, int warps, int stages, int chunkStri
 }
 
 cudaError_t ll_set_smem(int W, int topk, size_t bytes) {
-    return for_world_ll(W, topk, [&](auto k) {
-        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    });
+    return for_world_ll(W, topk, [&](auto k) { return raise_smem(k, bytes); });
 }
 
 cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out) {
@@ -1579,6 +1800,16 @@ cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, 
 cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s) {
     const cudaError_t e = fp32 ? launch_pdl(combine_kernel<CombineF32>, blocks, warps * 32, 0, s, p)
                                : launch_pdl(combine_kernel<CombineBf16>, blocks, warps * 32, 0, s, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_comm_sync(const SyncParams& p, cudaStream_t s) {
+    const cudaError_t e = launch_pdl(ep_comm_sync_kernel, 1, 32, 0, s, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_comm_push(const PushParams& p, int blocks, cudaStream_t s) {
+    const cudaError_t e = launch_pdl(ep_comm_push_kernel, blocks, 256, 0, s, p);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -12,7 +12,7 @@ import textwrap
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "ep.h")
+HEADERS = [os.path.join(ROOT, "include", "ep.h"), os.path.join(ROOT, "include", "ep_comm.h")]
 
 
 @pytest.fixture(scope="module")
@@ -24,7 +24,7 @@ def ep():
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    src = "".join(open(h).read() for h in HEADERS)
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(ep_[a-z_]+)\s*\(", src)))
 
@@ -32,7 +32,8 @@ def declared_functions():
 def test_header_declares_the_api():
     names = declared_functions()
     for n in ("ep_plan_create", "ep_dispatch", "ep_combine", "ep_plan_destroy", "ep_last_error",
-              "ep_plan_info", "ep_plan_check_error", "ep_cfg_check", "ep_plan_query"):
+              "ep_plan_info", "ep_plan_check_error", "ep_cfg_check", "ep_plan_query", "ep_comm_create",
+              "ep_comm_handle", "ep_comm_connect", "ep_comm_dispatch", "ep_comm_combine", "ep_comm_destroy"):
         assert n in names
 
 
@@ -50,8 +51,9 @@ def test_library_exports_every_declared_symbol(ep):
 def test_struct_layout_matches_header(ep, tmp_path):
     """sizeof/offsetof from a C compile of include/ep.h against the ctypes mirror."""
     fields = {"EpCfg": [n for n, _ in ep.EpCfg._fields_],
-              "EpPlanInfo": [n for n, _ in ep.EpPlanInfo._fields_]}
-    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "ep.h"', 'int main(void) {']
+              "EpPlanInfo": [n for n, _ in ep.EpPlanInfo._fields_],
+              "EpCommInfo": [n for n, _ in ep.EpCommInfo._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "ep_comm.h"', 'int main(void) {']
     for st, names in fields.items():
         lines.append(f'  printf("{st} size %zu\\n", sizeof({st}));')
         for n in names:
@@ -74,7 +76,7 @@ def test_header_compiles_as_plain_c_and_cpp(tmp_path):
     """The ABI header needs no CUDA header and compiles as C and C++."""
     for lang, comp in (("c", "gcc"), ("cpp", "g++")):
         f = tmp_path / f"inc.{lang}"
-        f.write_text('#include "ep.h"\nint main(void){ EpCfg c = {0}; return (int)sizeof(c) - 32; }\n')
+        f.write_text('#include "ep_comm.h"\nint main(void){ EpCfg c = {0}; return (int)sizeof(c) - 32; }\n')
         subprocess.check_call([comp, "-I", os.path.join(ROOT, "include"), str(f), "-o", str(tmp_path / lang)])
         assert subprocess.run([str(tmp_path / lang)]).returncode == 0
 
