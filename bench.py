@@ -374,6 +374,8 @@ def time_graphs(calls: dict, dev, dist) -> dict:
 def run_ours(args, wl):
     import torch
     rank, world, local, dist = dist_setup(args.gpus)
+    if world > 1:
+        return run_comm(args, wl, rank, world, local, dist)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if dist is not None:
@@ -585,6 +587,231 @@ def run_ours(args, wl):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+# ------------------------------------------------------------------ ranks on separate GPUs
+NVLINK_PEER_GBS = 770.0  # measured peer copy per direction per GPU on this machine's B200s
+
+
+def comm_workload(wl, world: int):
+    """The workload with its W ranks real, one per GPU: every rank holds
+    wl.max_tok token rows (wl.ct live), the experts are shared out over the
+    ranks (same total E), and every rank can receive the worst case."""
+    if wl.E % world:
+        raise SystemExit(f"{wl.E} experts do not divide over {world} ranks")
+    return wl.replace(W=world, n_epr=wl.E // world, max_recv=world * wl.max_tok)
+
+
+def rank_inputs(cwl, rank: int) -> dict:
+    """Rank `rank`'s seeded tokens (x, ids over all E experts, weights), made
+    on that rank only."""
+    one = cwl.replace(W=1, n_epr=cwl.E, max_recv=0, seed=cwl.seed * 1000 + rank)
+    inp = make_inputs(one)
+    return {"x": inp["x"][0], "topk_idx": inp["topk_idx"][0],
+            "topk_w": None if inp["topk_w"] is None else inp["topk_w"][0]}
+
+
+def nccl_alltoallv_step(x, idx, w, world: int, n_epr: int, dist):
+    """The library-collective baseline of one dispatch + identity expert +
+    combine: torch gathers the rows of each destination, NCCL moves them with
+    all_to_all_single (sizes exchanged first, then read on the host), the
+    rows go back the same way, and torch folds them (index_add in float32;
+    its order is not fixed). x: uint8 [T][row bytes] of bf16 rows. Returns
+    (out as bf16 [T][h], the received rows)."""
+    import torch
+    T, k = idx.shape
+    pe = torch.where(idx >= 0, torch.div(idx, n_epr, rounding_mode="floor"), torch.full_like(idx, world))
+    hit = torch.zeros((T, world + 1), dtype=torch.bool, device=x.device)
+    hit.scatter_(1, pe.long(), True)
+    hit = hit[:, :world]
+    dest, tok = hit.t().nonzero(as_tuple=True)  # by destination, then token
+    send = x.index_select(0, tok)
+    send_counts = hit.sum(0).to(torch.int64)
+    recv_counts = torch.empty_like(send_counts)
+    dist.all_to_all_single(recv_counts, send_counts)
+    sc, rc = send_counts.tolist(), recv_counts.tolist()
+    recv = torch.empty((sum(rc),) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
+    dist.all_to_all_single(recv, send, rc, sc)
+    back = torch.empty_like(send)
+    dist.all_to_all_single(back, recv, sc, rc)  # identity expert: the rows come back
+    if w is None:
+        wsum = hit.to(torch.float32)
+    else:
+        wsum = torch.zeros((T, world + 1), dtype=torch.float32, device=x.device)
+        wsum.scatter_add_(1, pe.long(), w)
+        wsum = wsum[:, :world]
+    rows = back.view(torch.bfloat16).float() * wsum[tok, dest].unsqueeze(1)  # rows are bytes of bf16
+    out = torch.zeros((T, rows.shape[1]), dtype=torch.float32, device=x.device)
+    out.index_add_(0, tok, rows)
+    return out.to(torch.bfloat16), recv
+
+
+def run_comm(args, wl, rank, world, local, dist):
+    """N > 1: the W ranks are the N processes, one per GPU, connected by the
+    library's communicator (ep_comm_*): the rows cross NVLink. Timed as the
+    one-GPU step, max over ranks; the NCCL all-to-allv baseline beside it."""
+    import datetime
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    from combine_ep_dispatch_05_b200 import build as epbuild
+    if rank == 0:
+        epbuild.build()
+    dist.barrier()
+    import combine_ep_dispatch_05_b200 as ep
+    from combine_ep_dispatch_05_b200 import comm as epcomm
+
+    cwl = comm_workload(wl, world)
+    try:
+        comm = epcomm.create_and_connect(cwl.cfg(), dist, ep.EP_SYNC_DEVICE)
+        sync = "device"
+    except ep.EpError as e:  # ranks sharing a GPU: the host barrier instead
+        if e.code != ep.EP_ERR_UNSUPPORTED:
+            raise
+        comm = epcomm.create_and_connect(cwl.cfg(), dist, ep.EP_SYNC_HOST)
+        sync = "host"
+    info = ep.ep_comm_info(comm)
+    inp = rank_inputs(cwl, rank)
+    x = torch.from_numpy(inp["x"].view(np.uint8)).to(dev)
+    idx = torch.from_numpy(inp["topk_idx"]).to(dev)
+    w = None if inp["topk_w"] is None else torch.from_numpy(inp["topk_w"]).to(dev)
+    hc = info.combineRowBytes // 2
+    y = torch.as_tensor(_DeviceMemory(info.recvX, (info.maxRecv, hc), "<i2"), device=dev).view(torch.bfloat16)
+    out = torch.empty((cwl.max_tok, hc), dtype=torch.bfloat16, device=dev)
+    flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_out = torch.empty((), dtype=torch.int32, device=dev)
+    s = torch.cuda.current_stream(dev)
+
+    for i in range(max(args.warmup, 0)):
+        torch.amax(flush, dim=0, out=flush_out)
+        ep.ep_comm_dispatch(comm, x, idx, w, s)
+        ep.ep_comm_combine(comm, y, out, s)
+    torch.cuda.synchronize(dev)
+    if ep.ep_comm_check_error(comm):
+        raise RuntimeError("device error word after warm-up")
+    check_comm_step(cwl, inp, out, info, rank, world, dist, dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for i in range(args.steps):
+        torch.amax(flush, dim=0, out=flush_out)
+        evs[i][0].record(s)
+        ep.ep_comm_dispatch(comm, x, idx, w, s)
+        evs[i][1].record(s)
+        ep.ep_comm_combine(comm, y, out, s)
+        evs[i][2].record(s)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clocks = sampler.stop()
+    disp_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
+    comb_ms = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps))
+    step_ms = max_over_ranks(disp_ms + comb_ms, dist, dev)
+    disp_ms = max_over_ranks(disp_ms, dist, dev)
+    comb_ms = max_over_ranks(comb_ms, dist, dev)
+    if ep.ep_comm_check_error(comm):
+        raise RuntimeError("device error word after the timed steps")
+
+    # Rows that cross NVLink: every row a rank sends to another rank, and the
+    # same rows coming back in the combine (the busiest rank sets the pace).
+    recv_n = int(torch.as_tensor(_DeviceMemory(info.recvCount, (1,), "<i4"), device=dev).cpu()[0])
+    T = cwl.max_tok
+    ids = inp["topk_idx"]
+    dest = np.where(ids >= 0, ids // cwl.n_epr, -1)
+    hit = np.zeros((T, world), dtype=bool)
+    for j in range(cwl.k):
+        m = dest[:, j] >= 0
+        hit[np.nonzero(m)[0], dest[m, j]] = True
+    sent_remote = int(hit.sum() - hit[:, rank].sum())
+    link_bytes = max_over_ranks(float(sent_remote * info.rowBytes), dist, dev)
+    link_gbs = link_bytes / (max(disp_ms, comb_ms) * 1e-3) / 1e9
+
+    # The library-collective baseline on the same tokens.
+    xb = x.view(cwl.max_tok, -1)
+    for _ in range(2):
+        nccl_alltoallv_step(xb, idx, w, world, cwl.n_epr, dist)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nb = max(3, min(args.steps, 20))
+    e0.record(s)
+    for _ in range(nb):
+        nccl_alltoallv_step(xb, idx, w, world, cwl.n_epr, dist)
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    nccl_ms = max_over_ranks(e0.elapsed_time(e1) / nb, dist, dev)
+
+    dist.barrier()
+    ep.ep_comm_destroy(comm)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": step_ms * 1e3, "unit": "us", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {**describe(cwl), "flush": "read",
+                       "parallelism": f"expert parallel: {world} ranks, one per GPU, rows over NVLink "
+                                      f"(communicator, {sync} barriers)"},
+            "dispatch_us": disp_ms * 1e3, "combine_us": comb_ms * 1e3,
+            "rows_received_rank0": recv_n,
+            "roofline": {"bound": "nvlink", "kernel": "ep_comm dispatch / combine",
+                         "achieved": link_gbs, "peak": NVLINK_PEER_GBS,
+                         "peak_source": "measured peer copy per direction per GPU (fallback figure)",
+                         "unit": "GB/s", "frac": link_gbs / NVLINK_PEER_GBS, "traffic": None,
+                         "bytes_per_launch": link_bytes, "avg_launch_us": max(disp_ms, comb_ms) * 1e3},
+            "nccl_baseline": {"step_us": nccl_ms * 1e3, "impl": "torch gather + NCCL all_to_all_single "
+                              "(sizes read on the host) + torch index_add fold"},
+            "cpu_baseline": None, "e2e": None, "clocks": clocks,
+            "gpu_launches": 7 * args.steps, "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
+def check_comm_step(cwl, inp, out, info, rank, world, dist, dev):
+    """Self-check of the last warm-up step, from this rank's own inputs: the
+    rows this rank received must number what every rank's routing sends it
+    (count rows gathered from all ranks), and with the identity expert every
+    output row must be the row times the sum of its weight sums, within the
+    spec's tolerance (float64 reference)."""
+    import torch
+    T, k, W = cwl.max_tok, cwl.k, world
+    ids = inp["topk_idx"]
+    dest = np.where(ids >= 0, ids // cwl.n_epr, -1)
+    hit = np.zeros((T, W), dtype=bool)
+    for j in range(k):
+        m = dest[:, j] >= 0
+        hit[np.nonzero(m)[0], dest[m, j]] = True
+    counts = torch.from_numpy(hit.sum(0).astype(np.int64)).to(dev)
+    table = [torch.empty_like(counts) for _ in range(W)]
+    dist.all_gather(table, counts)
+    expect = int(sum(int(t[rank]) for t in table))
+    got = int(torch.as_tensor(_DeviceMemory(info.recvCount, (1,), "<i4"), device=dev).cpu()[0])
+    if got != expect:
+        raise RuntimeError(f"rank {rank}: received {got} rows, the routing sends {expect}")
+    xw = inp["x"].view(np.uint16).astype(np.uint32) << 16
+    xf = xw.view(np.float32).astype(np.float64)
+    if inp["topk_w"] is None:
+        scale = hit.sum(1).astype(np.float64)
+    else:
+        scale = np.where(ids >= 0, inp["topk_w"], 0.0).astype(np.float64).sum(1)
+    ref = xf * scale[:, None]
+    o = out.float().cpu().numpy().astype(np.float64)
+    bad = np.abs(o - ref) > 2.0 ** -7 * np.abs(ref) + 1e-3
+    if bad.any():
+        raise RuntimeError(f"rank {rank}: {int(bad.sum())} output elements outside tolerance")
+
+
+class _DeviceMemory:
+    """A view of library-owned device memory for torch.as_tensor."""
+
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
 
 
 def main():

@@ -13,13 +13,15 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libep_b200.so")
+# EP_B200_LIBRARY=debug loads the bounds-checking build (libep_b200_debug.so).
+LIB_PATH = os.path.join(_PKG, "libep_b200_debug.so" if os.environ.get("EP_B200_LIBRARY") == "debug"
+                        else "libep_b200.so")
 
 EP_BF16, EP_FP32, EP_FP8, EP_FP4X2 = 0, 1, 2, 3
 EP_OK = 0
 EP_ERR_INVALID, EP_ERR_UNSUPPORTED, EP_ERR_NOMEM, EP_ERR_CUDA = -1, -2, -3, -4
 EP_ERR_STATE, EP_ERR_ALIGN, EP_ERR_DEVICE = -5, -6, -7
-EP_DEVERR_EXPERT_RANGE, EP_DEVERR_TIMEOUT, EP_DEVERR_CAPACITY = 1, 2, 4
+EP_DEVERR_EXPERT_RANGE, EP_DEVERR_TIMEOUT, EP_DEVERR_CAPACITY, EP_DEVERR_BOUNDS = 1, 2, 4, 8
 
 EXPORTED = ("ep_cfg_check", "ep_plan_query", "ep_plan_create", "ep_plan_destroy", "ep_plan_info",
             "ep_dispatch", "ep_combine", "ep_plan_check_error", "ep_last_error", "ep_dispatch_noalloc",

@@ -54,6 +54,8 @@ struct EpPlan {
     unsigned* ll_done;
     unsigned* ll_epoch;
     unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
+    int boundsRows;         // bounds-checking build: rows of each destination's buffers it checks against
+    int prefetchBlocks;     // route_count's L2 prefetch blocks (EP_ROUTE_PREFETCH_BLOCKS, 0: none)
     int fanoutSwitch;       // x100, see ScatterParams
     bool dispatched;
 };
@@ -494,6 +496,10 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         // EP_DEVERR_TIMEOUT.
         if (const char* t = std::getenv("EP_TEST_UNREACHABLE_BARRIER"))
             plan->barrierSlack = std::strcmp(t, "1") == 0 ? 1u : 0u;
+        // Test hook of the bounds-checking build: check the receive buffers
+        // against fewer rows than they have, so that the checks must fire.
+        plan->boundsRows = std::min(env_int("EP_TEST_BOUNDS_ROWS", plan->info.maxRecv), plan->info.maxRecv);
+        plan->prefetchBlocks = env_int("EP_ROUTE_PREFETCH_BLOCKS", sms, 0);
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
         plan->dense = !fused && dense;
@@ -664,6 +670,7 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         sp.scales = static_cast<const uint32_t*>(scales);
         sp.recv_scales = static_cast<uint32_t*>(recv_scales);
         sp.scaleWords = scaleWords;
+        sp.boundsRows = plan->boundsRows;
         if (plan->ll) {
             // One launch: every block routes and scans the batch, then copies its share.
             const int nEpr = c.numExpertPerRank;
@@ -707,6 +714,7 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         }
         rp.x = static_cast<const uint8_t*>(x);
         rp.rowBytes = plan->info.rowBytes;
+        rp.prefetchBlocks = plan->prefetchBlocks;
         rp.prefetchTokens = ep::prefetch_tokens(plan->G, plan->info.rowBytes,
                                                 (long long)plan->info.scatterBlocks * plan->info.scatterWarps,
                                                 plan->info.scatterStages);
@@ -749,6 +757,8 @@ int ep_combine(EpPlan* plan, const void* y, void* out, void* stream) {
         cp.G = plan->G;
         cp.W = plan->cfg.worldSize;
         cp.maxRecv = plan->maxRecv;
+        cp.err = plan->err;
+        cp.yBytes = plan->info.yBytes;
         cudaError_t e = ep::launch_combine(cp, plan->info.combineDtype == EP_FP32, plan->info.combineBlocks,
                                            plan->info.combineWarps,
                                            static_cast<cudaStream_t>(stream));

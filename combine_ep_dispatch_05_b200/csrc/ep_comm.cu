@@ -367,6 +367,7 @@ int ep_comm_dispatch(EpComm* c, const void* x, const int32_t* topk_idx, const fl
         rp.lastScan = 1;
         rp.x = static_cast<const uint8_t*>(x);
         rp.rowBytes = c->rowBytes;
+        rp.prefetchBlocks = c->geo.numSMs;
         rp.prefetchTokens =
             ep::prefetch_tokens(c->T, c->rowBytes, (long long)c->geo.blocks * c->geo.warps, c->geo.stages);
         cudaError_t e = ep::launch_route_count(rp, c->dense, s);
@@ -408,6 +409,7 @@ int ep_comm_dispatch(EpComm* c, const void* x, const int32_t* topk_idx, const fl
         sp.rank = c->rank;
         sp.counts = reinterpret_cast<const int32_t*>(c->shared + c->offCounts);
         sp.recv_total = reinterpret_cast<int32_t*>(lb + c->offRecvTotal);
+        sp.boundsRows = c->maxRecv;
         e = ep::launch_scatter_rows(sp, c->dense, c->geo.blocks, c->geo.warps, c->geo.smem, s);
         if (e != cudaSuccess) return cuda_err(e, "launch scatter_rows");
 
@@ -469,6 +471,7 @@ int ep_comm_combine(EpComm* c, const void* y, void* out, void* stream) {
         cp.counts = reinterpret_cast<const int32_t*>(c->shared + c->offCounts);
         cp.rank = c->rank;
         cp.err = pp.err;
+        cp.yBytes = (long long)c->maxLanding * c->crow;
         e = ep::launch_combine(cp, c->cfg.dtype == EP_FP32, c->geo.combineBlocks, c->geo.combineWarps, s);
         if (e != cudaSuccess) return cuda_err(e, "launch combine");
         return EP_OK;

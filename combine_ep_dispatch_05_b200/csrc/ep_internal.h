@@ -27,6 +27,14 @@ constexpr int kLlMaxTiles = 256;
 // Shared memory kept back from the dynamic budget for the kernels' static
 // shared memory.
 constexpr size_t kStaticSmemReserve = 2048;
+// The bounds-checking build (-DEP_DEBUG_BOUNDS, libep_b200_debug.so) checks
+// every row, record and scale-row address of the copies against its buffer's
+// extent; an access outside it is skipped and EP_DEVERR_BOUNDS is set.
+#ifdef EP_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
 // Bounded waits give up after this many SM clock cycles (about 1 s at 1.9 GHz).
 constexpr long long kWaitCycles = 2000000000LL;
 
@@ -55,17 +63,20 @@ struct RouteParams {
     int32_t* err;           // device error word
     int G, W, k, nEpr, E, numTiles, maxRecv, useWeights;
     int lastScan;           // 1: the last block scans the tile counts; 0: the scatter does
-    // The rows of present tokens g < prefetchTokens are prefetched into L2:
-    // the scatter's copy engines load them first (see prefetch_tokens).
+    // Blocks numTiles.. of the launch only prefetch into L2 the rows of the
+    // present tokens g < prefetchTokens, which the scatter's copy engines load
+    // first, so that those reads overlap the routing instead of following it.
     const uint8_t* x;       // [G][rowBytes]
     long long rowBytes;
     int prefetchTokens;
+    int prefetchBlocks;
 };
 
-// Tokens whose rows route_count prefetches into L2 for a scatter of `engines`
-// copy engines with `stages` stages each: every engine's first stages - 1
-// tokens (the hand-out gives engine w the tokens w, w + engines, ... first),
-// or every token when the whole batch takes at most 32 MB.
+// Tokens whose rows route_count's prefetch blocks bring into L2 for a
+// scatter of `engines` copy engines with `stages` stages each: the first
+// stages - 1 rounds of the hand-out (workers are numbered so that round i is
+// the tokens i * engines .. (i + 1) * engines - 1), or every token when the
+// whole batch takes at most 32 MB.
 inline int prefetch_tokens(long long G, long long rowBytes, long long engines, int stages) {
     const long long early = engines * (long long)(stages > 1 ? stages - 1 : 1);
     if (G * rowBytes <= (32LL << 20) || early >= G) return (int)G;
@@ -106,6 +117,7 @@ struct ScatterParams {
     int rank;                // this rank (source of every token of the call)
     const int32_t* counts;   // this rank's count table [W][W], complete (after the exchange)
     int32_t* recv_total;     // rows this rank receives, stored by block 0
+    int boundsRows;          // bounds-checking build: rows of each destination's buffers (maxRecv)
     // Only the fused dispatch (route + scan + scatter in one launch) uses these:
     const float* w;          // [G][k] or nullptr
     uint32_t* tok_mask_w;    // = tok_mask, written by the routing phase
@@ -144,6 +156,7 @@ struct CombineParams {
     const int32_t* counts;
     int rank;
     int32_t* err;          // the call is skipped when a barrier of it gave up (counts != nullptr)
+    long long yBytes;      // bounds-checking build: bytes of y
 };
 
 // The count exchange and the barrier of ranks in separate processes (one

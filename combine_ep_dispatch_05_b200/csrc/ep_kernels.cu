@@ -54,6 +54,10 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void mbar_fence_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -102,7 +106,7 @@ __device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t byt
                  : "memory");
 }
 
-// Bring [p, p + bytes) into L2 (no completion to wait for).
+// Bring [p, p + bytes) into L2 (nothing to wait for).
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -140,6 +144,10 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
 // tail (the spread of a worker's total over ~100 tokens is a few percent).
 // With fewer than eight tokens per worker the split is static only: the
 // counter would put thousands of atomics on one address for little balance.
+// Workers are numbered warp-major (worker = warp * blocks + block), so that
+// the static rounds give every block, i.e. every SM, the same number of
+// tokens to within one per warp (block-major numbering gave the first blocks
+// all the extra tokens: 15 against 12 per SM for 2048 tokens on 444 engines).
 // =====================================================================
 struct TokenSource {
     int w, nU, R, G, i;
@@ -229,6 +237,26 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     pdl_wait();     // the ids may come from the previous kernel of the stream
     pdl_trigger();  // let the scatter's launch and prologue overlap this kernel
 
+    if ((int)blockIdx.x >= p.numTiles) {
+        // A prefetch block: the rows of present early tokens, one token per
+        // thread (the blocks spread the prefetches over many SMs, whose
+        // copy units each issue them one after another).
+        for (int t = (blockIdx.x - p.numTiles) * kCountTile + threadIdx.x; t < p.prefetchTokens;
+             t += p.prefetchBlocks * kCountTile) {
+            bool present = false;
+            for (int j = 0; j < p.k; ++j) {
+                const int e = p.idx[(size_t)t * p.k + j];
+                present |= e >= 0 && e < p.E;
+            }
+            if (!present) continue;
+            const uint8_t* row = p.x + (size_t)t * p.rowBytes;
+            const long long n = p.rowBytes < (64 << 10) ? p.rowBytes : (64 << 10);
+            for (long long off = 0; off < n; off += 16384)
+                prefetch_l2(row + off, (uint32_t)(n - off < 16384 ? n - off : 16384));
+        }
+        return;
+    }
+
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = blockIdx.x * kCountTile + tid;
     const int W = p.W, k = p.k, C = kDense ? W : W + 1;
@@ -240,14 +268,6 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
     float ws[kW];
     if (g < p.G) mask = route_token<kW, kK>(p.idx, p.w, g, k, p.nEpr, p.E, ws, bad);
     if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
-    // The scatter's first tokens: their rows start towards L2 now, while the
-    // tile counts are still being made, instead of after the scatter starts.
-    if (mask != 0u && g < p.prefetchTokens) {
-        const uint8_t* row = p.x + (size_t)g * p.rowBytes;
-        const long long n = p.rowBytes < (64 << 10) ? p.rowBytes : (64 << 10);
-        for (long long off = 0; off < n; off += 16384)
-            prefetch_l2(row + off, (uint32_t)(n - off < 16384 ? n - off : 16384));
-    }
 
     // Per-warp histogram by ballot; column W counts the present tokens.
 #pragma unroll
@@ -439,6 +459,21 @@ __shared__ uint8_t* s_dst_x[kMaxWorld];
 __shared__ int32_t* s_dst_meta[kMaxWorld];
 __shared__ uint32_t* s_dst_scales[kMaxWorld];
 __shared__ int s_dst_cap[kMaxWorld];
+// Bounds-checking build: the end of each destination's receive rows, meta
+// records and scale rows.
+__shared__ const uint8_t* s_dst_x_end[kDebugBounds ? kMaxWorld : 1];
+__shared__ const int32_t* s_dst_meta_end[kDebugBounds ? kMaxWorld : 1];
+__shared__ const uint32_t* s_dst_scales_end[kDebugBounds ? kMaxWorld : 1];
+
+// Bounds-checking build: false (and EP_DEVERR_BOUNDS) when [p, p + bytes)
+// is not inside [lo, hi).
+__device__ __forceinline__ bool in_bounds(const void* p, long long bytes, const void* lo, const void* hi, int32_t* err) {
+    if (!kDebugBounds) return true;
+    const char* a = static_cast<const char*>(p);
+    if (a >= static_cast<const char*>(lo) && a + bytes <= static_cast<const char*>(hi)) return true;
+    atomicOr(err, EP_DEVERR_BOUNDS);
+    return false;
+}
 
 // Every thread of the block calls it (it ends with __syncthreads); with
 // peers, after the count table is complete. Block 0 stores the rows this rank
@@ -467,6 +502,12 @@ __device__ __forceinline__ bool dest_setup(const ScatterParams& p) {
         s_dst_meta[pe] = meta + first * p.M;
         s_dst_scales[pe] = sc != nullptr ? sc + first * p.scaleWords : nullptr;
         s_dst_cap[pe] = p.peers != nullptr ? p.maxRecv - (int)first : p.maxRecv;
+        if (kDebugBounds) {
+            const long long end = (p.peers != nullptr ? 0 : (long long)pe * p.maxRecv) + p.boundsRows;
+            s_dst_x_end[pe] = x + end * p.rowBytes;
+            s_dst_meta_end[pe] = meta + end * p.M;
+            s_dst_scales_end[pe] = sc != nullptr ? sc + end * p.scaleWords : nullptr;
+        }
     }
     const bool go = __syncthreads_and(p.peers == nullptr || (__ldcg(p.err) & EP_DEVERR_TIMEOUT) == 0) != 0;
     if (go && p.peers != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
@@ -488,7 +529,9 @@ __device__ __forceinline__ void write_scales(const ScatterParams& p, int g, uint
         for (uint32_t m = mask; m; m &= m - 1) {
             const int pe = __ffs(m) - 1;
             const int slot = __shfl_sync(kFull, my_slot, pe);
-            if (wi < p.scaleWords) s_dst_scales[pe][(size_t)slot * p.scaleWords + wi] = v;
+            uint32_t* dst = s_dst_scales[pe] + (size_t)slot * p.scaleWords + wi;
+            if (wi < p.scaleWords && in_bounds(dst, 4, s_dst_scales[pe], s_dst_scales_end[kDebugBounds ? pe : 0], p.err))
+                *dst = v;
         }
     }
 }
@@ -509,6 +552,7 @@ __device__ __forceinline__ void write_records(const ScatterParams& p, int g, uin
         const int slot = __shfl_sync(kFull, my_slot, pe);
         const int wb = __shfl_sync(kFull, wb_lane, pe);
         int32_t* rec = s_dst_meta[pe] + (size_t)slot * p.M;
+        if (!in_bounds(rec, 4LL * p.M, s_dst_meta[pe], s_dst_meta_end[kDebugBounds ? pe : 0], p.err)) continue;
         int v0;
         if (lane == 0) v0 = r;
         else if (lane == 1) v0 = t;
@@ -799,9 +843,13 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
             const uint32_t bytes = (uint32_t)(rem < p.chunkBytes ? rem : p.chunkBytes);
             item_tok[s] = pg;
             item_chunk[s] = pc;
-            mbar_arrive_expect_tx(bar0 + 8u * s, bytes);
-            bulk_load(stage0_addr + (uint32_t)s * p.chunkStride, p.x + (size_t)feed.row(p, pg) * p.rowBytes + off,
-                      bytes, bar0 + 8u * s);
+            const uint8_t* src = p.x + (size_t)feed.row(p, pg) * p.rowBytes + off;
+            if (in_bounds(src, bytes, p.x, p.x + (size_t)p.G * p.rowBytes, p.err)) {
+                mbar_arrive_expect_tx(bar0 + 8u * s, bytes);
+                bulk_load(stage0_addr + (uint32_t)s * p.chunkStride, src, bytes, bar0 + 8u * s);
+            } else {
+                mbar_arrive(bar0 + 8u * s);  // the stage completes without data
+            }
         }
         ++issued;
         if (++pc == p.numChunks) {
@@ -851,9 +899,9 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
         for (uint32_t m = cur_mask; m; m &= m - 1) {
             const int pe = __ffs(m) - 1;
             const int slot = __shfl_sync(kFull, my_slot, pe);
-            if (lane == 0)
-                bulk_store(s_dst_x[pe] + (size_t)slot * p.rowBytes + off,
-                           stage0_addr + (uint32_t)s * p.chunkStride, bytes);
+            uint8_t* dst = s_dst_x[pe] + (size_t)slot * p.rowBytes + off;
+            if (lane == 0 && in_bounds(dst, bytes, s_dst_x[pe], s_dst_x_end[kDebugBounds ? pe : 0], p.err))
+                bulk_store(dst, stage0_addr + (uint32_t)s * p.chunkStride, bytes);
         }
         if (lane == 0) bulk_commit();
         ++consumed;
@@ -908,7 +956,7 @@ __device__ __forceinline__ void global_copy_engines(const ScatterParams& p, cons
                                                     int warp, int nwarps, int P, int rows, const int* s_base) {
     const int engines = active_engines(p, nwarps, lane, rows);
     if (warp >= engines) return;  // this engine's stages stay unused
-    const TokenSource src = make_source(blockIdx.x * engines + warp, gridDim.x * engines, p.G, p.work, P);
+    const TokenSource src = make_source(warp * gridDim.x + blockIdx.x, gridDim.x * engines, p.G, p.work, P);
     if (s_base != nullptr) run_split_engine<kPend, true>(p, es, lane, src, s_base);
     else run_split_engine<kPend, false>(p, es, lane, src, nullptr);
 }
@@ -930,7 +978,7 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
         const int engines = active_engines(p, nwarps, lane, -1);
         if (warp >= engines) return;  // this engine's stages stay unused
         DynFeed<false> feed;
-        feed.init(p, make_source(blockIdx.x * engines + warp, gridDim.x * engines, p.G, p.work, p.G), lane,
+        feed.init(p, make_source(warp * gridDim.x + blockIdx.x, gridDim.x * engines, p.G, p.work, p.G), lane,
                   nullptr);
         copy_engine<kPend>(p, es, lane, feed);
         return;
@@ -1414,7 +1462,7 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
     // Tokens come from the shared hand-out (a token's cost grows with its
     // number of destinations, so a purely static split would leave a tail);
     // the next token and its routing row are fetched one token ahead.
-    TokenSource src = make_source(blockIdx.x * (blockDim.x >> 5) + warp, gridDim.x * (blockDim.x >> 5),
+    TokenSource src = make_source(warp * gridDim.x + blockIdx.x, gridDim.x * (blockDim.x >> 5),
                                   p.G, p.work, p.G);
     int next = 0;
     if (lane == 0) next = source_next(src);
@@ -1437,7 +1485,9 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
         const int n = __popc(mask);
         if (rr.x >= 0) {
             const int pos = __popc(mask & lanemask_lt());
-            s_row[warp][pos] = ybase + (size_t)rr.x * p.rowBytes;
+            const uint8_t* row = ybase + (size_t)rr.x * p.rowBytes;
+            if (!in_bounds(row, p.rowBytes, p.y, p.y + p.yBytes, p.err)) row = p.y;  // skipped: reads y's first row
+            s_row[warp][pos] = row;
             s_w[warp][pos] = __int_as_float(rr.y);
         }
         __syncwarp();
@@ -1610,7 +1660,7 @@ cudaError_t launch_pdl(void (*kernel)(P), int grid, int block, size_t smem, cuda
 namespace {
 template <bool kDense>
 cudaError_t launch_route_count_as(const RouteParams& p, cudaStream_t s) {
-    auto go = [&](auto kernel) { return launch_pdl(kernel, p.numTiles, kCountTile, 0, s, p); };
+    auto go = [&](auto kernel) { return launch_pdl(kernel, p.numTiles + p.prefetchBlocks, kCountTile, 0, s, p); };
     if (p.W <= 8)
         return p.k <= 8    ? go(ep_route_count_kernel<8, 8, kDense>)
                : p.k <= 16 ? go(ep_route_count_kernel<8, 16, kDense>)

@@ -174,6 +174,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         rp.useWeights = cfg->useWeights;
         rp.x = static_cast<const uint8_t*>(x);
         rp.rowBytes = info.rowBytes;
+        rp.prefetchBlocks = ds.numSMs;
         rp.prefetchTokens = ep::prefetch_tokens(G, info.rowBytes, (long long)ds.numSMs * perSm * warps, stages);
         if ((e = ep::launch_route_count(rp, false, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch route_count: %s", cudaGetErrorString(e));
@@ -204,6 +205,7 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         sp.stages = stages;
         sp.baseShift = 8;  // route_count's 256-token tiles
         sp.baseStride = W + 1;
+        sp.boundsRows = info.maxRecv;
         if ((e = ep::launch_scatter_rows(sp, false, ds.numSMs * perSm, warps, smem, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch scatter_rows: %s", cudaGetErrorString(e));
         return EP_OK;

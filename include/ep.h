@@ -127,7 +127,9 @@ enum {
 enum {
     EP_DEVERR_EXPERT_RANGE = 1, /* an expert id >= E was seen; it was treated as masked */
     EP_DEVERR_TIMEOUT = 2,      /* a bounded wait on a shared-memory barrier gave up */
-    EP_DEVERR_CAPACITY = 4      /* a destination received more than maxRecv rows */
+    EP_DEVERR_CAPACITY = 4,     /* a destination received more than maxRecv rows */
+    EP_DEVERR_BOUNDS = 8        /* bounds-checking build only (libep_b200_debug.so): an access
+                                   fell outside its buffer; it was skipped */
 };
 
 /* Validate a configuration on the host (no CUDA call). Returns EP_OK, or
@@ -157,14 +159,18 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * default, 0 never), EP_SCATTER_SCAN ("route": route_count's last block scans
  * the tile counts even when the scatter could), EP_DISPATCH_DENSE (1 / 0: the
  * large-batch form of the split dispatch for every plan / for none; by default
- * plans of more than 16384 tokens, W*T, take it). Test hook:
+ * plans of more than 16384 tokens, W*T, take it), EP_ROUTE_PREFETCH_BLOCKS
+ * (route_count's extra blocks that prefetch the scatter's first rows into L2;
+ * one per SM by default, 0 none). Test hooks:
  * EP_TEST_UNREACHABLE_BARRIER=1 makes the fused dispatch's grid barrier (with
  * EP_DISPATCH_FUSED=1), or the low-latency
  * dispatch's wait for the counts of earlier tiles, unreachable, so that the
  * bounded wait runs out: the waiting blocks report EP_DEVERR_TIMEOUT, issue no
  * copy and return about one second later (the low-latency dispatch's first
  * tile waits on nothing and writes its meta records before it gives up), and
- * the context stays usable. */
+ * the context stays usable; EP_TEST_BOUNDS_ROWS=n makes the bounds-checking
+ * build (libep_b200_debug.so) check the receive buffers against n rows per
+ * destination instead of maxRecv. */
 EpPlan* ep_plan_create(const EpCfg* cfg);
 
 /* Free the plan and its scratch. NULL is a no-op. The caller must make sure no

@@ -78,3 +78,63 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     assert cpu["cores"] >= 1 and cpu["nproc"] >= 1 and cpu["cpu_model"]
     assert cpu["single_core_us"] > 0 and "full tiny workload" in cpu["sample"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+
+
+def _nccl_baseline_worker(rank, world, port, q):
+    """The bench's all-to-allv baseline on gloo ranks (CPU tensors): its
+    received rows are the oracle's, in the same (source rank, token) order,
+    and its output rows are within the spec's tolerance of the oracle's."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import bench
+        import oracle
+        wl = bench.comm_workload(bench.get_workload("tiny").replace(h=64, max_tok=16, ct=12), world)
+        parts = [bench.rank_inputs(wl, r) for r in range(world)]
+        full = {k: np.stack([p[k] for p in parts]) for k in ("x", "topk_idx", "topk_w")}
+        ref = oracle.dispatch(wl.cfg(), full["x"], full["topk_idx"], full["topk_w"])
+        ref_out = oracle.combine(wl.cfg(), ref["recv_x"], ref["slotmap"], ref["wsum"])
+        mine = parts[rank]
+        x = torch.from_numpy(mine["x"].view(np.uint8).reshape(wl.max_tok, -1))
+        out, recv = bench.nccl_alltoallv_step(x, torch.from_numpy(mine["topk_idx"]),
+                                             torch.from_numpy(mine["topk_w"]), world, wl.n_epr, dist)
+        n = int(ref["recv_count"][rank])
+        ok_rows = recv.shape[0] == n and np.array_equal(recv.numpy().view(np.uint16).reshape(n, -1),
+                                                         ref["recv_x"][rank, :n])
+        got = out.float().numpy()
+        exp = torch.from_numpy(ref_out[rank].view(np.int16)).view(torch.bfloat16).float().numpy()
+        ok_out = bool((np.abs(got - exp) <= 2.0 ** -7 * np.abs(exp) + 1e-3).all())
+        q.put((rank, ok_rows, ok_out))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_nccl_baseline_logic_on_gloo():
+    import torch.multiprocessing as tmp
+    ctx = tmp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_nccl_baseline_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ok_rows, ok_out in got:
+        assert ok_rows, f"rank {rank}: received rows differ from the oracle's"
+        assert ok_out, f"rank {rank}: output outside tolerance"
+
+
+def test_comm_workload_keeps_the_expert_count():
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = bench.get_workload("main")
+    for n in (1, 2, 4, 8):
+        c = bench.comm_workload(wl, n)
+        assert c.W == n and c.E == wl.E and c.max_recv == n * wl.max_tok and c.max_tok == wl.max_tok
