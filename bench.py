@@ -649,12 +649,22 @@ def nccl_alltoallv_step(x, idx, w, world: int, n_epr: int, dist):
 def run_comm(args, wl, rank, world, local, dist):
     """N > 1: the W ranks are the N processes, one per GPU, connected by the
     library's communicator (ep_comm_*): the rows cross NVLink. Timed as the
-    one-GPU step, max over ranks; the NCCL all-to-allv baseline beside it."""
+    one-GPU step, max over ranks; the NCCL all-to-allv baseline beside it.
+    EP_BENCH_SHARE_GPU=1 puts every rank on GPU 0 with host barriers and a
+    gloo process group, to run this path where there is one GPU (no NCCL
+    baseline then)."""
     import datetime
     import torch
+    share = os.environ.get("EP_BENCH_SHARE_GPU") == "1"
+    if share:
+        local = 0
     dev = torch.device("cuda", local)
     torch.cuda.set_device(local)
-    dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    if share:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    else:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    cdev = torch.device("cpu") if share else dev  # where the bench's own collectives run
     from combine_ep_dispatch_05_b200 import build as epbuild
     if rank == 0:
         epbuild.build()
@@ -663,14 +673,12 @@ def run_comm(args, wl, rank, world, local, dist):
     from combine_ep_dispatch_05_b200 import comm as epcomm
 
     cwl = comm_workload(wl, world)
-    try:
-        comm = epcomm.create_and_connect(cwl.cfg(), dist, ep.EP_SYNC_DEVICE)
-        sync = "device"
-    except ep.EpError as e:  # ranks sharing a GPU: the host barrier instead
-        if e.code != ep.EP_ERR_UNSUPPORTED:
-            raise
+    if share:
         comm = epcomm.create_and_connect(cwl.cfg(), dist, ep.EP_SYNC_HOST)
         sync = "host"
+    else:
+        comm = epcomm.create_and_connect(cwl.cfg(), dist, ep.EP_SYNC_DEVICE)
+        sync = "device"
     info = ep.ep_comm_info(comm)
     inp = rank_inputs(cwl, rank)
     x = torch.from_numpy(inp["x"].view(np.uint8)).to(dev)
@@ -690,7 +698,7 @@ def run_comm(args, wl, rank, world, local, dist):
     torch.cuda.synchronize(dev)
     if ep.ep_comm_check_error(comm):
         raise RuntimeError("device error word after warm-up")
-    check_comm_step(cwl, inp, out, info, rank, world, dist, dev)
+    check_comm_step(cwl, inp, out, info, rank, world, dist, dev, cdev)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     dist.barrier()
@@ -708,9 +716,9 @@ def run_comm(args, wl, rank, world, local, dist):
     clocks = sampler.stop()
     disp_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
     comb_ms = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps))
-    step_ms = max_over_ranks(disp_ms + comb_ms, dist, dev)
-    disp_ms = max_over_ranks(disp_ms, dist, dev)
-    comb_ms = max_over_ranks(comb_ms, dist, dev)
+    step_ms = max_over_ranks(disp_ms + comb_ms, dist, cdev)
+    disp_ms = max_over_ranks(disp_ms, dist, cdev)
+    comb_ms = max_over_ranks(comb_ms, dist, cdev)
     if ep.ep_comm_check_error(comm):
         raise RuntimeError("device error word after the timed steps")
 
@@ -725,23 +733,60 @@ def run_comm(args, wl, rank, world, local, dist):
         m = dest[:, j] >= 0
         hit[np.nonzero(m)[0], dest[m, j]] = True
     sent_remote = int(hit.sum() - hit[:, rank].sum())
-    link_bytes = max_over_ranks(float(sent_remote * info.rowBytes), dist, dev)
+    link_bytes = max_over_ranks(float(sent_remote * info.rowBytes), dist, cdev)
     link_gbs = link_bytes / (max(disp_ms, comb_ms) * 1e-3) / 1e9
 
     # The library-collective baseline on the same tokens.
-    xb = x.view(cwl.max_tok, -1)
-    for _ in range(2):
-        nccl_alltoallv_step(xb, idx, w, world, cwl.n_epr, dist)
-    torch.cuda.synchronize(dev)
-    dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    nb = max(3, min(args.steps, 20))
-    e0.record(s)
-    for _ in range(nb):
-        nccl_alltoallv_step(xb, idx, w, world, cwl.n_epr, dist)
-    e1.record(s)
-    torch.cuda.synchronize(dev)
-    nccl_ms = max_over_ranks(e0.elapsed_time(e1) / nb, dist, dev)
+    nccl = None
+    if not share:
+        xb = x.view(cwl.max_tok, -1)
+        for _ in range(2):
+            nccl_alltoallv_step(xb, idx, w, world, cwl.n_epr, dist)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nb = max(3, min(args.steps, 20))
+        e0.record(s)
+        for _ in range(nb):
+            nccl_alltoallv_step(xb, idx, w, world, cwl.n_epr, dist)
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+        nccl = {"step_us": max_over_ranks(e0.elapsed_time(e1) / nb, dist, cdev) * 1e3,
+                "impl": "torch gather + NCCL all_to_all_single (sizes read on the host) + torch index_add fold"}
+
+    # End to end through the same calls: every step uploads this rank's
+    # inputs from pinned host memory and downloads its output rows.
+    e2e = None
+    if not args.no_e2e:
+        x_h = torch.from_numpy(inp["x"].view(np.uint8)).pin_memory()
+        idx_h = torch.from_numpy(inp["topk_idx"]).pin_memory()
+        w_h = None if w is None else torch.from_numpy(inp["topk_w"]).pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_h, non_blocking=True)
+            idx.copy_(idx_h, non_blocking=True)
+            if w_h is not None:
+                w.copy_(w_h, non_blocking=True)
+            ep.ep_comm_dispatch(comm, x, idx, w, s)
+            ep.ep_comm_combine(comm, y, out, s)
+            out_h.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        n_e2e = max(2, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, cdev)
+        h2d = x_h.numel() + idx_h.numel() * 4 + (0 if w_h is None else w_h.numel() * 4)
+        e2e = {"value": e2e_ms * 1e3, "unit": "us", "h2d_bytes_per_step": int(h2d) * world,
+               "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size()) * world, "steps": n_e2e,
+               "pipeline": "sequential on each rank; bytes are all ranks' together"}
 
     dist.barrier()
     ep.ep_comm_destroy(comm)
@@ -761,9 +806,8 @@ def run_comm(args, wl, rank, world, local, dist):
                          "peak_source": "measured peer copy per direction per GPU (fallback figure)",
                          "unit": "GB/s", "frac": link_gbs / NVLINK_PEER_GBS, "traffic": None,
                          "bytes_per_launch": link_bytes, "avg_launch_us": max(disp_ms, comb_ms) * 1e3},
-            "nccl_baseline": {"step_us": nccl_ms * 1e3, "impl": "torch gather + NCCL all_to_all_single "
-                              "(sizes read on the host) + torch index_add fold"},
-            "cpu_baseline": None, "e2e": None, "clocks": clocks,
+            "nccl_baseline": nccl,
+            "cpu_baseline": None, "e2e": e2e, "clocks": clocks,
             "gpu_launches": 7 * args.steps, "impl": "ours",
         }
         print(json.dumps(line), flush=True)
@@ -772,7 +816,7 @@ def run_comm(args, wl, rank, world, local, dist):
     return 0
 
 
-def check_comm_step(cwl, inp, out, info, rank, world, dist, dev):
+def check_comm_step(cwl, inp, out, info, rank, world, dist, dev, cdev):
     """Self-check of the last warm-up step, from this rank's own inputs: the
     rows this rank received must number what every rank's routing sends it
     (count rows gathered from all ranks), and with the identity expert every
@@ -786,7 +830,7 @@ def check_comm_step(cwl, inp, out, info, rank, world, dist, dev):
     for j in range(k):
         m = dest[:, j] >= 0
         hit[np.nonzero(m)[0], dest[m, j]] = True
-    counts = torch.from_numpy(hit.sum(0).astype(np.int64)).to(dev)
+    counts = torch.from_numpy(hit.sum(0).astype(np.int64)).to(cdev)
     table = [torch.empty_like(counts) for _ in range(W)]
     dist.all_gather(table, counts)
     expect = int(sum(int(t[rank]) for t in table))

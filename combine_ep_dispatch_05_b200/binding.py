@@ -26,7 +26,8 @@ EP_DEVERR_EXPERT_RANGE, EP_DEVERR_TIMEOUT, EP_DEVERR_CAPACITY, EP_DEVERR_BOUNDS 
 EXPORTED = ("ep_cfg_check", "ep_plan_query", "ep_plan_create", "ep_plan_destroy", "ep_plan_info",
             "ep_dispatch", "ep_combine", "ep_plan_check_error", "ep_last_error", "ep_dispatch_noalloc",
             "ep_dispatch_scaled", "ep_comm_create", "ep_comm_handle", "ep_comm_connect", "ep_comm_info",
-            "ep_comm_dispatch", "ep_comm_combine", "ep_comm_check_error", "ep_comm_destroy")
+            "ep_comm_dispatch", "ep_comm_combine", "ep_comm_check_error", "ep_comm_destroy",
+            "ep_comm_barrier_selftest")
 EP_SYNC_DEVICE, EP_SYNC_HOST = 0, 1
 EP_ERR_PEER = -8
 EP_COMM_HANDLE_BYTES = 256
@@ -110,6 +111,7 @@ def _load() -> ctypes.CDLL:
         "ep_comm_combine": ([P, P, P, P], I32),
         "ep_comm_check_error": ([P], I32),
         "ep_comm_destroy": ([P], None),
+        "ep_comm_barrier_selftest": ([ctypes.c_int32] * 4 + [P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -273,6 +275,13 @@ def ep_comm_combine(comm: int, y, out, stream=None) -> int:
 
 def ep_comm_check_error(comm: int) -> int:
     return _check(_lib.ep_comm_check_error(comm), "ep_comm_check_error")
+
+
+def ep_comm_barrier_selftest(W: int, rounds: int, absent_rank: int = -1, absent_from: int = 0):
+    """Returns (barriers completed, error words, early reads), a list of W each."""
+    arr = [(ctypes.c_int32 * W)() for _ in range(3)]
+    _check(_lib.ep_comm_barrier_selftest(W, rounds, absent_rank, absent_from, *arr), "ep_comm_barrier_selftest")
+    return tuple(list(a) for a in arr)
 
 
 def ep_comm_destroy(comm: int) -> None:

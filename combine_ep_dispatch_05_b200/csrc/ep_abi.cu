@@ -55,7 +55,6 @@ struct EpPlan {
     unsigned* ll_epoch;
     unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
     int boundsRows;         // bounds-checking build: rows of each destination's buffers it checks against
-    int prefetchBlocks;     // route_count's L2 prefetch blocks (EP_ROUTE_PREFETCH_BLOCKS, 0: none)
     int fanoutSwitch;       // x100, see ScatterParams
     bool dispatched;
 };
@@ -499,7 +498,6 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         // Test hook of the bounds-checking build: check the receive buffers
         // against fewer rows than they have, so that the checks must fire.
         plan->boundsRows = std::min(env_int("EP_TEST_BOUNDS_ROWS", plan->info.maxRecv), plan->info.maxRecv);
-        plan->prefetchBlocks = env_int("EP_ROUTE_PREFETCH_BLOCKS", sms, 0);
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
         plan->dense = !fused && dense;
@@ -712,12 +710,6 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
             plan->dispatched = true;
             return EP_OK;
         }
-        rp.x = static_cast<const uint8_t*>(x);
-        rp.rowBytes = plan->info.rowBytes;
-        rp.prefetchBlocks = plan->prefetchBlocks;
-        rp.prefetchTokens = ep::prefetch_tokens(plan->G, plan->info.rowBytes,
-                                                (long long)plan->info.scatterBlocks * plan->info.scatterWarps,
-                                                plan->info.scatterStages);
         e = ep::launch_route_count(rp, plan->dense, s);
         if (e != cudaSuccess) return cuda_fail(e, "launch route_count");
         sp.baseShift = 8;  // route_count's 256-token tiles

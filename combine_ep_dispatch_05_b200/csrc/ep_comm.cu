@@ -365,11 +365,6 @@ int ep_comm_dispatch(EpComm* c, const void* x, const int32_t* topk_idx, const fl
         rp.maxRecv = c->maxRecv;
         rp.useWeights = c->cfg.useWeights;
         rp.lastScan = 1;
-        rp.x = static_cast<const uint8_t*>(x);
-        rp.rowBytes = c->rowBytes;
-        rp.prefetchBlocks = c->geo.numSMs;
-        rp.prefetchTokens =
-            ep::prefetch_tokens(c->T, c->rowBytes, (long long)c->geo.blocks * c->geo.warps, c->geo.stages);
         cudaError_t e = ep::launch_route_count(rp, c->dense, s);
         if (e != cudaSuccess) return cuda_err(e, "launch route_count");
 
@@ -496,5 +491,56 @@ int ep_comm_check_error(EpComm* c) {
 }
 
 void ep_comm_destroy(EpComm* c) { free_comm(c); }
+
+int ep_comm_barrier_selftest(int32_t W, int32_t rounds, int32_t absentRank, int32_t absentFrom,
+                             int32_t* roundsDone, int32_t* errors, int32_t* violations) {
+    try {
+        if (W < 1 || W > ep::kMaxWorld) return err(EP_ERR_INVALID, "W outside 1..32");
+        if (rounds < 1 || rounds > 100000) return err(EP_ERR_INVALID, "rounds outside 1..100000");
+        const size_t flagsOff = up256(sizeof(ep::PeerTable));
+        const size_t epochsOff = flagsOff + up256(sizeof(unsigned) * W * W);
+        const size_t errsOff = epochsOff + up256(sizeof(unsigned) * W);
+        const size_t dataOff = errsOff + up256(sizeof(int32_t) * W);
+        const size_t doneOff = dataOff + up256(sizeof(int32_t) * (size_t)W * rounds);
+        const size_t violOff = doneOff + up256(sizeof(int32_t) * W);
+        const size_t total = violOff + up256(sizeof(int32_t) * W);
+        unsigned char* mem = nullptr;
+        cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&mem), total);
+        if (e != cudaSuccess) return cuda_err(e, "cudaMalloc");
+        ep::PeerTable t;
+        std::memset(&t, 0, sizeof t);
+        for (int r = 0; r < W; ++r) t.flags[r] = reinterpret_cast<unsigned*>(mem + flagsOff) + (size_t)r * W;
+        ep::BarrierTestParams p{};
+        p.peers = reinterpret_cast<ep::PeerTable*>(mem);
+        p.epochs = reinterpret_cast<unsigned*>(mem + epochsOff);
+        p.errs = reinterpret_cast<int32_t*>(mem + errsOff);
+        p.data = reinterpret_cast<int32_t*>(mem + dataOff);
+        p.rounds_done = reinterpret_cast<int32_t*>(mem + doneOff);
+        p.violations = reinterpret_cast<int32_t*>(mem + violOff);
+        p.W = W;
+        p.rounds = rounds;
+        p.absent = absentRank;
+        p.absentFrom = absentFrom;
+        int32_t out[3][ep::kMaxWorld];
+        if ((e = cudaMemset(mem, 0, total)) != cudaSuccess ||
+            (e = cudaMemcpy(mem, &t, sizeof t, cudaMemcpyHostToDevice)) != cudaSuccess ||
+            (e = ep::launch_comm_barrier_test(p, nullptr)) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess ||
+            (e = cudaMemcpy(out[0], p.rounds_done, sizeof(int32_t) * W, cudaMemcpyDeviceToHost)) != cudaSuccess ||
+            (e = cudaMemcpy(out[1], p.errs, sizeof(int32_t) * W, cudaMemcpyDeviceToHost)) != cudaSuccess ||
+            (e = cudaMemcpy(out[2], p.violations, sizeof(int32_t) * W, cudaMemcpyDeviceToHost)) != cudaSuccess) {
+            cudaFree(mem);
+            return cuda_err(e, "barrier self-test");
+        }
+        cudaFree(mem);
+        for (int r = 0; r < W; ++r) {
+            if (roundsDone) roundsDone[r] = out[0][r];
+            if (errors) errors[r] = out[1][r];
+            if (violations) violations[r] = out[2][r];
+        }
+        return EP_OK;
+    } catch (...) {
+        return err(EP_ERR_INVALID, "unexpected exception");
+    }
+}
 
 }  // extern "C"

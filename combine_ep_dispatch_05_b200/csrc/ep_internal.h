@@ -63,25 +63,7 @@ struct RouteParams {
     int32_t* err;           // device error word
     int G, W, k, nEpr, E, numTiles, maxRecv, useWeights;
     int lastScan;           // 1: the last block scans the tile counts; 0: the scatter does
-    // Blocks numTiles.. of the launch only prefetch into L2 the rows of the
-    // present tokens g < prefetchTokens, which the scatter's copy engines load
-    // first, so that those reads overlap the routing instead of following it.
-    const uint8_t* x;       // [G][rowBytes]
-    long long rowBytes;
-    int prefetchTokens;
-    int prefetchBlocks;
 };
-
-// Tokens whose rows route_count's prefetch blocks bring into L2 for a
-// scatter of `engines` copy engines with `stages` stages each: the first
-// stages - 1 rounds of the hand-out (workers are numbered so that round i is
-// the tokens i * engines .. (i + 1) * engines - 1), or every token when the
-// whole batch takes at most 32 MB.
-inline int prefetch_tokens(long long G, long long rowBytes, long long engines, int stages) {
-    const long long early = engines * (long long)(stages > 1 ? stages - 1 : 1);
-    if (G * rowBytes <= (32LL << 20) || early >= G) return (int)G;
-    return (int)early;
-}
 
 struct ScatterParams {
     const uint8_t* x;          // [G][rowBytes]
@@ -255,6 +237,19 @@ cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, 
 
 // Ranks in separate processes: the count exchange / barrier, and the push.
 cudaError_t launch_comm_sync(const SyncParams& p, cudaStream_t s);
+
+// The barrier of EP_SYNC_DEVICE with W ranks emulated by the W blocks of one
+// cooperative launch on this GPU (ep_comm_barrier_selftest).
+struct BarrierTestParams {
+    PeerTable* peers;      // flags[r] = rank r's flags [W]
+    unsigned* epochs;      // [W] each emulated rank's epoch
+    int32_t* errs;         // [W] each rank's error word
+    int32_t* data;         // [W][rounds] what each rank wrote before each barrier
+    int32_t* rounds_done;  // [W] barriers each rank completed
+    int32_t* violations;   // [W] values a rank read after a barrier that were not yet written
+    int W, rounds, absent, absentFrom;
+};
+cudaError_t launch_comm_barrier_test(const BarrierTestParams& p, cudaStream_t s);
 cudaError_t launch_comm_push(const PushParams& p, int blocks, cudaStream_t s);
 
 // Shared-memory bytes the scatter kernel needs for a geometry.

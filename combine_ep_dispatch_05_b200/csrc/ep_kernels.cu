@@ -106,11 +106,6 @@ __device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t byt
                  : "memory");
 }
 
-// Bring [p, p + bytes) into L2 (nothing to wait for).
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -236,26 +231,6 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
 
     pdl_wait();     // the ids may come from the previous kernel of the stream
     pdl_trigger();  // let the scatter's launch and prologue overlap this kernel
-
-    if ((int)blockIdx.x >= p.numTiles) {
-        // A prefetch block: the rows of present early tokens, one token per
-        // thread (the blocks spread the prefetches over many SMs, whose
-        // copy units each issue them one after another).
-        for (int t = (blockIdx.x - p.numTiles) * kCountTile + threadIdx.x; t < p.prefetchTokens;
-             t += p.prefetchBlocks * kCountTile) {
-            bool present = false;
-            for (int j = 0; j < p.k; ++j) {
-                const int e = p.idx[(size_t)t * p.k + j];
-                present |= e >= 0 && e < p.E;
-            }
-            if (!present) continue;
-            const uint8_t* row = p.x + (size_t)t * p.rowBytes;
-            const long long n = p.rowBytes < (64 << 10) ? p.rowBytes : (64 << 10);
-            for (long long off = 0; off < n; off += 16384)
-                prefetch_l2(row + off, (uint32_t)(n - off < 16384 ? n - off : 16384));
-        }
-        return;
-    }
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = blockIdx.x * kCountTile + tid;
@@ -1565,6 +1540,35 @@ __device__ __forceinline__ bool comm_barrier(const SyncParams& p, int lane) {
     return ok;
 }
 
+// W ranks emulated by the W blocks of one cooperative launch (so that all of
+// them run at once): rank r writes its word of round i, passes the barrier,
+// then reads every rank's word of round i, which the barrier must have made
+// visible. Rank `absent` stops arriving from round absentFrom on; the others
+// must then give up (bounded wait) with EP_DEVERR_TIMEOUT.
+__global__ void __launch_bounds__(32) ep_comm_barrier_test_kernel(BarrierTestParams p) {
+    const int r = blockIdx.x, lane = threadIdx.x;
+    SyncParams sp{};
+    sp.peers = p.peers;
+    sp.epoch = p.epochs + r;
+    sp.err = p.errs + r;
+    sp.rank = r;
+    sp.W = p.W;
+    int done = 0, bad = 0;
+    for (int i = 0; i < p.rounds; ++i) {
+        if (r == p.absent && i >= p.absentFrom) break;
+        if (lane == 0) *reinterpret_cast<volatile int32_t*>(p.data + (size_t)r * p.rounds + i) = i + 1;
+        if (!comm_barrier(sp, lane)) break;
+        ++done;
+        if (lane < p.W && *reinterpret_cast<volatile int32_t*>(p.data + (size_t)lane * p.rounds + i) != i + 1)
+            ++bad;
+    }
+    for (int off = 16; off > 0; off >>= 1) bad += __shfl_xor_sync(kFull, bad, off);
+    if (lane == 0) {
+        p.rounds_done[r] = done;
+        p.violations[r] = bad;
+    }
+}
+
 __global__ void __launch_bounds__(32) ep_comm_sync_kernel(SyncParams p) {
     pdl_wait();  // the count row and the rows of the previous kernel are complete
     const int lane = threadIdx.x;
@@ -1660,7 +1664,7 @@ cudaError_t launch_pdl(void (*kernel)(P), int grid, int block, size_t smem, cuda
 namespace {
 template <bool kDense>
 cudaError_t launch_route_count_as(const RouteParams& p, cudaStream_t s) {
-    auto go = [&](auto kernel) { return launch_pdl(kernel, p.numTiles + p.prefetchBlocks, kCountTile, 0, s, p); };
+    auto go = [&](auto kernel) { return launch_pdl(kernel, p.numTiles, kCountTile, 0, s, p); };
     if (p.W <= 8)
         return p.k <= 8    ? go(ep_route_count_kernel<8, 8, kDense>)
                : p.k <= 16 ? go(ep_route_count_kernel<8, 16, kDense>)
@@ -1850,6 +1854,20 @@ cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, 
 cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s) {
     const cudaError_t e = fp32 ? launch_pdl(combine_kernel<CombineF32>, blocks, warps * 32, 0, s, p)
                                : launch_pdl(combine_kernel<CombineBf16>, blocks, warps * 32, 0, s, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_comm_barrier_test(const BarrierTestParams& p, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.W);
+    cfg.blockDim = dim3(32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, ep_comm_barrier_test_kernel, p);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

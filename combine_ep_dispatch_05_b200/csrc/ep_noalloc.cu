@@ -172,10 +172,6 @@ extern "C" int ep_dispatch_noalloc(const EpCfg* cfg, const void* x, const int32_
         rp.numTiles = info.numTiles;
         rp.maxRecv = info.maxRecv;
         rp.useWeights = cfg->useWeights;
-        rp.x = static_cast<const uint8_t*>(x);
-        rp.rowBytes = info.rowBytes;
-        rp.prefetchBlocks = ds.numSMs;
-        rp.prefetchTokens = ep::prefetch_tokens(G, info.rowBytes, (long long)ds.numSMs * perSm * warps, stages);
         if ((e = ep::launch_route_count(rp, false, s)) != cudaSuccess)
             return noalloc_fail(EP_ERR_CUDA, "launch route_count: %s", cudaGetErrorString(e));
 

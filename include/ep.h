@@ -159,9 +159,7 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * default, 0 never), EP_SCATTER_SCAN ("route": route_count's last block scans
  * the tile counts even when the scatter could), EP_DISPATCH_DENSE (1 / 0: the
  * large-batch form of the split dispatch for every plan / for none; by default
- * plans of more than 16384 tokens, W*T, take it), EP_ROUTE_PREFETCH_BLOCKS
- * (route_count's extra blocks that prefetch the scatter's first rows into L2;
- * one per SM by default, 0 none). Test hooks:
+ * plans of more than 16384 tokens, W*T, take it). Test hooks:
  * EP_TEST_UNREACHABLE_BARRIER=1 makes the fused dispatch's grid barrier (with
  * EP_DISPATCH_FUSED=1), or the low-latency
  * dispatch's wait for the counts of earlier tiles, unreachable, so that the

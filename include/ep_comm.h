@@ -139,6 +139,19 @@ int ep_comm_check_error(EpComm* comm);
  * of any rank may still be running that uses this rank's memory. */
 void ep_comm_destroy(EpComm* comm);
 
+/* Self-test of the EP_SYNC_DEVICE barrier on the current GPU, without other
+ * GPUs: W ranks (1..32) are the W blocks of one cooperative launch (so they
+ * all run at once), each with its own flags, epoch and error word, meeting
+ * `rounds` times. Before each barrier a rank writes a word; after it, it
+ * reads every rank's word of that round, which must be there. Rank
+ * `absentRank` (-1: none) stops arriving from round `absentFrom`; the others
+ * then give up after about a second with EP_DEVERR_TIMEOUT. Per rank, into
+ * host arrays of W (each may be NULL): barriers completed, error word, words
+ * read too early. Synchronous; allocates and frees its own device memory.
+ * Returns EP_OK or a negative code. */
+int ep_comm_barrier_selftest(int32_t W, int32_t rounds, int32_t absentRank, int32_t absentFrom,
+                             int32_t* roundsDone, int32_t* errors, int32_t* violations);
+
 #ifdef __cplusplus
 }
 #endif

@@ -150,3 +150,24 @@ def test_connect_refuses_mismatched_records():
     finally:
         ep.ep_comm_destroy(a)
         ep.ep_comm_destroy(b)
+
+
+@pytest.mark.parametrize("W", [2, 3, 8, 32])
+def test_device_barrier_protocol_with_emulated_ranks(W):
+    """The EP_SYNC_DEVICE barrier among W ranks, emulated by the W blocks of
+    one cooperative launch on this GPU: every round completes on every rank,
+    and what each rank wrote before a barrier is visible to all after it."""
+    done, errs, early = ep.ep_comm_barrier_selftest(W, 200)
+    assert done == [200] * W and errs == [0] * W and early == [0] * W
+
+
+def test_device_barrier_gives_up_when_a_rank_stops_arriving():
+    """Rank 1 stops at round 3: the others complete 3 rounds, then their wait
+    gives up (about a second) with EP_DEVERR_TIMEOUT; no rank hangs."""
+    done, errs, early = ep.ep_comm_barrier_selftest(4, 10, 1, 3)
+    assert done == [3, 3, 3, 3] and early == [0] * 4
+    assert errs[1] == 0 and all(errs[r] & ep.EP_DEVERR_TIMEOUT for r in (0, 2, 3))
+    from gpu_harness import run_and_compare  # the device keeps working
+    from synth.inputs import make_inputs
+    run, _ = run_and_compare(workload("tiny").cfg(), make_inputs(workload("tiny")))
+    run.close()
