@@ -342,22 +342,29 @@ __global__ void __launch_bounds__(kCountTile) ep_route_count_kernel(RouteParams 
 // Returns the call's present tokens; *rows = the rows of all destinations.
 // Returns -1 (after setting EP_DEVERR_TIMEOUT) when the copy of the counts
 // did not arrive within the bounded wait.
-__device__ int scan_tile_bases(const ScatterParams& p, int* s_base, int* rows) {
-    __shared__ int s_tot[kMaxWorld + 1];
-    __shared__ __align__(8) uint64_t s_bar;
-    const int C = p.W + 1, n = p.numTiles * C;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    // One bulk copy brings the whole table (rounded up to 16 bytes: the
-    // table's region is padded to 256) into shared memory.
-    const uint32_t bar = smem_addr(&s_bar);
+// The scan is split in two so that the copy engines can issue their first
+// row loads while the table is on its way: scan_tile_bases_begin (thread 0
+// issues one bulk copy of the whole table, rounded up to 16 bytes: the
+// table's region is padded to 256) and scan_tile_bases_end (every thread).
+__shared__ __align__(8) uint64_t s_scan_bar;
+
+__device__ __forceinline__ void scan_tile_bases_begin(const ScatterParams& p, int* s_base) {
     if (threadIdx.x == 0) {
+        const uint32_t bar = smem_addr(&s_scan_bar);
         mbar_init(bar, 1u);
         mbar_fence_init();
-        const uint32_t bytes = ((uint32_t)n * 4u + 15u) & ~15u;
+        const uint32_t bytes = ((uint32_t)p.numTiles * (p.W + 1) * 4u + 15u) & ~15u;
         mbar_arrive_expect_tx(bar, bytes);
         bulk_load(smem_addr(s_base), p.tile_cnt, bytes, bar);
     }
-    __syncthreads();
+}
+
+__device__ int scan_tile_bases_end(const ScatterParams& p, int* s_base, int* rows) {
+    __shared__ int s_tot[kMaxWorld + 1];
+    const int C = p.W + 1;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const uint32_t bar = smem_addr(&s_scan_bar);
+    __syncthreads();  // the barrier is initialised
     if (!__syncthreads_and(mbar_wait_bounded(bar, 0u))) {
         if (threadIdx.x == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
         return -1;
@@ -387,6 +394,11 @@ __device__ int scan_tile_bases(const ScatterParams& p, int* s_base, int* rows) {
     for (int pe = 0; pe < p.W; ++pe) r += s_tot[pe];
     *rows = r;
     return s_tot[p.W];
+}
+
+__device__ int scan_tile_bases(const ScatterParams& p, int* s_base, int* rows) {
+    scan_tile_bases_begin(p, s_base);
+    return scan_tile_bases_end(p, s_base, rows);
 }
 
 // =====================================================================
@@ -798,8 +810,12 @@ struct PlistFeed {
 // row piece by row piece through an S-stage shared-memory ring, S - kPend
 // loads ahead, with kPend items' bulk stores left draining when a stage is
 // refilled.
-template <int kPend, class Feed>
-__device__ __forceinline__ void copy_engine(const ScatterParams& p, const EngineSmem& es, int lane, Feed& feed) {
+// `ready` runs once every warp of the block has issued its first loads and
+// before any store (every thread of the block calls it, so it may hold a
+// block-wide barrier); false: copy nothing, only drain the loads.
+template <int kPend, class Feed, class Ready>
+__device__ __forceinline__ void copy_engine(const ScatterParams& p, const EngineSmem& es, int lane, Feed& feed,
+                                            Ready&& ready) {
     const int S = p.stages;  // > kPend (checked on the host)
     const uint32_t stage0_addr = es.stage0_addr, bar0 = es.bar0;
     int* item_tok = es.item_tok;
@@ -835,6 +851,10 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
 
     const int lookahead = S - kPend;
     for (int i = 0; i < lookahead && pg < p.G; ++i) issue();
+    if (!ready()) {
+        ok = false;
+        pg = p.G;
+    }
 
     // Per-token state kept across the chunks of one token.
     TokenInputs pre;
@@ -843,7 +863,7 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
     uint32_t cur_mask = 0;
     int my_slot = -1;  // lane pe: slot of the current token at pe
 
-    while (consumed < issued) {
+    while (ok && consumed < issued) {
         const int s = consumed % S;
         const uint32_t parity = (uint32_t)(consumed / S) & 1u;
         __syncwarp();
@@ -914,11 +934,11 @@ __device__ __forceinline__ void run_split_engine(const ScatterParams& p, const E
     if (src.dyn) {
         DynFeed<kSmemBase> feed;
         feed.init(p, src, lane, s_base);
-        copy_engine<kPend>(p, es, lane, feed);
+        copy_engine<kPend>(p, es, lane, feed, [] { return true; });
     } else {
         StaticFeed<kSmemBase> feed;
         feed.init(p, src, lane, s_base);
-        copy_engine<kPend>(p, es, lane, feed);
+        copy_engine<kPend>(p, es, lane, feed, [] { return true; });
     }
 }
 
@@ -955,13 +975,27 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
         DynFeed<false> feed;
         feed.init(p, make_source(warp * gridDim.x + blockIdx.x, gridDim.x * engines, p.G, p.work, p.G), lane,
                   nullptr);
-        copy_engine<kPend>(p, es, lane, feed);
+        copy_engine<kPend>(p, es, lane, feed, [] { return true; });
         return;
     }
     int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem + p.baseOffset) : nullptr;
     const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, nwarps, lane);
     pdl_wait();     // routing written by route_count is visible from here on
     if (!dest_setup(p)) return;
+    const int nAll = gridDim.x * nwarps;
+    if (s_base != nullptr && p.G < 8 * nAll) {
+        // Fewer than 8 tokens per engine: the hand-out is static whatever the
+        // counts say, so every engine starts at once (all of them: the
+        // fan-out switch would need the counts) and issues its first row
+        // loads while the tile counts are still on their way; the scan
+        // completes before the first store.
+        scan_tile_bases_begin(p, s_base);
+        StaticFeed<true> feed;
+        feed.init(p, make_source(warp * gridDim.x + blockIdx.x, nAll, p.G, p.work, 0), lane, s_base);
+        int rows;
+        copy_engine<kPend>(p, es, lane, feed, [&] { return scan_tile_bases_end(p, s_base, &rows) >= 0; });
+        return;
+    }
     int P, rows = -1;
     if (s_base != nullptr) {
         P = scan_tile_bases(p, s_base, &rows);
@@ -1196,7 +1230,7 @@ __global__ void __launch_bounds__(kLlThreads, 1) ep_dispatch_ll_kernel(ScatterPa
     feed.i = warp;
     feed.step = engines;
     feed.tag = tag;
-    copy_engine<1>(p, es, lane, feed);
+    copy_engine<1>(p, es, lane, feed, [] { return true; });
 }
 
 // =====================================================================
@@ -1747,12 +1781,15 @@ cudaError_t scatter_blocks_per_sm(int warps, size_t smem, int* out) {
 }
 
 namespace {
-// The combine instance: 2 columns x 8 rows of 16-byte loads in flight per
-// lane, 2 blocks of 256 threads per SM (B200: tiles of 2 x 4 at 4 or 3 blocks
-// per SM and 1 x 8 at 4 measured slower at the main workload and within 2% on
-// skewed routing).
+// The combine instance: 4 columns x 4 rows of 16-byte loads in flight per
+// lane, 2 blocks of 256 threads per SM. A token's rows go in batches of 4, so
+// a token with few destinations still keeps 16 loads in flight per lane.
+// B200, against 2 columns x 8 rows: the 512-token workload (3.4 rows a token)
+// 20.5 vs 24.8 us, skewed routing (2.7) 287 vs 304 us, main (5.3) 453.9 vs
+// 453.7 us; 3 x 6 took 476 us at main; 2 x 4 at 4 or 3 blocks per SM and
+// 1 x 8 at 4 were slower at main as well.
 template <class Elem>
-constexpr auto combine_kernel = ep_combine_kernel<Elem, 2, 8, 2>;
+constexpr auto combine_kernel = ep_combine_kernel<Elem, 4, 4, 2>;
 }  // namespace
 
 cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out) {

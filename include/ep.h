@@ -231,7 +231,8 @@ int ep_dispatch_scaled(EpPlan* plan, const void* x, const int32_t* topk_idx, con
  *                          aligned; only rows < recv_count are read
  *   out  [W][T][hc]        16-byte aligned; every row is written
  * Both are float32 for an EP_FP32 plan and bfloat16 otherwise; hc =
- * combineHidden of ep_plan_info (2*h for EP_FP4X2, else h).
+ * combineHidden of ep_plan_info (2*h for EP_FP4X2, else h). A NaN in y gives
+ * a NaN out element; its sign and payload bits are not specified.
  * Returns EP_OK, EP_ERR_STATE before any dispatch, or a negative code.
  */
 int ep_combine(EpPlan* plan, const void* y, void* out, void* stream);
