@@ -298,6 +298,8 @@ def run_reference(args, wl):
     rank, world, local, dist = dist_setup(args.gpus)
     if rank != 0:
         return 0
+    if world > 1:  # the arm's config: the same workload with its W ranks on the N GPUs
+        wl = comm_workload(wl, world)
     inputs = make_inputs(wl)
     cpu = cpu_baseline(wl, inputs, args.steps, args.warmup)
     us = cpu["value"]

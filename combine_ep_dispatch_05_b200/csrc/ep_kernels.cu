@@ -703,9 +703,22 @@ struct StaticFeed {
     uint32_t mnext;  // this lane's mask in the next 32 rounds
     const int* s_base;
 
+    // Whether the token of round i is present, from its ids (an id in
+    // [0, E)): the ids are an input of the call, so this needs nothing from
+    // route_count and may run before the scatter waits for it.
     __device__ __forceinline__ uint32_t round_mask(const ScatterParams& p, int i) const {
         const long long t = src.w + (long long)i * src.nU;
-        return (i < src.R && t < p.G) ? __ldcg(p.tok_mask + t) : 0u;
+        if (i >= src.R || t >= p.G) return 0u;
+        const int32_t* ids = p.idx + (size_t)t * p.k;
+        bool any = false;
+        for (int j0 = 0; j0 < p.k; j0 += 8) {
+            int e[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) e[j] = j0 + j < p.k ? ids[j0 + j] : -1;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) any |= e[j] >= 0 && e[j] < p.E;
+        }
+        return any ? 1u : 0u;
     }
     __device__ __forceinline__ void init(const ScatterParams& p, const TokenSource& s0, int lane,
                                          const int* bases) {
@@ -980,22 +993,29 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     }
     int* s_base = p.baseSmemBytes > 0 ? reinterpret_cast<int*>(smem + p.baseOffset) : nullptr;
     const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, nwarps, lane);
-    pdl_wait();     // routing written by route_count is visible from here on
-    if (!dest_setup(p)) return;
     const int nAll = gridDim.x * nwarps;
     if (s_base != nullptr && p.G < 8 * nAll) {
         // Fewer than 8 tokens per engine: the hand-out is static whatever the
         // counts say, so every engine starts at once (all of them: the
-        // fan-out switch would need the counts) and issues its first row
-        // loads while the tile counts are still on their way; the scan
-        // completes before the first store.
-        scan_tile_bases_begin(p, s_base);
+        // fan-out switch would need the counts). It finds its tokens from
+        // their ids and issues their first row loads before waiting for
+        // route_count: x and the ids come from work that finished before
+        // route_count could start, and this kernel only launches once
+        // route_count has passed its own wait. The wait, the copy of the
+        // tile counts and their scan complete before the first store.
         StaticFeed<true> feed;
         feed.init(p, make_source(warp * gridDim.x + blockIdx.x, nAll, p.G, p.work, 0), lane, s_base);
         int rows;
-        copy_engine<kPend>(p, es, lane, feed, [&] { return scan_tile_bases_end(p, s_base, &rows) >= 0; });
+        copy_engine<kPend>(p, es, lane, feed, [&] {
+            pdl_wait();  // routing written by route_count is visible from here on
+            if (!dest_setup(p)) return false;
+            scan_tile_bases_begin(p, s_base);
+            return scan_tile_bases_end(p, s_base, &rows) >= 0;
+        });
         return;
     }
+    pdl_wait();     // routing written by route_count is visible from here on
+    if (!dest_setup(p)) return;
     int P, rows = -1;
     if (s_base != nullptr) {
         P = scan_tile_bases(p, s_base, &rows);

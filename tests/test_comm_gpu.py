@@ -171,3 +171,42 @@ def test_device_barrier_gives_up_when_a_rank_stops_arriving():
     from synth.inputs import make_inputs
     run, _ = run_and_compare(workload("tiny").cfg(), make_inputs(workload("tiny")))
     run.close()
+
+
+def test_device_sync_calls_replay_in_a_cuda_graph():
+    """EP_SYNC_DEVICE calls do no host synchronisation, so they can be
+    captured: a graph of dispatch + combine, replayed three times, gives the
+    eager results each time (the barrier epoch advances on the device)."""
+    wl = workload("pr599").replace(W=1, n_epr=32, max_recv=0, h=1024)
+    comm = _single_rank_comm(wl)
+    try:
+        from gpu_harness import as_bytes, to_dev
+        from synth.inputs import make_inputs
+        inputs = make_inputs(wl)
+        info = ep.ep_comm_info(comm)
+        x = to_dev(as_bytes(inputs["x"][0]))
+        idx = to_dev(inputs["topk_idx"][0])
+        w = to_dev(inputs["topk_w"][0])
+        recv_x = comm_harness.device_tensor(info.recvX, (info.maxRecv, info.rowBytes), "|u1")
+        y = recv_x.view(torch.bfloat16).view(info.maxRecv, -1)
+        out = torch.empty((wl.max_tok, wl.h), dtype=torch.bfloat16, device="cuda")
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            ep.ep_comm_dispatch(comm, x, idx, w, s)
+            ep.ep_comm_combine(comm, y, out, s)
+        s.synchronize()
+        eager = out.clone()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                ep.ep_comm_dispatch(comm, x, idx, w, s)
+                ep.ep_comm_combine(comm, y, out, s)
+        for _ in range(3):
+            out.fill_(0)
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(out, eager)
+        assert ep.ep_comm_check_error(comm) == 0
+        del g
+    finally:
+        ep.ep_comm_destroy(comm)
