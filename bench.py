@@ -37,9 +37,12 @@ from synth.inputs import make_inputs, workload  # noqa: E402
 METRIC = "dispatch+combine µs and HBM GB/s (% of B200 peak) at W=8 ct=4096 h=7168 topk8"
 FALLBACK_HBM_GBS = 6650.0
 FLUSH_BYTES = 256 << 20
+# The device code whose DRAM traffic profiles/ncu_traffic.json records; the
+# launch geometry it was taken with is recorded beside it.
 KERNEL_SOURCES = ["combine_ep_dispatch_05_b200/csrc/ep_kernels.cu",
-                  "combine_ep_dispatch_05_b200/csrc/ep_abi.cu",
                   "combine_ep_dispatch_05_b200/csrc/ep_internal.h"]
+TRAFFIC_GEOMETRY = ("scatterWarps", "scatterStages", "scatterChunkBytes", "scatterBlocks", "combineWarps",
+                    "combineBlocks")
 
 
 def parse():
@@ -137,15 +140,18 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, wl_name: str):
+def ncu_traffic(kernel: str, wl_name: str, geometry: dict):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    the current kernel code with the launch geometry this run has; else None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
         e = d[kernel]
         if e.get("source_sha") != source_hash():
+            return None
+        rec = d["geometry"][wl_name]
+        if any(rec[k] != geometry.get(k) for k in TRAFFIC_GEOMETRY):
             return None
         return e["per_launch_bytes"].get(wl_name)
     except Exception:
@@ -376,7 +382,9 @@ def time_graphs(calls: dict, dev, dist) -> dict:
 def run_ours(args, wl):
     import torch
     rank, world, local, dist = dist_setup(args.gpus)
-    if world > 1:
+    # EP_BENCH_COMM=1 (under torchrun) runs the communicator path with one rank
+    # as well: the device-barrier path of a multi-GPU run, on one GPU.
+    if world > 1 or (dist is not None and os.environ.get("EP_BENCH_COMM") == "1"):
         return run_comm(args, wl, rank, world, local, dist)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -488,7 +496,8 @@ def run_ours(args, wl):
         dom = {"kernel": "ep_combine_kernel", "bytes": cb, "ms": comb_ms_max, "gbs": c_gbs}
     else:
         dom = {"kernel": dispatch_kernels(info), "bytes": db, "ms": disp_ms_max, "gbs": d_gbs}
-    traffic = ncu_traffic("ep_combine_kernel" if dom["kernel"] == "ep_combine_kernel" else "ep_dispatch", wl.name)
+    traffic = ncu_traffic("ep_combine_kernel" if dom["kernel"] == "ep_combine_kernel" else "ep_dispatch", wl.name,
+                          info.as_dict())
 
     # End to end: every step copies its inputs from pinned host memory to the
     # device, runs dispatch and combine, and copies its result back to pinned

@@ -160,11 +160,16 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
     g.chunkBytes = chunk;
     g.chunkStride = (chunk + 127) & ~127;
     g.numChunks = (int)((rowBytes + chunk - 1) / chunk);
-    const int budget = 215 * 1024;
-    // Rows of 8 KB and more: a third engine, which sits out at a high fan-out
-    // (see copy_engine). Smaller rows already give several blocks per SM.
+    // Rows of 8 KB and more: one block per SM of about 215 KB, with a third
+    // engine that sits out at a high fan-out (see copy_engine). Smaller rows:
+    // two engines per block and two blocks per SM, each within about 110 KB
+    // (an SM has 228 KB, and each block also holds its static shared memory
+    // and 1 KB the system keeps). B200, fp8 rows of 7 KB at the main workload:
+    // 8 stages left one block per SM once the static shared memory grew
+    // (419 us), 7 stages keep two (245 us).
     int warps = g.chunkStride >= 8192 ? 3 : 2;
-    int stages = budget / (warps * g.chunkStride);
+    const int budget = 215 * 1024;
+    int stages = (warps == 3 ? budget : 110 * 1024) / (warps * g.chunkStride);
     if (stages < 4) {
         warps = 2;
         stages = budget / (warps * g.chunkStride);
@@ -310,9 +315,11 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info) {
         const Geometry geo = pick_geometry(cfg, false);
         fill_info(cfg, geo, info);
         const int sms = 148;  // B200
-        info->scatterBlocks = sms * std::max(1, (200 * 1024) / (int)ep::scatter_smem_bytes(
-                                                                   geo.scatterWarps, std::max(geo.scatterStages, 1),
-                                                                   geo.chunkStride));
+        // Blocks per SM: the SM's 228 KB over the block's shared memory, its
+        // static shared memory and the 1 KB the system keeps per block.
+        const size_t perBlock = ep::scatter_smem_bytes(geo.scatterWarps, std::max(geo.scatterStages, 1),
+                                                       geo.chunkStride) + ep::kStaticSmemReserve + 1024;
+        info->scatterBlocks = sms * std::max(1, (int)((228 * 1024) / perBlock));
         info->combineBlocks = sms * 2;
         size_t llSmem = 0;
         int llTile = 0;

@@ -32,21 +32,25 @@ def test_source_hash_ignores_comments_and_whitespace(src_copy):
 
 def test_source_hash_sees_code_changes(src_copy):
     base = bench.source_hash()
-    p = src_copy / bench.KERNEL_SOURCES[2]
+    p = src_copy / bench.KERNEL_SOURCES[1]
     p.write_text(p.read_text() + "\nconstexpr int kAnotherConstant = 1;\n")
     assert bench.source_hash() != base
 
 
 def test_traffic_record_is_keyed_by_the_source_hash(src_copy):
-    """The recorded traffic applies to the code it was captured on and to
-    nothing else: any code edit makes bench report it as unknown."""
-    rec = bench.ncu_traffic("ep_dispatch", "main")
+    """The recorded traffic applies to the code and the launch geometry it was
+    captured with and to nothing else: a code edit or another geometry makes
+    bench report it as unknown."""
+    import json
+    geo = json.load(open(src_copy / "profiles" / "ncu_traffic.json"))["geometry"]["main"]
+    rec = bench.ncu_traffic("ep_dispatch", "main", dict(geo))
     if rec is None:
         pytest.skip("the traffic record predates the current kernel code (profile again)")
     assert rec > 2.5e9
-    p = src_copy / bench.KERNEL_SOURCES[1]
+    assert bench.ncu_traffic("ep_dispatch", "main", dict(geo, scatterStages=geo["scatterStages"] + 1)) is None
+    p = src_copy / bench.KERNEL_SOURCES[0]
     p.write_text(p.read_text() + "\nstatic int edited_code = 0;\n")
-    assert bench.ncu_traffic("ep_dispatch", "main") is None
+    assert bench.ncu_traffic("ep_dispatch", "main", dict(geo)) is None
 
 
 def test_algorithmic_bytes_of_the_main_workload():
