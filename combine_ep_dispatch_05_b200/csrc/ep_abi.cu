@@ -53,6 +53,14 @@ struct EpPlan {
     int32_t* ll_ticket;
     unsigned* ll_done;
     unsigned* ll_epoch;
+    bool local;           // small-batch single launch with per-block routing (dispatch_local)
+    size_t localSmem;     // its dynamic shared memory: routing area, then the copy engines
+    size_t localEngineOffset;
+    int localOwn;         // the most tokens one of its blocks owns
+    int localBlocks;      // its grid
+    unsigned long long* local_agg;  // its scratch: the blocks' published totals, call epoch, blocks done
+    unsigned* local_epoch;
+    unsigned* local_done;
     unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
     int boundsRows;         // bounds-checking build: rows of each destination's buffers it checks against
     int fanoutSwitch;       // x100, see ScatterParams
@@ -198,6 +206,9 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
 // hides (ct = 1 workload: 19.5 vs 17.4 us; the 512-token workload: 32.9 vs
 // 33.8 us), since its own handoffs cost as many dependent memory round trips.
 constexpr int kLlDefaultMaxTokens = 0;
+
+// Largest batch (W * maxTokPerRank tokens) that takes dispatch_local.
+constexpr int kLocalDefaultMaxTokens = 0;
 
 // Returns the stages per copy engine of the low-latency dispatch that fit
 // `smemOptin` (the shared memory in *smem, the tile in *tile), or 0 when the
@@ -494,7 +505,54 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
                 }
             }
         }
-        plan->info.dispatchLowLatency = plan->ll ? 1 : 0;
+        // Small batches: dispatch_local, one launch in which every block
+        // routes the batch itself, when each block owns at most kLocalMaxOwn
+        // tokens and the batch has at most EP_LOCAL_MAX_TOKENS tokens.
+        plan->local = false;
+        {
+            const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
+            const int localMax = env_int("EP_LOCAL_MAX_TOKENS", kLocalDefaultMaxTokens, 0);
+            int blocks = plan->info.scatterBlocks;
+            if (!fused && !plan->ll && G <= localMax && geo.scatterWarps <= ep::kLocalWarps) {
+                // The grid: the scatter's, at most one block a token, at most
+                // what fits the SMs at once (the routing area may cost a block
+                // per SM, which changes the tokens a block owns: try again).
+                const size_t limit = (size_t)smemOptin - ep::kStaticSmemReserve;
+                blocks = (int)std::min<long long>(blocks, G);
+                for (int attempt = 0; attempt < 3 && blocks >= 1; ++attempt) {
+                    const int own = (int)((G + blocks - 1) / blocks);
+                    if (own > ep::kLocalMaxOwn) break;
+                    const size_t area = ep::local_layout(own, cfg->worldSize, ep::kLocalWarps).total;
+                    int stages = geo.scatterStages;
+                    size_t lsm = area + ep::scatter_smem_bytes(geo.scatterWarps, stages, geo.chunkStride);
+                    while (lsm > limit && stages > 2)
+                        lsm = area + ep::scatter_smem_bytes(geo.scatterWarps, --stages, geo.chunkStride);
+                    if (lsm > limit) break;
+                    int per = 0;
+                    if ((e = ep::local_set_smem(cfg->worldSize, cfg->numExpertPerToken, lsm)) != cudaSuccess ||
+                        (e = ep::local_blocks_per_sm(cfg->worldSize, cfg->numExpertPerToken, lsm, &per)) !=
+                            cudaSuccess) {
+                        cuda_fail(e, "dispatch_local set-up");
+                        delete plan;
+                        return nullptr;
+                    }
+                    if (per < 1) break;
+                    if (blocks > sms * per) {
+                        blocks = sms * per;
+                        continue;
+                    }
+                    plan->local = true;
+                    plan->localSmem = lsm;
+                    plan->localEngineOffset = area;
+                    plan->localOwn = own;
+                    plan->localBlocks = blocks;
+                    plan->info.scatterBlocks = blocks;
+                    plan->info.scatterStages = stages;
+                    break;
+                }
+            }
+        }
+        plan->info.dispatchLowLatency = (plan->ll || plan->local) ? 1 : 0;
         plan->fanoutSwitch = env_int("EP_SCATTER_FANOUT_SWITCH", 375, 0);
         // Test hook for the failure path: the fused dispatch's grid barrier,
         // or the low-latency dispatch's wait for earlier tiles, can never
@@ -514,7 +572,8 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
         plan->maxRecv = plan->info.maxRecv;
 
-        const ep::ScratchLayout L = ep::scratch_layout(plan->G, cfg->worldSize, plan->info.numTiles, plan->ll);
+        const ep::ScratchLayout L = ep::scratch_layout(plan->G, cfg->worldSize, plan->info.numTiles, plan->ll,
+                                                       plan->local ? plan->localBlocks : 0);
         plan->info.scratchBytes = (long long)L.total;
         const size_t total = L.total;
         if ((e = cudaMalloc(&plan->scratch, total)) != cudaSuccess) {
@@ -550,6 +609,9 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->ll_ticket = reinterpret_cast<int32_t*>(base + L.ll_ticket);
         plan->ll_done = reinterpret_cast<unsigned*>(base + L.ll_done);
         plan->ll_epoch = reinterpret_cast<unsigned*>(base + L.ll_epoch);
+        plan->local_agg = reinterpret_cast<unsigned long long*>(base + L.local_agg);
+        plan->local_epoch = reinterpret_cast<unsigned*>(base + L.local_epoch);
+        plan->local_done = reinterpret_cast<unsigned*>(base + L.local_done);
         plan->dispatched = false;
         g_last_error[0] = '\0';
         return plan;
@@ -676,6 +738,24 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         sp.recv_scales = static_cast<uint32_t*>(recv_scales);
         sp.scaleWords = scaleWords;
         sp.boundsRows = plan->boundsRows;
+        if (plan->local) {
+            // One launch: every block routes the tokens up to its own, then copies its own.
+            const int nEpr = c.numExpertPerRank;
+            sp.w = c.useWeights ? topk_w : nullptr;
+            sp.useWeights = c.useWeights;
+            sp.nEprShift = (nEpr & (nEpr - 1)) == 0 ? __builtin_ctz((unsigned)nEpr) : -1;
+            sp.localOwn = plan->localOwn;
+            sp.localEngines = plan->info.scatterWarps;
+            sp.engineOffset = (int)plan->localEngineOffset;
+            sp.local_agg = plan->local_agg;
+            sp.local_epoch = plan->local_epoch;
+            sp.local_done = plan->local_done;
+            sp.barrierSlack = plan->barrierSlack;
+            e = ep::launch_dispatch_local(sp, plan->localBlocks, plan->localSmem, s);
+            if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_local");
+            plan->dispatched = true;
+            return EP_OK;
+        }
         if (plan->ll) {
             // One launch: every block routes and scans the batch, then copies its share.
             const int nEpr = c.numExpertPerRank;

@@ -24,6 +24,11 @@ constexpr int kMaxCombineWarps = 8;
 constexpr int kLlThreads = 512;
 constexpr int kLlWarps = kLlThreads / 32;
 constexpr int kLlMaxTiles = 256;
+// Warps of a dispatch_local block (its first warps are the copy engines), and
+// the most tokens one block may own (the plan takes dispatch_local only when
+// ceil(G / blocks) is at most this).
+constexpr int kLocalWarps = 8;
+constexpr int kLocalMaxOwn = 64;
 // Shared memory kept back from the dynamic budget for the kernels' static
 // shared memory.
 constexpr size_t kStaticSmemReserve = 2048;
@@ -122,7 +127,39 @@ struct ScatterParams {
     int32_t* ll_ticket;      // next tile to hand out (0 at the start of each call)
     unsigned* ll_done;       // blocks past the hand-out; the last one resets ticket and done
     unsigned* ll_epoch;      // calls so far (tags the status words of this call)
+    // Only dispatch_local uses these (and w, recv_count, useWeights, nEprShift,
+    // engineOffset, barrierSlack): the most tokens a block owns, its copy-engine
+    // warps, the blocks' published totals [blocks][ceil(W / 6)], the call epoch
+    // and the blocks past their look-back (the last one advances the epoch).
+    int localOwn;
+    int localEngines;
+    unsigned long long* local_agg;
+    unsigned* local_epoch;
+    unsigned* local_done;
 };
+
+// Byte offsets of dispatch_local's routing area in shared memory (each
+// 16-byte aligned): masks of the own chunks' tokens [chunks * 32], their own
+// tokens per destination, then bases [chunks][W], the own tokens' slots
+// [own][W], the present own tokens [own], and counters: [0] present own
+// tokens, [1] next one to hand out, [2 + pe] the block's total at pe. own: the
+// most tokens a block owns; its tokens span at most (own + 62) / 32 chunks.
+struct LocalLayout {
+    size_t cmask, ccnt, slot, list, ctr, total;
+};
+__host__ __device__ inline size_t local_up16(size_t n) { return (n + 15) & ~(size_t)15; }
+__host__ __device__ inline LocalLayout local_layout(int own, int W, int warps) {
+    (void)warps;
+    const size_t chunks = (size_t)(own + 62) / 32;
+    LocalLayout L;
+    L.cmask = 0;
+    L.ccnt = L.cmask + local_up16(chunks * 32 * 4);
+    L.slot = L.ccnt + local_up16(chunks * (size_t)W * 4);
+    L.list = L.slot + local_up16((size_t)own * W * 4);
+    L.ctr = L.list + local_up16((size_t)own * 4);
+    L.total = (L.ctr + (2 + kMaxWorld) * 4 + 127) & ~(size_t)127;
+    return L;
+}
 
 struct CombineParams {
     const uint8_t* y;      // [W][maxRecv][rowBytes]
@@ -175,12 +212,14 @@ struct PushParams {
 // barrier, fused blocks done, low-latency tile ticket, blocks done, call epoch
 // and present total, route_count's present-token total), error word.
 struct ScratchLayout {
-    size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base, ll_status, ll_agg, ll_plist;
-    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, ptotal, err, total;
+    size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base, ll_status, ll_agg, ll_plist, local_agg;
+    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, ptotal, local_epoch,
+        local_done, err, total;
 };
 
-// ll: the plan takes the single-launch dispatch (its regions are empty otherwise).
-inline ScratchLayout scratch_layout(long long G, int W, int numTiles, bool ll = false) {
+// ll: the plan takes the single-launch dispatch (its regions are empty
+// otherwise); localBlocks: the grid of dispatch_local (0: not taken).
+inline ScratchLayout scratch_layout(long long G, int W, int numTiles, bool ll = false, int localBlocks = 0) {
     auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
     const size_t numChunks32 = (size_t)((G + 31) / 32);
     ScratchLayout L;
@@ -194,7 +233,8 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles, bool ll = 
     L.ll_status = L.chunk_base + up(sizeof(int32_t) * numChunks32 * W);
     L.ll_agg = L.ll_status + up(sizeof(uint32_t) * llTiles);
     L.ll_plist = L.ll_agg + up(sizeof(int32_t) * llTiles * (W + 1));
-    L.ticket = L.ll_plist + (ll ? up(sizeof(int32_t) * (size_t)G * (W + 2)) : 0);
+    L.local_agg = L.ll_plist + (ll ? up(sizeof(int32_t) * (size_t)G * (W + 2)) : 0);
+    L.ticket = L.local_agg + up(sizeof(unsigned long long) * (size_t)localBlocks * ((W + 5) / 6));
     L.work = L.ticket + 4;
     L.cwork = L.ticket + 8;
     L.cdone = L.ticket + 12;
@@ -205,6 +245,8 @@ inline ScratchLayout scratch_layout(long long G, int W, int numTiles, bool ll = 
     L.ll_epoch = L.ticket + 32;
     L.ll_ptotal = L.ticket + 40;
     L.ptotal = L.ticket + 48;
+    L.local_epoch = L.ticket + 52;
+    L.local_done = L.ticket + 56;
     L.err = L.ticket + 256;
     L.total = L.err + 256;
     return L;
@@ -234,6 +276,12 @@ size_t ll_smem_bytes(int tileTokens, int W, int warps, int stages, int chunkStri
 cudaError_t ll_set_smem(int W, int topk, size_t bytes);
 cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out);
 cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s);
+
+// Single-launch dispatch of small batches with per-block routing
+// (dispatch_local, kLocalWarps warps per block): opt-in, occupancy, launch.
+cudaError_t local_set_smem(int W, int topk, size_t bytes);
+cudaError_t local_blocks_per_sm(int W, int topk, size_t smem, int* out);
+cudaError_t launch_dispatch_local(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s);
 
 // Ranks in separate processes: the count exchange / barrier, and the push.
 cudaError_t launch_comm_sync(const SyncParams& p, cudaStream_t s);

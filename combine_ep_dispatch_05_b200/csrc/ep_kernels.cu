@@ -1254,6 +1254,286 @@ __global__ void __launch_bounds__(kLlThreads, 1) ep_dispatch_ll_kernel(ScatterPa
 }
 
 // =====================================================================
+// dispatch_local: the whole dispatch of a small batch in one launch. Block b
+// owns the tokens [lo, hi) of an even, contiguous split of the batch (every
+// block owns at least one), routes them and copies them itself:
+//   1. the chunks of 32 tokens holding own tokens: destination masks (shared
+//      memory) and, per chunk and destination, the own tokens that go there;
+//      the present own tokens form a list;
+//   2. the block publishes its totals per destination in words tagged with
+//      the call's epoch (decoupled look-back, as in single-pass prefix
+//      scans); the copy-engine warps issue the row loads of the first present
+//      own tokens;
+//   3. every thread adds up a share of the earlier blocks' words, each loaded
+//      once its tag shows this call (a bounded wait: blocks publish before
+//      they wait and wait only on lower-numbered ones, so the waits end), into
+//      the block's base at each destination; slots of the own tokens (base +
+//      rank among the own tokens going there; -1: not sent there, -2: beyond
+//      maxRecv); routing rows of the absent own tokens; the last block stores
+//      recv_count;
+//   4. the engines copy the present own tokens, handed out through a
+//      shared-memory counter: per token its routing row and meta records (and
+//      scale rows), then the row's bulk stores.
+// A block's word q holds its totals at destinations 6q .. 6q+5 (8 bits each:
+// a block owns at most kLocalMaxOwn < 256 tokens) under a 16-bit tag, so that
+// one 64-bit load brings a count and the proof that it is this call's. The
+// epoch advances once every block has read it (the last block to get past
+// its look-back), so replays of a captured graph stay in step.
+// Shared memory: the routing area (LocalLayout) at 0, the copy engines'
+// barriers and stages at engineOffset.
+// =====================================================================
+constexpr int kLocalPerWord = 6;
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Destination mask of token g from its ids (ids outside [0, E) are masked;
+// `bad` reports ids >= E). All k loads are issued before any is used.
+template <int kK>
+__device__ __forceinline__ uint32_t local_mask(const ScatterParams& p, int g, bool& bad) {
+    const int32_t* ids = p.idx + (size_t)g * p.k;
+    int e[kK];
+#pragma unroll
+    for (int j = 0; j < kK; ++j) e[j] = j < p.k ? ids[j] : -1;
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < kK; ++j) {
+        if (e[j] >= p.E) bad = true;
+        if (e[j] >= 0 && e[j] < p.E) m |= 1u << dest_pe(e[j], p.nEpr, p.nEprShift);
+    }
+    return m;
+}
+
+// The own tokens' feed: list entry i (a present own token) is handle i.
+struct LocalFeed {
+    const int* list;  // present own tokens, ascending
+    int* ctr;         // next entry to hand out (shared memory)
+    const int* slot;  // [own][W]: slot of own token g - lo at each destination
+    int n, lo;
+
+    __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
+        int i = 0;
+        if (lane == 0) i = atomicAdd(ctr, 1);
+        i = __shfl_sync(kFull, i, 0);
+        return i < n ? i : p.G;
+    }
+    __device__ __forceinline__ int row(const ScatterParams&, int h) const { return list[h]; }
+    __device__ __forceinline__ TokenInputs load(const ScatterParams& p, int h, int lane) const {
+        TokenInputs in;
+        in.h = h;
+        in.g = list[h];
+        in.rr = make_int2(lane < p.W ? slot[(in.g - lo) * p.W + lane] : -1, 0);
+        in.base = 0;
+        in.e = lane < p.k ? p.idx[(size_t)in.g * p.k + lane] : -1;
+        in.wt = (lane < p.k && p.w != nullptr) ? p.w[(size_t)in.g * p.k + lane] : 0.0f;
+        return in;
+    }
+    // Lane pe: the token's weight sum at pe (float32, topk order), its routing
+    // row and, for every destination it reaches, its meta record.
+    __device__ __forceinline__ uint32_t prepare(const ScatterParams& p, const TokenInputs& in, int lane,
+                                                int& my_slot) const {
+        const int pe_e = (in.e >= 0 && in.e < p.E) ? dest_pe(in.e, p.nEpr, p.nEprShift) : -1;
+        float ws = 0.0f;
+        for (int j = 0; j < p.k; ++j) {
+            const int q = __shfl_sync(kFull, pe_e, j);
+            const float wj = __shfl_sync(kFull, in.wt, j);
+            if (q == lane) ws = ws + wj;
+        }
+        const int s = in.rr.x;
+        my_slot = s >= 0 ? s : -1;
+        const int wb = s != -1 ? __float_as_int(p.useWeights ? ws : 1.0f) : 0;
+        if (lane < p.W) p.route[(size_t)in.g * p.W + lane] = make_int2(my_slot, wb);
+        const uint32_t mask = __ballot_sync(kFull, my_slot >= 0);
+        write_records(p, in.g, mask, my_slot, wb, in.e, lane);
+        return mask;
+    }
+};
+
+template <int kW, int kK>
+__global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(ScatterParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_base[kW];
+    __shared__ unsigned s_tag;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int G = p.G, W = p.W, b = blockIdx.x;
+    const int lo = (int)((long long)b * G / gridDim.x);
+    const int hi = (int)((long long)(b + 1) * G / gridDim.x);  // > lo: the grid has at most G blocks
+    const LocalLayout L = local_layout(p.localOwn, W, nwarps);
+    uint32_t* cmask = reinterpret_cast<uint32_t*>(smem + L.cmask);
+    int* ccnt = reinterpret_cast<int*>(smem + L.ccnt);
+    int* slot = reinterpret_cast<int*>(smem + L.slot);
+    int* list = reinterpret_cast<int*>(smem + L.list);
+    int* ctr = reinterpret_cast<int*>(smem + L.ctr);
+    const int c_lo = lo >> 5, nch = ((hi + 31) >> 5) - c_lo;
+    const int nw = (W + kLocalPerWord - 1) / kLocalPerWord;  // words per block
+
+    pdl_wait();  // the ids, x and the previous call's words are visible from here on
+    if (tid == 0) s_tag = ((__ldcg(p.local_epoch) << 1) | 1u) & 0xffffu;
+    if (tid < kW) s_base[tid] = 0;
+
+    // 1. Masks of the own chunks' tokens; own tokens per chunk and destination.
+    for (int i = warp; i < nch; i += nwarps) {
+        const int g = (c_lo + i) * 32 + lane;
+        const bool own = g >= lo && g < hi;
+        bool bad = false;
+        const uint32_t m = own ? local_mask<kK>(p, g, bad) : 0u;
+        if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
+        cmask[i * 32 + lane] = m;
+#pragma unroll
+        for (int pe = 0; pe < kW; ++pe) {
+            if (pe < W) {
+                const uint32_t bb = __ballot_sync(kFull, (m >> pe) & 1u);
+                if (lane == pe) ccnt[i * W + pe] = __popc(bb);
+            }
+        }
+    }
+    dest_setup(p);  // ends with a block barrier (one GPU: always goes ahead)
+
+    // 2. Publish this block's totals; list the present own tokens.
+    if (warp == 0) {
+        int tot = 0;
+        if (lane < W)
+            for (int i = 0; i < nch; ++i) tot += ccnt[i * W + lane];
+        const unsigned tag = s_tag;
+        for (int q = 0; q < nw; ++q) {
+            unsigned long long v = tag;
+#pragma unroll
+            for (int u = 0; u < kLocalPerWord; ++u) {
+                const int c = __shfl_sync(kFull, tot, (q * kLocalPerWord + u) & 31);
+                if (q * kLocalPerWord + u < W) v |= (unsigned long long)c << (16 + 8 * u);
+            }
+            if (lane == 0) st_relaxed_u64(p.local_agg + (size_t)b * nw + q, v);
+        }
+        if (hi == G && lane < W) ctr[2 + lane] = tot;  // the last block's own totals, for recv_count
+        const int own = hi - lo, off = lo - c_lo * 32;
+        int n = 0;
+        for (int j0 = 0; j0 < own; j0 += 32) {
+            const int j = j0 + lane;
+            const bool present = j < own && cmask[off + j] != 0u;
+            const uint32_t bb = __ballot_sync(kFull, present);
+            if (present) list[n + __popc(bb & lanemask_lt())] = lo + j;
+            n += __popc(bb);
+        }
+        if (lane == 0) {
+            ctr[0] = n;
+            ctr[1] = 0;
+        }
+    }
+    __syncthreads();
+
+    // 3; every thread of the block runs this once (the engines after issuing
+    // their first row loads).
+    auto route_rest = [&]() -> bool {
+        const unsigned want = (s_tag + (p.barrierSlack << 1)) & 0xffffu;
+        const int words = b * nw;
+        int ok = 1;
+        for (int i0 = 0; i0 < words; i0 += 4 * (int)blockDim.x) {
+            unsigned long long v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * blockDim.x + tid;
+                v[u] = i < words ? ld_relaxed_u64(p.local_agg + i) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * blockDim.x + tid;
+                if (i >= words) continue;
+                if ((unsigned)(v[u] & 0xffffu) != want) {  // not yet published: wait, bounded
+                    const long long t0 = clock64();
+                    do {
+                        if (clock64() - t0 > kWaitCycles) {
+                            ok = 0;
+                            break;
+                        }
+                        __nanosleep(32);
+                        v[u] = ld_relaxed_u64(p.local_agg + i);
+                    } while ((unsigned)(v[u] & 0xffffu) != want);
+                    if (!ok) break;
+                }
+                const int q = i % nw;
+#pragma unroll
+                for (int c = 0; c < kLocalPerWord; ++c) {
+                    const int pe = q * kLocalPerWord + c;
+                    const int n = (int)((v[u] >> (16 + 8 * c)) & 0xffu);
+                    if (pe < W && n != 0) atomicAdd(&s_base[pe], n);
+                }
+            }
+            if (!ok) break;
+        }
+        if (tid == 0 && atomicAdd(p.local_done, 1u) == gridDim.x - 1) {
+            *p.local_done = 0u;  // every block has read the epoch: the next call's
+            atomicAdd(p.local_epoch, 1u);
+        }
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
+            return false;  // the bases are unknown: nothing is copied
+        }
+        if (warp == 0 && lane < W) {
+            int run = s_base[lane];
+            if (hi == G) {
+                const int total = run + ctr[2 + lane];
+                p.recv_count[lane] = total;  // stored, not accumulated
+                if (total > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
+            }
+            for (int i = 0; i < nch; ++i) {
+                const int c = ccnt[i * W + lane];
+                ccnt[i * W + lane] = run;
+                run += c;
+            }
+        }
+        __syncthreads();
+        const uint32_t lt = lanemask_lt();
+        for (int i = warp; i < nch; i += nwarps) {
+            const int g = (c_lo + i) * 32 + lane;
+            const uint32_t m = cmask[i * 32 + lane];  // 0 for tokens that are not own
+            const bool own = g >= lo && g < hi;
+#pragma unroll
+            for (int pe = 0; pe < kW; ++pe) {
+                if (pe < W) {
+                    const bool hit = (m >> pe) & 1u;
+                    const uint32_t bb = __ballot_sync(kFull, hit);
+                    if (own) {
+                        int sl = -1;
+                        if (hit) {
+                            sl = ccnt[i * W + pe] + __popc(bb & lt);
+                            if (sl >= p.maxRecv) {  // only when maxRecv is exceeded
+                                atomicOr(p.err, EP_DEVERR_CAPACITY);
+                                sl = -2;
+                            }
+                        }
+                        slot[(g - lo) * W + pe] = sl;
+                        if (m == 0u) p.route[(size_t)g * W + pe] = make_int2(-1, 0);  // absent: no engine sees it
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        return true;
+    };
+
+    const int engines = p.localEngines;
+    if (warp < engines) {
+        const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, engines, lane);
+        LocalFeed feed;
+        feed.list = list;
+        feed.ctr = ctr + 1;
+        feed.slot = slot;
+        feed.n = ctr[0];
+        feed.lo = lo;
+        copy_engine<1>(p, es, lane, feed, route_rest);
+    } else {
+        route_rest();
+    }
+}
+
+// =====================================================================
 // dispatch_fused: route, scan and scatter in one cooperative launch (an
 // option, EP_DISPATCH_FUSED=1: on B200 it measured slower than route_count +
 // scatter_rows, since ~300 copy-engine warps route the tokens instead of
@@ -1905,6 +2185,36 @@ cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out) {
 
 cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s) {
     cudaError_t e = for_world_ll(p.W, p.k, [&](auto k) { return launch_pdl(k, blocks, kLlThreads, smem, s, p); });
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+namespace {
+template <typename F>
+cudaError_t for_world_local(int W, int k, F&& f) {
+    if (W <= 8)
+        return k <= 8 ? f(ep_dispatch_local_kernel<8, 8>) : k <= 16 ? f(ep_dispatch_local_kernel<8, 16>)
+                                                             : f(ep_dispatch_local_kernel<8, 32>);
+    if (W <= 16)
+        return k <= 8 ? f(ep_dispatch_local_kernel<16, 8>) : k <= 16 ? f(ep_dispatch_local_kernel<16, 16>)
+                                                              : f(ep_dispatch_local_kernel<16, 32>);
+    return k <= 8 ? f(ep_dispatch_local_kernel<32, 8>) : k <= 16 ? f(ep_dispatch_local_kernel<32, 16>)
+                                                          : f(ep_dispatch_local_kernel<32, 32>);
+}
+}  // namespace
+
+cudaError_t local_set_smem(int W, int topk, size_t bytes) {
+    return for_world_local(W, topk, [&](auto k) { return raise_smem(k, bytes); });
+}
+
+cudaError_t local_blocks_per_sm(int W, int topk, size_t smem, int* out) {
+    return for_world_local(W, topk, [&](auto k) {
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, kLocalWarps * 32, smem);
+    });
+}
+
+cudaError_t launch_dispatch_local(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s) {
+    cudaError_t e =
+        for_world_local(p.W, p.k, [&](auto k) { return launch_pdl(k, blocks, kLocalWarps * 32, smem, s, p); });
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
