@@ -322,15 +322,13 @@ def run_reference(args, wl):
 # ------------------------------------------------------------------ our arm
 def dispatch_kernels(info) -> str:
     """The kernels one dispatch of this plan launches."""
-    if info.dispatchLowLatency:
-        return "ep_dispatch_ll (one launch)"
     if info.dispatchFused:
-        return "ep_dispatch_fused (one cooperative launch)"
+        return "ep_dispatch_fused (one launch)"
     return "ep_dispatch (route_count + scatter_rows)"
 
 
 def dispatch_launches(info) -> int:
-    return 1 if (info.dispatchLowLatency or info.dispatchFused) else 2
+    return 1 if info.dispatchFused else 2
 
 
 GRAPH_CALLS = 20   # calls captured back to back in one CUDA graph

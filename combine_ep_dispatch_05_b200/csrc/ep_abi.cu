@@ -32,36 +32,21 @@ struct EpPlan {
     int32_t* ptotal;      // route_count's present-token total (last-block scan)
     int32_t* cwork;
     uint32_t* cdone;
-    int32_t* chunk_cnt;   // fused dispatch: [ceil(G/32)][W]
-    int32_t* chunk_base;
-    uint32_t* fbar;
-    uint32_t* fdone;
     int32_t* err;
     size_t scatterSmem;
     bool dense;           // large batches: route_count's earlier form, tile bases in global memory
     size_t baseSmem;      // > 0: the scatter scans the tile counts into this much shared memory
     size_t baseOffset;    // its offset in the scatter's shared memory, and the engines'
     size_t engineOffset;
-    bool fused;           // route + scan + scatter in one cooperative launch
-    bool ll;              // small-batch single launch (dispatch_ll)
-    size_t llSmem;        // its dynamic shared memory
-    int llTile;           // its tokens per block
-    unsigned* ll_status;  // its scratch: tile status words, tile counts, present list, counters
-    int32_t* ll_agg;
-    int32_t* ll_plist;
-    unsigned long long* ll_ptotal;
-    int32_t* ll_ticket;
-    unsigned* ll_done;
-    unsigned* ll_epoch;
-    bool local;           // small-batch single launch with per-block routing (dispatch_local)
-    size_t localSmem;     // its dynamic shared memory: routing area, then the copy engines
-    size_t localEngineOffset;
-    int localOwn;         // the most tokens one of its blocks owns
-    int localBlocks;      // its grid
-    unsigned long long* local_agg;  // its scratch: the blocks' published totals, call epoch, blocks done
-    unsigned* local_epoch;
-    unsigned* local_done;
-    unsigned barrierSlack;  // test hook: 1 makes the fused grid barrier unreachable
+    bool fused;           // the fused dispatch (dispatch_fused): one launch, per-block routing
+    size_t fusedSmem;     // its dynamic shared memory: routing area, then the copy engines
+    size_t fusedEngineOffset;
+    int fusedOwn;         // the most tokens one of its blocks owns
+    int fusedBlocks;      // its grid
+    unsigned long long* fused_agg;  // its scratch: the blocks' published totals, call epoch, blocks done
+    unsigned* fused_epoch;
+    unsigned* fused_done;
+    unsigned barrierSlack;  // test hook: 1 makes the fused dispatch's look-back unreachable
     int boundsRows;         // bounds-checking build: rows of each destination's buffers it checks against
     int fanoutSwitch;       // x100, see ScatterParams
     bool dispatched;
@@ -197,36 +182,16 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
     return g;
 }
 
-// Plans of at most EP_LL_MAX_TOKENS tokens per rank (the design page's
-// internode dispatch switches to its low-latency family at 512 tokens a
-// launch) may take the single-launch low-latency dispatch (dispatch_ll); a
-// tile (a block's tokens) must fit one block's threads. It is off by default
-// (kLlDefaultMaxTokens = 0): on B200 it measured no faster than route_count +
-// scatter_rows, whose launch boundary programmatic dependent launch already
-// hides (ct = 1 workload: 19.5 vs 17.4 us; the 512-token workload: 32.9 vs
-// 33.8 us), since its own handoffs cost as many dependent memory round trips.
-constexpr int kLlDefaultMaxTokens = 0;
-
-// Largest batch (W * maxTokPerRank tokens) that takes dispatch_local.
-constexpr int kLocalDefaultMaxTokens = 0;
-
-// Returns the stages per copy engine of the low-latency dispatch that fit
-// `smemOptin` (the shared memory in *smem, the tile in *tile), or 0 when the
-// plan does not take it.
-int ll_stages(const EpCfg* c, const Geometry& geo, bool fused, int blocks, size_t smemOptin, size_t* smem,
-              int* tile) {
-    const long long G = (long long)c->worldSize * c->maxTokPerRank;
-    const int llMax = env_int("EP_LL_MAX_TOKENS", kLlDefaultMaxTokens, 0);
-    if (fused || geo.scatterWarps > ep::kLlWarps ||
-        c->maxTokPerRank > llMax || blocks < 1)
-        return 0;
-    *tile = ep::ll_tile_tokens(G, blocks);
-    if (*tile > ep::kLlThreads) return 0;
-    for (int st = geo.scatterStages; st >= 2; --st) {
-        *smem = ep::ll_smem_bytes(*tile, c->worldSize, geo.scatterWarps, st, geo.chunkStride);
-        if (*smem <= smemOptin) return st;
-    }
-    return 0;
+// The fused dispatch (dispatch_fused, EP_DISPATCH_FUSED=1): one launch in
+// which every block routes its own share of the batch and copies it, for
+// plans where no block owns more than kFusedMaxOwn tokens. Taken only on
+// request: on B200 it measured about as fast as route_count + scatter_rows at
+// the 512-token workload (28.4-28.9 vs 29.7 us) and slower where a few
+// present tokens cluster (ct = 8 of 512 tokens a rank: 17.7 vs 15.2 us),
+// since a block's present tokens all go through that block's engines.
+bool want_fused() {
+    const char* v = std::getenv("EP_DISPATCH_FUSED");
+    return v && std::strcmp(v, "1") == 0;
 }
 
 void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
@@ -332,15 +297,12 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info) {
                                                        geo.chunkStride) + ep::kStaticSmemReserve + 1024;
         info->scatterBlocks = sms * std::max(1, (int)((228 * 1024) / perBlock));
         info->combineBlocks = sms * 2;
-        size_t llSmem = 0;
-        int llTile = 0;
-        const int llStages = ll_stages(cfg, geo, false, sms, 227 * 1024 - 4096, &llSmem, &llTile);
-        if (llStages > 0) {
-            const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
-            info->dispatchLowLatency = 1;
-            info->scatterBlocks = (int)((G + llTile - 1) / llTile);
-            info->scatterStages = llStages;
-            info->scratchBytes = (long long)ep::scratch_layout(G, cfg->worldSize, info->numTiles, true).total;
+        const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
+        const int fusedBlocks = (int)std::min<long long>(info->scatterBlocks, G);
+        if (want_fused() && (G + fusedBlocks - 1) / fusedBlocks <= ep::kFusedMaxOwn) {
+            info->dispatchFused = 1;
+            info->scatterBlocks = fusedBlocks;
+            info->scratchBytes = (long long)ep::scratch_layout(G, cfg->worldSize, info->numTiles, fusedBlocks).total;
         }
         return EP_OK;
     } catch (...) {
@@ -377,19 +339,17 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         const long long Gtok = (long long)cfg->worldSize * cfg->maxTokPerRank;
         const int denseEnv = env_int("EP_DISPATCH_DENSE", -1, 0);
         const bool dense = denseEnv >= 0 ? denseEnv != 0 : Gtok > kDenseMinTokens;
-        const char* fusedEnv = std::getenv("EP_DISPATCH_FUSED");
-        const bool wantFused = fusedEnv && std::strcmp(fusedEnv, "1") == 0;
         {
             // The scatter scans route_count's tile counts itself when they
             // fit a few KB of shared memory (route_count then ends without a
-            // last-block scan); the fused dispatch has its own. Shared memory:
+            // last-block scan). Shared memory:
             // the tile bases (if any) first, then the copy engines.
             const int numTiles =
                 (int)(((long long)cfg->worldSize * cfg->maxTokPerRank + ep::kCountTile - 1) / ep::kCountTile);
             const size_t bs = ep::scatter_base_smem_bytes(numTiles, cfg->worldSize);
             const char* scanEnv = std::getenv("EP_SCATTER_SCAN");
             const bool scanInRoute = scanEnv && std::strcmp(scanEnv, "route") == 0;
-            if (!wantFused && !scanInRoute && !dense && bs <= ep::kMaxBaseSmemBytes) baseSmem = bs;
+            if (!scanInRoute && !dense && bs <= ep::kMaxBaseSmemBytes) baseSmem = bs;
             const size_t limit = (size_t)smemOptin - ep::kStaticSmemReserve;
             auto engines = [&]() {
                 return ep::scatter_smem_bytes(geo.scatterWarps, geo.scatterStages, geo.chunkStride);
@@ -451,69 +411,12 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->info.device = dev;
         plan->info.numSMs = sms;
         plan->info.scatterBlocks = env_int("EP_SCATTER_BLOCKS", sms * sPerSm);
-        // Dispatch in one cooperative launch (route + scan + scatter) only on
-        // request (EP_DISPATCH_FUSED=1): on B200 the two launches of
-        // route_count + scatter_rows measured faster at every size (main
-        // workload 476 vs 500 us, ct=1 workload 17.4 vs 20.5 us).
-        bool fused = wantFused;
-        int coop = 0;
-        if (fused && (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop))
-            fused = false;
-        if (fused) {
-            int fPerSm = 0;
-            if ((e = ep::fused_set_smem(cfg->worldSize, cfg->numExpertPerToken, smem)) != cudaSuccess ||
-                (e = ep::fused_blocks_per_sm(cfg->worldSize, cfg->numExpertPerToken, geo.scatterWarps, smem,
-                                             &fPerSm)) != cudaSuccess) {
-                cuda_fail(e, "fused dispatch set-up");
-                delete plan;
-                return nullptr;
-            }
-            if (fPerSm < 1)
-                fused = false;
-            else  // a cooperative launch needs every block resident at once
-                plan->info.scatterBlocks = std::min(plan->info.scatterBlocks, sms * fPerSm);
-        }
-        plan->fused = fused;
-        plan->info.dispatchFused = fused ? 1 : 0;
-        // Small batches: the single-launch low-latency dispatch (ll_stages).
-        // The kernel's static shared memory (under 4 KB) comes on top.
-        plan->ll = false;
-        plan->llSmem = 0;
-        plan->llTile = 0;
-        {
-            const int llBlocks = std::max(1, env_int("EP_SCATTER_BLOCKS", sms));
-            size_t llSmem = 0;
-            int llTile = 0;
-            const int llStages =
-                ll_stages(cfg, geo, fused, llBlocks, (size_t)smemOptin - 4096, &llSmem, &llTile);
-            if (llStages > 0) {
-                int per = 0;
-                if ((e = ep::ll_set_smem(cfg->worldSize, cfg->numExpertPerToken, llSmem)) != cudaSuccess ||
-                    (e = ep::ll_blocks_per_sm(cfg->worldSize, cfg->numExpertPerToken, llSmem, &per)) !=
-                        cudaSuccess) {
-                    cuda_fail(e, "low-latency dispatch set-up");
-                    delete plan;
-                    return nullptr;
-                }
-                if (per >= 1) {
-                    const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
-                    plan->ll = true;
-                    plan->llSmem = llSmem;
-                    plan->llTile = llTile;
-                    plan->info.scatterBlocks = (int)((G + llTile - 1) / llTile);
-                    plan->info.scatterStages = llStages;
-                }
-            }
-        }
-        // Small batches: dispatch_local, one launch in which every block
-        // routes the batch itself, when each block owns at most kLocalMaxOwn
-        // tokens and the batch has at most EP_LOCAL_MAX_TOKENS tokens.
-        plan->local = false;
+        // The fused dispatch, on request (want_fused).
+        plan->fused = false;
         {
             const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
-            const int localMax = env_int("EP_LOCAL_MAX_TOKENS", kLocalDefaultMaxTokens, 0);
             int blocks = plan->info.scatterBlocks;
-            if (!fused && !plan->ll && G <= localMax && geo.scatterWarps <= ep::kLocalWarps) {
+            if (want_fused() && geo.scatterWarps <= ep::kFusedWarps) {
                 // The grid: the scatter's, at most one block a token, at most
                 // what fits the SMs at once (the routing area may cost a block
                 // per SM, which changes the tokens a block owns: try again).
@@ -521,18 +424,18 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
                 blocks = (int)std::min<long long>(blocks, G);
                 for (int attempt = 0; attempt < 3 && blocks >= 1; ++attempt) {
                     const int own = (int)((G + blocks - 1) / blocks);
-                    if (own > ep::kLocalMaxOwn) break;
-                    const size_t area = ep::local_layout(own, cfg->worldSize, ep::kLocalWarps).total;
+                    if (own > ep::kFusedMaxOwn) break;
+                    const size_t area = ep::fused_layout(own, cfg->worldSize, ep::kFusedWarps).total;
                     int stages = geo.scatterStages;
                     size_t lsm = area + ep::scatter_smem_bytes(geo.scatterWarps, stages, geo.chunkStride);
                     while (lsm > limit && stages > 2)
                         lsm = area + ep::scatter_smem_bytes(geo.scatterWarps, --stages, geo.chunkStride);
                     if (lsm > limit) break;
                     int per = 0;
-                    if ((e = ep::local_set_smem(cfg->worldSize, cfg->numExpertPerToken, lsm)) != cudaSuccess ||
-                        (e = ep::local_blocks_per_sm(cfg->worldSize, cfg->numExpertPerToken, lsm, &per)) !=
+                    if ((e = ep::fused_set_smem(cfg->worldSize, cfg->numExpertPerToken, lsm)) != cudaSuccess ||
+                        (e = ep::fused_blocks_per_sm(cfg->worldSize, cfg->numExpertPerToken, lsm, &per)) !=
                             cudaSuccess) {
-                        cuda_fail(e, "dispatch_local set-up");
+                        cuda_fail(e, "dispatch_fused set-up");
                         delete plan;
                         return nullptr;
                     }
@@ -541,23 +444,22 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
                         blocks = sms * per;
                         continue;
                     }
-                    plan->local = true;
-                    plan->localSmem = lsm;
-                    plan->localEngineOffset = area;
-                    plan->localOwn = own;
-                    plan->localBlocks = blocks;
+                    plan->fused = true;
+                    plan->fusedSmem = lsm;
+                    plan->fusedEngineOffset = area;
+                    plan->fusedOwn = own;
+                    plan->fusedBlocks = blocks;
                     plan->info.scatterBlocks = blocks;
                     plan->info.scatterStages = stages;
                     break;
                 }
             }
         }
-        plan->info.dispatchLowLatency = (plan->ll || plan->local) ? 1 : 0;
+        plan->info.dispatchFused = plan->fused ? 1 : 0;
         plan->fanoutSwitch = env_int("EP_SCATTER_FANOUT_SWITCH", 375, 0);
-        // Test hook for the failure path: the fused dispatch's grid barrier,
-        // or the low-latency dispatch's wait for earlier tiles, can never
-        // complete, so the blocks give up after their bounded wait and report
-        // EP_DEVERR_TIMEOUT.
+        // Test hook for the failure path: the fused dispatch's wait for the
+        // earlier blocks' totals can never complete, so the blocks give up
+        // after their bounded wait and report EP_DEVERR_TIMEOUT.
         if (const char* t = std::getenv("EP_TEST_UNREACHABLE_BARRIER"))
             plan->barrierSlack = std::strcmp(t, "1") == 0 ? 1u : 0u;
         // Test hook of the bounds-checking build: check the receive buffers
@@ -565,15 +467,15 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->boundsRows = std::min(env_int("EP_TEST_BOUNDS_ROWS", plan->info.maxRecv), plan->info.maxRecv);
         plan->info.combineBlocks = env_int("EP_COMBINE_BLOCKS", sms * cPerSm);
         plan->scatterSmem = smem;
-        plan->dense = !fused && dense;
-        plan->baseSmem = fused ? 0 : baseSmem;
-        plan->baseOffset = fused ? 0 : baseOffset;
-        plan->engineOffset = fused ? 0 : engineOffset;
+        plan->dense = dense;
+        plan->baseSmem = baseSmem;
+        plan->baseOffset = baseOffset;
+        plan->engineOffset = engineOffset;
         plan->G = cfg->worldSize * cfg->maxTokPerRank;
         plan->maxRecv = plan->info.maxRecv;
 
-        const ep::ScratchLayout L = ep::scratch_layout(plan->G, cfg->worldSize, plan->info.numTiles, plan->ll,
-                                                       plan->local ? plan->localBlocks : 0);
+        const ep::ScratchLayout L =
+            ep::scratch_layout(plan->G, cfg->worldSize, plan->info.numTiles, plan->fused ? plan->fusedBlocks : 0);
         plan->info.scratchBytes = (long long)L.total;
         const size_t total = L.total;
         if ((e = cudaMalloc(&plan->scratch, total)) != cudaSuccess) {
@@ -597,21 +499,10 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         plan->ptotal = reinterpret_cast<int32_t*>(base + L.ptotal);
         plan->cwork = reinterpret_cast<int32_t*>(base + L.cwork);
         plan->cdone = reinterpret_cast<uint32_t*>(base + L.cdone);
-        plan->chunk_cnt = reinterpret_cast<int32_t*>(base + L.chunk_cnt);
-        plan->chunk_base = reinterpret_cast<int32_t*>(base + L.chunk_base);
-        plan->fbar = reinterpret_cast<uint32_t*>(base + L.fbar);
-        plan->fdone = reinterpret_cast<uint32_t*>(base + L.fdone);
         plan->err = reinterpret_cast<int32_t*>(base + L.err);
-        plan->ll_status = reinterpret_cast<unsigned*>(base + L.ll_status);
-        plan->ll_agg = reinterpret_cast<int32_t*>(base + L.ll_agg);
-        plan->ll_plist = reinterpret_cast<int32_t*>(base + L.ll_plist);
-        plan->ll_ptotal = reinterpret_cast<unsigned long long*>(base + L.ll_ptotal);
-        plan->ll_ticket = reinterpret_cast<int32_t*>(base + L.ll_ticket);
-        plan->ll_done = reinterpret_cast<unsigned*>(base + L.ll_done);
-        plan->ll_epoch = reinterpret_cast<unsigned*>(base + L.ll_epoch);
-        plan->local_agg = reinterpret_cast<unsigned long long*>(base + L.local_agg);
-        plan->local_epoch = reinterpret_cast<unsigned*>(base + L.local_epoch);
-        plan->local_done = reinterpret_cast<unsigned*>(base + L.local_done);
+        plan->fused_agg = reinterpret_cast<unsigned long long*>(base + L.fused_agg);
+        plan->fused_epoch = reinterpret_cast<unsigned*>(base + L.fused_epoch);
+        plan->fused_done = reinterpret_cast<unsigned*>(base + L.fused_done);
         plan->dispatched = false;
         g_last_error[0] = '\0';
         return plan;
@@ -738,61 +629,20 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
         sp.recv_scales = static_cast<uint32_t*>(recv_scales);
         sp.scaleWords = scaleWords;
         sp.boundsRows = plan->boundsRows;
-        if (plan->local) {
-            // One launch: every block routes the tokens up to its own, then copies its own.
-            const int nEpr = c.numExpertPerRank;
-            sp.w = c.useWeights ? topk_w : nullptr;
-            sp.useWeights = c.useWeights;
-            sp.nEprShift = (nEpr & (nEpr - 1)) == 0 ? __builtin_ctz((unsigned)nEpr) : -1;
-            sp.localOwn = plan->localOwn;
-            sp.localEngines = plan->info.scatterWarps;
-            sp.engineOffset = (int)plan->localEngineOffset;
-            sp.local_agg = plan->local_agg;
-            sp.local_epoch = plan->local_epoch;
-            sp.local_done = plan->local_done;
-            sp.barrierSlack = plan->barrierSlack;
-            e = ep::launch_dispatch_local(sp, plan->localBlocks, plan->localSmem, s);
-            if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_local");
-            plan->dispatched = true;
-            return EP_OK;
-        }
-        if (plan->ll) {
-            // One launch: every block routes and scans the batch, then copies its share.
-            const int nEpr = c.numExpertPerRank;
-            sp.w = c.useWeights ? topk_w : nullptr;
-            sp.useWeights = c.useWeights;
-            sp.nEprShift = (nEpr & (nEpr - 1)) == 0 ? __builtin_ctz((unsigned)nEpr) : -1;
-            sp.llListCap = plan->llTile;
-            sp.llEngines = plan->info.scatterWarps;
-            sp.ll_status = plan->ll_status;
-            sp.ll_agg = plan->ll_agg;
-            sp.ll_plist = plan->ll_plist;
-            sp.ll_ptotal = plan->ll_ptotal;
-            sp.ll_ticket = plan->ll_ticket;
-            sp.ll_done = plan->ll_done;
-            sp.ll_epoch = plan->ll_epoch;
-            sp.barrierSlack = plan->barrierSlack;
-            e = ep::launch_dispatch_ll(sp, plan->info.scatterBlocks, plan->llSmem, s);
-            if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_ll");
-            plan->dispatched = true;
-            return EP_OK;
-        }
         if (plan->fused) {
-            // One cooperative launch: routing phase, chunk scan, copy engines.
-            sp.baseShift = 5;
-            sp.baseStride = c.worldSize;
-            sp.tile_base = plan->chunk_base;
+            // One launch: each block routes its own tokens, adds up the earlier blocks' totals, copies its own.
+            const int nEpr = c.numExpertPerRank;
             sp.w = c.useWeights ? topk_w : nullptr;
-            sp.tok_mask_w = plan->tok_mask;
-            sp.chunk_cnt = plan->chunk_cnt;
-            sp.chunk_base_w = plan->chunk_base;
-            sp.recv_count = recv_count;
-            sp.bar = plan->fbar;
-            sp.done = plan->fdone;
-            sp.numChunks32 = (plan->G + 31) / 32;
             sp.useWeights = c.useWeights;
+            sp.nEprShift = (nEpr & (nEpr - 1)) == 0 ? __builtin_ctz((unsigned)nEpr) : -1;
+            sp.fusedOwn = plan->fusedOwn;
+            sp.fusedEngines = plan->info.scatterWarps;
+            sp.engineOffset = (int)plan->fusedEngineOffset;
+            sp.fused_agg = plan->fused_agg;
+            sp.fused_epoch = plan->fused_epoch;
+            sp.fused_done = plan->fused_done;
             sp.barrierSlack = plan->barrierSlack;
-            e = ep::launch_dispatch_fused(sp, plan->info.scatterBlocks, plan->info.scatterWarps, plan->scatterSmem, s);
+            e = ep::launch_dispatch_fused(sp, plan->fusedBlocks, plan->fusedSmem, s);
             if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_fused");
             plan->dispatched = true;
             return EP_OK;

@@ -18,17 +18,11 @@ constexpr int kMaxWorld = 32;   // one destination bit per lane of a 32-bit mask
 constexpr int kMaxTopk = 32;    // one topk entry per lane
 constexpr int kMaxScatterWarps = 16;
 constexpr int kMaxCombineWarps = 8;
-// Threads of a low-latency dispatch block (its first warps are the copy
-// engines); a block routes a tile of at most kLlThreads tokens, and a launch
-// has at most kLlMaxTiles tiles.
-constexpr int kLlThreads = 512;
-constexpr int kLlWarps = kLlThreads / 32;
-constexpr int kLlMaxTiles = 256;
-// Warps of a dispatch_local block (its first warps are the copy engines), and
-// the most tokens one block may own (the plan takes dispatch_local only when
+// Warps of a dispatch_fused block (its first warps are the copy engines), and
+// the most tokens one block may own (the plan takes dispatch_fused only when
 // ceil(G / blocks) is at most this).
-constexpr int kLocalWarps = 8;
-constexpr int kLocalMaxOwn = 64;
+constexpr int kFusedWarps = 8;
+constexpr int kFusedMaxOwn = 64;
 // Shared memory kept back from the dynamic budget for the kernels' static
 // shared memory.
 constexpr size_t kStaticSmemReserve = 2048;
@@ -105,58 +99,41 @@ struct ScatterParams {
     const int32_t* counts;   // this rank's count table [W][W], complete (after the exchange)
     int32_t* recv_total;     // rows this rank receives, stored by block 0
     int boundsRows;          // bounds-checking build: rows of each destination's buffers (maxRecv)
-    // Only the fused dispatch (route + scan + scatter in one launch) uses these:
+    // Only dispatch_fused uses these, and the fields below:
     const float* w;          // [G][k] or nullptr
-    uint32_t* tok_mask_w;    // = tok_mask, written by the routing phase
-    int32_t* chunk_cnt;      // [numChunks32][W]
-    int32_t* chunk_base_w;   // = tile_base, written by the scan phase
     int32_t* recv_count;     // [W]
-    unsigned* bar;           // grid-barrier counter
-    unsigned* done;          // blocks finished; the last one resets bar, work, done
-    int numChunks32;         // ceil(G / 32)
     int useWeights;
-    unsigned barrierSlack;   // 0; 1 makes the first grid barrier unreachable (tests of the timeout path)
-    // Only the low-latency dispatch uses these (and w, recv_count, useWeights):
+    unsigned barrierSlack;   // 0; 1 makes the look-back wait for a tag no block publishes (tests of the timeout path)
     int nEprShift;           // log2(nEpr) when nEpr is a power of two, else -1
-    int llListCap;           // tokens per tile (<= kLlThreads); gridDim.x = ceil(G / llListCap)
-    int llEngines;           // copy-engine warps per block (<= kLlWarps)
-    unsigned* ll_status;     // [kLlMaxTiles]: (epoch << 1) | 1 once the tile's counts are published
-    int32_t* ll_agg;         // [kLlMaxTiles][W + 1]: rows of each tile at each destination, present tokens
-    int32_t* ll_plist;       // [G][W + 2]: present token q: tag, token, slot at each destination
-    unsigned long long* ll_ptotal;  // (tag << 32) | present tokens of the call, from the last tile
-    int32_t* ll_ticket;      // next tile to hand out (0 at the start of each call)
-    unsigned* ll_done;       // blocks past the hand-out; the last one resets ticket and done
-    unsigned* ll_epoch;      // calls so far (tags the status words of this call)
-    // Only dispatch_local uses these (and w, recv_count, useWeights, nEprShift,
-    // engineOffset, barrierSlack): the most tokens a block owns, its copy-engine
-    // warps, the blocks' published totals [blocks][ceil(W / 6)], the call epoch
-    // and the blocks past their look-back (the last one advances the epoch).
-    int localOwn;
-    int localEngines;
-    unsigned long long* local_agg;
-    unsigned* local_epoch;
-    unsigned* local_done;
+    // (and engineOffset): the most tokens a block owns, its copy-engine warps,
+    // the blocks' published totals [blocks][ceil(W / 6)], the call epoch and
+    // the blocks past their look-back (the last one advances the epoch).
+    int fusedOwn;
+    int fusedEngines;
+    unsigned long long* fused_agg;
+    unsigned* fused_epoch;
+    unsigned* fused_done;
 };
 
-// Byte offsets of dispatch_local's routing area in shared memory (each
+// Byte offsets of dispatch_fused's routing area in shared memory (each
 // 16-byte aligned): masks of the own chunks' tokens [chunks * 32], their own
 // tokens per destination, then bases [chunks][W], the own tokens' slots
 // [own][W], the present own tokens [own], and counters: [0] present own
 // tokens, [1] next one to hand out, [2 + pe] the block's total at pe. own: the
 // most tokens a block owns; its tokens span at most (own + 62) / 32 chunks.
-struct LocalLayout {
+struct FusedLayout {
     size_t cmask, ccnt, slot, list, ctr, total;
 };
-__host__ __device__ inline size_t local_up16(size_t n) { return (n + 15) & ~(size_t)15; }
-__host__ __device__ inline LocalLayout local_layout(int own, int W, int warps) {
+__host__ __device__ inline size_t fused_up16(size_t n) { return (n + 15) & ~(size_t)15; }
+__host__ __device__ inline FusedLayout fused_layout(int own, int W, int warps) {
     (void)warps;
     const size_t chunks = (size_t)(own + 62) / 32;
-    LocalLayout L;
+    FusedLayout L;
     L.cmask = 0;
-    L.ccnt = L.cmask + local_up16(chunks * 32 * 4);
-    L.slot = L.ccnt + local_up16(chunks * (size_t)W * 4);
-    L.list = L.slot + local_up16((size_t)own * W * 4);
-    L.ctr = L.list + local_up16((size_t)own * 4);
+    L.ccnt = L.cmask + fused_up16(chunks * 32 * 4);
+    L.slot = L.ccnt + fused_up16(chunks * (size_t)W * 4);
+    L.list = L.slot + fused_up16((size_t)own * W * 4);
+    L.ctr = L.list + fused_up16((size_t)own * 4);
     L.total = (L.ctr + (2 + kMaxWorld) * 4 + 127) & ~(size_t)127;
     return L;
 }
@@ -205,48 +182,31 @@ struct PushParams {
 
 // Byte offsets of the dispatch scratch regions (each 256-byte aligned):
 // routing table, token masks, tile counts, tile bases (256-token tiles of the
-// split dispatch), chunk counts and bases (32-token chunks of the fused
-// dispatch), the low-latency dispatch's tile status words, tile counts and
-// present-token list, the counters (one 256-byte region: tile ticket, scatter
-// token counter, combine token counter, combine blocks done, fused grid
-// barrier, fused blocks done, low-latency tile ticket, blocks done, call epoch
-// and present total, route_count's present-token total), error word.
+// split dispatch), the fused dispatch's published totals, the counters (one
+// 256-byte region: tile ticket, scatter token counter, combine token counter,
+// combine blocks done, route_count's present-token total, the fused
+// dispatch's call epoch and blocks done), error word.
 struct ScratchLayout {
-    size_t route, tok_mask, tile_cnt, tile_base, chunk_cnt, chunk_base, ll_status, ll_agg, ll_plist, local_agg;
-    size_t ticket, work, cwork, cdone, fbar, fdone, ll_ticket, ll_done, ll_epoch, ll_ptotal, ptotal, local_epoch,
-        local_done, err, total;
+    size_t route, tok_mask, tile_cnt, tile_base, fused_agg;
+    size_t ticket, work, cwork, cdone, ptotal, fused_epoch, fused_done, err, total;
 };
 
-// ll: the plan takes the single-launch dispatch (its regions are empty
-// otherwise); localBlocks: the grid of dispatch_local (0: not taken).
-inline ScratchLayout scratch_layout(long long G, int W, int numTiles, bool ll = false, int localBlocks = 0) {
+// fusedBlocks: the grid of dispatch_fused (0: the plan does not take it).
+inline ScratchLayout scratch_layout(long long G, int W, int numTiles, int fusedBlocks = 0) {
     auto up = [](size_t n) { return (n + 255) & ~(size_t)255; };
-    const size_t numChunks32 = (size_t)((G + 31) / 32);
     ScratchLayout L;
     L.route = 0;
     L.tok_mask = L.route + up(sizeof(int2) * (size_t)G * W);
     L.tile_cnt = L.tok_mask + up(sizeof(uint32_t) * (size_t)G);
     L.tile_base = L.tile_cnt + up(sizeof(int32_t) * (size_t)numTiles * (W + 1));
-    L.chunk_cnt = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * (W + 1));
-    L.chunk_base = L.chunk_cnt + up(sizeof(int32_t) * numChunks32 * W);
-    const size_t llTiles = ll ? (size_t)(G < kLlMaxTiles ? G : kLlMaxTiles) : 0;
-    L.ll_status = L.chunk_base + up(sizeof(int32_t) * numChunks32 * W);
-    L.ll_agg = L.ll_status + up(sizeof(uint32_t) * llTiles);
-    L.ll_plist = L.ll_agg + up(sizeof(int32_t) * llTiles * (W + 1));
-    L.local_agg = L.ll_plist + (ll ? up(sizeof(int32_t) * (size_t)G * (W + 2)) : 0);
-    L.ticket = L.local_agg + up(sizeof(unsigned long long) * (size_t)localBlocks * ((W + 5) / 6));
+    L.fused_agg = L.tile_base + up(sizeof(int32_t) * (size_t)numTiles * (W + 1));
+    L.ticket = L.fused_agg + up(sizeof(unsigned long long) * (size_t)fusedBlocks * ((W + 5) / 6));
     L.work = L.ticket + 4;
     L.cwork = L.ticket + 8;
     L.cdone = L.ticket + 12;
-    L.fbar = L.ticket + 16;
-    L.fdone = L.ticket + 20;
-    L.ll_ticket = L.ticket + 24;
-    L.ll_done = L.ticket + 28;
-    L.ll_epoch = L.ticket + 32;
-    L.ll_ptotal = L.ticket + 40;
-    L.ptotal = L.ticket + 48;
-    L.local_epoch = L.ticket + 52;
-    L.local_done = L.ticket + 56;
+    L.ptotal = L.ticket + 16;
+    L.fused_epoch = L.ticket + 20;
+    L.fused_done = L.ticket + 24;
     L.err = L.ticket + 256;
     L.total = L.err + 256;
     return L;
@@ -263,25 +223,11 @@ cudaError_t launch_scatter_rows(const ScatterParams& p, bool dense, int blocks, 
                                 cudaStream_t s);
 // fp32: float32 combine leg (an fp32 plan); bf16 otherwise.
 cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s);
-// Fused dispatch (route + scan + scatter), a cooperative launch: blocks must
-// not exceed the co-resident capacity (fused_blocks_per_sm * SMs).
-cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s);
+// The fused dispatch of small batches: one launch, per-block routing
+// (dispatch_fused, kFusedWarps warps per block): opt-in, occupancy, launch.
 cudaError_t fused_set_smem(int W, int topk, size_t bytes);
-cudaError_t fused_blocks_per_sm(int W, int topk, int warps, size_t smem, int* out);
-// Low-latency dispatch (one launch, no dependency between blocks) for small
-// batches: shared memory it needs, opt-in, occupancy, launch (kLlThreads
-// threads per block).
-int ll_tile_tokens(long long G, int blocks);
-size_t ll_smem_bytes(int tileTokens, int W, int warps, int stages, int chunkStride);
-cudaError_t ll_set_smem(int W, int topk, size_t bytes);
-cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out);
-cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s);
-
-// Single-launch dispatch of small batches with per-block routing
-// (dispatch_local, kLocalWarps warps per block): opt-in, occupancy, launch.
-cudaError_t local_set_smem(int W, int topk, size_t bytes);
-cudaError_t local_blocks_per_sm(int W, int topk, size_t smem, int* out);
-cudaError_t launch_dispatch_local(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s);
+cudaError_t fused_blocks_per_sm(int W, int topk, size_t smem, int* out);
+cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s);
 
 // Ranks in separate processes: the count exchange / barrier, and the push.
 cudaError_t launch_comm_sync(const SyncParams& p, cudaStream_t s);

@@ -21,12 +21,13 @@
 //   combine      one warp per token: up to 8 destination rows in flight per
 //                16-byte column, float32 fma fold in destPe order; bf16 RNE out
 //                (float32 out, unrounded, for a float32 plan).
-// Options: dispatch_ll (one launch; blocks publish tile counts and read their
-// predecessors') and dispatch_fused (one cooperative launch, grid barriers).
+// Option: dispatch_fused, the whole dispatch of a small batch in one launch
+// (each block routes and copies its own share of the batch; the bases come
+// from the other blocks' published counts by decoupled look-back).
 //
-// No kernel traps or spins without a bound: waits on shared-memory barriers,
-// grid barriers and other blocks' published words give up after
-// kWaitCycles, set EP_DEVERR_TIMEOUT and drain their copies.
+// No kernel traps or spins without a bound: waits on shared-memory barriers
+// and on other blocks' published words give up after kWaitCycles, set
+// EP_DEVERR_TIMEOUT and drain their copies.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -410,7 +411,7 @@ __device__ int scan_tile_bases(const ScatterParams& p, int* s_base, int* rows) {
 struct TokenInputs {
     int h;     // the feed's handle of the token, or -1 when nothing is loaded
     int g;     // token
-    int2 rr;   // lane < W: (tile-local rank or -1, weight bits); list feed: (slot or -1, -)
+    int2 rr;   // lane < W: (tile-local rank or -1, weight bits); OwnFeed: (slot, or -1 / -2, -)
     int base;  // lane < W: base of the token's tile at destination lane
     int e;     // lane < k: topk id
     float wt;  // lane < k: topk weight (list feed only)
@@ -750,75 +751,6 @@ struct StaticFeed {
     }
 };
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Wait (bounded) until *p == want; false when the wait gave up.
-__device__ __forceinline__ bool wait_tag(const unsigned* p, unsigned want) {
-    if (ld_acquire_u32(p) == want) return true;
-    const long long t0 = clock64();
-    while (ld_acquire_u32(p) != want) {
-        if (clock64() - t0 > kWaitCycles) return false;
-        __nanosleep(32);
-    }
-    return true;
-}
-
-// Single-launch small-batch dispatch: the call's present tokens are a list
-// in global memory (entry q: tag, token, slot at each destination), written
-// by the blocks that routed them; this block copies entries b, b + nb, ...
-// (handle i = entry b + i*nb). The routing rows and meta records are already
-// written; the engine copies the rows (and the scale rows, when the call has
-// them).
-struct PlistFeed {
-    const int32_t* plist;  // [P][W + 2]
-    int b, nb, n, i, step;
-    unsigned tag;
-
-    __device__ __forceinline__ const int32_t* entry(const ScatterParams& p, int h) const {
-        return plist + (size_t)(b + (size_t)h * nb) * (p.W + 2);
-    }
-    // Next handle, once its entry is published (lane 0 waits, bounded).
-    __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
-        int h = p.G;
-        if (i < n) {
-            h = i;
-            i += step;
-            int ok = 1;
-            if (lane == 0) ok = wait_tag(reinterpret_cast<const unsigned*>(entry(p, h)), tag);
-            __syncwarp();
-            if (!__shfl_sync(kFull, ok, 0)) {
-                if (lane == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
-                n = 0;  // copy nothing more
-                h = p.G;
-            }
-        }
-        return h;
-    }
-    __device__ __forceinline__ int row(const ScatterParams& p, int h) const { return __ldcg(entry(p, h) + 1); }
-    __device__ __forceinline__ TokenInputs load(const ScatterParams& p, int h, int lane) const {
-        const int32_t* e = entry(p, h);
-        TokenInputs in;
-        in.h = h;
-        in.g = __ldcg(e + 1);
-        in.rr = make_int2(lane < p.W ? __ldcg(e + 2 + lane) : -1, 0);
-        in.base = 0;
-        in.e = -1;
-        in.wt = 0.0f;
-        return in;
-    }
-    __device__ __forceinline__ uint32_t prepare(const ScatterParams& p, const TokenInputs& in, int lane,
-                                                int& my_slot) const {
-        my_slot = in.rr.x;
-        const uint32_t mask = __ballot_sync(kFull, my_slot >= 0);
-        if (p.scaleWords > 0) write_scales(p, in.g, mask, my_slot, lane);
-        return mask;
-    }
-};
-
 // One copy engine (a warp): the present tokens its feed hands out are copied
 // row piece by row piece through an S-stage shared-memory ring, S - kPend
 // loads ahead, with kPend items' bulk stores left draining when a stage is
@@ -1026,235 +958,10 @@ __global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_scatter_rows_kernel(
     global_copy_engines<kPend>(p, es, lane, warp, nwarps, P, rows, s_base);
 }
 
-// =====================================================================
-// dispatch_ll: the whole dispatch of a small batch in one launch (the
-// low-latency family; the pages switch to theirs at 512 tokens a launch).
-// Block = tile of up to kLlThreads consecutive tokens, one thread per token:
-//   1. the block takes the next tile from a ticket, routes its tokens
-//      (destination masks; counts per 32-token chunk by ballot) and publishes
-//      the tile's count at every destination and of present tokens, then a
-//      status word tagged with this call's epoch;
-//   2. it adds up the counts of all earlier tiles, each loaded as soon as its
-//      status is published (a bounded wait). Tiles are handed out in order,
-//      so a block only waits on blocks that are already running, and no
-//      block waits before publishing: the waits end. The last tile stores
-//      recv_count and publishes the number of present tokens P;
-//   3. each thread of a present token computes its slots (tile base + chunk
-//      base + rank in the chunk), writes the token's routing row and meta
-//      records, and publishes the token as entry q of the present list (q =
-//      its number among the call's present tokens, in (srcRank, token)
-//      order); absent tokens get their routing rows;
-//   4. the block's copy engines copy entries b, b + nb, ... (b = its tile),
-//      each once it is published: the copies spread over all blocks however
-//      the present tokens cluster.
-// Shared memory: [slots of the tile's present tokens: T x W], then the copy
-// engines' barriers and stages.
-// =====================================================================
 __device__ __forceinline__ int dest_pe(int e, int nEpr, int shift) { return shift >= 0 ? e >> shift : e / nEpr; }
 
-__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-template <int kW, int kK>
-__global__ void __launch_bounds__(kLlThreads, 1) ep_dispatch_ll_kernel(ScatterParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_cnt[kLlWarps][kW + 1];  // per chunk: rows at each destination, present tokens
-    __shared__ int s_base[kW + 1];           // the same for all earlier tiles
-    __shared__ int s_agg[kW + 1];            // the same for this tile
-    __shared__ int s_tile, s_present, s_ok;
-    __shared__ unsigned s_tag;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int G = p.G, W = p.W, k = p.k, C = W + 1;
-    const int TT = p.llListCap;
-    int* tile_slot = reinterpret_cast<int*>(smem);  // [TT][W]
-    uint8_t* area = smem + (((size_t)TT * W * sizeof(int) + 127) & ~(size_t)127);
-
-    pdl_wait();  // the ids and the counters of the previous call are visible from here on
-    pdl_trigger();
-    dest_setup(p);
-    if (tid == 0) {
-        s_tile = atomicAdd(p.ll_ticket, 1);
-        s_tag = (__ldcg(p.ll_epoch) << 1) | 1u;
-    }
-    if (tid <= kW) s_base[tid] = 0;
-    __syncthreads();
-    const int t = s_tile;
-    const unsigned tag = s_tag;
-    // Every block has its tile: the last one to get here resets the hand-out
-    // for the next call and advances the epoch (the blocks of this call keep
-    // the tag they read).
-    if (tid == 0 && atomicAdd(p.ll_done, 1u) == gridDim.x - 1) {
-        *p.ll_ticket = 0;
-        *p.ll_done = 0u;
-        atomicAdd(p.ll_epoch, 1u);
-    }
-
-    // 1. Route this tile: thread i takes token t*TT + i. Its ids (entries
-    // that are masked or out of range become -1) and weights stay in
-    // registers for step 3.
-    const int g = t * TT + tid;
-    const bool live = tid < TT && g < G;
-    uint32_t mask = 0;
-    bool bad = false;
-    int e[kK];
-    float wj[kK];
-#pragma unroll
-    for (int j = 0; j < kK; ++j) {
-        e[j] = (live && j < k) ? p.idx[(size_t)g * k + j] : -1;
-        wj[j] = (live && j < k && p.w != nullptr) ? p.w[(size_t)g * k + j] : 0.0f;
-    }
-#pragma unroll
-    for (int j = 0; j < kK; ++j) {
-        if (e[j] >= p.E) {  // contract violation: report, treat as masked
-            bad = true;
-            e[j] = -1;
-        }
-        if (e[j] >= 0) mask |= 1u << dest_pe(e[j], p.nEpr, p.nEprShift);
-    }
-    if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
-    int cnt = 0;
-#pragma unroll
-    for (int pe = 0; pe < kW; ++pe) {
-        if (pe < W) {
-            const uint32_t bb = __ballot_sync(kFull, (mask >> pe) & 1u);
-            if (lane == pe) cnt = __popc(bb);
-        }
-    }
-    const uint32_t bp = __ballot_sync(kFull, mask != 0u);
-    if (lane < W) s_cnt[warp][lane] = cnt;
-    if (lane == 0) s_cnt[warp][W] = __popc(bp);
-    __syncthreads();
-    // Chunk bases within the tile (in place) and the tile's counts; publish.
-    if (warp == 0) {
-        for (int col = lane; col < C; col += 32) {  // 33 columns when W = 32
-            int run = 0;
-            for (int w = 0; w < kLlWarps; ++w) {
-                const int c = s_cnt[w][col];
-                s_cnt[w][col] = run;
-                run += c;
-            }
-            s_agg[col] = run;
-            p.ll_agg[(size_t)t * C + col] = run;
-        }
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) st_release_u32(p.ll_status + t, tag);
-    }
-
-    // 2. Counts of the earlier tiles. (barrierSlack, a test hook, 0
-    // otherwise, makes the awaited tag one that no block writes.)
-    const unsigned want = tag + (p.barrierSlack << 1);
-    int ok = 1;
-    for (int i = tid; i < t; i += kLlThreads) {
-        if (!wait_tag(p.ll_status + i, want)) {
-            ok = 0;
-            break;
-        }
-        for (int c = 0; c < C; ++c) atomicAdd(&s_base[c], __ldcg(p.ll_agg + (size_t)i * C + c));
-    }
-    if (!__syncthreads_and(ok)) {
-        if (tid == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
-        return;  // nothing copied: the counts are unknown
-    }
-    if (t == (int)gridDim.x - 1) {
-        if (tid < W) {
-            const int total = s_base[tid] + s_agg[tid];
-            p.recv_count[tid] = total;  // stored, not accumulated
-            if (total > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
-        }
-        if (tid == 0)
-            st_release_u64(p.ll_ptotal, ((unsigned long long)tag << 32) | (unsigned)(s_base[W] + s_agg[W]));
-    }
-
-    // 3. Slots, routing rows, meta records and present-list entries of this
-    // tile's tokens.
-    const uint32_t lt = lanemask_lt();
-    const int li = s_cnt[warp][W] + __popc(bp & lt);  // present token number within the tile
-#pragma unroll
-    for (int pe = 0; pe < kW; ++pe) {
-        if (pe < W) {
-            const bool hit = (mask >> pe) & 1u;
-            const uint32_t bb = __ballot_sync(kFull, hit);
-            if (live && mask != 0u) {
-                int slot = hit ? s_base[pe] + s_cnt[warp][pe] + __popc(bb & lt) : -1;
-                if (slot >= p.maxRecv) {  // only when the counts were corrupted
-                    atomicOr(p.err, EP_DEVERR_CAPACITY);
-                    slot = -1;
-                }
-                tile_slot[li * W + pe] = slot;
-            }
-        }
-    }
-    if (live) {
-        const int r = g / p.T, tok = g - r * p.T;
-        int32_t* ent = p.ll_plist + (size_t)(s_base[W] + li) * (W + 2);
-        if (mask != 0u) ent[1] = g;
-        for (int pe = 0; pe < W; ++pe) {
-            const int slot = mask != 0u ? tile_slot[li * W + pe] : -1;
-            if (mask != 0u) ent[2 + pe] = slot;
-            if (slot < 0) {
-                p.route[(size_t)g * W + pe] = make_int2(-1, 0);
-                continue;
-            }
-            float ws = 0.0f;
-#pragma unroll
-            for (int j = 0; j < kK; ++j)
-                if (e[j] >= 0 && dest_pe(e[j], p.nEpr, p.nEprShift) == pe) ws = ws + wj[j];
-            const int wb = __float_as_int(p.useWeights ? ws : 1.0f);
-            p.route[(size_t)g * W + pe] = make_int2(slot, wb);
-            int32_t* rec = p.recv_meta + ((size_t)pe * p.maxRecv + slot) * p.M;
-            rec[0] = r;
-            rec[1] = tok;
-            rec[2] = wb;
-#pragma unroll
-            for (int j = 0; j < kK; ++j)
-                if (j < k) rec[3 + j] = (e[j] >= 0 && dest_pe(e[j], p.nEpr, p.nEprShift) == pe) ? e[j] - pe * p.nEpr : -1;
-        }
-        if (mask != 0u) st_release_u32(reinterpret_cast<unsigned*>(ent), tag);  // after the entry's fields
-    }
-
-    // 4. Copy engines, once the number of present tokens is known.
-    if (tid == 0) {
-        const unsigned long long wantP = (unsigned long long)want;
-        unsigned long long v = ld_acquire_u64(p.ll_ptotal);
-        const long long t0 = clock64();
-        while ((v >> 32) != wantP && clock64() - t0 <= kWaitCycles) {
-            __nanosleep(32);
-            v = ld_acquire_u64(p.ll_ptotal);
-        }
-        s_ok = (v >> 32) == wantP;
-        s_present = (int)(v & 0xffffffffu);
-        if (!s_ok) atomicOr(p.err, EP_DEVERR_TIMEOUT);
-    }
-    __syncthreads();
-    const int engines = p.llEngines;
-    if (!s_ok || warp >= engines) return;
-    const int present = s_present, nb = gridDim.x;
-    const EngineSmem es = engine_smem_init(area, p, warp, engines, lane);
-    PlistFeed feed;
-    feed.plist = p.ll_plist;
-    feed.b = t;
-    feed.nb = nb;
-    feed.n = present > t ? (present - 1 - t) / nb + 1 : 0;
-    feed.i = warp;
-    feed.step = engines;
-    feed.tag = tag;
-    copy_engine<1>(p, es, lane, feed, [] { return true; });
-}
-
 // =====================================================================
-// dispatch_local: the whole dispatch of a small batch in one launch. Block b
+// dispatch_fused: the whole dispatch of a small batch in one launch. Block b
 // owns the tokens [lo, hi) of an even, contiguous split of the batch (every
 // block owns at least one), routes them and copies them itself:
 //   1. the chunks of 32 tokens holding own tokens: destination masks (shared
@@ -1275,14 +982,14 @@ __global__ void __launch_bounds__(kLlThreads, 1) ep_dispatch_ll_kernel(ScatterPa
 //      shared-memory counter: per token its routing row and meta records (and
 //      scale rows), then the row's bulk stores.
 // A block's word q holds its totals at destinations 6q .. 6q+5 (8 bits each:
-// a block owns at most kLocalMaxOwn < 256 tokens) under a 16-bit tag, so that
+// a block owns at most kFusedMaxOwn < 256 tokens) under a 16-bit tag, so that
 // one 64-bit load brings a count and the proof that it is this call's. The
 // epoch advances once every block has read it (the last block to get past
 // its look-back), so replays of a captured graph stay in step.
-// Shared memory: the routing area (LocalLayout) at 0, the copy engines'
+// Shared memory: the routing area (FusedLayout) at 0, the copy engines'
 // barriers and stages at engineOffset.
 // =====================================================================
-constexpr int kLocalPerWord = 6;
+constexpr int kFusedPerWord = 6;
 
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
     unsigned long long v;
@@ -1297,7 +1004,7 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
 // Destination mask of token g from its ids (ids outside [0, E) are masked;
 // `bad` reports ids >= E). All k loads are issued before any is used.
 template <int kK>
-__device__ __forceinline__ uint32_t local_mask(const ScatterParams& p, int g, bool& bad) {
+__device__ __forceinline__ uint32_t token_dest_mask(const ScatterParams& p, int g, bool& bad) {
     const int32_t* ids = p.idx + (size_t)g * p.k;
     int e[kK];
 #pragma unroll
@@ -1312,7 +1019,7 @@ __device__ __forceinline__ uint32_t local_mask(const ScatterParams& p, int g, bo
 }
 
 // The own tokens' feed: list entry i (a present own token) is handle i.
-struct LocalFeed {
+struct OwnFeed {
     const int* list;  // present own tokens, ascending
     int* ctr;         // next entry to hand out (shared memory)
     const int* slot;  // [own][W]: slot of own token g - lo at each destination
@@ -1357,7 +1064,7 @@ struct LocalFeed {
 };
 
 template <int kW, int kK>
-__global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(ScatterParams p) {
+__global__ void __launch_bounds__(kFusedWarps * 32, 1) ep_dispatch_fused_kernel(ScatterParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_base[kW];
     __shared__ unsigned s_tag;
@@ -1365,17 +1072,17 @@ __global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(
     const int G = p.G, W = p.W, b = blockIdx.x;
     const int lo = (int)((long long)b * G / gridDim.x);
     const int hi = (int)((long long)(b + 1) * G / gridDim.x);  // > lo: the grid has at most G blocks
-    const LocalLayout L = local_layout(p.localOwn, W, nwarps);
+    const FusedLayout L = fused_layout(p.fusedOwn, W, nwarps);
     uint32_t* cmask = reinterpret_cast<uint32_t*>(smem + L.cmask);
     int* ccnt = reinterpret_cast<int*>(smem + L.ccnt);
     int* slot = reinterpret_cast<int*>(smem + L.slot);
     int* list = reinterpret_cast<int*>(smem + L.list);
     int* ctr = reinterpret_cast<int*>(smem + L.ctr);
     const int c_lo = lo >> 5, nch = ((hi + 31) >> 5) - c_lo;
-    const int nw = (W + kLocalPerWord - 1) / kLocalPerWord;  // words per block
+    const int nw = (W + kFusedPerWord - 1) / kFusedPerWord;  // words per block
 
     pdl_wait();  // the ids, x and the previous call's words are visible from here on
-    if (tid == 0) s_tag = ((__ldcg(p.local_epoch) << 1) | 1u) & 0xffffu;
+    if (tid == 0) s_tag = ((__ldcg(p.fused_epoch) << 1) | 1u) & 0xffffu;
     if (tid < kW) s_base[tid] = 0;
 
     // 1. Masks of the own chunks' tokens; own tokens per chunk and destination.
@@ -1383,7 +1090,7 @@ __global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(
         const int g = (c_lo + i) * 32 + lane;
         const bool own = g >= lo && g < hi;
         bool bad = false;
-        const uint32_t m = own ? local_mask<kK>(p, g, bad) : 0u;
+        const uint32_t m = own ? token_dest_mask<kK>(p, g, bad) : 0u;
         if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
         cmask[i * 32 + lane] = m;
 #pragma unroll
@@ -1405,11 +1112,11 @@ __global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(
         for (int q = 0; q < nw; ++q) {
             unsigned long long v = tag;
 #pragma unroll
-            for (int u = 0; u < kLocalPerWord; ++u) {
-                const int c = __shfl_sync(kFull, tot, (q * kLocalPerWord + u) & 31);
-                if (q * kLocalPerWord + u < W) v |= (unsigned long long)c << (16 + 8 * u);
+            for (int u = 0; u < kFusedPerWord; ++u) {
+                const int c = __shfl_sync(kFull, tot, (q * kFusedPerWord + u) & 31);
+                if (q * kFusedPerWord + u < W) v |= (unsigned long long)c << (16 + 8 * u);
             }
-            if (lane == 0) st_relaxed_u64(p.local_agg + (size_t)b * nw + q, v);
+            if (lane == 0) st_relaxed_u64(p.fused_agg + (size_t)b * nw + q, v);
         }
         if (hi == G && lane < W) ctr[2 + lane] = tot;  // the last block's own totals, for recv_count
         const int own = hi - lo, off = lo - c_lo * 32;
@@ -1439,7 +1146,7 @@ __global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int i = i0 + u * blockDim.x + tid;
-                v[u] = i < words ? ld_relaxed_u64(p.local_agg + i) : 0ull;
+                v[u] = i < words ? ld_relaxed_u64(p.fused_agg + i) : 0ull;
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -1453,23 +1160,23 @@ __global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(
                             break;
                         }
                         __nanosleep(32);
-                        v[u] = ld_relaxed_u64(p.local_agg + i);
+                        v[u] = ld_relaxed_u64(p.fused_agg + i);
                     } while ((unsigned)(v[u] & 0xffffu) != want);
                     if (!ok) break;
                 }
                 const int q = i % nw;
 #pragma unroll
-                for (int c = 0; c < kLocalPerWord; ++c) {
-                    const int pe = q * kLocalPerWord + c;
+                for (int c = 0; c < kFusedPerWord; ++c) {
+                    const int pe = q * kFusedPerWord + c;
                     const int n = (int)((v[u] >> (16 + 8 * c)) & 0xffu);
                     if (pe < W && n != 0) atomicAdd(&s_base[pe], n);
                 }
             }
             if (!ok) break;
         }
-        if (tid == 0 && atomicAdd(p.local_done, 1u) == gridDim.x - 1) {
-            *p.local_done = 0u;  // every block has read the epoch: the next call's
-            atomicAdd(p.local_epoch, 1u);
+        if (tid == 0 && atomicAdd(p.fused_done, 1u) == gridDim.x - 1) {
+            *p.fused_done = 0u;  // every block has read the epoch: the next call's
+            atomicAdd(p.fused_epoch, 1u);
         }
         if (!__syncthreads_and(ok)) {
             if (tid == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
@@ -1518,10 +1225,10 @@ __global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(
         return true;
     };
 
-    const int engines = p.localEngines;
+    const int engines = p.fusedEngines;
     if (warp < engines) {
         const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, engines, lane);
-        LocalFeed feed;
+        OwnFeed feed;
         feed.list = list;
         feed.ctr = ctr + 1;
         feed.slot = slot;
@@ -1530,122 +1237,6 @@ __global__ void __launch_bounds__(kLocalWarps * 32, 1) ep_dispatch_local_kernel(
         copy_engine<1>(p, es, lane, feed, route_rest);
     } else {
         route_rest();
-    }
-}
-
-// =====================================================================
-// dispatch_fused: route, scan and scatter in one cooperative launch (an
-// option, EP_DISPATCH_FUSED=1: on B200 it measured slower than route_count +
-// scatter_rows, since ~300 copy-engine warps route the tokens instead of
-// route_count's thousand, and two grid barriers and a one-warp-per-destination
-// scan cost more than the launch they save).
-//   1. every warp routes 32-token chunks: destination masks, weight sums,
-//      chunk-local ranks and chunk counts by ballot;
-//   2. grid barrier; warps scan the chunk counts, one destination each, into
-//      chunk bases and store recv_count;
-//   3. grid barrier; the copy engines run as in scatter_rows.
-// The barriers spin on a global counter with a bound; a cooperative launch
-// keeps every block resident, so they complete. The last block to finish
-// resets the counters for the next call.
-// =====================================================================
-__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned target) {
-    __threadfence();  // every thread's writes of this phase, before the arrival
-    __syncthreads();
-    int ok = 1;
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(bar, 1u);
-        const long long t0 = clock64();
-        for (;;) {
-            unsigned v;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-            if (v >= target) break;
-            if (clock64() - t0 > kWaitCycles) {
-                ok = 0;
-                break;
-            }
-            __nanosleep(64);
-        }
-        __threadfence();
-    }
-    return __syncthreads_and(ok) != 0;
-}
-
-template <int kW, int kK>
-__global__ void __launch_bounds__(kMaxScatterWarps * 32) ep_dispatch_fused_kernel(ScatterParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const int gw = blockIdx.x * nwarps + warp, nW = gridDim.x * nwarps;
-    const int W = p.W;
-    const EngineSmem es = engine_smem_init(smem, p, warp, nwarps, lane);
-    pdl_wait();  // the ids may come from the previous kernel of the stream
-    dest_setup(p);
-
-    // 1. route 32-token chunks
-    const uint32_t lt = lanemask_lt();
-    for (int c = gw; c < p.numChunks32; c += nW) {
-        const int g = c * 32 + lane;
-        uint32_t mask = 0;
-        bool bad = false;
-        float ws[kW];
-        if (g < p.G) mask = route_token<kW, kK>(p.idx, p.w, g, p.k, p.nEpr, p.E, ws, bad);
-        if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
-        if (g < p.G) p.tok_mask_w[g] = mask;
-        int my_cnt = 0;
-#pragma unroll
-        for (int pe = 0; pe < kW; ++pe) {
-            if (pe < W) {
-                const bool hit = (mask >> pe) & 1u;
-                const uint32_t b = __ballot_sync(kFull, hit);
-                if (lane == pe) my_cnt = __popc(b);
-                if (g < p.G) {
-                    const float wsum = hit ? (p.useWeights ? ws[pe] : 1.0f) : 0.0f;
-                    p.route[(size_t)g * W + pe] = make_int2(hit ? __popc(b & lt) : -1, __float_as_int(wsum));
-                }
-            }
-        }
-        if (lane < W) p.chunk_cnt[(size_t)c * W + lane] = my_cnt;
-    }
-
-    bool ok = grid_barrier(p.bar, gridDim.x + p.barrierSlack);
-
-    // 2. one warp per destination scans the chunk counts
-    for (int pe = gw; ok && pe < W; pe += nW) {
-        int running = 0;
-        for (int c0 = 0; c0 < p.numChunks32; c0 += 32) {
-            const int c = c0 + lane;
-            const int v = c < p.numChunks32 ? __ldcg(p.chunk_cnt + (size_t)c * W + pe) : 0;
-            int incl = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int n = __shfl_up_sync(kFull, incl, off);
-                if (lane >= off) incl += n;
-            }
-            if (c < p.numChunks32) p.chunk_base_w[(size_t)c * W + pe] = running + incl - v;
-            running += __shfl_sync(kFull, incl, 31);
-        }
-        if (lane == 0) {
-            p.recv_count[pe] = running;  // stored, not accumulated
-            if (running > p.maxRecv) atomicOr(p.err, EP_DEVERR_CAPACITY);
-        }
-    }
-
-    ok = ok && grid_barrier(p.bar, 2u * gridDim.x + p.barrierSlack);
-
-    // 3. copy engines
-    if (ok) global_copy_engines<1>(p, es, lane, warp, nwarps, p.G, -1, nullptr);
-    else if (threadIdx.x == 0) atomicOr(p.err, EP_DEVERR_TIMEOUT);
-
-    // The last block to finish resets the counters for the next call.
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
-            *p.bar = 0u;
-            *p.work = 0;
-            *p.done = 0u;
-            __threadfence();
-        }
     }
 }
 
@@ -2105,7 +1696,7 @@ cudaError_t launch_scatter_rows(const ScatterParams& p, bool dense, int blocks, 
 
 namespace {
 template <typename F>
-cudaError_t for_world(int W, int k, F&& f) {
+cudaError_t for_world_fused(int W, int k, F&& f) {
     if (W <= 8)
         return k <= 8 ? f(ep_dispatch_fused_kernel<8, 8>) : k <= 16 ? f(ep_dispatch_fused_kernel<8, 16>)
                                                              : f(ep_dispatch_fused_kernel<8, 32>);
@@ -2118,103 +1709,18 @@ cudaError_t for_world(int W, int k, F&& f) {
 }  // namespace
 
 cudaError_t fused_set_smem(int W, int topk, size_t bytes) {
-    return for_world(W, topk, [&](auto k) { return raise_smem(k, bytes); });
+    return for_world_fused(W, topk, [&](auto k) { return raise_smem(k, bytes); });
 }
 
-cudaError_t fused_blocks_per_sm(int W, int topk, int warps, size_t smem, int* out) {
-    return for_world(W, topk, [&](auto k) {
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, warps * 32, smem);
+cudaError_t fused_blocks_per_sm(int W, int topk, size_t smem, int* out) {
+    return for_world_fused(W, topk, [&](auto k) {
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, kFusedWarps * 32, smem);
     });
 }
 
-cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, int warps, size_t smem, cudaStream_t s) {
-    cudaError_t e = for_world(p.W, p.k, [&](auto k) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(blocks);
-        cfg.blockDim = dim3(warps * 32);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, k, p);
-    });
-    return e != cudaSuccess ? e : cudaGetLastError();
-}
-
-namespace {
-template <typename F>
-cudaError_t for_world_ll(int W, int k, F&& f) {
-    if (W <= 8)
-        return k <= 8 ? f(ep_dispatch_ll_kernel<8, 8>) : k <= 16 ? f(ep_dispatch_ll_kernel<8, 16>)
-                                                          : f(ep_dispatch_ll_kernel<8, 32>);
-    if (W <= 16)
-        return k <= 8 ? f(ep_dispatch_ll_kernel<16, 8>) : k <= 16 ? f(ep_dispatch_ll_kernel<16, 16>)
-                                                           : f(ep_dispatch_ll_kernel<16, 32>);
-    return k <= 8 ? f(ep_dispatch_ll_kernel<32, 8>) : k <= 16 ? f(ep_dispatch_ll_kernel<32, 16>)
-                                                       : f(ep_dispatch_ll_kernel<32, 32>);
-}
-}  // namespace
-
-int ll_tile_tokens(long long G, int blocks) {
-    // Tokens per tile: the batch spread over `blocks` blocks, at least enough
-    // that there are no more than kLlMaxTiles tiles.
-    long long tt = (G + blocks - 1) / blocks;
-    const long long minTt = (G + kLlMaxTiles - 1) / kLlMaxTiles;
-    if (tt < minTt) tt = minTt;
-    if (tt < 1) tt = 1;
-    return (int)tt;
-}
-
-size_t ll_smem_bytes(int tileTokens, int W, int warps, int stages, int chunkStride) {
-    const size_t list = ((size_t)tileTokens * (size_t)W * sizeof(int) + 127) & ~(size_t)127;
-    return list + scatter_smem_bytes(warps, stages, chunkStride);
-}
-
-cudaError_t ll_set_smem(int W, int topk, size_t bytes) {
-    return for_world_ll(W, topk, [&](auto k) { return raise_smem(k, bytes); });
-}
-
-cudaError_t ll_blocks_per_sm(int W, int topk, size_t smem, int* out) {
-    return for_world_ll(W, topk, [&](auto k) {
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, kLlThreads, smem);
-    });
-}
-
-cudaError_t launch_dispatch_ll(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s) {
-    cudaError_t e = for_world_ll(p.W, p.k, [&](auto k) { return launch_pdl(k, blocks, kLlThreads, smem, s, p); });
-    return e != cudaSuccess ? e : cudaGetLastError();
-}
-
-namespace {
-template <typename F>
-cudaError_t for_world_local(int W, int k, F&& f) {
-    if (W <= 8)
-        return k <= 8 ? f(ep_dispatch_local_kernel<8, 8>) : k <= 16 ? f(ep_dispatch_local_kernel<8, 16>)
-                                                             : f(ep_dispatch_local_kernel<8, 32>);
-    if (W <= 16)
-        return k <= 8 ? f(ep_dispatch_local_kernel<16, 8>) : k <= 16 ? f(ep_dispatch_local_kernel<16, 16>)
-                                                              : f(ep_dispatch_local_kernel<16, 32>);
-    return k <= 8 ? f(ep_dispatch_local_kernel<32, 8>) : k <= 16 ? f(ep_dispatch_local_kernel<32, 16>)
-                                                          : f(ep_dispatch_local_kernel<32, 32>);
-}
-}  // namespace
-
-cudaError_t local_set_smem(int W, int topk, size_t bytes) {
-    return for_world_local(W, topk, [&](auto k) { return raise_smem(k, bytes); });
-}
-
-cudaError_t local_blocks_per_sm(int W, int topk, size_t smem, int* out) {
-    return for_world_local(W, topk, [&](auto k) {
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, k, kLocalWarps * 32, smem);
-    });
-}
-
-cudaError_t launch_dispatch_local(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s) {
+cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, size_t smem, cudaStream_t s) {
     cudaError_t e =
-        for_world_local(p.W, p.k, [&](auto k) { return launch_pdl(k, blocks, kLocalWarps * 32, smem, s, p); });
+        for_world_fused(p.W, p.k, [&](auto k) { return launch_pdl(k, blocks, kFusedWarps * 32, smem, s, p); });
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -96,16 +96,13 @@ typedef struct EpPlanInfo {
     int64_t combineRowBytes;  /* bytes of a y / out row */
     int64_t yBytes;           /* bytes of y: W*maxRecv*combineRowBytes */
     int64_t outBytes;         /* bytes of out: W*T*combineRowBytes */
-    int32_t dispatchFused;    /* 1: dispatch is one cooperative launch (route, scan, scatter);
-                                 0: two launches (route_count, scatter_rows) */
-    int32_t dispatchLowLatency; /* 1: dispatch is the small-batch single launch: each block
-                                 routes one tile of tokens (scatterBlocks tiles), adds up the
-                                 counts that earlier tiles publish, writes its tokens' slots
-                                 and records, and copies every scatterBlocks-th present token.
-                                 Taken when maxTokPerRank <= EP_LL_MAX_TOKENS (0, i.e. off,
-                                 by default; the design page's internode dispatch switches
-                                 to its low-latency family at 512 tokens a launch, §9).
-                                 Results are identical either way. */
+    int32_t dispatchFused;    /* 1: dispatch is one launch (EP_DISPATCH_FUSED=1, where every
+                                 block owns at most 64 tokens): block b routes its own
+                                 contiguous share of the W*T tokens (scatterBlocks blocks),
+                                 publishes its per-destination totals, adds up the earlier
+                                 blocks' totals (decoupled look-back, a bounded wait) and
+                                 copies its own tokens; 0: two launches (route_count,
+                                 scatter_rows). Results are identical either way. */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
@@ -141,7 +138,7 @@ int ep_cfg_check(const EpCfg* cfg);
 
 /* Host-only sizing: fill *info for cfg as a plan on a generic device would
  * resolve it (device = -1, numSMs = 0, geometry from a 148-SM B200 without
- * the geometry overrides; EP_LL_MAX_TOKENS is honoured). Lets a
+ * the geometry overrides; EP_DISPATCH_FUSED is honoured). Lets a
  * caller size recv_x / recv_meta before creating a plan. Returns EP_OK or a
  * negative code. */
 int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
@@ -152,21 +149,19 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * ticket, the error word). Returns NULL on failure (ep_last_error() says why).
  * Environment overrides, read here only (for geometry sweeps):
  * EP_SCATTER_BLOCKS, EP_SCATTER_WARPS, EP_SCATTER_STAGES, EP_SCATTER_CHUNK, EP_COMBINE_BLOCKS,
- * EP_COMBINE_WARPS, EP_DISPATCH_FUSED (1: one cooperative launch instead of
- * two), EP_LL_MAX_TOKENS (largest maxTokPerRank that takes the low-latency
- * dispatch; 0, i.e. off, by default), EP_SCATTER_FANOUT_SWITCH (100 x
+ * EP_COMBINE_WARPS, EP_DISPATCH_FUSED (1: the one-launch dispatch of
+ * dispatchFused, where every block owns at most 64 tokens; off by default),
+ * EP_SCATTER_FANOUT_SWITCH (100 x
  * the mean fan-out above which one copy engine per block sits out; 375 by
  * default, 0 never), EP_SCATTER_SCAN ("route": route_count's last block scans
  * the tile counts even when the scatter could), EP_DISPATCH_DENSE (1 / 0: the
  * large-batch form of the split dispatch for every plan / for none; by default
  * plans of more than 16384 tokens, W*T, take it). Test hooks:
- * EP_TEST_UNREACHABLE_BARRIER=1 makes the fused dispatch's grid barrier (with
- * EP_DISPATCH_FUSED=1), or the low-latency
- * dispatch's wait for the counts of earlier tiles, unreachable, so that the
- * bounded wait runs out: the waiting blocks report EP_DEVERR_TIMEOUT, issue no
- * copy and return about one second later (the low-latency dispatch's first
- * tile waits on nothing and writes its meta records before it gives up), and
- * the context stays usable; EP_TEST_BOUNDS_ROWS=n makes the bounds-checking
+ * EP_TEST_UNREACHABLE_BARRIER=1 makes the one-launch dispatch's wait for the
+ * earlier blocks' totals unreachable, so that the bounded wait runs out: every
+ * block but the first (which waits on nothing and copies its own tokens)
+ * reports EP_DEVERR_TIMEOUT, copies nothing and returns about one second
+ * later, and the context stays usable; EP_TEST_BOUNDS_ROWS=n makes the bounds-checking
  * build (libep_b200_debug.so) check the receive buffers against n rows per
  * destination instead of maxRecv. */
 EpPlan* ep_plan_create(const EpCfg* cfg);

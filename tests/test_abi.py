@@ -148,33 +148,35 @@ def test_plan_query_dtype_legs(ep, dtype, h, row, chid, crow, cdt):
     assert info.yBytes == 8 * 32768 * crow and info.outBytes == 8 * 4096 * crow
 
 
-@pytest.mark.parametrize("kw,ll", [
-    (dict(), 0),                                                       # main shape: 4096 tokens a rank
-    (dict(maxTokPerRank=512, maxRecv=0), 1),                           # 512 tokens a rank: low latency
-    (dict(maxTokPerRank=513, maxRecv=0), 0),                           # above the switch
+@pytest.mark.parametrize("kw,fused", [
+    (dict(), 0),                                                       # main shape: 222 tokens a block
+    (dict(maxTokPerRank=512, maxRecv=0), 1),                           # 4096 tokens: 28 a block
+    (dict(maxTokPerRank=513, maxRecv=0), 1),
     (dict(worldSize=4, maxTokPerRank=512, numExpertPerRank=8, numExpertPerToken=6, maxRecv=0), 1),
     (dict(maxTokPerRank=512, numExpertPerToken=32, maxRecv=0), 1),     # topk 32
-    (dict(worldSize=32, maxTokPerRank=512, numExpertPerToken=8, maxRecv=0), 1),  # 16384 tokens: 111 a block
-    (dict(maxTokPerRank=1, maxRecv=0), 1),
+    (dict(worldSize=32, maxTokPerRank=512, numExpertPerToken=8, maxRecv=0), 0),  # 16384 tokens: 111 a block
+    (dict(maxTokPerRank=1, maxRecv=0), 1),                             # 8 tokens: 8 blocks of one
     (dict(maxTokPerRank=512, maxRecv=0, dtype=1), 1),                  # fp32 rows of 28672 bytes
     (dict(maxTokPerRank=512, maxRecv=0, hiddenDim=100000), 1),         # rows copied in pieces
 ])
-def test_plan_query_dispatch_family(ep, kw, ll, monkeypatch):
-    """With EP_LL_MAX_TOKENS=512, plans of at most 512 tokens a rank take the
-    single-launch low-latency dispatch; the rest take route_count +
-    scatter_rows. Both give identical results. By default the low-latency
-    dispatch is off."""
-    assert ep.ep_plan_query(_cfg(**kw)).dispatchLowLatency == 0
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", "512")
+def test_plan_query_dispatch_form(ep, kw, fused, monkeypatch):
+    """With EP_DISPATCH_FUSED=1, plans where no block owns more than 64 tokens
+    take the one-launch fused dispatch (a grid of at most one block a token);
+    the rest take route_count + scatter_rows. Both give identical results. By
+    default the fused dispatch is off."""
+    assert ep.ep_plan_query(_cfg(**kw)).dispatchFused == 0
+    plain = ep.ep_plan_query(_cfg(**kw))
+    monkeypatch.setenv("EP_DISPATCH_FUSED", "1")
     cfg = _cfg(**kw)
     info = ep.ep_plan_query(cfg)
-    assert info.dispatchLowLatency == ll
-    assert info.dispatchFused == 0
-    if ll:
-        G = cfg["worldSize"] * cfg["maxTokPerRank"]
-        tile = -(-G // 148)
-        assert info.scatterBlocks == -(-G // tile) <= 148
-        assert info.scatterStages >= 2
+    assert info.dispatchFused == fused
+    G = cfg["worldSize"] * cfg["maxTokPerRank"]
+    if fused:
+        assert info.scatterBlocks == min(plain.scatterBlocks, G)
+        assert -(-G // info.scatterBlocks) <= 64
+        assert info.scratchBytes > plain.scratchBytes  # the blocks' published totals
+    else:
+        assert info.scatterBlocks == plain.scatterBlocks and info.scratchBytes == plain.scratchBytes
 
 
 def test_entry_points_reject_without_crashing(ep):

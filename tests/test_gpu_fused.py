@@ -1,10 +1,11 @@
-"""dispatch_local (one launch; every block routes the batch up to its own
-tokens) against the CPU oracle, through the C ABI (needs a B200).
+"""The fused dispatch (EP_DISPATCH_FUSED=1: one launch; every block routes
+its own share of the batch, adds up the earlier blocks' published totals and
+copies its own tokens) against the CPU oracle, through the C ABI (needs a
+B200).
 
 The same bar as test_gpu_parity: dispatch bit-exact, rows and records past
 recv_count keep their canaries, combine bit-exact with the oracle's fold.
-EP_LOCAL_MAX_TOKENS raises the size limit so that every case below that the
-per-block token bound admits takes this dispatch.
+Every case below that the per-block token bound admits takes this dispatch.
 """
 import numpy as np
 import pytest
@@ -22,38 +23,38 @@ from gpu_harness import (CANARY_META, DeviceRun, compare_combine, compare_dispat
                          to_dev)
 from synth.inputs import make_inputs, workload  # noqa: E402
 
-LOCAL_MAX_OWN = 64  # tokens a block may own (kLocalMaxOwn)
+FUSED_MAX_OWN = 64  # tokens a block may own (kFusedMaxOwn)
 
 
 @pytest.fixture(autouse=True)
-def _local(monkeypatch):
-    monkeypatch.setenv("EP_LOCAL_MAX_TOKENS", "1000000")
+def _fused(monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_FUSED", "1")
 
 
-def _expect_local(info, G, k=None):
+def _expect_fused(info, G, k=None):
     blocks = info.scatterBlocks
-    if -(-G // min(blocks, G)) <= LOCAL_MAX_OWN:
-        assert info.dispatchLowLatency == 1
+    if -(-G // min(blocks, G)) <= FUSED_MAX_OWN:
+        assert info.dispatchFused == 1
         assert blocks <= G
 
 
 @pytest.mark.parametrize("name", ["tiny", "pr599", "latency1", "latency8"])
-def test_local_workloads(name):
+def test_fused_workloads(name):
     wl = workload(name)
     run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
-    assert run.info.dispatchLowLatency == 1
+    assert run.info.dispatchFused == 1
     run.close()
 
 
 @pytest.mark.parametrize("ct,topk", [(512, 6), (512, 8), (1024, 6), (2048, 8), (1, 6), (8, 6)])
-def test_local_pr599_matrix(ct, topk):
+def test_fused_pr599_matrix(ct, topk):
     """mori PR #599's correctness matrix ("Perf/ep disp 1250 ship",
     correctness section) at the sizes this dispatch takes."""
     max_tok = max(ct, 512)
     wl = workload("pr599").replace(h=2048, ct=ct, max_tok=max_tok, max_recv=4 * max_tok, k=topk,
                                    seed=2000 + ct + topk)
     run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
-    _expect_local(run.info, wl.W * wl.max_tok, wl.k)
+    _expect_fused(run.info, wl.W * wl.max_tok, wl.k)
     run.close()
 
 
@@ -68,7 +69,7 @@ def test_local_pr599_matrix(ct, topk):
     (7, 3, 256, 3, 3, True, 0),         # fewer tokens than blocks
     (16, 100, 512, 16, 3, True, 0),     # topk 16 (second ids instance), nEpr not a power of two
 ])
-def test_local_random(case):
+def test_fused_random(case):
     W, T, h, k, nEpr, use_w, max_recv = case
     rng = np.random.default_rng(hash(case) % (1 << 32))
     E = W * nEpr
@@ -78,21 +79,21 @@ def test_local_random(case):
     cfg = dict(worldSize=W, hiddenDim=h, maxTokPerRank=T, numExpertPerRank=nEpr,
                numExpertPerToken=k, maxRecv=max_recv, dtype=0, useWeights=int(use_w))
     run, _ = run_and_compare(cfg, dict(x=xb, topk_idx=idx, topk_w=w))
-    _expect_local(run.info, W * T, k)
+    _expect_fused(run.info, W * T, k)
     run.close()
 
 
 @pytest.mark.parametrize("dtype", [0, 1, 2, 3], ids=["bf16", "fp32", "fp8", "fp4x2"])
-def test_local_dtype_random_small(dtype):
+def test_fused_dtype_random_small(dtype):
     rng = np.random.default_rng(300 + dtype)
     for _ in range(6):
         cfg, xb, idx, w = P.random_small_case(rng, dtype=dtype)
         run, _ = run_and_compare(cfg, dict(x=xb, topk_idx=idx, topk_w=w))
-        assert run.info.dispatchLowLatency == 1
+        assert run.info.dispatchFused == 1
         run.close()
 
 
-def test_local_scaled():
+def test_fused_scaled():
     """Scale rows travel with the payload (ep_dispatch_scaled)."""
     rng = np.random.default_rng(41)
     for case in range(6):
@@ -102,7 +103,7 @@ def test_local_scaled():
         scales = rng.standard_normal((W, T, sw)).astype(np.float32)
         ref = oracle.dispatch(cfg, xb, idx, w, scales=scales)
         with DeviceRun(cfg, dict(x=xb, topk_idx=idx, topk_w=w)) as run:
-            assert run.info.dispatchLowLatency == 1
+            assert run.info.dispatchFused == 1
             R = run.info.maxRecv
             rs = torch.full((W, R, sw), 0x0C0FFEE, dtype=torch.int32, device="cuda")
             ep.ep_dispatch_scaled(run.plan, run.x, run.idx, run.w, to_dev(scales), sw, run.recv_x,
@@ -117,7 +118,7 @@ def test_local_scaled():
             assert run.error_word() == 0
 
 
-def test_local_out_of_range_ids():
+def test_fused_out_of_range_ids():
     rng = np.random.default_rng(5)
     W, T, k, nEpr = 4, 64, 4, 4
     idx = rng.integers(-2, W * nEpr + 3, size=(W, T, k)).astype(np.int32)
@@ -131,7 +132,7 @@ def test_local_out_of_range_ids():
     run.close()
 
 
-def test_local_empty_call():
+def test_fused_empty_call():
     wl = workload("latency1")
     inputs = make_inputs(wl)
     inputs["topk_idx"][:] = -1
@@ -141,7 +142,7 @@ def test_local_empty_call():
     run.close()
 
 
-def test_local_repeated_calls_and_graph():
+def test_fused_repeated_calls_and_graph():
     """Two routings on one plan, then dispatch + combine captured in a CUDA
     graph and replayed: every replay matches the eager results."""
     wl = workload("pr599").replace(h=512)
@@ -186,20 +187,20 @@ def test_local_repeated_calls_and_graph():
     {"EP_SCATTER_BLOCKS": "40"},                             # 52 tokens a block
     {"EP_SCATTER_BLOCKS": "31"},                             # 67 a block: over the bound, split dispatch
 ])
-def test_local_geometry(env, monkeypatch):
+def test_fused_geometry(env, monkeypatch):
     for k_, v in env.items():
         monkeypatch.setenv(k_, v)
     wl = workload("pr599").replace(h=1536)
     run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
     G = wl.W * wl.max_tok
     if env.get("EP_SCATTER_BLOCKS") == "31":
-        assert run.info.dispatchLowLatency == 0
+        assert run.info.dispatchFused == 0
     else:
-        _expect_local(run.info, G, wl.k)
+        _expect_fused(run.info, G, wl.k)
     run.close()
 
 
-def test_local_lookback_wait_runs_out(monkeypatch):
+def test_fused_lookback_wait_runs_out(monkeypatch):
     """Failure detection without a GPU fault: the test hook makes every block
     wait for a tag that no block publishes. Block 0, which waits on nothing,
     copies its own tokens; every other block gives up after its bounded wait
@@ -209,7 +210,7 @@ def test_local_lookback_wait_runs_out(monkeypatch):
     wl = workload("latency8")
     inputs = make_inputs(wl)
     with DeviceRun(wl.cfg(), inputs) as run:
-        assert run.info.dispatchLowLatency == 1
+        assert run.info.dispatchFused == 1
         run.dispatch()
         err = run.error_word()  # synchronises: the kernel has returned
         assert err & ep.EP_DEVERR_TIMEOUT

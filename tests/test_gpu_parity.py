@@ -19,9 +19,20 @@ if not torch.cuda.is_available():  # pragma: no cover - collected on CPU machines t
 import combine_ep_dispatch_05_b200 as ep  # noqa: E402
 import oracle  # noqa: E402
 import oracle_pins as P  # noqa: E402
-from gpu_harness import (CANARY_META, DeviceRun, compare_combine, compare_dispatch, run_and_compare,  # noqa: E402
+from gpu_harness import (DeviceRun, compare_combine, compare_dispatch, run_and_compare,  # noqa: E402
                          to_dev)
 from synth.inputs import WORKLOADS, make_inputs, workload  # noqa: E402
+
+
+FUSED_MAX_OWN = 64  # tokens a block of the fused dispatch may own (kFusedMaxOwn)
+
+
+def _fused_expected(info, fused, G):
+    """EP_DISPATCH_FUSED=1 takes the one-launch dispatch when no block owns
+    more than FUSED_MAX_OWN tokens."""
+    if fused == "1" and info.dispatchFused:
+        assert -(-G // info.scatterBlocks) <= FUSED_MAX_OWN
+    return fused == "1" and -(-G // min(info.scatterBlocks, G)) <= FUSED_MAX_OWN
 
 
 def test_library_is_in_tree():
@@ -36,25 +47,17 @@ def test_workload_parity(name):
     run.close()
 
 
-@pytest.mark.parametrize("fused", ["0", "1"])
-@pytest.mark.parametrize("name", ["main", "latency8"])
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["split", "fused"])
+@pytest.mark.parametrize("name", ["tiny", "pr599", "latency1", "latency8", "main"])
 def test_workload_parity_both_dispatch_modes(name, fused, monkeypatch):
+    """The workloads through both dispatch forms: route_count + scatter_rows,
+    and the one-launch fused dispatch (which main, at 222 tokens a block, does
+    not take)."""
     monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
     wl = workload(name)
     run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
-    assert run.info.dispatchFused == int(fused)
-    run.close()
-
-
-@pytest.mark.parametrize("ll", ["0", "512"], ids=["split", "lowlat"])
-@pytest.mark.parametrize("name", ["tiny", "pr599", "latency1", "latency8"])
-def test_workload_parity_dispatch_families(name, ll, monkeypatch):
-    """The small workloads through both dispatch families: route_count +
-    scatter_rows, and the single-launch low-latency dispatch."""
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", ll)
-    wl = workload(name)
-    run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
-    assert run.info.dispatchLowLatency == (ll != "0")
+    assert run.info.dispatchFused == _fused_expected(run.info, fused, wl.W * wl.max_tok)
+    assert run.info.dispatchFused == (fused == "1" and name != "main")
     run.close()
 
 
@@ -107,14 +110,14 @@ def _small_random_cfg(rng, W, T, h, k, nEpr, use_w, max_recv=0, dup=True, oob=Fa
     (2, 40, 20000, 3, 4, True, 0),      # 40000-byte rows: copied in three pieces
     (8, 1000, 1024, 6, 8, True, 0),     # 4 tiles, ragged
 ])
-@pytest.mark.parametrize("ll", ["0", "100000"], ids=["split", "lowlat"])
-def test_random_parity(case, ll, monkeypatch):
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", ll)
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["split", "fused"])
+def test_random_parity(case, fused, monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
     W, T, h, k, nEpr, use_w, max_recv = case
     rng = np.random.default_rng(hash(case) % (1 << 32))
     cfg, inputs = _small_random_cfg(rng, W, T, h, k, nEpr, use_w, max_recv)
     run, _ = run_and_compare(cfg, inputs)
-    assert run.info.dispatchLowLatency == (ll != "0")
+    assert run.info.dispatchFused == _fused_expected(run.info, fused, W * T)
     run.close()
 
 
@@ -129,10 +132,10 @@ def test_dtype_parity(dtype, h):
     run.close()
 
 
-@pytest.mark.parametrize("ll", ["0", "512"], ids=["split", "lowlat"])
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["split", "fused"])
 @pytest.mark.parametrize("dtype", [0, 1, 2, 3], ids=["bf16", "fp32", "fp8", "fp4x2"])
-def test_dtype_random_small(dtype, ll, monkeypatch):
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", ll)
+def test_dtype_random_small(dtype, fused, monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
     """Arbitrary payload bits (NaN and inf patterns included for fp32), duplicate
     ids, masked entries, maxRecv above W*T."""
     rng = np.random.default_rng(100 + dtype)
@@ -176,7 +179,7 @@ def _check_scaled(cfg, inputs, sw, seed=7):
         assert run.error_word() == 0
 
 
-@pytest.mark.parametrize("fused", ["0", "1"])
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["split", "fused"])
 @pytest.mark.parametrize("dtype,h,sw", [(2, 7168, 56), (0, 1024, 1), (3, 512, 33)],
                          ids=["fp8-block-scales", "bf16-one-scale", "fp4x2-33-words"])
 def test_dispatch_scaled(dtype, h, sw, fused, monkeypatch):
@@ -186,18 +189,18 @@ def test_dispatch_scaled(dtype, h, sw, fused, monkeypatch):
     _check_scaled(wl.cfg(), make_inputs(wl), sw)
 
 
-@pytest.mark.parametrize("ll", ["0", "512"], ids=["split", "lowlat"])
-def test_dispatch_scaled_random_small(ll, monkeypatch):
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", ll)
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["split", "fused"])
+def test_dispatch_scaled_random_small(fused, monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
     rng = np.random.default_rng(31)
     for case in range(6):
         cfg, xb, idx, w = P.random_small_case(rng, dtype=case % 4)
         _check_scaled(cfg, dict(x=xb, topk_idx=idx, topk_w=w), int(rng.integers(1, 80)), seed=case)
 
 
-@pytest.mark.parametrize("ll", ["0", "512"], ids=["split", "lowlat"])
-def test_out_of_range_ids_reported_and_masked(ll, monkeypatch):
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", ll)
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["split", "fused"])
+def test_out_of_range_ids_reported_and_masked(fused, monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
     rng = np.random.default_rng(5)
     cfg, inputs = _small_random_cfg(rng, 4, 64, 64, 4, 4, True, oob=True)
     assert (inputs["topk_idx"] >= 16).any()
@@ -215,10 +218,10 @@ def test_fma_single_rounding_case():
     run.close()
 
 
-@pytest.mark.parametrize("ll", ["0", "512"], ids=["split", "lowlat"])
-def test_absent_tokens_and_empty_call(ll, monkeypatch):
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["split", "fused"])
+def test_absent_tokens_and_empty_call(fused, monkeypatch):
     """All ids masked: nothing received, zero counts, zero output rows."""
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", ll)
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
     wl = workload("latency1")
     inputs = make_inputs(wl)
     inputs["topk_idx"][:] = -1
@@ -307,17 +310,12 @@ def test_graph_capture_replay():
     {"EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2", "EP_SCATTER_CHUNK": "1024"},
     {"EP_COMBINE_WARPS": "1", "EP_COMBINE_BLOCKS": "3"},
     {"EP_DISPATCH_FUSED": "0"},                              # two launches: route_count + scatter_rows
-    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_BLOCKS": "3"},    # fused, few blocks: long chunk loops
+    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_BLOCKS": "40"},   # fused, 52 tokens a block
     {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "8", "EP_SCATTER_STAGES": "2", "EP_SCATTER_CHUNK": "1024"},
-    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "1", "EP_SCATTER_BLOCKS": "1"},  # fewer warps than W
-    {"EP_LL_MAX_TOKENS": "0"},                               # split dispatch at this size
+    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_WARPS": "1"},    # fused, one engine a block
     {"EP_SCATTER_SCAN": "route"},                            # route_count's last block scans the counts
     {"EP_DISPATCH_DENSE": "1"},                              # route_count's large-batch form
-    {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "4"},   # four tiles of 512 tokens
-    {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "7", "EP_SCATTER_WARPS": "16", "EP_SCATTER_STAGES": "2",
-     "EP_SCATTER_CHUNK": "512"},                             # many engines, rows in six pieces
-    {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_BLOCKS": "2000"},  # capped at 256 tiles of 8 tokens
-    {"EP_LL_MAX_TOKENS": "512", "EP_SCATTER_WARPS": "1"},   # one engine a tile
+    {"EP_DISPATCH_FUSED": "1", "EP_SCATTER_BLOCKS": "7"},    # 293 tokens a block: over the bound, split
 ])
 def test_geometry_overrides(env, monkeypatch):
     for k_, v in env.items():
@@ -325,59 +323,10 @@ def test_geometry_overrides(env, monkeypatch):
     wl = workload("pr599").replace(h=1536)
     run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
     info = run.info
-    if "EP_SCATTER_BLOCKS" in env and not info.dispatchLowLatency:
+    if "EP_SCATTER_BLOCKS" in env:
         assert info.scatterBlocks == int(env["EP_SCATTER_BLOCKS"])
-    if info.dispatchLowLatency:  # one block a tile
-        G = wl.W * wl.max_tok
-        tile = max(-(-G // int(env.get("EP_SCATTER_BLOCKS", info.numSMs))), -(-G // 256))
-        assert info.scatterBlocks == -(-G // tile)
     if "EP_DISPATCH_FUSED" in env:
-        assert info.dispatchFused == int(env["EP_DISPATCH_FUSED"])
-    if "EP_LL_MAX_TOKENS" in env:
-        assert info.dispatchLowLatency == (env["EP_LL_MAX_TOKENS"] != "0")
-    run.close()
-
-
-@pytest.mark.parametrize("family", ["fused", "lowlat"])
-def test_bounded_wait_runs_out_and_reports(family, monkeypatch):
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", "512" if family == "lowlat" else "0")
-    """Failure detection without a GPU fault: a wait that nothing can complete
-    (test hook: the fused dispatch's grid barrier, or the low-latency
-    dispatch's wait for the counts of earlier tiles) makes the waiting blocks
-    give up after their bounded wait; the host reads EP_DEVERR_TIMEOUT from
-    the error word, and the context and a fresh plan keep working."""
-    monkeypatch.setenv("EP_DISPATCH_FUSED", "1" if family == "fused" else "0")
-    monkeypatch.setenv("EP_TEST_UNREACHABLE_BARRIER", "1")
-    wl = workload("latency8")
-    inputs = make_inputs(wl)
-    with DeviceRun(wl.cfg(), inputs) as run:
-        assert run.info.dispatchFused == (family == "fused")
-        assert run.info.dispatchLowLatency == (family == "lowlat")
-        run.dispatch()
-        err = run.error_word()  # synchronises: the kernel has returned
-        assert err & ep.EP_DEVERR_TIMEOUT
-        if family == "fused":
-            assert bool((run.recv_x == 0xAB).all())  # no copy was issued
-        else:
-            # Only the first tile (tokens 0..tile-1, all of source rank 0),
-            # which waits on nothing, got its meta records written: at each
-            # destination they are the oracle's first records, and nothing
-            # lies past them. No row was copied: copies wait for the number of
-            # present tokens, which no block could publish.
-            assert bool((run.recv_x == 0xAB).all())
-            G = wl.W * wl.max_tok
-            tile = -(-G // run.info.numSMs)
-            assert tile <= wl.max_tok
-            ref = oracle.dispatch(wl.cfg(), inputs["x"], inputs["topk_idx"], inputs["topk_w"])
-            meta = run.recv_meta.cpu().numpy()
-            for pe in range(wl.W):
-                n0 = int(((ref["recv_meta"][pe, :, 0] == 0) &
-                          (ref["recv_meta"][pe, :, 1] < tile) &
-                          (np.arange(ref["recv_meta"].shape[1]) < ref["recv_count"][pe])).sum())
-                assert np.array_equal(meta[pe, :n0], ref["recv_meta"][pe, :n0])
-                assert (meta[pe, n0:] == CANARY_META).all()
-    monkeypatch.delenv("EP_TEST_UNREACHABLE_BARRIER")
-    run, _ = run_and_compare(wl.cfg(), inputs)  # the device is healthy
+        assert info.dispatchFused == _fused_expected(info, env["EP_DISPATCH_FUSED"], wl.W * wl.max_tok)
     run.close()
 
 

@@ -41,10 +41,10 @@ def scatter_smem(warps, stages, chunk_stride):
     return head + warps * stages * chunk_stride
 
 
-@pytest.mark.parametrize("ll", ["0", "512"], ids=["default", "single-launch-enabled"])
-def test_random_plan_geometry(ep, ll, monkeypatch):
-    monkeypatch.setenv("EP_LL_MAX_TOKENS", ll)
-    for cfg in random_cfgs(400, 7 + int(ll)):
+@pytest.mark.parametrize("fused", ["0", "1"], ids=["default", "fused-enabled"])
+def test_random_plan_geometry(ep, fused, monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_FUSED", fused)
+    for cfg in random_cfgs(400, 7 + 505 * int(fused)):
         assert ep.ep_cfg_check(cfg) == 0, (cfg, ep.ep_last_error())
         info = ep.ep_plan_query(cfg)
         W, T, k = cfg["worldSize"], cfg["maxTokPerRank"], cfg["numExpertPerToken"]
@@ -60,16 +60,10 @@ def test_random_plan_geometry(ep, ll, monkeypatch):
         assert -(-row // chunk) * chunk >= row
         stride = (chunk + 127) & ~127
         assert info.scatterStages >= 2 and info.scatterWarps >= 1
-        if info.dispatchLowLatency:
-            assert ll == "512" and T <= 512
-            tile = -(-G // 148)
-            tile = max(tile, -(-G // 256))
-            assert tile <= 512
-            assert info.scatterBlocks == -(-G // tile) <= 256
-            lst = (tile * W * 4 + 127) & ~127
-            assert lst + scatter_smem(info.scatterWarps, info.scatterStages, stride) <= SMEM_OPTIN
-        else:
-            assert scatter_smem(info.scatterWarps, info.scatterStages, stride) <= SMEM_OPTIN
+        assert scatter_smem(info.scatterWarps, info.scatterStages, stride) <= SMEM_OPTIN
+        if info.dispatchFused:  # one launch: at most 64 tokens a block, at most one block a token
+            assert fused == "1"
+            assert info.scatterBlocks <= G and -(-G // info.scatterBlocks) <= 64
         # scratch holds at least the routing table and the token masks
         assert info.scratchBytes >= G * W * 8 + G * 4
         # the combine leg
