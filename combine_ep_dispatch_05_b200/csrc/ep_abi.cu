@@ -416,7 +416,18 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
         {
             const long long G = (long long)cfg->worldSize * cfg->maxTokPerRank;
             int blocks = plan->info.scatterBlocks;
-            if (want_fused() && geo.scatterWarps <= ep::kFusedWarps) {
+            // Copy engines: a block's present tokens all go through its own
+            // engines, so where rows are small there are more of them (with at
+            // least 3 stages each, in the split scatter's shared memory),
+            // unless the geometry is set by hand.
+            int fEngines = geo.scatterWarps, fStages = geo.scatterStages;
+            if (!std::getenv("EP_SCATTER_WARPS") && !std::getenv("EP_SCATTER_STAGES")) {
+                const long long budget = (long long)geo.scatterWarps * geo.scatterStages * geo.chunkStride;
+                fEngines = (int)std::max<long long>(geo.scatterWarps,
+                                                    std::min<long long>(ep::kFusedWarps, budget / (3LL * geo.chunkStride)));
+                fStages = (int)std::max<long long>(2, std::min<long long>(8, budget / ((long long)fEngines * geo.chunkStride)));
+            }
+            if (want_fused() && fEngines <= ep::kFusedWarps) {
                 // The grid: the scatter's, at most one block a token, at most
                 // what fits the SMs at once (the routing area may cost a block
                 // per SM, which changes the tokens a block owns: try again).
@@ -425,11 +436,12 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
                 for (int attempt = 0; attempt < 3 && blocks >= 1; ++attempt) {
                     const int own = (int)((G + blocks - 1) / blocks);
                     if (own > ep::kFusedMaxOwn) break;
-                    const size_t area = ep::fused_layout(own, cfg->worldSize, ep::kFusedWarps).total;
-                    int stages = geo.scatterStages;
-                    size_t lsm = area + ep::scatter_smem_bytes(geo.scatterWarps, stages, geo.chunkStride);
+                    const size_t area =
+                        ep::fused_layout(own, cfg->worldSize, ep::kFusedWarps, cfg->numExpertPerToken).total;
+                    int stages = fStages;
+                    size_t lsm = area + ep::scatter_smem_bytes(fEngines, stages, geo.chunkStride);
                     while (lsm > limit && stages > 2)
-                        lsm = area + ep::scatter_smem_bytes(geo.scatterWarps, --stages, geo.chunkStride);
+                        lsm = area + ep::scatter_smem_bytes(fEngines, --stages, geo.chunkStride);
                     if (lsm > limit) break;
                     int per = 0;
                     if ((e = ep::fused_set_smem(cfg->worldSize, cfg->numExpertPerToken, lsm)) != cudaSuccess ||
@@ -450,6 +462,7 @@ EpPlan* ep_plan_create(const EpCfg* cfg) {
                     plan->fusedOwn = own;
                     plan->fusedBlocks = blocks;
                     plan->info.scatterBlocks = blocks;
+                    plan->info.scatterWarps = fEngines;
                     plan->info.scatterStages = stages;
                     break;
                 }

@@ -118,14 +118,15 @@ struct ScatterParams {
 // Byte offsets of dispatch_fused's routing area in shared memory (each
 // 16-byte aligned): masks of the own chunks' tokens [chunks * 32], their own
 // tokens per destination, then bases [chunks][W], the own tokens' slots
-// [own][W], the present own tokens [own], and counters: [0] present own
-// tokens, [1] next one to hand out, [2 + pe] the block's total at pe. own: the
-// most tokens a block owns; its tokens span at most (own + 62) / 32 chunks.
+// [own][W], the present own tokens [own], counters ([0] present own tokens,
+// [1] next one to hand out, [2 + pe] the block's total at pe), and the own
+// tokens' topk ids and weights [own][k] each. own: the most tokens a block
+// owns; its tokens span at most (own + 62) / 32 chunks.
 struct FusedLayout {
-    size_t cmask, ccnt, slot, list, ctr, total;
+    size_t cmask, ccnt, slot, list, ctr, ids, wts, total;
 };
 __host__ __device__ inline size_t fused_up16(size_t n) { return (n + 15) & ~(size_t)15; }
-__host__ __device__ inline FusedLayout fused_layout(int own, int W, int warps) {
+__host__ __device__ inline FusedLayout fused_layout(int own, int W, int warps, int k) {
     (void)warps;
     const size_t chunks = (size_t)(own + 62) / 32;
     FusedLayout L;
@@ -134,7 +135,9 @@ __host__ __device__ inline FusedLayout fused_layout(int own, int W, int warps) {
     L.slot = L.ccnt + fused_up16(chunks * (size_t)W * 4);
     L.list = L.slot + fused_up16((size_t)own * W * 4);
     L.ctr = L.list + fused_up16((size_t)own * 4);
-    L.total = (L.ctr + (2 + kMaxWorld) * 4 + 127) & ~(size_t)127;
+    L.ids = L.ctr + fused_up16((2 + kMaxWorld) * 4);
+    L.wts = L.ids + fused_up16((size_t)own * k * 4);
+    L.total = (L.wts + (size_t)own * k * 4 + 127) & ~(size_t)127;
     return L;
 }
 

@@ -1002,16 +1002,27 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
 }
 
 // Destination mask of token g from its ids (ids outside [0, E) are masked;
-// `bad` reports ids >= E). All k loads are issued before any is used.
+// `bad` reports ids >= E); its k ids and weights (0 without weights) are also
+// kept in sid / sw for the copy engines. All loads are issued before any is
+// used.
 template <int kK>
-__device__ __forceinline__ uint32_t token_dest_mask(const ScatterParams& p, int g, bool& bad) {
+__device__ __forceinline__ uint32_t token_dest_mask(const ScatterParams& p, int g, bool& bad, int* sid, float* sw) {
     const int32_t* ids = p.idx + (size_t)g * p.k;
+    const float* wts = p.w != nullptr ? p.w + (size_t)g * p.k : nullptr;
     int e[kK];
+    float w[kK];
 #pragma unroll
-    for (int j = 0; j < kK; ++j) e[j] = j < p.k ? ids[j] : -1;
+    for (int j = 0; j < kK; ++j) {
+        e[j] = j < p.k ? ids[j] : -1;
+        w[j] = (j < p.k && wts != nullptr) ? wts[j] : 0.0f;
+    }
     uint32_t m = 0;
 #pragma unroll
     for (int j = 0; j < kK; ++j) {
+        if (j < p.k) {
+            sid[j] = e[j];
+            sw[j] = w[j];
+        }
         if (e[j] >= p.E) bad = true;
         if (e[j] >= 0 && e[j] < p.E) m |= 1u << dest_pe(e[j], p.nEpr, p.nEprShift);
     }
@@ -1023,6 +1034,8 @@ struct OwnFeed {
     const int* list;  // present own tokens, ascending
     int* ctr;         // next entry to hand out (shared memory)
     const int* slot;  // [own][W]: slot of own token g - lo at each destination
+    const int* ids;   // [own][k]: its topk ids, and weights
+    const float* wts;
     int n, lo;
 
     __device__ __forceinline__ int next(const ScatterParams& p, int lane) {
@@ -1038,8 +1051,8 @@ struct OwnFeed {
         in.g = list[h];
         in.rr = make_int2(lane < p.W ? slot[(in.g - lo) * p.W + lane] : -1, 0);
         in.base = 0;
-        in.e = lane < p.k ? p.idx[(size_t)in.g * p.k + lane] : -1;
-        in.wt = (lane < p.k && p.w != nullptr) ? p.w[(size_t)in.g * p.k + lane] : 0.0f;
+        in.e = lane < p.k ? ids[(in.g - lo) * p.k + lane] : -1;
+        in.wt = lane < p.k ? wts[(in.g - lo) * p.k + lane] : 0.0f;
         return in;
     }
     // Lane pe: the token's weight sum at pe (float32, topk order), its routing
@@ -1072,12 +1085,14 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) ep_dispatch_fused_kernel(
     const int G = p.G, W = p.W, b = blockIdx.x;
     const int lo = (int)((long long)b * G / gridDim.x);
     const int hi = (int)((long long)(b + 1) * G / gridDim.x);  // > lo: the grid has at most G blocks
-    const FusedLayout L = fused_layout(p.fusedOwn, W, nwarps);
+    const FusedLayout L = fused_layout(p.fusedOwn, W, nwarps, p.k);
     uint32_t* cmask = reinterpret_cast<uint32_t*>(smem + L.cmask);
     int* ccnt = reinterpret_cast<int*>(smem + L.ccnt);
     int* slot = reinterpret_cast<int*>(smem + L.slot);
     int* list = reinterpret_cast<int*>(smem + L.list);
     int* ctr = reinterpret_cast<int*>(smem + L.ctr);
+    int* sids = reinterpret_cast<int*>(smem + L.ids);
+    float* swts = reinterpret_cast<float*>(smem + L.wts);
     const int c_lo = lo >> 5, nch = ((hi + 31) >> 5) - c_lo;
     const int nw = (W + kFusedPerWord - 1) / kFusedPerWord;  // words per block
 
@@ -1090,7 +1105,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) ep_dispatch_fused_kernel(
         const int g = (c_lo + i) * 32 + lane;
         const bool own = g >= lo && g < hi;
         bool bad = false;
-        const uint32_t m = own ? token_dest_mask<kK>(p, g, bad) : 0u;
+        const uint32_t m = own ? token_dest_mask<kK>(p, g, bad, sids + (g - lo) * p.k, swts + (g - lo) * p.k) : 0u;
         if (bad) atomicOr(p.err, EP_DEVERR_EXPERT_RANGE);
         cmask[i * 32 + lane] = m;
 #pragma unroll
@@ -1232,6 +1247,8 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) ep_dispatch_fused_kernel(
         feed.list = list;
         feed.ctr = ctr + 1;
         feed.slot = slot;
+        feed.ids = sids;
+        feed.wts = swts;
         feed.n = ctr[0];
         feed.lo = lo;
         copy_engine<1>(p, es, lane, feed, route_rest);
