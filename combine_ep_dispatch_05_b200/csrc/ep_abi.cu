@@ -655,6 +655,10 @@ static int dispatch_impl(EpPlan* plan, const void* x, const int32_t* topk_idx, c
             sp.fused_epoch = plan->fused_epoch;
             sp.fused_done = plan->fused_done;
             sp.barrierSlack = plan->barrierSlack;
+            // One row load per copy engine before the look-back: B200, one run at the
+            // 512-token workload, none 27.7 us, one 27.1, two 28.8, all (three) 28.7:
+            // more rows in flight delay the look-back's loads behind them.
+            sp.earlyIssue = 1;
             e = ep::launch_dispatch_fused(sp, plan->fusedBlocks, plan->fusedSmem, s);
             if (e != cudaSuccess) return cuda_fail(e, "launch dispatch_fused");
             plan->dispatched = true;

@@ -99,6 +99,7 @@ struct ScatterParams {
     const int32_t* counts;   // this rank's count table [W][W], complete (after the exchange)
     int32_t* recv_total;     // rows this rank receives, stored by block 0
     int boundsRows;          // bounds-checking build: rows of each destination's buffers (maxRecv)
+    int earlyIssue;          // row loads a copy engine issues before its ready hook: 0 all, n > 0 at most n, < 0 none
     // Only dispatch_fused uses these, and the fields below:
     const float* w;          // [G][k] or nullptr
     int32_t* recv_count;     // [W]

@@ -795,11 +795,15 @@ __device__ __forceinline__ void copy_engine(const ScatterParams& p, const Engine
     };
 
     const int lookahead = S - kPend;
-    for (int i = 0; i < lookahead && pg < p.G; ++i) issue();
+    // Loads issued before the ready hook: the whole lookahead, unless the
+    // kernel caps them (earlyIssue > 0: at most that many; < 0: none).
+    const int early = p.earlyIssue == 0 ? lookahead : min(lookahead, max(p.earlyIssue, 0));
+    for (int i = 0; i < early && pg < p.G; ++i) issue();
     if (!ready()) {
         ok = false;
         pg = p.G;
     }
+    while (ok && issued < lookahead && pg < p.G) issue();
 
     // Per-token state kept across the chunks of one token.
     TokenInputs pre;
@@ -966,11 +970,12 @@ __device__ __forceinline__ int dest_pe(int e, int nEpr, int shift) { return shif
 // block owns at least one), routes them and copies them itself:
 //   1. the chunks of 32 tokens holding own tokens: destination masks (shared
 //      memory) and, per chunk and destination, the own tokens that go there;
-//      the present own tokens form a list;
+//      the own tokens' ids and weights (shared memory); the present own
+//      tokens form a list;
 //   2. the block publishes its totals per destination in words tagged with
 //      the call's epoch (decoupled look-back, as in single-pass prefix
-//      scans); the copy-engine warps issue the row loads of the first present
-//      own tokens;
+//      scans); each copy-engine warp issues the row load of its first present
+//      own token;
 //   3. every thread adds up a share of the earlier blocks' words, each loaded
 //      once its tag shows this call (a bounded wait: blocks publish before
 //      they wait and wait only on lower-numbered ones, so the waits end), into
@@ -1240,9 +1245,10 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 1) ep_dispatch_fused_kernel(
         return true;
     };
 
-    const int engines = p.fusedEngines;
-    if (warp < engines) {
-        const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, engines, lane);
+    // 4. The copies: each engine issues its first row load (p.earlyIssue) before
+    // it joins the look-back, the rest once the slots are known.
+    if (warp < p.fusedEngines) {
+        const EngineSmem es = engine_smem_init(smem + p.engineOffset, p, warp, p.fusedEngines, lane);
         OwnFeed feed;
         feed.list = list;
         feed.ctr = ctr + 1;
