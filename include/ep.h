@@ -102,7 +102,10 @@ typedef struct EpPlanInfo {
                                  publishes its per-destination totals, adds up the earlier
                                  blocks' totals (decoupled look-back, a bounded wait) and
                                  copies its own tokens; 0: two launches (route_count,
-                                 scatter_rows). Results are identical either way. */
+                                 scatter_rows). Results are identical either way. The
+                                 one-launch form suits full batches: where only the first
+                                 tokens of each rank are live, a few blocks do all the
+                                 copies. */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
