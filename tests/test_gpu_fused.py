@@ -68,6 +68,7 @@ def test_fused_pr599_matrix(ct, topk):
     (8, 1000, 1024, 6, 8, True, 0),     # 55 tokens a block
     (7, 3, 256, 3, 3, True, 0),         # fewer tokens than blocks
     (16, 100, 512, 16, 3, True, 0),     # topk 16 (second ids instance), nEpr not a power of two
+    (32, 296, 64, 32, 1, True, 0),      # 9472 tokens: 64 a block, W = k = 32, the largest routing area
 ])
 def test_fused_random(case):
     W, T, h, k, nEpr, use_w, max_recv = case
