@@ -154,15 +154,24 @@ Geometry pick_geometry(const EpCfg* c, bool use_env) {
     g.chunkStride = (chunk + 127) & ~127;
     g.numChunks = (int)((rowBytes + chunk - 1) / chunk);
     // Rows of 8 KB and more: one block per SM of about 215 KB, with a third
-    // engine that sits out at a high fan-out (see copy_engine). Smaller rows:
-    // two engines per block and two blocks per SM, each within about 110 KB
-    // (an SM has 228 KB, and each block also holds its static shared memory
-    // and 1 KB the system keeps). B200, fp8 rows of 7 KB at the main workload:
-    // 8 stages left one block per SM once the static shared memory grew
-    // (419 us), 7 stages keep two (245 us).
+    // engine that sits out at a high fan-out (see copy_engine). Rows between
+    // 4 and 8 KB: two engines per block and two blocks per SM, each within
+    // about 110 KB (an SM has 228 KB, and each block also holds its static
+    // shared memory and 1 KB the system keeps). B200, fp8 rows of 7 KB at the
+    // main workload: 8 stages left one block per SM once the static shared
+    // memory grew (419 us), 7 stages keep two (245 us); 3 x 4, 3 x 5 and 2 x 6
+    // measured 246-248 us. Rows of at most 4 KB: three engines of 5 stages, as
+    // many blocks as fit an SM (per-token work weighs more against small rows):
+    // fp4x2 rows of 3.5 KB at the main workload 135.4 vs 160.9 us with 2 x 8
+    // (5 x 5 136.3, 4 x 5 142.1, 8 x 3 144.9), the ct = 1 workload's 4 KB rows
+    // 14.3 vs 15.3 us.
     int warps = g.chunkStride >= 8192 ? 3 : 2;
     const int budget = 215 * 1024;
     int stages = (warps == 3 ? budget : 110 * 1024) / (warps * g.chunkStride);
+    if (g.chunkStride <= 4096) {
+        warps = 3;
+        stages = 5;
+    }
     if (stages < 4) {
         warps = 2;
         stages = budget / (warps * g.chunkStride);

@@ -245,11 +245,13 @@ def test_noalloc_rejects_misaligned_buffers_before_any_launch(ep, which):
     assert "aligned" in ep.ep_last_error()
 
 
-@pytest.mark.parametrize("dtype,h,blocks_per_sm", [(0, 7168, 1), (2, 7168, 2), (3, 3584, 3), (1, 7168, 1)])
+@pytest.mark.parametrize("dtype,h,blocks_per_sm", [(0, 7168, 1), (2, 7168, 2), (3, 3584, 4), (1, 7168, 1)])
 def test_plan_query_blocks_per_sm(ep, dtype, h, blocks_per_sm):
-    """Rows under 8 KB take two engines per block and stages few enough that
-    two or more blocks share an SM's 228 KB (with each block's static shared
-    memory and the 1 KB the system keeps); rows of 8 KB and more, one block."""
+    """Rows between 4 and 8 KB take two engines per block and stages few
+    enough that two blocks share an SM's 228 KB (with each block's static
+    shared memory and the 1 KB the system keeps); rows of at most 4 KB, three
+    engines of 5 stages, as many blocks as fit; rows of 8 KB and more, one
+    block."""
     info = ep.ep_plan_query(_cfg(dtype=dtype, hiddenDim=h))
     assert info.scatterBlocks == 148 * blocks_per_sm
     per_block = info.scatterWarps * info.scatterStages * ((info.scatterChunkBytes + 127) // 128 * 128)
