@@ -103,9 +103,9 @@ typedef struct EpPlanInfo {
                                  blocks' totals (decoupled look-back, a bounded wait) and
                                  copies its own tokens; 0: two launches (route_count,
                                  scatter_rows). Results are identical either way. The
-                                 one-launch form suits full batches: where only the first
-                                 tokens of each rank are live, a few blocks do all the
-                                 copies. */
+                                 one-launch form suits full, small batches (up to ~20
+                                 tokens a block): where only the first tokens of each rank
+                                 are live, a few blocks do all the copies. */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
