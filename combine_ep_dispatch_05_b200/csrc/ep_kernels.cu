@@ -755,9 +755,10 @@ struct StaticFeed {
 // row piece by row piece through an S-stage shared-memory ring, S - kPend
 // loads ahead, with kPend items' bulk stores left draining when a stage is
 // refilled.
-// `ready` runs once every warp of the block has issued its first loads and
-// before any store (every thread of the block calls it, so it may hold a
-// block-wide barrier); false: copy nothing, only drain the loads.
+// `ready` runs once the engine has issued its first loads (its whole
+// lookahead, or p.earlyIssue of them) and before any store; every thread of
+// the block calls it, so it may hold a block-wide barrier. false: copy
+// nothing, only drain the loads.
 template <int kPend, class Feed, class Ready>
 __device__ __forceinline__ void copy_engine(const ScatterParams& p, const EngineSmem& es, int lane, Feed& feed,
                                             Ready&& ready) {
