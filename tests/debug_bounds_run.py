@@ -28,6 +28,13 @@ def main(mode: str) -> int:
         for wl in cases:
             run, _ = run_and_compare(wl.cfg(), make_inputs(wl))  # also asserts a clean error word
             run.close()
+        # the same through the fused one-launch dispatch (read at plan creation)
+        os.environ["EP_DISPATCH_FUSED"] = "1"
+        for wl in cases[:3]:
+            run, _ = run_and_compare(wl.cfg(), make_inputs(wl))
+            assert run.info.dispatchFused == 1
+            run.close()
+        del os.environ["EP_DISPATCH_FUSED"]
         # the scaled dispatch: scale rows checked as well
         wl = workload("pr599").replace(h=512)
         inputs = make_inputs(wl)
@@ -43,16 +50,20 @@ def main(mode: str) -> int:
         wl = workload("pr599").replace(h=1024)
         half = wl.max_recv // 2
         os.environ["EP_TEST_BOUNDS_ROWS"] = str(half)
-        run = DeviceRun(wl.cfg(), make_inputs(wl))
-        run.dispatch()
-        torch.cuda.synchronize()
-        err = run.error_word()
-        assert err & ep.EP_DEVERR_BOUNDS, err
-        counts = run.recv_count.cpu().numpy()
-        assert (counts > half).any(), counts  # the case reaches past the checked rows
-        for pe in range(wl.W):
-            assert bool((run.recv_x[pe, half:] == CANARY_BYTE).all()), pe  # stopped rows stayed unwritten
-        run.close()
+        for fused in ("0", "1"):  # both dispatch forms
+            os.environ["EP_DISPATCH_FUSED"] = fused
+            run = DeviceRun(wl.cfg(), make_inputs(wl))
+            assert run.info.dispatchFused == int(fused)
+            run.dispatch()
+            torch.cuda.synchronize()
+            err = run.error_word()
+            assert err & ep.EP_DEVERR_BOUNDS, err
+            counts = run.recv_count.cpu().numpy()
+            assert (counts > half).any(), counts  # the case reaches past the checked rows
+            for pe in range(wl.W):
+                assert bool((run.recv_x[pe, half:] == CANARY_BYTE).all()), pe  # stopped rows stayed unwritten
+            run.close()
+        del os.environ["EP_DISPATCH_FUSED"]
     print("ok")
     return 0
 
