@@ -162,8 +162,9 @@ def test_device_barrier_protocol_with_emulated_ranks(W):
 
 
 def test_device_barrier_gives_up_when_a_rank_stops_arriving():
-    """Rank 1 stops at round 3: the others complete 3 rounds, then their wait
-    gives up (about a second) with EP_DEVERR_TIMEOUT; no rank hangs."""
+    """Rank 1 stops arriving after its third barrier: the others pass 3
+    barriers, then their wait gives up (about a second) with EP_DEVERR_TIMEOUT;
+    no rank hangs."""
     done, errs, early = ep.ep_comm_barrier_selftest(4, 10, 1, 3)
     assert done == [3, 3, 3, 3] and early == [0] * 4
     assert errs[1] == 0 and all(errs[r] & ep.EP_DEVERR_TIMEOUT for r in (0, 2, 3))
