@@ -126,7 +126,9 @@ enum {
  * they record the problem here and keep going or return. */
 enum {
     EP_DEVERR_EXPERT_RANGE = 1, /* an expert id >= E was seen; it was treated as masked */
-    EP_DEVERR_TIMEOUT = 2,      /* a bounded wait on a shared-memory barrier gave up */
+    EP_DEVERR_TIMEOUT = 2,      /* a bounded wait gave up: on a copy's shared-memory barrier,
+                                   on another block's published totals (dispatchFused), or on
+                                   another rank's barrier flag (ep_comm.h) */
     EP_DEVERR_CAPACITY = 4,     /* a destination received more than maxRecv rows */
     EP_DEVERR_BOUNDS = 8        /* bounds-checking build only (libep_b200_debug.so): an access
                                    fell outside its buffer; it was skipped */
