@@ -55,7 +55,7 @@ class EpPlanInfo(ctypes.Structure):
                 ("scatterPend", ctypes.c_int32), ("combineDtype", ctypes.c_int32),
                 ("combineHidden", ctypes.c_int32), ("combineRowBytes", ctypes.c_int64),
                 ("yBytes", ctypes.c_int64), ("outBytes", ctypes.c_int64),
-                ("dispatchFused", ctypes.c_int32)]
+                ("dispatchFused", ctypes.c_int32), ("combineLoadBytes", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}

@@ -467,7 +467,7 @@ int ep_comm_combine(EpComm* c, const void* y, void* out, void* stream) {
         cp.rank = c->rank;
         cp.err = pp.err;
         cp.yBytes = (long long)c->maxLanding * c->crow;
-        e = ep::launch_combine(cp, c->cfg.dtype == EP_FP32, c->geo.combineBlocks, c->geo.combineWarps, s);
+        e = ep::launch_combine(cp, c->cfg.dtype == EP_FP32, false, c->geo.combineBlocks, c->geo.combineWarps, s);
         if (e != cudaSuccess) return cuda_err(e, "launch combine");
         return EP_OK;
     } catch (...) {

@@ -225,8 +225,9 @@ cudaError_t launch_route_count(const RouteParams& p, bool dense, cudaStream_t s)
 // stride W, no scan of its own).
 cudaError_t launch_scatter_rows(const ScatterParams& p, bool dense, int blocks, int warps, size_t smem,
                                 cudaStream_t s);
-// fp32: float32 combine leg (an fp32 plan); bf16 otherwise.
-cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s);
+// fp32: float32 combine leg (an fp32 plan); bf16 otherwise. wide: 32-byte
+// loads of y (y and rowBytes multiples of 32 bytes).
+cudaError_t launch_combine(const CombineParams& p, bool fp32, bool wide, int blocks, int warps, cudaStream_t s);
 // The fused dispatch of small batches: one launch, per-block routing
 // (dispatch_fused, kFusedWarps warps per block): opt-in, occupancy, launch.
 cudaError_t fused_set_smem(int W, int topk, size_t bytes);

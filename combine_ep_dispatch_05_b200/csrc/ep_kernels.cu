@@ -132,6 +132,13 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return v;
 }
 
+// 32 bytes (two 16-byte vectors) in one load; p must be 32-byte aligned.
+__device__ __forceinline__ void ld_stream_v8(const void* p, uint4& a, uint4& b) {
+    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+        : "l"(p));
+}
+
 // =====================================================================
 // Token hand-out shared by the scatter engines and the combine warps. Worker w
 // of nU takes tokens w, w + nU, ... for R rounds (no coordination), then the
@@ -152,15 +159,17 @@ struct TokenSource {
 };
 
 // P: the tokens that carry work (present tokens when the caller knows them,
-// else G); the counter is used only when there are 8 of them per worker.
-__device__ __forceinline__ TokenSource make_source(int w, int nU, int G, int32_t* ctr, int P) {
+// else G); the counter is used only when there are minPer of them per worker
+// (8 for the scatter; the combine's 4: B200, main shape at 2048 tokens a
+// rank, 235.4 us with the counter against 240.9 without).
+__device__ __forceinline__ TokenSource make_source(int w, int nU, int G, int32_t* ctr, int P, int minPer = 8) {
     TokenSource s;
     s.w = w;
     s.nU = nU;
     s.G = G;
     s.i = 0;
     s.ctr = ctr;
-    s.dyn = G >= 8 * nU && P >= 8 * nU;
+    s.dyn = G >= minPer * nU && P >= minPer * nU;
     s.R = s.dyn ? max(0, (int)((7LL * G) / (8LL * nU)) - 1) : (G + nU - 1) / nU;
     return s;
 }
@@ -1313,26 +1322,37 @@ struct CombineF32 {
 
 // One token's output row: for each group of kU 16-byte columns per lane, the
 // loads of up to kB destination rows are issued together, then folded in
-// destination order (so the result does not depend on kU or kB).
-template <class Elem, int kU, int kB>
+// destination order (so the result does not depend on kU, kB or kWide).
+// kWide: a lane's columns come in adjacent pairs, each pair one 32-byte load
+// (rows 32-byte aligned, V even: checked on the host).
+template <class Elem, int kU, int kB, bool kWide>
 __device__ __forceinline__ void combine_columns(const uint8_t* const* rows, const float* wts, int n, uint4* orow,
                                                 int V, int lane) {
-    for (int v0 = lane; v0 < V; v0 += 32 * kU) {
-        float acc[kU][Elem::kPer];
+    constexpr int kP = kWide ? 2 : 1;  // 16-byte columns per load
+    constexpr int kL = kU / kP;        // loads per lane and row in a pass
+    static_assert(kU % kP == 0, "kU must be a multiple of the load width");
+    const int VL = V / kP;             // loads across a row
+    for (int v0 = lane; v0 < VL; v0 += 32 * kL) {
+        float acc[kL][kP][Elem::kPer];
 #pragma unroll
-        for (int u = 0; u < kU; ++u)
+        for (int u = 0; u < kL; ++u)
 #pragma unroll
-            for (int i = 0; i < Elem::kPer; ++i) acc[u][i] = 0.0f;
+            for (int h = 0; h < kP; ++h)
+#pragma unroll
+                for (int i = 0; i < Elem::kPer; ++i) acc[u][h][i] = 0.0f;
         for (int b = 0; b < n; b += kB) {
-            uint4 val[kU][kB];
+            uint4 val[kL][kB][kP];
 #pragma unroll
             for (int i = 0; i < kB; ++i) {
                 if (b + i < n) {
                     const uint8_t* row = rows[b + i];
 #pragma unroll
-                    for (int u = 0; u < kU; ++u) {
+                    for (int u = 0; u < kL; ++u) {
                         const int v = v0 + 32 * u;
-                        if (v < V) val[u][i] = ld_stream_v4(row + (size_t)v * 16);
+                        if (v < VL) {
+                            if constexpr (kWide) ld_stream_v8(row + (size_t)v * 32, val[u][i][0], val[u][i][kP - 1]);
+                            else val[u][i][0] = ld_stream_v4(row + (size_t)v * 16);
+                        }
                     }
                 }
             }
@@ -1341,22 +1361,26 @@ __device__ __forceinline__ void combine_columns(const uint8_t* const* rows, cons
                 if (b + i < n) {
                     const float w = wts[b + i];
 #pragma unroll
-                    for (int u = 0; u < kU; ++u)
-                        if (v0 + 32 * u < V) Elem::fma(acc[u], w, val[u][i]);
+                    for (int u = 0; u < kL; ++u)
+                        if (v0 + 32 * u < VL)
+#pragma unroll
+                            for (int h = 0; h < kP; ++h) Elem::fma(acc[u][h], w, val[u][i][h]);
                 }
             }
         }
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < kL; ++u) {
             const int v = v0 + 32 * u;
-            if (v < V) orow[v] = Elem::pack(acc[u]);
+            if (v < VL)
+#pragma unroll
+                for (int h = 0; h < kP; ++h) orow[v * kP + h] = Elem::pack(acc[u][h]);
         }
     }
 }
 
 // kCols x kRows loads in flight per lane and pass; kMinBlocks blocks of 256
 // threads per SM bound the registers (65536 / (256 * kMinBlocks)).
-template <class Elem, int kCols, int kRows, int kMinBlocks>
+template <class Elem, int kCols, int kRows, int kMinBlocks, bool kWide>
 __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_kernel(CombineParams p) {
     __shared__ const uint8_t* s_row[kMaxCombineWarps][kMaxWorld];
     __shared__ float s_w[kMaxCombineWarps][kMaxWorld];
@@ -1387,7 +1411,7 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
     // number of destinations, so a purely static split would leave a tail);
     // the next token and its routing row are fetched one token ahead.
     TokenSource src = make_source(warp * gridDim.x + blockIdx.x, gridDim.x * (blockDim.x >> 5),
-                                  p.G, p.work, p.G);
+                                  p.G, p.work, p.G, 4);
     int next = 0;
     if (lane == 0) next = source_next(src);
     int g = __shfl_sync(kFull, next, 0);
@@ -1416,7 +1440,7 @@ __global__ void __launch_bounds__(kMaxCombineWarps * 32, kMinBlocks) ep_combine_
         }
         __syncwarp();
 
-        combine_columns<Elem, kCols, kRows>(s_row[warp], s_w[warp], n, orow, V, lane);
+        combine_columns<Elem, kCols, kRows, kWide>(s_row[warp], s_w[warp], n, orow, V, lane);
         __syncwarp();
         g = g_next;
     }
@@ -1703,8 +1727,14 @@ namespace {
 // 20.5 vs 24.8 us, skewed routing (2.7) 287 vs 304 us, main (5.3) 453.9 vs
 // 453.7 us; 3 x 6 took 476 us at main; 2 x 4 at 4 or 3 blocks per SM and
 // 1 x 8 at 4 were slower at main as well.
-template <class Elem>
-constexpr auto combine_kernel = ep_combine_kernel<Elem, 4, 4, 2>;
+// kWide: the same tile in 32-byte loads, for large batches (the host picks
+// it). B200, main shape (W=8, h=7168, topk 8), 16- vs 32-byte loads: 4096
+// tokens a rank 453.9 vs 441.7 us (fp32 rows 892.5 vs 868.2, skewed routing
+// 287.4 vs 279.5), 2048 tokens 235.4 vs 233.9, but 1024 tokens 128.7 vs 136.1
+// and the 512-token workload 20.6 vs 22.7: the wide loads pay only on large
+// batches.
+template <class Elem, bool kWide = false>
+constexpr auto combine_kernel = ep_combine_kernel<Elem, 4, 4, 2, kWide>;
 }  // namespace
 
 cudaError_t combine_blocks_per_sm(int warps, bool fp32, int* out) {
@@ -1748,9 +1778,12 @@ cudaError_t launch_dispatch_fused(const ScatterParams& p, int blocks, size_t sme
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_combine(const CombineParams& p, bool fp32, int blocks, int warps, cudaStream_t s) {
-    const cudaError_t e = fp32 ? launch_pdl(combine_kernel<CombineF32>, blocks, warps * 32, 0, s, p)
-                               : launch_pdl(combine_kernel<CombineBf16>, blocks, warps * 32, 0, s, p);
+cudaError_t launch_combine(const CombineParams& p, bool fp32, bool wide, int blocks, int warps, cudaStream_t s) {
+    const cudaError_t e =
+        fp32 ? (wide ? launch_pdl(combine_kernel<CombineF32, true>, blocks, warps * 32, 0, s, p)
+                     : launch_pdl(combine_kernel<CombineF32>, blocks, warps * 32, 0, s, p))
+             : (wide ? launch_pdl(combine_kernel<CombineBf16, true>, blocks, warps * 32, 0, s, p)
+                     : launch_pdl(combine_kernel<CombineBf16>, blocks, warps * 32, 0, s, p));
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

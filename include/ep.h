@@ -106,6 +106,10 @@ typedef struct EpPlanInfo {
                                  one-launch form suits full, small batches (up to ~20
                                  tokens a block): where only the first tokens of each rank
                                  are live, a few blocks do all the copies. */
+    int32_t combineLoadBytes; /* 32: the combine reads y in 32-byte loads (batches of more
+                                 than 16384 tokens, combine rows a multiple of 32 bytes; a
+                                 call whose y is not 32-byte aligned takes 16-byte loads);
+                                 16 otherwise. Results are identical either way. */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
@@ -143,7 +147,8 @@ int ep_cfg_check(const EpCfg* cfg);
 
 /* Host-only sizing: fill *info for cfg as a plan on a generic device would
  * resolve it (device = -1, numSMs = 0, geometry from a 148-SM B200 without
- * the geometry overrides; EP_DISPATCH_FUSED is honoured). Lets a
+ * the geometry overrides; EP_DISPATCH_FUSED and EP_COMBINE_WIDE are
+ * honoured). Lets a
  * caller size recv_x / recv_meta before creating a plan. Returns EP_OK or a
  * negative code. */
 int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
@@ -161,7 +166,9 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * default, 0 never), EP_SCATTER_SCAN ("route": route_count's last block scans
  * the tile counts even when the scatter could), EP_DISPATCH_DENSE (1 / 0: the
  * large-batch form of the split dispatch for every plan / for none; by default
- * plans of more than 16384 tokens, W*T, take it). Test hooks:
+ * plans of more than 16384 tokens, W*T, take it), EP_COMBINE_WIDE (1 / 0:
+ * 32-byte combine loads for every plan whose combine rows are a multiple of
+ * 32 bytes / for none; by default plans of more than 16384 tokens). Test hooks:
  * EP_TEST_UNREACHABLE_BARRIER=1 makes the one-launch dispatch's wait for the
  * earlier blocks' totals unreachable, so that the bounded wait runs out: every
  * block but the first (which waits on nothing and copies its own tokens)

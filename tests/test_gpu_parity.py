@@ -145,6 +145,65 @@ def test_dtype_random_small(dtype, fused, monkeypatch):
         run.close()
 
 
+@pytest.mark.parametrize("case", [
+    # W, T, h, k, nEpr, weights, maxRecv -- combine rows a multiple of 32 bytes
+    (3, 300, 272, 5, 3, True, 0),       # 544-byte rows: 17 loads a row, a partial warp
+    (8, 1000, 1024, 6, 8, True, 0),     # 4 tiles, ragged
+    (2, 40, 20000, 3, 4, True, 0),      # 40000-byte rows
+    (5, 77, 16, 7, 1, False, 500),      # one 32-byte load a row, no weights
+])
+def test_wide_combine_parity(case, monkeypatch):
+    """The combine's 32-byte loads, forced on small plans (EP_COMBINE_WIDE=1):
+    bit-exact against the oracle like the 16-byte loads."""
+    monkeypatch.setenv("EP_COMBINE_WIDE", "1")
+    W, T, h, k, nEpr, use_w, max_recv = case
+    rng = np.random.default_rng(hash(case) % (1 << 32))
+    cfg, inputs = _small_random_cfg(rng, W, T, h, k, nEpr, use_w, max_recv)
+    run, _ = run_and_compare(cfg, inputs)
+    assert run.info.combineLoadBytes == 32
+    run.close()
+
+
+@pytest.mark.parametrize("dtype", [1, 2, 3], ids=["fp32", "fp8", "fp4x2"])
+def test_wide_combine_dtypes_random_small(dtype, monkeypatch):
+    """32-byte combine loads over the other combine legs: fp32 (arbitrary bits,
+    NaN and inf included) and the bf16 leg of byte payloads."""
+    monkeypatch.setenv("EP_COMBINE_WIDE", "1")
+    rng = np.random.default_rng(300 + dtype)
+    wide = 0
+    for _ in range(8):
+        cfg, xb, idx, w = P.random_small_case(rng, dtype=dtype)
+        run, _ = run_and_compare(cfg, dict(x=xb, topk_idx=idx, topk_w=w))
+        wide += run.info.combineLoadBytes == 32
+        run.close()
+    assert wide > 0
+
+
+def test_wide_combine_misaligned_y_takes_narrow_loads(monkeypatch):
+    """A plan with 32-byte combine loads, called with a y that is 16- but not
+    32-byte aligned: the call takes the 16-byte loads, with the same results."""
+    monkeypatch.setenv("EP_COMBINE_WIDE", "1")
+    wl = workload("pr599").replace(h=1024)
+    cfg = wl.cfg()
+    inputs = make_inputs(wl)
+    run, ref = run_and_compare(cfg, inputs)
+    assert run.info.combineLoadBytes == 32
+    y = run.identity_y()
+    n = y.numel() * y.element_size()
+    buf = torch.empty(n + 64, dtype=torch.uint8, device="cuda")
+    off = (16 - buf.data_ptr() % 32) % 32  # the first 16- but not 32-byte aligned offset
+    yv = buf[off:off + n]
+    assert yv.data_ptr() % 32 == 16
+    yv.copy_(y.reshape(-1).view(torch.uint8))
+    run.reset_canaries()
+    run.dispatch()
+    run.combine(y=yv.view(y.dtype).view(y.shape))
+    torch.cuda.synchronize()
+    compare_combine(run, oracle.combine(cfg, ref["recv_x"], ref["slotmap"], ref["wsum"]))
+    assert run.error_word() == 0
+    run.close()
+
+
 @pytest.mark.parametrize("dtype,h", [(2, 7168), (3, 3584)], ids=["fp8", "fp4x2"])
 def test_dtype_main_dispatch(dtype, h):
     """The main workload with a one-byte payload, at full size: dispatch
