@@ -203,16 +203,19 @@ bool want_fused() {
     return v && std::strcmp(v, "1") == 0;
 }
 
-// The combine reads y in 32-byte loads for batches of more than 16384 tokens
-// whose combine rows are a multiple of 32 bytes (a call whose y is not 32-byte
-// aligned takes 16-byte loads): on B200 these ran 2.7 % faster at 32768
-// tokens and 5 % slower at 8192 (ep_kernels.cu, combine_kernel).
-// EP_COMBINE_WIDE=0/1 overrides the batch-size rule.
+// The combine reads y in 32-byte loads when its output, W*T combine rows, is
+// at least 192 MiB and the rows are a multiple of 32 bytes (a call whose y is
+// not 32-byte aligned takes 16-byte loads). B200, W=8, topk 8, output size ->
+// 16- vs 32-byte loads: 67 MB 72.7 vs 76.6 us, 117 MB 128.7 vs 136.1, 134 MB
+// (h=2048, 32768 tokens) 135.5 vs 140.0 and (h=4096, 16384 tokens) 139.9 vs
+// 144.8; 235 MB 235.4 vs 233.9, 268 MB 262.8 vs 259.6, 470 MB 454.0 vs 442.8
+// (h=7168) and 464.4 vs 452.5 (h=14336), 940 MB 902.5 vs 872.7.
+// EP_COMBINE_WIDE=0/1 overrides the size rule.
 bool combine_wide(const EpCfg* c) {
     if (combine_row_bytes(c) % 32 != 0) return false;
     const int env = env_int("EP_COMBINE_WIDE", -1, 0);
     if (env >= 0) return env != 0;
-    return (long long)c->worldSize * c->maxTokPerRank > 16384;
+    return (long long)c->worldSize * c->maxTokPerRank * combine_row_bytes(c) >= (192LL << 20);
 }
 
 void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {

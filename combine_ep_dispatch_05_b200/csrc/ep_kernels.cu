@@ -1727,12 +1727,12 @@ namespace {
 // 20.5 vs 24.8 us, skewed routing (2.7) 287 vs 304 us, main (5.3) 453.9 vs
 // 453.7 us; 3 x 6 took 476 us at main; 2 x 4 at 4 or 3 blocks per SM and
 // 1 x 8 at 4 were slower at main as well.
-// kWide: the same tile in 32-byte loads, for large batches (the host picks
+// kWide: the same tile in 32-byte loads, for large outputs (the host picks
 // it). B200, main shape (W=8, h=7168, topk 8), 16- vs 32-byte loads: 4096
 // tokens a rank 453.9 vs 441.7 us (fp32 rows 892.5 vs 868.2, skewed routing
 // 287.4 vs 279.5), 2048 tokens 235.4 vs 233.9, but 1024 tokens 128.7 vs 136.1
-// and the 512-token workload 20.6 vs 22.7: the wide loads pay only on large
-// batches.
+// and the 512-token workload 20.6 vs 22.7: the wide loads pay only once the
+// output is a few hundred MB.
 template <class Elem, bool kWide = false>
 constexpr auto combine_kernel = ep_combine_kernel<Elem, 4, 4, 2, kWide>;
 }  // namespace

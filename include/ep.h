@@ -106,10 +106,10 @@ typedef struct EpPlanInfo {
                                  one-launch form suits full, small batches (up to ~20
                                  tokens a block): where only the first tokens of each rank
                                  are live, a few blocks do all the copies. */
-    int32_t combineLoadBytes; /* 32: the combine reads y in 32-byte loads (batches of more
-                                 than 16384 tokens, combine rows a multiple of 32 bytes; a
-                                 call whose y is not 32-byte aligned takes 16-byte loads);
-                                 16 otherwise. Results are identical either way. */
+    int32_t combineLoadBytes; /* 32: the combine reads y in 32-byte loads (outBytes of at
+                                 least 192 MiB, combine rows a multiple of 32 bytes; a call
+                                 whose y is not 32-byte aligned takes 16-byte loads); 16
+                                 otherwise. Results are identical either way. */
 } EpPlanInfo;
 
 typedef struct EpPlan EpPlan;
@@ -168,7 +168,7 @@ int ep_plan_query(const EpCfg* cfg, EpPlanInfo* info);
  * large-batch form of the split dispatch for every plan / for none; by default
  * plans of more than 16384 tokens, W*T, take it), EP_COMBINE_WIDE (1 / 0:
  * 32-byte combine loads for every plan whose combine rows are a multiple of
- * 32 bytes / for none; by default plans of more than 16384 tokens). Test hooks:
+ * 32 bytes / for none; by default plans whose outBytes is at least 192 MiB). Test hooks:
  * EP_TEST_UNREACHABLE_BARRIER=1 makes the one-launch dispatch's wait for the
  * earlier blocks' totals unreachable, so that the bounded wait runs out: every
  * block but the first (which waits on nothing and copies its own tokens)

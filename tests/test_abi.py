@@ -180,17 +180,20 @@ def test_plan_query_dispatch_form(ep, kw, fused, monkeypatch):
 
 
 @pytest.mark.parametrize("kw,load", [
-    (dict(), 32),                                               # 32768 tokens, 14336-byte rows
+    (dict(), 32),                                               # output 470 MB, 14336-byte rows
     (dict(dtype=1), 32),                                        # fp32 leg, 28672-byte rows
     (dict(dtype=3, hiddenDim=3584), 32),                        # fp4x2 in, bf16 leg of 14336 bytes
-    (dict(maxTokPerRank=2048, maxRecv=16384), 16),              # 16384 tokens: not above the switch
+    (dict(maxTokPerRank=2048, maxRecv=16384), 32),              # 235 MB
+    (dict(maxTokPerRank=1024, maxRecv=8192), 16),               # 117 MB
+    (dict(hiddenDim=2048), 16),                                 # 134 MB
+    (dict(hiddenDim=14336, maxTokPerRank=2048, maxRecv=16384), 32),  # 470 MB from 16384 tokens
     (dict(worldSize=4, maxTokPerRank=512, numExpertPerRank=8, numExpertPerToken=6, maxRecv=0), 16),
     (dict(hiddenDim=7176), 16),                                 # 14352-byte rows: not a multiple of 32
 ])
 def test_plan_query_combine_load_width(ep, kw, load, monkeypatch):
-    """The combine reads y in 32-byte loads for batches of more than 16384
-    tokens whose combine rows are a multiple of 32 bytes; EP_COMBINE_WIDE
-    overrides the batch-size rule but never the row rule."""
+    """The combine reads y in 32-byte loads when its output is at least 192 MiB
+    and its rows are a multiple of 32 bytes; EP_COMBINE_WIDE overrides the size
+    rule but never the row rule."""
     cfg = _cfg(**kw)
     assert ep.ep_plan_query(cfg).combineLoadBytes == load
     row_ok = ep.ep_plan_query(cfg).combineRowBytes % 32 == 0
