@@ -467,6 +467,9 @@ int ep_comm_combine(EpComm* c, const void* y, void* out, void* stream) {
         cp.rank = c->rank;
         cp.err = pp.err;
         cp.yBytes = (long long)c->maxLanding * c->crow;
+        // 16-byte loads: a rank's output is its own T tokens, W times below a
+        // one-GPU plan's, and on B200 the 32-byte loads only paid from outputs of
+        // about 200 MB (ep_abi.cu, combine_wide).
         e = ep::launch_combine(cp, c->cfg.dtype == EP_FP32, false, c->geo.combineBlocks, c->geo.combineWarps, s);
         if (e != cudaSuccess) return cuda_err(e, "launch combine");
         return EP_OK;
