@@ -203,6 +203,13 @@ bool want_fused() {
     return v && std::strcmp(v, "1") == 0;
 }
 
+}  // namespace
+
+namespace ep {
+bool combine_wide_loads(long long outBytes, long long rowBytes);  // defined below
+}
+
+namespace {
 // The combine reads y in 32-byte loads when its output, W*T combine rows, is
 // at least 192 MiB and the rows are a multiple of 32 bytes (a call whose y is
 // not 32-byte aligned takes 16-byte loads). B200, W=8, topk 8, output size ->
@@ -212,10 +219,8 @@ bool want_fused() {
 // (h=7168) and 464.4 vs 452.5 (h=14336), 940 MB 902.5 vs 872.7.
 // EP_COMBINE_WIDE=0/1 overrides the size rule.
 bool combine_wide(const EpCfg* c) {
-    if (combine_row_bytes(c) % 32 != 0) return false;
-    const int env = env_int("EP_COMBINE_WIDE", -1, 0);
-    if (env >= 0) return env != 0;
-    return (long long)c->worldSize * c->maxTokPerRank * combine_row_bytes(c) >= (192LL << 20);
+    return ep::combine_wide_loads((long long)c->worldSize * c->maxTokPerRank * combine_row_bytes(c),
+                                  combine_row_bytes(c));
 }
 
 void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
@@ -251,6 +256,13 @@ void fill_info(const EpCfg* c, const Geometry& geo, EpPlanInfo* info) {
 
 namespace ep {
 void set_last_error(const char* msg) { std::snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+
+bool combine_wide_loads(long long outBytes, long long rowBytes) {
+    if (rowBytes % 32 != 0) return false;
+    const int env = env_int("EP_COMBINE_WIDE", -1, 0);
+    if (env >= 0) return env != 0;
+    return outBytes >= (192LL << 20);
+}
 
 int fail_code(int code, const char* msg) { return fail(code, "%s", msg); }
 

@@ -23,6 +23,12 @@
 #include "ep_comm.h"
 #include "ep_internal.h"
 
+namespace ep {
+// Whether the combine reads y in 32-byte loads (ep_abi.cu): outputs of at
+// least 192 MiB with rows a multiple of 32 bytes, unless EP_COMBINE_WIDE says.
+bool combine_wide_loads(long long outBytes, long long rowBytes);
+}
+
 namespace {
 
 constexpr char kMagic[8] = {'E', 'P', 'C', 'O', 'M', 'M', '1', '\0'};
@@ -467,10 +473,11 @@ int ep_comm_combine(EpComm* c, const void* y, void* out, void* stream) {
         cp.rank = c->rank;
         cp.err = pp.err;
         cp.yBytes = (long long)c->maxLanding * c->crow;
-        // 16-byte loads: a rank's output is its own T tokens, W times below a
-        // one-GPU plan's, and on B200 the 32-byte loads only paid from outputs of
-        // about 200 MB (ep_abi.cu, combine_wide).
-        e = ep::launch_combine(cp, c->cfg.dtype == EP_FP32, false, c->geo.combineBlocks, c->geo.combineWarps, s);
+        // 32-byte loads by the one-GPU plans' rule on this rank's output (its T
+        // tokens); the landing rows start 256-byte aligned, crow apart.
+        const bool wide = ep::combine_wide_loads((long long)c->T * c->crow, c->crow) &&
+                          reinterpret_cast<uintptr_t>(cp.y) % 32 == 0;
+        e = ep::launch_combine(cp, c->cfg.dtype == EP_FP32, wide, c->geo.combineBlocks, c->geo.combineWarps, s);
         if (e != cudaSuccess) return cuda_err(e, "launch combine");
         return EP_OK;
     } catch (...) {

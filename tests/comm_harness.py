@@ -108,9 +108,11 @@ def check_step(torch, ep, comm, wl, rank):
 
 
 def rank_main(rank, W, port, spec, q):
-    """spec: {"workload": name, "replace": {...}, "seeds": [...], "sync": 0|1}.
+    """spec: {"workload": name, "replace": {...}, "seeds": [...], "sync": 0|1,
+    "env": {...} (optional: environment of the library in this rank)}.
     Runs one step per seed on one communicator."""
     try:
+        os.environ.update(spec.get("env", {}))
         torch, dist = _setup(rank, W, port, spec.get("timeout_s", 60))
         import combine_ep_dispatch_05_b200 as ep
         from synth.inputs import workload

@@ -65,6 +65,10 @@ def _spawn(target, W, spec, extra=()):
                                           "n_epr": 8}, "seeds": [4]}),  # hot destination, W not a power of 2
     (2, {"workload": "tiny", "replace": {"dtype": 1, "h": 64}, "seeds": [6]}),     # fp32 rows and combine
     (2, {"workload": "tiny", "replace": {"dtype": 2, "h": 256}, "seeds": [7]}),    # fp8 rows, bf16 combine
+    (3, {"workload": "pr599", "replace": {"h": 1040}, "seeds": [8],                # the combine's 32-byte
+         "env": {"EP_COMBINE_WIDE": "1"}}),                                          # loads, 2080-byte rows
+    (2, {"workload": "tiny", "replace": {"dtype": 1, "h": 72}, "seeds": [9],       # and over fp32 rows
+         "env": {"EP_COMBINE_WIDE": "1"}}),
 ])
 def test_ranks_in_processes_match_the_oracle(W, spec):
     spec = dict(spec, sync=ep.EP_SYNC_HOST)
