@@ -18,9 +18,10 @@
 //                loops (WarpCopy on gfx9xx, one TDM tile per token on gfx1250,
 //                design page §9 and PR #599) are the prior art.
 // combine = combine (one launch)
-//   combine      one warp per token: up to 8 destination rows in flight per
-//                16-byte column, float32 fma fold in destPe order; bf16 RNE out
-//                (float32 out, unrounded, for a float32 plan).
+//   combine      one warp per token: 4 destination rows x 4 16-byte columns
+//                in flight per lane (read as 32-byte loads for large outputs),
+//                float32 fma fold in destPe order; bf16 RNE out (float32 out,
+//                unrounded, for a float32 plan).
 // Option: dispatch_fused, the whole dispatch of a small batch in one launch
 // (each block routes and copies its own share of the batch; the bases come
 // from the other blocks' published counts by decoupled look-back).
